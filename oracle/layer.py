@@ -1,0 +1,298 @@
+"""Retained-token Llama decoder layer, forward and backward (oracle).
+
+What the pages fix:
+* Jenga notes §4.1 / Jenga summary §4.1 (Fig. 5): per layer, the retained tokens
+  run through the attention block and the MLP block; eliminated tokens skip both.
+* §4.4 / §4.4.1 (Fig. 9): retained rows are read from the original input and the
+  sub-block outputs are added in place into those rows (residual add); eliminated
+  rows keep their input, so their gradient is the identity.
+* §4.4.2 (Fig. 10): segment-based peak cutting -- the sequence is cut into
+  segments, each segment's activations are rebuilt, its gradient computed and its
+  activations dropped; gradients are aggregated across segments.
+* Experimental setup: Llama-2 models (RMSNorm, rotary positions, SiLU-gated MLP),
+  LoRA fine-tuning, mixed bf16/fp32.
+
+Readings (the pages are silent on these):
+* RoPE uses the tokens' ORIGINAL positions; attention is causal among retained
+  tokens only (eliminated tokens are neither queries nor keys).  Because the kept
+  block list ascends, causality in compact order equals causality in original order.
+* RMSNorm eps 1e-5, learned gains applied after normalisation; RoPE theta 10000 with
+  the rotate-half convention (pairs d and d + D/2); LoRA on q_proj and v_proj,
+  delta W = scale * B @ A, no dropout, no biases.
+* One index set per layer serves both sub-blocks.
+* bf16 storage rounding (``rnd=True``) at: xn (normed attention input), q and k after
+  RoPE, v, the attention output o, h (after the attention residual add), hn (normed
+  MLP input), a = SiLU(g) * u, the layer output, and the input gradient dX.  All other
+  arithmetic is float64.  LoRA intermediates t = xn A^T and LoRA gradients stay
+  unrounded.  ``rnd=False`` gives the exact float64 layer.
+* Segmented backward: consecutive segments of ``segment_tokens`` retained rows (last
+  one short), processed last segment first; key/value gradients accumulate across
+  query segments, so a key segment is complete once every later query segment has
+  been processed.  Equal to the unsegmented backward up to float64 summation order.
+
+Shapes: x [n, h]; weights [out, in]; q, k, v, o [n, H, D]; LoRA A [r, h], B [H*D, r].
+"""
+from dataclasses import dataclass
+
+import numpy as np
+
+from .bf16 import from_bits, round_bf16
+from .movement import retained_rows
+
+
+@dataclass
+class Weights:
+    wq: np.ndarray
+    wk: np.ndarray
+    wv: np.ndarray
+    wo: np.ndarray
+    wg: np.ndarray
+    wu: np.ndarray
+    wd: np.ndarray
+    g1: np.ndarray
+    g2: np.ndarray
+    aq: np.ndarray
+    bq: np.ndarray
+    av: np.ndarray
+    bv: np.ndarray
+    heads: int
+    head_dim: int
+    eps: float = 1e-5
+    theta: float = 10000.0
+    lora_scale: float = 1.0
+
+    @classmethod
+    def from_bits(cls, p, shape):
+        """Build float64 weights from bf16 bit patterns (``synth.LayerParams``)."""
+        return cls(wq=from_bits(p.wq), wk=from_bits(p.wk), wv=from_bits(p.wv), wo=from_bits(p.wo),
+                   wg=from_bits(p.wg), wu=from_bits(p.wu), wd=from_bits(p.wd),
+                   g1=from_bits(p.attn_norm), g2=from_bits(p.mlp_norm),
+                   aq=from_bits(p.aq), bq=from_bits(p.bq), av=from_bits(p.av), bv=from_bits(p.bv),
+                   heads=shape.heads, head_dim=shape.head_dim, eps=shape.rms_eps,
+                   theta=shape.rope_theta, lora_scale=shape.lora_scale)
+
+
+def _r(x, rnd):
+    return round_bf16(x) if rnd else x
+
+
+# ------------------------------------------------------------------ building blocks
+
+
+def rms_norm(x, g, eps):
+    """y = x / sqrt(mean(x^2) + eps) * g (per row); returns y and the row factor."""
+    rstd = 1.0 / np.sqrt((x * x).mean(axis=1) + eps)
+    return x * rstd[:, None] * g[None, :], rstd
+
+
+def rms_norm_bwd(dy, x, g, rstd):
+    """Gradient of ``rms_norm`` w.r.t. x (derived by hand):
+    dx_j = r g_j dy_j - x_j r^3 / N * sum_i dy_i g_i x_i."""
+    N = x.shape[1]
+    dyg = dy * g[None, :]
+    dot = (dyg * x).sum(axis=1)
+    return dyg * rstd[:, None] - x * (rstd ** 3 * dot / N)[:, None]
+
+
+def rope_cos_sin(pos, D, theta):
+    """cos/sin of angle pos * theta^(-2i/D), i = 0 .. D/2-1; shape [n, D/2]."""
+    inv = theta ** (-np.arange(0, D, 2, dtype=np.float64) / D)
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * inv[None, :]
+    return np.cos(ang), np.sin(ang)
+
+
+def rope(x, cos, sin):
+    """Rotate-half rotary embedding of x [n, H, D]."""
+    half = x.shape[-1] // 2
+    x1, x2 = x[..., :half], x[..., half:]
+    c, s = cos[:, None, :], sin[:, None, :]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def rope_bwd(dy, cos, sin):
+    """Transpose of ``rope`` (rotation by the negative angle)."""
+    half = dy.shape[-1] // 2
+    d1, d2 = dy[..., :half], dy[..., half:]
+    c, s = cos[:, None, :], sin[:, None, :]
+    return np.concatenate([d1 * c + d2 * s, d2 * c - d1 * s], axis=-1)
+
+
+def sigmoid(z):
+    e = np.exp(-np.abs(z))
+    return np.where(z >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def silu(z):
+    return z * sigmoid(z)
+
+
+def silu_grad(z):
+    s = sigmoid(z)
+    return s * (1.0 + z * (1.0 - s))
+
+
+def attention_fwd(q, k, v, chunk=1024):
+    """Causal softmax attention per head (softmax(q k^T / sqrt(D)) v, keys j <= i).
+
+    Returns o [n, H, D] and the row log-sum-exp [H, n] of the scaled logits."""
+    n, H, D = q.shape
+    scale = 1.0 / np.sqrt(D)
+    o = np.zeros_like(q)
+    lse = np.zeros((H, n))
+    jj = np.arange(n)
+    for h in range(H):
+        for i0 in range(0, n, chunk):
+            i1 = min(n, i0 + chunk)
+            s = (q[i0:i1, h] @ k[:i1, h].T) * scale
+            s = np.where(jj[None, :i1] <= np.arange(i0, i1)[:, None], s, -np.inf)
+            m = s.max(axis=1, keepdims=True)
+            p = np.exp(s - m)
+            l = p.sum(axis=1, keepdims=True)
+            o[i0:i1, h] = (p / l) @ v[:i1, h]
+            lse[h, i0:i1] = (m + np.log(l))[:, 0]
+    return o, lse
+
+
+def attention_bwd_rows(q, k, v, do, r0, r1, dk_acc, dv_acc, chunk=1024):
+    """Backward of ``attention_fwd`` for the query rows [r0, r1).
+
+    Returns dq for those rows and ADDS their contribution to dk_acc / dv_acc (keys
+    [0, r1)).  dS = P * (dP - rowsum(P * dP)), dP = dO V^T, dQ = dS K / sqrt(D),
+    dK = dS^T Q / sqrt(D), dV = P^T dO (textbook softmax-attention backward)."""
+    n, H, D = q.shape
+    scale = 1.0 / np.sqrt(D)
+    dq = np.zeros((r1 - r0, H, D))
+    jj = np.arange(n)
+    for h in range(H):
+        for i0 in range(r0, r1, chunk):
+            i1 = min(r1, i0 + chunk)
+            s = (q[i0:i1, h] @ k[:i1, h].T) * scale
+            s = np.where(jj[None, :i1] <= np.arange(i0, i1)[:, None], s, -np.inf)
+            m = s.max(axis=1, keepdims=True)
+            p = np.exp(s - m)
+            p /= p.sum(axis=1, keepdims=True)
+            dp = do[i0:i1, h] @ v[:i1, h].T
+            delta = (p * dp).sum(axis=1, keepdims=True)
+            ds = p * (dp - delta)
+            dq[i0 - r0:i1 - r0, h] = (ds @ k[:i1, h]) * scale
+            dk_acc[:i1, h] += (ds.T @ q[i0:i1, h]) * scale
+            dv_acc[:i1, h] += p.T @ do[i0:i1, h]
+    return dq
+
+
+# ------------------------------------------------------------------ layer
+
+
+def layer_fwd(x, pos, W: Weights, rnd=True):
+    """Llama decoder layer on the retained rows x [n, h] at original positions ``pos``.
+
+    Returns (out [n, h], ctx) where ctx holds what the backward needs."""
+    x = np.asarray(x, np.float64)
+    n, hdim = x.shape
+    H, D, s = W.heads, W.head_dim, W.lora_scale
+    xn, rstd1 = rms_norm(x, W.g1, W.eps)
+    xn = _r(xn, rnd)
+    tq = xn @ W.aq.T
+    tv = xn @ W.av.T
+    q_lin = (xn @ W.wq.T + s * (tq @ W.bq.T)).reshape(n, H, D)
+    k_lin = (xn @ W.wk.T).reshape(n, H, D)
+    v = _r((xn @ W.wv.T + s * (tv @ W.bv.T)).reshape(n, H, D), rnd)
+    cos, sin = rope_cos_sin(pos, D, W.theta)
+    q = _r(rope(q_lin, cos, sin), rnd)
+    k = _r(rope(k_lin, cos, sin), rnd)
+    o, lse = attention_fwd(q, k, v)
+    o = _r(o, rnd)
+    h = _r(x + o.reshape(n, H * D) @ W.wo.T, rnd)
+    hn, rstd2 = rms_norm(h, W.g2, W.eps)
+    hn = _r(hn, rnd)
+    gt = hn @ W.wg.T
+    ut = hn @ W.wu.T
+    a = _r(silu(gt) * ut, rnd)
+    out = _r(h + a @ W.wd.T, rnd)
+    ctx = dict(x=x, pos=np.asarray(pos), xn=xn, rstd1=rstd1, tq=tq, tv=tv, q=q, k=k, v=v, o=o,
+               lse=lse, h=h, hn=hn, rstd2=rstd2, gt=gt, ut=ut, a=a, cos=cos, sin=sin, rnd=rnd)
+    return out, ctx
+
+
+def _segments(n, seg):
+    if seg is None or seg <= 0 or seg >= n:
+        return [(0, n)] if n else []
+    return [(s0, min(n, s0 + seg)) for s0 in range(0, n, seg)]
+
+
+def layer_bwd(ctx, G, W: Weights, segment_tokens=None):
+    """Backward of ``layer_fwd`` for loss = sum(out * G) (so dOut = G).
+
+    Frozen base weights get no gradient.  Returns (dx [n, h], grads) with grads the
+    LoRA gradients daq [r, h], dbq [H*D, r], dav, dbv.  ``segment_tokens`` splits the
+    retained rows into consecutive segments processed last-first (module docstring)."""
+    G = np.asarray(G, np.float64)
+    x, xn, h, hn = ctx["x"], ctx["xn"], ctx["h"], ctx["hn"]
+    q, k, v, o = ctx["q"], ctx["k"], ctx["v"], ctx["o"]
+    cos, sin = ctx["cos"], ctx["sin"]
+    n, hdim = x.shape
+    H, D, s = W.heads, W.head_dim, W.lora_scale
+    r = W.aq.shape[0]
+    dx = np.zeros((n, hdim))
+    grads = dict(daq=np.zeros_like(W.aq), dbq=np.zeros_like(W.bq),
+                 dav=np.zeros_like(W.av), dbv=np.zeros_like(W.bv))
+    dk_acc = np.zeros((n, H, D))
+    dv_acc = np.zeros((n, H, D))
+    for (s0, s1) in reversed(_segments(n, segment_tokens)):
+        sl = slice(s0, s1)
+        # --- MLP block: out = h + (silu(hn Wg^T) * (hn Wu^T)) Wd^T
+        Gs = G[sl]
+        da = Gs @ W.wd
+        gt, ut = ctx["gt"][sl], ctx["ut"][sl]
+        dut = da * silu(gt)
+        dgt = da * ut * silu_grad(gt)
+        dhn = dgt @ W.wg + dut @ W.wu
+        dh = Gs + rms_norm_bwd(dhn, h[sl], W.g2, ctx["rstd2"][sl])
+        # --- attention block: h = x + o Wo^T
+        do_full = np.zeros((n, H, D))
+        do_full[sl] = (dh @ W.wo).reshape(s1 - s0, H, D)
+        dq = attention_bwd_rows(q, k, v, do_full, s0, s1, dk_acc, dv_acc)
+        # keys/values of this segment are complete now
+        dq_lin = rope_bwd(dq, cos[sl], sin[sl]).reshape(s1 - s0, H * D)
+        dk_lin = rope_bwd(dk_acc[sl], cos[sl], sin[sl]).reshape(s1 - s0, H * D)
+        dv = dv_acc[sl].reshape(s1 - s0, H * D)
+        dtq = s * (dq_lin @ W.bq)                      # [ns, r]
+        dtv = s * (dv @ W.bv)
+        grads["dbq"] += s * (dq_lin.T @ ctx["tq"][sl])
+        grads["dbv"] += s * (dv.T @ ctx["tv"][sl])
+        grads["daq"] += dtq.T @ xn[sl]
+        grads["dav"] += dtv.T @ xn[sl]
+        dxn = dq_lin @ W.wq + dk_lin @ W.wk + dv @ W.wv + dtq @ W.aq + dtv @ W.av
+        dx[sl] = dh + rms_norm_bwd(dxn, x[sl], W.g1, ctx["rstd1"][sl])
+    del r
+    return _r(dx, ctx["rnd"]), grads
+
+
+# ------------------------------------------------------------------ whole sequence
+
+
+def sparse_layer_fwd(X, idx, n_kept, blk, W: Weights, rnd=True):
+    """Layer on the kept blocks of X [S, h]; eliminated rows pass through unchanged."""
+    X = np.asarray(X, np.float64)
+    rows = retained_rows(idx, n_kept, blk)
+    Xo = X.copy()
+    if rows.size == 0:
+        return Xo, None
+    out, ctx = layer_fwd(X[rows], rows, W, rnd)
+    Xo[rows] = out
+    ctx["rows"] = rows
+    return Xo, ctx
+
+
+def sparse_layer_bwd(ctx, G, W: Weights, segment_tokens=None):
+    """dX = G on eliminated rows; the layer backward on retained rows."""
+    G = np.asarray(G, np.float64)
+    dX = G.copy()
+    if ctx is None:
+        z = dict(daq=np.zeros_like(W.aq), dbq=np.zeros_like(W.bq),
+                 dav=np.zeros_like(W.av), dbv=np.zeros_like(W.bv))
+        return dX, z
+    rows = ctx["rows"]
+    dx, grads = layer_bwd(ctx, G[rows], W, segment_tokens)
+    dX[rows] = dx
+    return dX, grads
