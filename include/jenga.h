@@ -1,0 +1,257 @@
+/*
+ * jenga.h -- C ABI of the token-sparse layer library (B200, sm_100a).
+ *
+ * The operations follow the Jenga paper ("Jenga: Enhancing LLM Long-Context
+ * Fine-tuning with Contextual Token Sparsity", ATC'25), as described by the
+ * papercache.org deep notes ("Jenga notes") and the aipaper.cc summary ("Jenga
+ * summary"):
+ *   - block informativeness scoring      Jenga summary §4.2.1 Eq. (1), §4.2.2 Eq. (2), §4.2.3
+ *   - threshold selection                Jenga notes §4.2 Algorithm 1; Jenga summary §4.2.3
+ *   - permutation-free gather / in-place residual scatter-add
+ *                                        Jenga notes §4.4; Jenga summary §4.4.1 (Fig. 9)
+ *   - retained-token layer forward/backward, segment-wise gradients
+ *                                        Jenga summary §4.1 (Fig. 5), §4.4.2 (Fig. 10)
+ *   - block-score predictor              Jenga notes §4.3; Jenga summary §4.3.1 (Fig. 8)
+ *
+ * Conventions
+ * -----------
+ *  * Every function returns jenga_status; none aborts.  jenga_last_error() gives
+ *    the text of the last failure on the calling host thread.
+ *  * All tensor pointers are CALLER-OWNED DEVICE memory.  The library never
+ *    allocates or frees device memory; scratch space is passed in as a workspace
+ *    whose size is given by the matching *_workspace_bytes / *_bytes query.
+ *  * Every call is asynchronous on the given CUDA stream (NULL = legacy default
+ *    stream) and does not synchronise the host.  Argument checks that need only
+ *    host values are done before launch (JENGA_EINVAL).  Faults that only the
+ *    device can see (an index out of range, an n_kept above the stated maximum, a
+ *    pipeline wait that ran past its time budget) are recorded in a device error
+ *    word; jenga_check_device_status() synchronises the stream, reads and clears it.
+ *  * Layouts are row-major.  Activations are token-major [B, S, hidden]; per-head
+ *    tensors are [B, S, H, D] (a token's H*D values contiguous, token pitch ld);
+ *    weights are [out, in] (PyTorch Linear).  bf16 = IEEE bfloat16 bits.
+ *  * Block indices are int32, ascending, kept blocks first; entries past n_kept
+ *    are -1.  Token t of kept block i (0 <= t < blk) is sequence row
+ *    idx[i] * blk + t and compact row i * blk + t.
+ */
+#ifndef JENGA_H_
+#define JENGA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define JENGA_API __attribute__((visibility("default")))
+#else
+#define JENGA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* jenga_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+  JENGA_OK = 0,
+  JENGA_EINVAL = 1,       /* bad argument (shape, pointer, mode) */
+  JENGA_EUNSUPPORTED = 2, /* valid but not implemented for these sizes / dtypes */
+  JENGA_ECUDA = 3,        /* a CUDA runtime call failed */
+  JENGA_ETIMEOUT = 4,     /* a device-side wait ran past its budget */
+  JENGA_EWORKSPACE = 5,   /* workspace / saved buffer smaller than required */
+  JENGA_EINTERNAL = 6,    /* device detected an internal inconsistency (bad index) */
+} jenga_status;
+
+typedef enum { JENGA_F32 = 0, JENGA_BF16 = 1 } jenga_dtype;
+
+typedef enum {
+  /* Jenga summary §4.2.1 Eq. (1) with S_ij the causal softmax probability of query i on
+   * key j (diagonal included), summed over queries and heads (no 1/N_head), then over
+   * the tokens of each key block (§4.2.3).  Per sequence the scores sum to H * S. */
+  JENGA_SCORE_SOFTMAX_MASS = 0,
+  /* Jenga summary §4.2.2 Eq. (2): for each (query block, key block) score block the
+   * max over causal entries of sum_h max(q_i.k_j/sqrt(D), 0) / N_head, summed over
+   * query blocks (§4.2.3). */
+  JENGA_SCORE_PAPER_BLOCKMAX = 1,
+} jenga_score_mode;
+
+typedef enum {
+  JENGA_SELECT_MEAN_GE = 0,   /* keep score >= average block score (Algorithm 1, step 1) */
+  JENGA_SELECT_TOPK_FRAC = 1, /* keep k = ceil(param * nb - 1e-6) blocks, rank (score desc, index asc) */
+  JENGA_SELECT_ABS_GE = 2,    /* keep score >= param */
+  JENGA_SELECT_TOPK = 3,      /* keep k = (int)param blocks, same ranking */
+} jenga_select_mode;
+
+/* ------------------------------------------------------------------ status */
+JENGA_API const char* jenga_status_string(jenga_status st);
+/* Copies the last error message of this host thread (NUL-terminated, truncated). */
+JENGA_API size_t jenga_last_error(char* buf, size_t len);
+/* Synchronises `stream`, returns the first device-recorded fault since the last call
+ * (JENGA_OK if none) and clears it.  detail (nullable) gets {site, info}. */
+JENGA_API jenga_status jenga_check_device_status(jenga_stream_t stream, uint32_t* detail2);
+/* Device-side wait budget in nanoseconds for every pipeline wait (default 2e9).
+ * Applies to launches made after the call. */
+JENGA_API jenga_status jenga_set_wait_budget_ns(uint64_t ns);
+/* Library version and build string. */
+JENGA_API const char* jenga_version(void);
+/* Launch timing for measurement: while enabled, every kernel the library launches is
+ * bracketed by two CUDA events recorded on the launch's own stream (host-thread
+ * local use; no device memory).  Enabling clears previous records. */
+JENGA_API jenga_status jenga_profile_enable(int on);
+/* Waits for the recorded events, writes {"kernel": {"launches": n, "ms": total}, ...}
+ * (NUL-terminated, truncated to len) and clears the records; returns the full length. */
+JENGA_API size_t jenga_profile_report(char* buf, size_t len);
+
+/* ------------------------------------------------------------------ scoring
+ * jenga_score_blocks -- block informativeness (a2 + a3 of the path).
+ *   q, k     : [B, S, H, D] of dtype dt; token pitch ldq / ldk elements (>= H*D),
+ *              batch pitch S * ld.  q and k may alias one fused [S, 2*H*D] buffer.
+ *   blk      : tokens per block, S % blk == 0; nb = S / blk.
+ *   causal   : 1 = query i attends keys j <= i (the scoring the path uses); 0 = all j.
+ *   scores   : [B, nb] fp32 out.  Deterministic (fixed reduction order).
+ *   ws       : workspace of jenga_score_workspace_bytes(...) bytes (row LSE [B,H,S]
+ *              and per-head partial scores [B,H,nb]).
+ * fp32 inputs use exact fp32 SIMT dot products (D <= 128); bf16 inputs use the
+ * tensor-core kernels and need D == 128.  Errors: EINVAL (shapes), EWORKSPACE,
+ * EUNSUPPORTED (D / dtype / mode combination not built). */
+JENGA_API size_t jenga_score_workspace_bytes(int B, int S, int H, int D, int blk);
+JENGA_API jenga_status jenga_score_blocks(const void* q, int64_t ldq, const void* k, int64_t ldk, int B, int S, int H,
+                                int D, int blk, int causal, jenga_dtype dt, jenga_score_mode mode,
+                                float* scores, void* ws, size_t ws_bytes, jenga_stream_t stream);
+
+/* ------------------------------------------------------------------ selection
+ * jenga_select -- threshold / top-k selection and compaction (a4).
+ *   scores : [B, nb] fp32 (NaN compares as -inf).
+ *   idx    : [B, nb] int32 out, ascending kept block indices then -1.
+ *   n_kept : [B] int32 out.   mask : [B, nb] uint8 out (nullable).
+ *   ws     : jenga_select_workspace_bytes(B, nb) bytes (0 for nb <= 8192).
+ * MEAN_GE forms the average as a float64 sum of the scores divided by nb and
+ * compares each score as float64.  TOPK modes are exact (rank counting).  Large nb
+ * (> 8192) supports MEAN_GE and ABS_GE (multi-CTA ballot + prefix-sum compaction). */
+JENGA_API size_t jenga_select_workspace_bytes(int B, int nb);
+JENGA_API jenga_status jenga_select(const float* scores, int B, int nb, jenga_select_mode mode, float param,
+                          int32_t* idx, int32_t* n_kept, uint8_t* mask, void* ws, size_t ws_bytes,
+                          jenga_stream_t stream);
+
+/* ------------------------------------------------------------------ token movement
+ * jenga_gather -- out[b, i*blk + t, :] = x[b, idx[b,i]*blk + t, :] for i < n_kept[b] (a5).
+ *   x   : [B, S, h] (row pitch ldx elements), out : [B, n_cap, h] (row pitch ldo),
+ *   n_cap = rows of out per batch (>= n_kept[b]*blk, checked on device).  Rows of out
+ *   past n_kept[b]*blk are not written.  dt: F32 or BF16.  h * elem % 16 == 0 and
+ *   16-byte aligned rows use 128-bit moves. */
+JENGA_API jenga_status jenga_gather(const void* x, int64_t ldx, int B, int S, int h, int blk, const int32_t* idx,
+                          const int32_t* n_kept, jenga_dtype dt, void* out, int64_t ldo, int n_cap,
+                          jenga_stream_t stream);
+
+/* jenga_scatter_add -- in-place residual add of a retained-row result (a7):
+ *   x[b, idx[b,i]*blk + t, :] = round(x + alpha * y[b, i*blk + t, :]); other rows untouched.
+ *   The sum is one fp32 fused multiply-add, rounded once more to bf16 for bf16 data. */
+JENGA_API jenga_status jenga_scatter_add(void* x, int64_t ldx, const void* y, int64_t ldy, int B, int S, int h, int blk,
+                               const int32_t* idx, const int32_t* n_kept, float alpha, jenga_dtype dt,
+                               int n_cap, jenga_stream_t stream);
+
+/* jenga_scale_rows -- x[b, rows[b,i], :] *= factor for i < n_rows (salient-token
+ * emphasis of synthetic inputs, and its backward as the same diagonal). */
+JENGA_API jenga_status jenga_scale_rows(void* x, int64_t ldx, int B, int S, int h, const int32_t* rows, int n_rows,
+                              float factor, jenga_dtype dt, jenga_stream_t stream);
+
+/* ------------------------------------------------------------------ layer
+ * A Llama-2 decoder layer (RMSNorm -> q/k/v with RoPE -> causal attention -> o_proj
+ * -> residual; RMSNorm -> SiLU-gated MLP -> residual) with LoRA on q_proj and v_proj,
+ * run only on the retained rows (Jenga summary §4.1, §4.4.1).  bf16 storage, fp32
+ * accumulation.  RoPE uses each token's ORIGINAL position (rotate-half, pairs d and
+ * d + D/2, angle pos * theta^(-2i/D)); attention is causal among retained tokens.
+ * head_dim must be 128, hidden and ffn multiples of 128, lora rank 16. */
+typedef struct jenga_layer_weights {
+  int hidden, heads, head_dim, ffn;
+  float rms_eps, rope_theta;
+  const void* attn_norm; /* [hidden] bf16 RMSNorm gain before attention */
+  const void* mlp_norm;  /* [hidden] bf16 RMSNorm gain before the MLP */
+  const void* wq;        /* [H*D, hidden] bf16 */
+  const void* wk;        /* [H*D, hidden] bf16 */
+  const void* wv;        /* [H*D, hidden] bf16 */
+  const void* wo;        /* [hidden, H*D] bf16 */
+  const void* wg;        /* [ffn, hidden] bf16 gate_proj */
+  const void* wu;        /* [ffn, hidden] bf16 up_proj */
+  const void* wd;        /* [hidden, ffn] bf16 down_proj */
+} jenga_layer_weights;
+
+typedef struct jenga_lora {
+  int rank;       /* 16 */
+  float scale;    /* alpha / rank */
+  const void* aq; /* [rank, hidden] bf16 */
+  const void* bq; /* [H*D, rank] bf16 */
+  const void* av; /* [rank, hidden] bf16 */
+  const void* bv; /* [H*D, rank] bf16 */
+} jenga_lora;
+
+typedef struct jenga_lora_grads { /* fp32, ACCUMULATED into (+=) */
+  float* daq;                     /* [rank, hidden] */
+  float* dbq;                     /* [H*D, rank] */
+  float* dav;
+  float* dbv;
+} jenga_lora_grads;
+
+/* Packed (re-laid-out) copies of the frozen weights the kernels read: fused QKV,
+ * gate/up interleaved in 64-row groups, and the transposes the backward needs.
+ * Built once per layer with jenga_layer_pack; read-only afterwards. */
+JENGA_API size_t jenga_layer_pack_bytes(const jenga_layer_weights* w, const jenga_lora* lora);
+JENGA_API jenga_status jenga_layer_pack(const jenga_layer_weights* w, const jenga_lora* lora, void* packed,
+                              size_t packed_bytes, jenga_stream_t stream);
+
+/* jenga_layer_score_qk -- a1: q and k of ALL S tokens for scoring (no grad):
+ *   qk[b, s, 0:H*D] = RoPE(RMSNorm(x) Wq^T + scale (RMSNorm(x) Aq^T) Bq^T)
+ *   qk[b, s, H*D:2*H*D] = RoPE(RMSNorm(x) Wk^T), positions s.  qk: [B, S, 2*H*D] bf16. */
+JENGA_API size_t jenga_layer_score_qk_workspace_bytes(const jenga_layer_weights* w, int B, int S);
+JENGA_API jenga_status jenga_layer_score_qk(const jenga_layer_weights* w, const jenga_lora* lora, const void* packed,
+                                  const void* x, int B, int S, void* qk, void* ws, size_t ws_bytes,
+                                  jenga_stream_t stream);
+
+/* jenga_sparse_layer_fwd -- a5 + a6 + a7: the layer on the kept blocks of x, in place.
+ *   x      : [B, S, hidden] bf16, updated in place on retained rows only.
+ *   idx, n_kept : from jenga_select; n_kept_max: host bound on every n_kept[b].
+ *   saved  : jenga_layer_saved_bytes(...) bytes; written here, read by the backward.
+ *   ws     : jenga_layer_fwd_workspace_bytes(...) bytes of scratch. */
+JENGA_API size_t jenga_layer_saved_bytes(const jenga_layer_weights* w, int B, int blk, int n_kept_max);
+JENGA_API size_t jenga_layer_fwd_workspace_bytes(const jenga_layer_weights* w, int B, int blk, int n_kept_max);
+JENGA_API jenga_status jenga_sparse_layer_fwd(const jenga_layer_weights* w, const jenga_lora* lora, const void* packed,
+                                    void* x, int B, int S, int blk, const int32_t* idx, const int32_t* n_kept,
+                                    int n_kept_max, void* saved, size_t saved_bytes, void* ws, size_t ws_bytes,
+                                    jenga_stream_t stream);
+
+/* jenga_sparse_layer_bwd -- a8 + a9: backward of jenga_sparse_layer_fwd for an upstream
+ * gradient G held in dx ([B, S, hidden] bf16).  On return dx holds dL/dx: eliminated
+ * rows keep G (identity through the residual), retained rows get the layer backward.
+ * Frozen base weights get no gradient; LoRA gradients are ACCUMULATED into grads.
+ * The retained rows are processed in consecutive segments of segment_tokens rows
+ * (multiple of 128; last one short), last segment first, so per-segment scratch is
+ * bounded by the segment length (Jenga summary §4.4.2). */
+JENGA_API size_t jenga_layer_bwd_workspace_bytes(const jenga_layer_weights* w, int B, int blk, int n_kept_max,
+                                       int segment_tokens);
+JENGA_API jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, const jenga_lora* lora, const void* packed,
+                                    void* dx, int B, int S, int blk, const int32_t* idx, const int32_t* n_kept,
+                                    int n_kept_max, const void* saved, size_t saved_bytes, jenga_lora_grads* grads,
+                                    int segment_tokens, void* ws, size_t ws_bytes, jenga_stream_t stream);
+
+/* ------------------------------------------------------------------ predictor
+ * jenga_predict_blocks -- a10 (Jenga notes §4.3; Jenga summary §4.3.1): per block the
+ * mean of its rows of x (raw layer input), then s = W2 . GELU(W1 xbar + b1) + b2
+ * with exact-erf GELU.  x [B, S, h] bf16; W1 [m, h] bf16, b1 [m] fp32, W2 [m] bf16,
+ * b2 [1] fp32 (device); scores [B, nb] fp32.  m <= 256.
+ * ws: jenga_predict_workspace_bytes bytes (pooled block means, fp32). */
+JENGA_API size_t jenga_predict_workspace_bytes(int B, int S, int h, int blk);
+JENGA_API jenga_status jenga_predict_blocks(const void* x, int B, int S, int h, int blk, const void* w1, const float* b1,
+                                  const void* w2, const float* b2, int m, float* scores, void* ws,
+                                  size_t ws_bytes, jenga_stream_t stream);
+
+/* ------------------------------------------------------------------ test hook
+ * jenga_test_gemm -- C[M, N] = A[M, K] * B[N, K]^T through the tcgen05 GEMM the layer
+ * uses (bf16 inputs, fp32 accumulate; C fp32 if out_f32 else bf16).  bn: 256 or 32
+ * (output tile width).  K % 64 == 0; rows 16-byte aligned.  For kernel tests only. */
+JENGA_API jenga_status jenga_test_gemm(const void* A, int64_t lda, const void* B, int64_t ldb, int M, int N, int K,
+                                       void* C, int64_t ldc, int out_f32, int bn, jenga_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JENGA_H_ */

@@ -1,0 +1,196 @@
+"""GPU parity of the single-step kernels (through the C ABI) against the CPU oracle.
+
+Bars: indices/masks/gathers bit-exact; fp32 scores within 1e-3 relative; bf16
+scores within 2e-2 relative; GEMM against an fp32 PyTorch reference."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import movement as omv
+from oracle import predictor as opr
+from oracle import scores as osc
+from oracle import select as osel
+from oracle.bf16 import from_bits
+from tests.layer_harness import bits_to_torch, rel_max, torch_to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def J():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import token_sparse_long_b200 as J
+    J._lib.load()
+    return J
+
+
+# ------------------------------------------------------------------ tcgen05 GEMM
+@pytest.mark.parametrize("M,N,K,bn", [(128, 256, 64, 256), (200, 512, 128, 256), (384, 768, 1024, 256),
+                                      (130, 32, 4096, 32), (1000, 1024, 4096, 256)])
+def test_gemm_against_fp32_matmul(J, M, N, K, bn):
+    g = torch.Generator(device="cuda").manual_seed(M + N + K)
+    a = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+    b = torch.randn(N, K, device="cuda", generator=g).to(torch.bfloat16)
+    c = J.jenga_test_gemm(a, b, out_f32=True, bn=bn)
+    J.jenga_check_device_status()
+    ref = a.float() @ b.float().t()
+    err = (c - ref).abs().max().item() / ref.abs().max().item()
+    assert err < 1e-4, err
+    if bn == 256:
+        cb = J.jenga_test_gemm(a, b, out_f32=False, bn=bn)
+        assert (cb.float() - ref).abs().max().item() / ref.abs().max().item() < 1e-2
+
+
+# ------------------------------------------------------------------ scoring
+def test_score_fp32_workload_against_oracle(J):
+    c = synth.gen_score_case(0)
+    q = torch.from_numpy(c.q).cuda()
+    k = torch.from_numpy(c.k).cuda()
+    sc = J.jenga_score_blocks(q, k, c.H, c.D, c.blk)
+    J.jenga_check_device_status()
+    ref = osc.block_scores_softmax_mass(c.q.reshape(c.S, c.H, c.D).astype(np.float64),
+                                        c.k.reshape(c.S, c.H, c.D).astype(np.float64), c.blk)
+    got = sc.cpu().numpy().astype(np.float64)
+    assert np.abs(got - ref).max() / np.abs(ref).max() < 1e-3
+    assert np.all(np.abs(got - ref) / ref < 1e-3)
+    assert abs(got.sum() - c.H * c.S) < 1e-3 * c.H * c.S
+    # selection: GPU scores through the oracle's mean threshold -> bit-exact indices
+    idx, nk, mask = J.jenga_select(sc, "mean_ge")
+    (oi, on, om), mean = osel.select_mean_ge(sc.cpu().numpy())
+    assert int(nk[0]) == on and (idx.cpu().numpy() == oi).all() and (mask.cpu().numpy() == om).all()
+    # gathered [n_kept * 32, 256] X and the scatter-add of 2 x the gathered rows
+    x = torch.from_numpy(c.x).cuda()
+    n_rows = on * c.blk
+    xg = J.jenga_gather(x, idx, nk, c.blk, n_rows)
+    ref_g = omv.gather(c.x.astype(np.float64), oi, on, c.blk)
+    assert np.array_equal(xg.cpu().numpy().astype(np.float64), ref_g)
+    x2 = x.clone()
+    J.jenga_scatter_add(x2, xg, idx, nk, c.blk, 2.0)
+    ref_s = omv.scatter_add(c.x.astype(np.float64), ref_g, oi, on, c.blk, 2.0, "f32")
+    assert np.array_equal(x2.cpu().numpy().astype(np.float64), ref_s)
+    J.jenga_check_device_status()
+
+
+@pytest.mark.parametrize("S,H,causal", [(512, 2, True), (1024, 3, True), (256, 2, False)])
+def test_score_bf16_against_oracle(J, S, H, causal):
+    g = torch.Generator(device="cuda").manual_seed(S + H)
+    q = (torch.randn(S, H * 128, device="cuda", generator=g) * 0.25).to(torch.bfloat16)
+    k = (torch.randn(S, H * 128, device="cuda", generator=g) * 0.25).to(torch.bfloat16)
+    sc = J.jenga_score_blocks(q, k, H, 128, 64, causal=causal)
+    J.jenga_check_device_status()
+    ref = osc.block_scores_softmax_mass(torch_to_f64(q).reshape(S, H, 128), torch_to_f64(k).reshape(S, H, 128), 64,
+                                        causal=causal)
+    got = sc.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - ref) / np.abs(ref) < 2e-2), np.abs(got - ref).max()
+    assert abs(got.sum() - H * S) < 2e-3 * H * S
+
+
+def test_score_bf16_fused_qk_buffer_and_batch(J):
+    S, H = 512, 2
+    g = torch.Generator(device="cuda").manual_seed(7)
+    qk = (torch.randn(2, S, 2 * H * 128, device="cuda", generator=g) * 0.3).to(torch.bfloat16)
+    sc = J.jenga_score_blocks(qk[:, :, :H * 128], qk[:, :, H * 128:], H, 128, 128)
+    for b in range(2):
+        qb = torch_to_f64(qk[b, :, :H * 128]).reshape(S, H, 128)
+        kb = torch_to_f64(qk[b, :, H * 128:]).reshape(S, H, 128)
+        ref = osc.block_scores_softmax_mass(qb, kb, 128)
+        assert np.all(np.abs(sc[b].cpu().numpy() - ref) / ref < 2e-2)
+
+
+def test_score_paper_blockmax(J):
+    S, H, D, blk = 64, 2, 16, 8
+    g = torch.Generator(device="cuda").manual_seed(9)
+    q = torch.randn(S, H * D, device="cuda", generator=g, dtype=torch.float32)
+    k = torch.randn(S, H * D, device="cuda", generator=g, dtype=torch.float32)
+    sc = J.jenga_score_blocks(q, k, H, D, blk, mode="paper_blockmax")
+    ref = osc.block_scores_paper_blockmax(torch_to_f64(q).reshape(S, H, D), torch_to_f64(k).reshape(S, H, D), blk)
+    assert np.allclose(sc.cpu().numpy(), ref, rtol=1e-4, atol=1e-5)
+
+
+# ------------------------------------------------------------------ selection
+@pytest.mark.parametrize("nb,mode,param,dist", [(256, "topk_frac", 0.8, "normal"), (256, "topk_frac", 0.4, "ties"),
+                                               (16, "mean_ge", 0, "normal"), (1000, "mean_ge", 0, "ties"),
+                                               (8192, "abs_ge", 0.5, "normal"), (300, "topk", 7, "ties"),
+                                               (64, "topk_frac", 0.0, "normal"), (64, "topk_frac", 1.0, "normal")])
+def test_select_bit_exact(J, nb, mode, param, dist):
+    sc = synth.gen_scores(nb, 3, nb, dist)
+    idx, nk, mask = J.jenga_select(torch.from_numpy(sc).cuda(), mode, param)
+    J.jenga_check_device_status()
+    oi, on, om = osel.select(sc, mode, param)
+    assert np.array_equal(nk.cpu().numpy(), on)
+    assert np.array_equal(idx.cpu().numpy(), oi)
+    assert np.array_equal(mask.cpu().numpy(), om)
+
+
+@pytest.mark.parametrize("mode,param", [("abs_ge", 0.25), ("mean_ge", 0)])
+def test_select_large_multi_cta(J, mode, param):
+    nb = (1 << 20) + 777
+    sc = synth.gen_scores(5, 2, nb)
+    idx, nk, mask = J.jenga_select(torch.from_numpy(sc).cuda(), mode, param)
+    J.jenga_check_device_status()
+    for b in range(2):
+        if mode == "abs_ge":
+            oi, on, om = osel.select_abs_ge(sc[b], param)
+        else:
+            (oi, on, om), _ = osel.select_mean_ge(sc[b])
+        assert int(nk[b]) == on
+        assert np.array_equal(idx[b].cpu().numpy(), oi)
+        assert np.array_equal(mask[b].cpu().numpy(), om)
+
+
+# ------------------------------------------------------------------ movement
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_gather_scatter_random(J, dtype):
+    S, h, blk = 1024, 384, 64
+    g = torch.Generator(device="cuda").manual_seed(11)
+    x = torch.randn(S, h, device="cuda", generator=g).to(dtype)
+    sc = synth.gen_scores(12, 1, S // blk)
+    idx, nk, _ = J.jenga_select(torch.from_numpy(sc).cuda(), "topk_frac", 0.5)
+    n_cap = (S // blk) * blk
+    out = torch.full((n_cap, h), 7.0, device="cuda", dtype=dtype)
+    J.jenga_gather(x, idx, nk, blk, n_cap, out=out)
+    xi = idx.cpu().numpy()[0]
+    n = int(nk[0])
+    ref = omv.gather(torch_to_f64(x), xi, n, blk)
+    assert np.array_equal(torch_to_f64(out[: n * blk]), ref)
+    assert (out[n * blk:] == 7.0).all()
+    y = torch.randn(n * blk, h, device="cuda", generator=g).to(dtype)
+    x2 = x.clone()
+    J.jenga_scatter_add(x2, y, idx, nk, blk, 1.0)
+    ref2 = omv.scatter_add(torch_to_f64(x), torch_to_f64(y), xi, n, blk, 1.0,
+                           "bf16" if dtype == torch.bfloat16 else "f32")
+    assert np.array_equal(torch_to_f64(x2), ref2)
+    # keep-none: nothing moves
+    z = torch.zeros(1, dtype=torch.int32, device="cuda")
+    x3 = x.clone()
+    J.jenga_scatter_add(x3, y, idx, z, blk, 1.0)
+    assert torch.equal(x3, x)
+
+
+def test_scale_rows(J):
+    x = torch.randn(64, 256, device="cuda").to(torch.bfloat16)
+    rows = torch.tensor([3, 17, 40], dtype=torch.int32, device="cuda")
+    y = x.clone()
+    J.jenga_scale_rows(y, rows, 3.0)
+    ref = torch_to_f64(x)
+    ref[[3, 17, 40]] = torch_to_f64(x[[3, 17, 40]].float().mul(3).to(torch.bfloat16))
+    assert np.array_equal(torch_to_f64(y), ref)
+
+
+# ------------------------------------------------------------------ predictor
+def test_predictor_against_oracle(J):
+    shape = synth.LayerShape(hidden=512, heads=4, head_dim=128, ffn=1024)
+    case = synth.gen_layer_case(4, S=2048, blk=128, shape=shape, salient_frac=0.0, predictor_hidden=128)
+    pr = case.predictor
+    x = bits_to_torch(case.x)
+    w1 = bits_to_torch(pr["w1"])
+    w2 = bits_to_torch(pr["w2"]).reshape(-1)
+    b1 = torch.from_numpy(pr["b1"]).cuda()
+    b2 = torch.from_numpy(pr["b2"]).cuda()
+    s = J.jenga_predict_blocks(x, 128, w1, b1, w2, b2)
+    J.jenga_check_device_status()
+    ref = opr.predict_blocks(from_bits(case.x), 128, from_bits(pr["w1"]), pr["b1"], from_bits(pr["w2"]), pr["b2"])
+    got = s.cpu().numpy().astype(np.float64)
+    assert rel_max(got, ref) < 1e-3

@@ -1,0 +1,96 @@
+"""GPU parity of the retained-token layer (a1..a9) against the CPU oracle.
+
+The oracle runs on the GPU's kept-block list and the same seeded inputs, so a
+selection difference cannot cascade.  Bar: max |gpu - oracle| / rms(oracle) <= 3e-2
+on the layer's contribution (out - x) and the backward's contribution (dX - G) -- with
+one bf16 ulp of the stored result forgiven, since that final rounding may land on either
+neighbour -- and on each LoRA gradient; eliminated rows exactly unchanged."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import select as osel
+from tests.layer_harness import (SMALL, oracle_layer, oracle_scores_from_qk, rel_delta_ulp, rel_max, run_layer_gpu,
+                                 small_case, torch_to_f64)
+
+pytestmark = pytest.mark.gpu
+TOL = 3e-2
+
+
+@pytest.fixture(scope="module")
+def J():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import token_sparse_long_b200 as J
+    J._lib.load()
+    return J
+
+
+def _check(case, gpu, seg=None):
+    Xo, dX, grads, X, G = oracle_layer(case, gpu, seg=seg)
+    rows = np.zeros(case.S, bool)
+    for b in gpu["idx"][: gpu["n_kept"]]:
+        rows[b * case.blk:(b + 1) * case.blk] = True
+    assert np.array_equal(gpu["out"][~rows], X[~rows]), "eliminated rows must pass through unchanged"
+    assert np.array_equal(gpu["dx"][~rows], G[~rows]), "eliminated rows: identity gradient"
+    e_out = rel_delta_ulp(gpu["out"][rows], Xo[rows], X[rows])
+    e_dx = rel_delta_ulp(gpu["dx"][rows], dX[rows], G[rows])
+    assert e_out < TOL, e_out
+    assert e_dx < TOL, e_dx
+    for k in grads:
+        if np.abs(grads[k]).max() == 0:
+            assert np.abs(gpu["grads"][k]).max() == 0, k
+        else:
+            assert rel_max(gpu["grads"][k], grads[k]) < TOL, (k, rel_max(gpu["grads"][k], grads[k]))
+    return e_out, e_dx
+
+
+@pytest.mark.parametrize("keep,seg,lora_b", [(0.5, 4096, 0.02), (0.25, 128, 0.02), (1.0, 256, 0.0),
+                                             (0.75, 4096, 0.0)])
+def test_small_layer(J, keep, seg, lora_b):
+    case = small_case(seed=5, S=1024, blk=64, lora_b_std=lora_b)
+    gpu = run_layer_gpu(case, keep=keep, seg=seg)
+    ref_sc = oracle_scores_from_qk(torch_to_f64(gpu["qk"]), SMALL.heads, SMALL.head_dim, case.blk)
+    assert np.all(np.abs(gpu["scores"] - ref_sc) / ref_sc < 2e-2)
+    oi, on, _ = osel.select_topk(gpu["scores"], osel.topk_count(keep, case.S // case.blk))
+    assert on == gpu["n_kept"] and np.array_equal(oi, gpu["idx"])
+    _check(case, gpu)
+
+
+def test_mean_threshold_layer_device_count(J):
+    # data-dependent n_kept (mean threshold): grids sized for all blocks, kernels read
+    # the count on the device
+    case = small_case(seed=6, S=512, blk=128)
+    gpu = run_layer_gpu(case, keep=0.0, seg=256, mode="mean_ge")
+    (oi, on, _), _ = osel.select_mean_ge(gpu["scores"])
+    assert on == gpu["n_kept"] and np.array_equal(oi, gpu["idx"])
+    _check(case, gpu)
+
+
+def test_keep_none(J):
+    case = small_case(seed=7, S=512, blk=64)
+    gpu = run_layer_gpu(case, keep=0.0, seg=4096)
+    assert gpu["n_kept"] == 0
+    X = gpu["x_in"]
+    assert np.array_equal(gpu["out"], X)
+    assert all(np.abs(v).max() == 0 for v in gpu["grads"].values())
+
+
+def test_segmented_equals_unsegmented(J):
+    case = small_case(seed=8, S=1024, blk=64)
+    a = run_layer_gpu(case, keep=0.75, seg=4096)
+    b = run_layer_gpu(case, keep=0.75, seg=128, handle=a["handle"])
+    assert np.array_equal(a["out"], b["out"])
+    assert rel_max(b["dx"] - a["x_in"] * 0, a["dx"]) < 1e-2
+    for k in a["grads"]:
+        assert rel_max(b["grads"][k], a["grads"][k]) < 1e-2
+
+
+def test_llama7b_shape_s4k_layer(J):
+    """One 7B-shaped layer at S=4096, block 64, keep 50% (the single-layer workload)."""
+    case = synth.gen_workload("llama7b_s4k", seed=0, lora_b_std=0.02)
+    gpu = run_layer_gpu(case, keep=0.5, seg=4096)
+    oi, on, _ = osel.select_topk(gpu["scores"], 32)
+    assert on == 32 and np.array_equal(oi, gpu["idx"])
+    _check(case, gpu)

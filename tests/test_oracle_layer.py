@@ -14,7 +14,14 @@ import torch
 from oracle import layer as oly
 from oracle.movement import retained_rows
 
-torch.set_default_dtype(torch.float64)
+
+
+@pytest.fixture(autouse=True)
+def _float64_default():
+    old = torch.get_default_dtype()
+    torch.set_default_dtype(torch.float64)
+    yield
+    torch.set_default_dtype(old)
 
 
 def _weights(seed, h=32, H=2, D=16, F=48, r=4, b_std=0.1, gain_noise=True, scale=2.0, eps=1e-5):

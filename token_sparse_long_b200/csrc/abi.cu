@@ -1,0 +1,190 @@
+// Status strings, per-thread error text, device error word, tensor-map encoding.
+#include <cstdarg>
+#include <map>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+
+namespace jenga {
+
+static thread_local std::string t_last_error;
+static unsigned long long s_host_budget = 2000000000ull;
+
+void set_last_error(const std::string& msg) { t_last_error = msg; }
+
+jenga_status fail(jenga_status st, const char* fmt, ...) {
+  char buf[1024];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return st;
+}
+
+unsigned long long host_wait_budget_ns() { return s_host_budget; }
+
+// ------------------------------------------------------------------ launch timing
+// One pair of CUDA events per launch while enabled (single host thread; events are
+// created once and reused; no device memory is allocated).
+struct ProfState {
+  bool on = false;
+  std::vector<cudaEvent_t> ev;
+  std::vector<const char*> names;
+  size_t n = 0;
+};
+static ProfState g_prof;
+
+int prof_begin(const char* name, cudaStream_t st) {
+  if (!g_prof.on) return -1;
+  const size_t slot = g_prof.n;
+  while (g_prof.ev.size() < 2 * (slot + 1)) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return -1;
+    g_prof.ev.push_back(e);
+  }
+  if (g_prof.names.size() < slot + 1) g_prof.names.resize(slot + 1);
+  g_prof.names[slot] = name;
+  if (cudaEventRecord(g_prof.ev[2 * slot], st) != cudaSuccess) return -1;
+  g_prof.n = slot + 1;
+  return (int)slot;
+}
+
+void prof_end(int slot, cudaStream_t st) {
+  if (slot < 0) return;
+  cudaEventRecord(g_prof.ev[2 * (size_t)slot + 1], st);
+}
+
+int sm_count() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static int cache[64] = {0};
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+jenga_status make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                            uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(JENGA_ECUDA, "cuTensorMapEncodeTiled entry point not available");
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (ld * 2) % 16 || rows == 0 || cols == 0)
+    return fail(JENGA_EINVAL, "tensor map: base must be 16-byte aligned and row pitch a multiple of 16 bytes");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(JENGA_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return JENGA_OK;
+}
+
+}  // namespace jenga
+
+using namespace jenga;
+
+extern "C" const char* jenga_status_string(jenga_status st) {
+  switch (st) {
+    case JENGA_OK: return "ok";
+    case JENGA_EINVAL: return "invalid argument";
+    case JENGA_EUNSUPPORTED: return "unsupported configuration";
+    case JENGA_ECUDA: return "CUDA error";
+    case JENGA_ETIMEOUT: return "device wait timed out";
+    case JENGA_EWORKSPACE: return "workspace too small";
+    case JENGA_EINTERNAL: return "device-detected internal error";
+  }
+  return "unknown status";
+}
+
+extern "C" size_t jenga_last_error(char* buf, size_t len) {
+  const std::string& s = t_last_error;
+  if (buf && len) {
+    size_t n = s.size() < len - 1 ? s.size() : len - 1;
+    memcpy(buf, s.data(), n);
+    buf[n] = 0;
+  }
+  return s.size();
+}
+
+extern "C" jenga_status jenga_check_device_status(jenga_stream_t stream, uint32_t* detail2) {
+  JENGA_CUDA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
+  unsigned int e[4];
+  JENGA_CUDA_TRY(cudaMemcpyFromSymbol(e, g_device_error, sizeof(e)));
+  if (detail2) {
+    detail2[0] = e[1];
+    detail2[1] = e[2];
+  }
+  if (e[0] == 0) return JENGA_OK;
+  unsigned int z[4] = {0, 0, 0, 0};
+  JENGA_CUDA_TRY(cudaMemcpyToSymbol(g_device_error, z, sizeof(z)));
+  return fail((jenga_status)e[0], "device reported %s at site %u (detail %u)", jenga_status_string((jenga_status)e[0]),
+              e[1], e[2]);
+}
+
+extern "C" jenga_status jenga_set_wait_budget_ns(uint64_t ns) {
+  unsigned long long v = ns;
+  JENGA_CUDA_TRY(cudaMemcpyToSymbol(g_wait_budget_ns, &v, sizeof(v)));
+  s_host_budget = v;
+  return JENGA_OK;
+}
+
+extern "C" const char* jenga_version(void) { return "jenga-b200 0.1 (sm_100a)"; }
+
+extern "C" jenga_status jenga_profile_enable(int on) {
+  g_prof.on = on != 0;
+  g_prof.n = 0;
+  return JENGA_OK;
+}
+
+extern "C" size_t jenga_profile_report(char* buf, size_t len) {
+  std::map<std::string, std::pair<long, double>> agg;  // name -> (launches, ms)
+  std::vector<std::string> order;
+  for (size_t i = 0; i < g_prof.n; ++i) {
+    float ms = 0.f;
+    cudaEventSynchronize(g_prof.ev[2 * i + 1]);
+    if (cudaEventElapsedTime(&ms, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]) != cudaSuccess) ms = -1.f;
+    const std::string k = g_prof.names[i];
+    if (!agg.count(k)) order.push_back(k);
+    agg[k].first += 1;
+    agg[k].second += ms;
+  }
+  std::string s = "{";
+  char tmp[256];
+  for (size_t i = 0; i < order.size(); ++i) {
+    snprintf(tmp, sizeof(tmp), "%s\"%s\": {\"launches\": %ld, \"ms\": %.6f}", i ? ", " : "", order[i].c_str(),
+             agg[order[i]].first, agg[order[i]].second);
+    s += tmp;
+  }
+  s += "}";
+  g_prof.n = 0;
+  if (buf && len) {
+    size_t n = s.size() < len - 1 ? s.size() : len - 1;
+    memcpy(buf, s.data(), n);
+    buf[n] = 0;
+  }
+  return s.size();
+}

@@ -1,0 +1,229 @@
+// Shared device/host helpers of the jenga library (sm_100a only).
+//
+// Error plumbing: every exported call returns jenga_status; kernels that detect a
+// fault (bounded wait expired, index out of range) record it in a module-global
+// device error word that jenga_check_device_status() reads and clears.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstdio>
+#include <string>
+
+#include "../../include/jenga.h"
+
+namespace jenga {
+
+typedef __nv_bfloat16 bf16;
+
+// ------------------------------------------------------------------ host errors
+void set_last_error(const std::string& msg);
+jenga_status fail(jenga_status st, const char* fmt, ...);
+
+#define JENGA_CUDA_TRY(expr)                                                        \
+  do {                                                                              \
+    cudaError_t _e = (expr);                                                        \
+    if (_e != cudaSuccess)                                                          \
+      return ::jenga::fail(JENGA_ECUDA, "%s failed: %s (%s:%d)", #expr,             \
+                           cudaGetErrorString(_e), __FILE__, __LINE__);             \
+  } while (0)
+
+#define JENGA_CHECK_ARG(cond, ...)                                                  \
+  do {                                                                              \
+    if (!(cond)) return ::jenga::fail(JENGA_EINVAL, __VA_ARGS__);                   \
+  } while (0)
+
+#define JENGA_LAUNCH_CHECK()                                                        \
+  do {                                                                              \
+    cudaError_t _e = cudaGetLastError();                                            \
+    if (_e != cudaSuccess)                                                          \
+      return ::jenga::fail(JENGA_ECUDA, "kernel launch failed: %s (%s:%d)",         \
+                           cudaGetErrorString(_e), __FILE__, __LINE__);             \
+  } while (0)
+
+// ------------------------------------------------------------------ device errors
+// err[0] = first error code (JENGA_E*), err[1] = site id, err[2] = detail.
+// Defined here: the library is one translation unit (csrc/jenga_all.cu).
+__device__ unsigned int g_device_error[4];
+
+enum ErrSite : unsigned int {
+  SITE_GEMM_PRODUCER = 1,
+  SITE_GEMM_MMA = 2,
+  SITE_GEMM_EPILOGUE = 3,
+  SITE_SCORE_TC = 4,
+  SITE_INDEX_RANGE = 5,
+  SITE_NKEPT_RANGE = 6,
+  SITE_ATTN = 7,
+};
+
+__device__ __forceinline__ void record_device_error(unsigned code, unsigned site, unsigned detail) {
+  if (atomicCAS(&g_device_error[0], 0u, code) == 0u) {
+    g_device_error[1] = site;
+    g_device_error[2] = detail;
+  }
+}
+
+// wait budget for mbarrier spins, in nanoseconds of %globaltimer (host-settable)
+__device__ unsigned long long g_wait_budget_ns = 2000000000ull;
+
+__device__ __forceinline__ unsigned long long global_timer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(phase)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: returns false (and records a timeout) if the phase does not
+// complete within the wait budget.  Never spins forever.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, unsigned site) {
+  if (mbar_try_wait(bar, phase)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  const unsigned long long budget = g_wait_budget_ns;
+  while (true) {
+    if (mbar_try_wait(bar, phase)) return true;
+    if (global_timer_ns() - t0 > budget) {
+      record_device_error(JENGA_ETIMEOUT, site, phase);
+      return false;
+    }
+  }
+}
+
+// 2D TMA tile load into shared memory, completion counted on an mbarrier.
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                            int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---- tcgen05 (5th-generation tensor core, accumulators in tensor memory)
+__device__ __forceinline__ void tmem_alloc(uint32_t* smem_holder, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_holder)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate (kind::f16)
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on an mbarrier once all previously issued tcgen05.mma of this thread complete.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+// Load 32 consecutive fp32 columns of this thread's TMEM lane (warp w reads lanes 32*(w%4)..).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+        "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+        "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor for a K-major tile whose rows are 128 bytes
+// (64 bf16), stored with the 128-byte swizzle in 1024-byte groups of 8 rows.
+__device__ __forceinline__ uint64_t umma_desc_k_sw128(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);          // start address (16-byte units)
+  d |= (uint64_t)1 << 16;                               // leading byte offset (unused for SW128 K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;                     // stride byte offset: 8-row group pitch
+  d |= (uint64_t)1 << 46;                               // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                               // layout: 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor: kind::f16, A/B bf16 K-major, D fp32, shape M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ float bf16_to_f(bf16 v) { return __bfloat162float(v); }
+
+// ------------------------------------------------------------------ host helpers
+// Encode a 2D row-major bf16 tensor map (rows x cols, row pitch ld elements) with a
+// box of box_rows x 64 columns and the 128-byte swizzle.
+jenga_status make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                            uint32_t box_rows);
+
+int sm_count();
+unsigned long long host_wait_budget_ns();
+
+// Per-launch timing (off by default): when enabled with jenga_profile_enable, every
+// kernel launch is bracketed by two CUDA events recorded on its own stream, and
+// jenga_profile_report aggregates launches and milliseconds per kernel name.
+int prof_begin(const char* name, cudaStream_t st);
+void prof_end(int slot, cudaStream_t st);
+
+}  // namespace jenga

@@ -1,0 +1,374 @@
+// tcgen05 GEMM for the retained-token layer projections (sm_100a).
+//
+//   C[M, N] = A1[M, K1] * B1[N, K1]^T  (+ A2[M, K2] * B2[N, K2]^T)     bf16 in, fp32 accumulate
+//
+// Both operands are K-major bf16 (row-major [rows, K]).  The optional second
+// operand pair extends the reduction (used to fold the LoRA up-projection into the
+// QKV projection, and the LoRA down-projection's input gradient into the dX GEMM).
+//
+// Structure (one 128 x BN output tile per CTA, 192 threads):
+//   warp 0      TMA producer: 128 x 64 A box + BN x 64 B box per stage into a
+//               STAGES-deep shared-memory ring (128-byte swizzle), mbarrier tx counts
+//   warp 1      allocates BN TMEM columns; one lane issues tcgen05.mma (M=128, N=BN,
+//               K=16) x 4 per stage and tcgen05.commit to release the stage
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time of their TMEM lane quarter
+//               (row = 32 * (warp % 4) + lane), fused epilogue, global stores
+// Every wait is bounded (see mbar_wait); rows past the device-side valid count are
+// neither loaded usefully nor stored.
+#pragma once
+
+#include "common.cuh"
+
+namespace jenga {
+
+constexpr int GEMM_BM = 128;
+constexpr int GEMM_BK = 64;
+constexpr int GEMM_THREADS = 192;
+
+enum GemmEpi : int {
+  EPI_STORE_BF16 = 0,   // out[m, n] = bf16(acc * alpha)
+  EPI_STORE_F32 = 1,    // out[m, n] = acc * alpha (fp32)
+  EPI_SCATTER_ADD = 2,  // x[row(m), n] = bf16(x + acc); aux[m, n] = same value (optional)
+  EPI_SWIGLU = 3,       // 64-col groups (gate, up) -> out[m, n/2 + j] = bf16(silu(g) * u)
+  EPI_QKV_ROPE = 4,     // q/k/v sections of width hd; RoPE(pos(m)) on q and k -> bf16
+  EPI_SWIGLU_BWD = 5,   // acc = dA; aux = (g, u) interleaved bf16 -> out = (dg, du) interleaved bf16
+  EPI_LORA_T = 6,       // out fp32 [m, 0:N] = beta * acc ; aux bf16 [m, 0:64] = bf16(alpha * acc), zero padded
+};
+
+struct EpiParams {
+  void* out = nullptr;
+  int64_t ldo = 0;
+  void* aux = nullptr;
+  int64_t ld_aux = 0;
+  bf16* x = nullptr;  // scatter target [x_rows, ldx]
+  int64_t ldx = 0;
+  int64_t x_rows = 0;
+  const int32_t* idx = nullptr;  // kept block list (row map); null = identity rows
+  int blk = 1;
+  int row_offset = 0;            // compact row of local row 0 (segment start)
+  const int32_t* n_valid = nullptr;  // device: valid rows = (*n_valid) * valid_mult - row_offset
+  int valid_mult = 1;
+  int m_host = 0;                // host bound on rows (M of the launch)
+  float alpha = 1.f;
+  float beta = 1.f;              // LORA_T: scale of the fp32 copy
+  int hd = 0;                    // QKV: H * D (section width)
+  const double* inv_freq = nullptr;  // QKV: RoPE inverse frequencies [64] (head_dim 128)
+};
+
+__device__ __forceinline__ int epi_valid_rows(const EpiParams& p) {
+  int v = p.m_host;
+  if (p.n_valid) {
+    int nv = (*p.n_valid) * p.valid_mult - p.row_offset;
+    v = min(v, max(nv, 0));
+  }
+  return v;
+}
+
+// sequence row of compact row c (through the kept-block list)
+__device__ __forceinline__ int64_t map_row(const EpiParams& p, int c) {
+  if (!p.idx) return c;
+  int b = c / p.blk;
+  return (int64_t)__ldg(p.idx + b) * p.blk + (c - b * p.blk);
+}
+
+__device__ __forceinline__ void store_bf16x32(bf16* dst, const float* v) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    uint32_t* ws = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
+      ws[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    d[q] = w;
+  }
+}
+
+__device__ __forceinline__ void load_bf16x32(const bf16* src, float* v) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w = s[q];
+    const uint32_t* ws = reinterpret_cast<const uint32_t*>(&w);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&ws[i]);
+      float2 f = __bfloat1622float2(h);
+      v[q * 8 + 2 * i] = f.x;
+      v[q * 8 + 2 * i + 1] = f.y;
+    }
+  }
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.f + __expf(-z)); }
+
+template <int BN>
+struct GemmSmem {
+  static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
+  static constexpr int A_BYTES = GEMM_BM * GEMM_BK * 2;
+  static constexpr int B_BYTES = BN * GEMM_BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int TOTAL = BAR_OFF + 256 + 1024;  // barriers + 1 KB alignment slack
+};
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                   const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, int nkb1,
+                   int nkb2, int N, EpiParams ep) {
+  using L = GemmSmem<BN>;
+  constexpr int STAGES = L::STAGES;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accum = empty + STAGES;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 1);
+  __shared__ double s_inv_freq[64];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * BN;
+  const int m0 = blockIdx.y * GEMM_BM;
+  const int valid = epi_valid_rows(ep);
+  if (m0 >= valid) return;  // whole tile past the valid rows (uniform per CTA)
+  const int nkb = nkb1 + nkb2;
+
+  if (EPI == EPI_QKV_ROPE) {
+    if (threadIdx.x < 64) s_inv_freq[threadIdx.x] = ep.inv_freq[threadIdx.x];
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accum, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, BN < 32 ? 32 : BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    prefetch_tmap(&tmA1);
+    prefetch_tmap(&tmB1);
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % STAGES;
+      if (kb >= STAGES && !mbar_wait(&empty[s], ((kb / STAGES) - 1) & 1, SITE_GEMM_PRODUCER)) break;
+      uint8_t* sa = smem + s * L::STAGE_BYTES;
+      uint8_t* sb = sa + L::A_BYTES;
+      mbar_arrive_expect_tx(&full[s], L::STAGE_BYTES);
+      if (kb < nkb1) {
+        tma_load_2d(sa, &tmA1, &full[s], kb * GEMM_BK, m0);
+        tma_load_2d(sb, &tmB1, &full[s], kb * GEMM_BK, n0);
+      } else {
+        tma_load_2d(sa, &tmA2, &full[s], (kb - nkb1) * GEMM_BK, m0);
+        tma_load_2d(sb, &tmB2, &full[s], (kb - nkb1) * GEMM_BK, n0);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    constexpr uint32_t idesc = umma_idesc_bf16(GEMM_BM, BN);
+    bool ok = true;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % STAGES;
+      if (!mbar_wait(&full[s], (kb / STAGES) & 1, SITE_GEMM_MMA)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t sa = smem_u32(smem + s * L::STAGE_BYTES);
+      const uint32_t sb = sa + L::A_BYTES;
+#pragma unroll
+      for (int k = 0; k < GEMM_BK / 16; ++k) {
+        umma_bf16(tmem, umma_desc_k_sw128(sa + k * 32), umma_desc_k_sw128(sb + k * 32), idesc,
+                  (kb > 0 || k > 0) ? 1u : 0u);
+      }
+      umma_commit(&empty[s]);
+    }
+    if (ok) umma_commit(accum);
+  } else if (warp >= 2) {
+    // ---------------- epilogue
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int m = m0 + r;
+    const bool ok = mbar_wait(accum, 0, SITE_GEMM_EPILOGUE);
+    tc_fence_after();
+    if (ok) {
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16);
+      const bool row_ok = m < valid;
+      float v[32];
+      if (EPI == EPI_STORE_BF16 || EPI == EPI_STORE_F32 || EPI == EPI_SCATTER_ADD) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          tmem_ld32(tbase + c * 32, v);
+          const int n = n0 + c * 32;
+          if (!row_ok || n >= N) continue;
+          if (EPI == EPI_STORE_BF16) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= ep.alpha;
+            store_bf16x32(reinterpret_cast<bf16*>(ep.out) + (int64_t)m * ep.ldo + n, v);
+          } else if (EPI == EPI_STORE_F32) {
+            float4* d = reinterpret_cast<float4*>(reinterpret_cast<float*>(ep.out) + (int64_t)m * ep.ldo + n);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              d[q] = make_float4(v[4 * q] * ep.alpha, v[4 * q + 1] * ep.alpha, v[4 * q + 2] * ep.alpha,
+                                 v[4 * q + 3] * ep.alpha);
+          } else {  // scatter-add into the residual rows
+            const int64_t row = map_row(ep, m + ep.row_offset);
+            if (row < 0 || row >= ep.x_rows) {
+              record_device_error(JENGA_EINTERNAL, SITE_INDEX_RANGE, (unsigned)row);
+              continue;
+            }
+            bf16* xp = ep.x + row * ep.ldx + n;
+            float xv[32];
+            load_bf16x32(xp, xv);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = xv[i] + v[i];
+            store_bf16x32(xp, v);
+            if (ep.aux) store_bf16x32(reinterpret_cast<bf16*>(ep.aux) + (int64_t)m * ep.ld_aux + n, v);
+          }
+        }
+      } else if (EPI == EPI_SWIGLU) {
+#pragma unroll 1
+        for (int g = 0; g < BN / 128; ++g) {
+#pragma unroll 1
+          for (int hh = 0; hh < 2; ++hh) {
+            float u[32];
+            tmem_ld32(tbase + g * 128 + hh * 32, v);
+            tmem_ld32(tbase + g * 128 + 64 + hh * 32, u);
+            const int n = n0 + g * 128;
+            if (!row_ok || n >= N) continue;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = silu_f(v[i]) * u[i];
+            store_bf16x32(reinterpret_cast<bf16*>(ep.out) + (int64_t)m * ep.ldo + (n >> 1) + hh * 32, v);
+          }
+        }
+      } else if (EPI == EPI_SWIGLU_BWD) {
+        // acc column j (of ffn) -> group j/64, gate at 128*group + j%64, up at +64
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          tmem_ld32(tbase + c * 32, v);
+          const int j = n0 + c * 32;
+          if (!row_ok || j >= N) continue;
+          const int64_t col = (int64_t)(j >> 6) * 128 + (j & 63);
+          const bf16* gu = reinterpret_cast<const bf16*>(ep.aux) + (int64_t)m * ep.ld_aux + col;
+          float gv[32], uv[32], dg[32];
+          load_bf16x32(gu, gv);
+          load_bf16x32(gu + 64, uv);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float sg = 1.f / (1.f + __expf(-gv[i]));
+            const float da = v[i];
+            dg[i] = da * uv[i] * sg * (1.f + gv[i] * (1.f - sg));
+            v[i] = da * gv[i] * sg;  // du = dA * silu(g)
+          }
+          bf16* o = reinterpret_cast<bf16*>(ep.out) + (int64_t)m * ep.ldo + col;
+          store_bf16x32(o, dg);
+          store_bf16x32(o + 64, v);
+        }
+      } else if (EPI == EPI_LORA_T) {
+        // N <= 32 (t_q, t_v): fp32 copy + scaled bf16 copy padded to 64 columns
+        tmem_ld32(tbase, v);
+        if (row_ok) {
+          float* o = reinterpret_cast<float*>(ep.out) + (int64_t)m * ep.ldo;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < N) o[i] = v[i] * ep.beta;
+          float w[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = i < N ? v[i] * ep.alpha : 0.f;
+          bf16* a = reinterpret_cast<bf16*>(ep.aux) + (int64_t)m * ep.ld_aux;
+          store_bf16x32(a, w);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = 0.f;
+          store_bf16x32(a + 32, w);
+        }
+      } else if (EPI == EPI_QKV_ROPE) {
+        // tile = BN/128 heads; section = (n / hd): 0 q, 1 k, 2 v; RoPE on q and k
+        const int64_t pos = row_ok ? map_row(ep, m + ep.row_offset) : 0;
+#pragma unroll 1
+        for (int g = 0; g < BN / 128; ++g) {
+          const int nh = n0 + g * 128;
+          const bool rope = nh < 2 * ep.hd;
+#pragma unroll 1
+          for (int hh = 0; hh < 2; ++hh) {
+            float u[32];
+            tmem_ld32(tbase + g * 128 + hh * 32, v);
+            tmem_ld32(tbase + g * 128 + 64 + hh * 32, u);
+            if (!row_ok || nh >= N) continue;
+            if (rope) {
+#pragma unroll 4
+              for (int i = 0; i < 32; ++i) {
+                const double ang = (double)pos * s_inv_freq[hh * 32 + i];
+                const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
+                float sn, cs;
+                sincosf((float)red, &sn, &cs);
+                const float a = v[i], b = u[i];
+                v[i] = a * cs - b * sn;
+                u[i] = b * cs + a * sn;
+              }
+            }
+            bf16* o = reinterpret_cast<bf16*>(ep.out) + (int64_t)m * ep.ldo + nh;
+            store_bf16x32(o + hh * 32, v);
+            store_bf16x32(o + 64 + hh * 32, u);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BN < 32 ? 32 : BN);
+  }
+}
+
+// ------------------------------------------------------------------ host launcher
+struct GemmOperand {
+  const void* ptr;
+  int64_t rows;  // tensor-map extent (rows may extend past the valid rows)
+  int64_t ld;    // row pitch in elements
+};
+
+template <int BN, int EPI>
+jenga_status launch_gemm(const GemmOperand& A1, const GemmOperand& B1, int K1, const GemmOperand* A2,
+                         const GemmOperand* B2, int K2, int M, int N, const EpiParams& ep, cudaStream_t st,
+                         const char* name = "gemm") {
+  using L = GemmSmem<BN>;
+  if (M <= 0 || N <= 0) return JENGA_OK;
+  if (K1 % GEMM_BK || K2 % GEMM_BK || K1 <= 0) return fail(JENGA_EINVAL, "gemm: K must be a multiple of 64");
+  CUtensorMap ta1, tb1, ta2, tb2;
+  jenga_status s;
+  if ((s = make_tmap_bf16(&ta1, A1.ptr, A1.rows, K1, A1.ld, GEMM_BM)) != JENGA_OK) return s;
+  if ((s = make_tmap_bf16(&tb1, B1.ptr, B1.rows, K1, B1.ld, BN)) != JENGA_OK) return s;
+  if (K2 > 0) {
+    if ((s = make_tmap_bf16(&ta2, A2->ptr, A2->rows, K2, A2->ld, GEMM_BM)) != JENGA_OK) return s;
+    if ((s = make_tmap_bf16(&tb2, B2->ptr, B2->rows, K2, B2->ld, BN)) != JENGA_OK) return s;
+  } else {
+    ta2 = ta1;
+    tb2 = tb1;
+  }
+  JENGA_CUDA_TRY(
+      cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL));
+  EpiParams p = ep;
+  p.m_host = M;
+  dim3 grid((N + BN - 1) / BN, (M + GEMM_BM - 1) / GEMM_BM);
+  const int ps = prof_begin(name, st);
+  gemm_tc_kernel<BN, EPI><<<grid, GEMM_THREADS, L::TOTAL, st>>>(ta1, tb1, ta2, tb2, K1 / GEMM_BK, K2 / GEMM_BK,
+                                                                 N, p);
+  prof_end(ps, st);
+  JENGA_LAUNCH_CHECK();
+  return JENGA_OK;
+}
+
+}  // namespace jenga

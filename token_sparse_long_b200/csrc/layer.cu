@@ -1,0 +1,617 @@
+// Retained-token Llama decoder layer: weight packing, all-S q/k projection for
+// scoring, forward, segment-wise backward (Jenga summary §4.1, §4.4.1, §4.4.2).
+#include "gemm_tc.cuh"
+#include "layer_kernels.cuh"
+
+namespace jenga {
+
+jenga_status attn_forward(const bf16* q, const bf16* k, const bf16* v, int64_t ld, bf16* o, int64_t ldo, float* lse,
+                          int64_t lse_ld, int H, const int32_t* n_valid, int valid_mult, int n_cap, cudaStream_t st);
+jenga_status attn_backward_segment(const bf16* q, const bf16* k, const bf16* v, int64_t ld, const bf16* o,
+                                   int64_t ldo, const float* lse, int64_t lse_ld, const bf16* dO, int64_t ld_do,
+                                   float* delta, int64_t delta_ld, float* dq, int64_t ld_dq, float* dk_acc,
+                                   float* dv_acc, int64_t ld_acc, int H, int s0, int s1, const int32_t* n_valid,
+                                   int valid_mult, int n_cap, cudaStream_t st);
+
+constexpr int LORA_R = 16;
+constexpr int LORA_PAD = 64;  // padded K of the LoRA operand pairs
+
+// A bump allocator over a caller buffer (256-byte aligned sub-buffers).
+struct Carve {
+  uintptr_t base, cur, end;
+  explicit Carve(void* p, size_t bytes = ~size_t(0) >> 1)
+      : base((uintptr_t)p), cur((uintptr_t)p), end(bytes == (~size_t(0) >> 1) ? ~uintptr_t(0) : (uintptr_t)p + bytes) {}
+  template <class T>
+  T* take(size_t count) {
+    cur = (cur + 255) & ~uintptr_t(255);
+    T* r = (T*)cur;
+    cur += count * sizeof(T);
+    return r;
+  }
+  size_t used() const { return (size_t)(cur - base) + 256; }
+  bool ok() const { return cur <= end; }
+};
+
+struct Dims {
+  int h, H, D, HD, F;
+};
+
+static jenga_status check_weights(const jenga_layer_weights* w, const jenga_lora* lora, Dims* d) {
+  JENGA_CHECK_ARG(w && lora, "layer: null weights");
+  JENGA_CHECK_ARG(w->head_dim == 128, "layer: head_dim must be 128 (got %d)", w->head_dim);
+  JENGA_CHECK_ARG(w->hidden > 0 && w->hidden % 256 == 0 && w->hidden <= 8192, "layer: hidden must be a multiple of 256, <= 8192");
+  JENGA_CHECK_ARG(w->heads > 0 && w->ffn > 0 && w->ffn % 256 == 0, "layer: ffn must be a multiple of 256");
+  JENGA_CHECK_ARG(lora->rank == LORA_R, "layer: LoRA rank must be 16");
+  JENGA_CHECK_ARG(w->wq && w->wk && w->wv && w->wo && w->wg && w->wu && w->wd && w->attn_norm && w->mlp_norm,
+                  "layer: null weight pointer");
+  JENGA_CHECK_ARG(lora->aq && lora->bq && lora->av && lora->bv, "layer: null LoRA pointer");
+  d->h = w->hidden;
+  d->H = w->heads;
+  d->D = w->head_dim;
+  d->HD = w->heads * w->head_dim;
+  d->F = w->ffn;
+  JENGA_CHECK_ARG(d->HD % 256 == 0, "layer: heads * head_dim must be a multiple of 256");
+  return JENGA_OK;
+}
+
+struct Packed {
+  bf16 *wqkv, *lorab, *aqv, *wgu, *woT, *wdT, *wguT, *wqkvT, *bcat, *aqvT;
+  double* inv_freq;
+};
+
+static size_t carve_packed(Carve& c, const Dims& d, Packed* p) {
+  p->wqkv = c.take<bf16>((size_t)3 * d.HD * d.h);
+  p->lorab = c.take<bf16>((size_t)3 * d.HD * LORA_PAD);
+  p->aqv = c.take<bf16>((size_t)2 * LORA_R * d.h);
+  p->wgu = c.take<bf16>((size_t)2 * d.F * d.h);
+  p->woT = c.take<bf16>((size_t)d.HD * d.h);
+  p->wdT = c.take<bf16>((size_t)d.F * d.h);
+  p->wguT = c.take<bf16>((size_t)d.h * 2 * d.F);
+  p->wqkvT = c.take<bf16>((size_t)d.h * 3 * d.HD);
+  p->bcat = c.take<bf16>((size_t)2 * LORA_R * 3 * d.HD);
+  p->aqvT = c.take<bf16>((size_t)d.h * LORA_PAD);
+  p->inv_freq = c.take<double>(64);
+  return c.used();
+}
+
+struct Saved {
+  bf16 *xr, *qkv, *o, *hres;
+  float *t, *lse, *rstd1, *rstd2;
+};
+
+static size_t carve_saved(Carve& c, const Dims& d, int nc, Saved* s) {
+  s->xr = c.take<bf16>((size_t)nc * d.h);
+  s->qkv = c.take<bf16>((size_t)nc * 3 * d.HD);
+  s->o = c.take<bf16>((size_t)nc * d.HD);
+  s->hres = c.take<bf16>((size_t)nc * d.h);
+  s->t = c.take<float>((size_t)nc * 2 * LORA_R);
+  s->lse = c.take<float>((size_t)d.H * nc);
+  s->rstd1 = c.take<float>(nc);
+  s->rstd2 = c.take<float>(nc);
+  return c.used();
+}
+
+struct FwdWs {
+  bf16 *xn, *tb, *a;
+};
+static size_t carve_fwd_ws(Carve& c, const Dims& d, int nc, FwdWs* w) {
+  w->xn = c.take<bf16>((size_t)nc * d.h);
+  w->tb = c.take<bf16>((size_t)nc * LORA_PAD);
+  w->a = c.take<bf16>((size_t)nc * d.F);
+  return c.used();
+}
+
+struct BwdWs {
+  float *dk_acc, *dv_acc;
+  bf16 *xn, *gu, *g, *dgu, *dhb, *dO, *dqkv, *dtb;
+  float *dhn, *dh, *delta, *dq, *dt, *part;
+};
+static size_t carve_bwd_ws(Carve& c, const Dims& d, int nc, int T, BwdWs* w) {
+  w->dk_acc = c.take<float>((size_t)nc * d.HD);
+  w->dv_acc = c.take<float>((size_t)nc * d.HD);
+  w->xn = c.take<bf16>((size_t)T * d.h);
+  w->gu = c.take<bf16>((size_t)T * 2 * d.F);
+  w->g = c.take<bf16>((size_t)T * d.h);
+  w->dgu = c.take<bf16>((size_t)T * 2 * d.F);
+  w->dhb = c.take<bf16>((size_t)T * d.h);
+  w->dO = c.take<bf16>((size_t)T * d.HD);
+  w->dqkv = c.take<bf16>((size_t)T * 3 * d.HD);
+  w->dtb = c.take<bf16>((size_t)T * LORA_PAD);
+  w->dhn = c.take<float>((size_t)T * d.h);
+  w->dh = c.take<float>((size_t)T * d.h);
+  w->delta = c.take<float>((size_t)d.H * T);
+  w->dq = c.take<float>((size_t)T * d.HD);
+  w->dt = c.take<float>((size_t)T * 2 * LORA_R);
+  const int chunks = (T + LG_CHUNK - 1) / LG_CHUNK;
+  const int cmax = d.HD > d.h ? d.HD : d.h;
+  w->part = c.take<float>((size_t)chunks * cmax * 16);
+  return c.used();
+}
+
+static int grid_cap(int64_t work, int per_block) {
+  int64_t g = (work + per_block - 1) / per_block;
+  int cap = sm_count() * 16;
+  if (g < 1) g = 1;
+  return (int)(g < cap ? g : cap);
+}
+
+static jenga_status transpose(const bf16* src, int64_t lds, bf16* dst, int64_t ldd, int R, int C, cudaStream_t st) {
+  dim3 g((C + 31) / 32, (R + 31) / 32);
+  {
+  const int _ps = ::jenga::prof_begin("transpose_bf16", st);
+  transpose_bf16_kernel<<<g, dim3(32, 8), 0, st>>>(src, lds, dst, ldd, R, C);
+  ::jenga::prof_end(_ps, st);
+  }
+  JENGA_LAUNCH_CHECK();
+  return JENGA_OK;
+}
+static jenga_status copy2d(const bf16* src, int64_t lds, bf16* dst, int64_t ldd, int R, int C, cudaStream_t st) {
+  {
+  const int _ps = ::jenga::prof_begin("copy_bf16", st);
+  copy_bf16_kernel<<<grid_cap((int64_t)R * C, 256), 256, 0, st>>>(src, lds, dst, ldd, R, C);
+  ::jenga::prof_end(_ps, st);
+  }
+  JENGA_LAUNCH_CHECK();
+  return JENGA_OK;
+}
+static jenga_status zero(bf16* dst, int64_t n, cudaStream_t st) {
+  {
+  const int _ps = ::jenga::prof_begin("zero_bf16", st);
+  zero_bf16_kernel<<<grid_cap(n, 256), 256, 0, st>>>(dst, n);
+  ::jenga::prof_end(_ps, st);
+  }
+  JENGA_LAUNCH_CHECK();
+  return JENGA_OK;
+}
+
+#define JENGA_TRY(expr)                   \
+  do {                                    \
+    jenga_status _s = (expr);             \
+    if (_s != JENGA_OK) return _s;        \
+  } while (0)
+
+static EpiParams epi_base(const int32_t* idx, int blk, const int32_t* n_kept, int row_offset) {
+  EpiParams e;
+  e.idx = idx;
+  e.blk = blk;
+  e.n_valid = n_kept;
+  e.valid_mult = blk;
+  e.row_offset = row_offset;
+  return e;
+}
+
+static jenga_status rmsnorm(const bf16* x, int64_t ldx, const int32_t* idx, int blk, int row_offset,
+                            const int32_t* n_valid, int mult, int rows, int h, float eps, const bf16* gain, bf16* xr,
+                            bf16* xn, float* rstd, cudaStream_t st, int64_t x_rows = 0) {
+  if (rows <= 0) return JENGA_OK;
+  {
+  const int _ps = ::jenga::prof_begin("rmsnorm_rows", st);
+  rmsnorm_rows_kernel<<<rows, ROW_THREADS, 0, st>>>(x, ldx, idx, blk, row_offset, n_valid, mult, h, eps, gain, xr, h,
+                                                    xn, h, rstd, x_rows ? x_rows : rows);
+  ::jenga::prof_end(_ps, st);
+  }
+  JENGA_LAUNCH_CHECK();
+  return JENGA_OK;
+}
+
+}  // namespace jenga
+
+using namespace jenga;
+
+// ==================================================================== pack
+extern "C" size_t jenga_layer_pack_bytes(const jenga_layer_weights* w, const jenga_lora* lora) {
+  Dims d;
+  if (check_weights(w, lora, &d) != JENGA_OK) return 0;
+  Carve c(nullptr);
+  Packed p;
+  return carve_packed(c, d, &p);
+}
+
+extern "C" jenga_status jenga_layer_pack(const jenga_layer_weights* w, const jenga_lora* lora, void* packed,
+                                         size_t packed_bytes, jenga_stream_t stream) {
+  Dims d;
+  JENGA_TRY(check_weights(w, lora, &d));
+  const size_t need = jenga_layer_pack_bytes(w, lora);
+  if (!packed || packed_bytes < need) return fail(JENGA_EWORKSPACE, "jenga_layer_pack: %zu < %zu bytes", packed_bytes, need);
+  cudaStream_t st = (cudaStream_t)stream;
+  Carve c(packed, packed_bytes);
+  Packed p;
+  carve_packed(c, d, &p);
+  const int h = d.h, HD = d.HD, F = d.F;
+  const bf16* wq = (const bf16*)w->wq;
+  const bf16* wk = (const bf16*)w->wk;
+  const bf16* wv = (const bf16*)w->wv;
+  const bf16* wg = (const bf16*)w->wg;
+  const bf16* wu = (const bf16*)w->wu;
+  // fused QKV [3HD, h]
+  JENGA_TRY(copy2d(wq, h, p.wqkv, h, HD, h, st));
+  JENGA_TRY(copy2d(wk, h, p.wqkv + (size_t)HD * h, h, HD, h, st));
+  JENGA_TRY(copy2d(wv, h, p.wqkv + (size_t)2 * HD * h, h, HD, h, st));
+  // LoRA up-projection as a K=64 operand: rows of q -> cols 0..15 = Bq, rows of v -> cols 16..31 = Bv
+  JENGA_TRY(zero(p.lorab, (int64_t)3 * HD * LORA_PAD, st));
+  JENGA_TRY(copy2d((const bf16*)lora->bq, LORA_R, p.lorab, LORA_PAD, HD, LORA_R, st));
+  JENGA_TRY(copy2d((const bf16*)lora->bv, LORA_R, p.lorab + (size_t)2 * HD * LORA_PAD + LORA_R, LORA_PAD, HD, LORA_R, st));
+  // LoRA down-projection [Aq; Av] (32 x h)
+  JENGA_TRY(copy2d((const bf16*)lora->aq, h, p.aqv, h, LORA_R, h, st));
+  JENGA_TRY(copy2d((const bf16*)lora->av, h, p.aqv + (size_t)LORA_R * h, h, LORA_R, h, st));
+  // gate/up interleaved in groups of 64 rows: [g 0..63, u 0..63, g 64..127, u 64..127, ...]
+  for (int grp = 0; grp < F / 64; ++grp) {
+    JENGA_TRY(copy2d(wg + (size_t)grp * 64 * h, h, p.wgu + (size_t)grp * 128 * h, h, 64, h, st));
+    JENGA_TRY(copy2d(wu + (size_t)grp * 64 * h, h, p.wgu + (size_t)(grp * 128 + 64) * h, h, 64, h, st));
+  }
+  // transposes for the backward
+  JENGA_TRY(transpose((const bf16*)w->wo, HD, p.woT, h, h, HD, st));          // Wo [h, HD] -> [HD, h]
+  JENGA_TRY(transpose((const bf16*)w->wd, F, p.wdT, h, h, F, st));            // Wd [h, F]  -> [F, h]
+  JENGA_TRY(transpose(p.wgu, h, p.wguT, 2 * F, 2 * F, h, st));                // [2F, h]    -> [h, 2F]
+  JENGA_TRY(transpose(p.wqkv, h, p.wqkvT, 3 * HD, 3 * HD, h, st));            // [3HD, h]   -> [h, 3HD]
+  // dt = dqkv * bcat^T : rows 0..15 = [Bq^T | 0 | 0], rows 16..31 = [0 | 0 | Bv^T]
+  JENGA_TRY(zero(p.bcat, (int64_t)2 * LORA_R * 3 * HD, st));
+  JENGA_TRY(transpose((const bf16*)lora->bq, LORA_R, p.bcat, 3 * HD, HD, LORA_R, st));
+  JENGA_TRY(transpose((const bf16*)lora->bv, LORA_R, p.bcat + (size_t)LORA_R * 3 * HD + 2 * HD, 3 * HD, HD, LORA_R, st));
+  // [Aq; Av]^T padded to 64 columns: [h, 64]
+  JENGA_TRY(zero(p.aqvT, (int64_t)h * LORA_PAD, st));
+  JENGA_TRY(transpose(p.aqv, h, p.aqvT, LORA_PAD, 2 * LORA_R, h, st));
+  {
+  const int _ps = ::jenga::prof_begin("inv_freq", st);
+  inv_freq_kernel<<<1, 64, 0, st>>>(p.inv_freq, d.D, log2((double)w->rope_theta));
+  ::jenga::prof_end(_ps, st);
+  }
+  JENGA_LAUNCH_CHECK();
+  return JENGA_OK;
+}
+
+// ==================================================================== score q/k (a1)
+extern "C" size_t jenga_layer_score_qk_workspace_bytes(const jenga_layer_weights* w, int B, int S) {
+  if (!w || B < 1 || S < 1) return 0;
+  Carve c(nullptr);
+  c.take<bf16>((size_t)S * w->hidden);
+  c.take<float>((size_t)S * 2 * LORA_R);
+  c.take<bf16>((size_t)S * LORA_PAD);
+  return c.used();
+}
+
+extern "C" jenga_status jenga_layer_score_qk(const jenga_layer_weights* w, const jenga_lora* lora, const void* packed,
+                                             const void* x, int B, int S, void* qk, void* ws, size_t ws_bytes,
+                                             jenga_stream_t stream) {
+  Dims d;
+  JENGA_TRY(check_weights(w, lora, &d));
+  JENGA_CHECK_ARG(packed && x && qk, "jenga_layer_score_qk: null pointer");
+  JENGA_CHECK_ARG(B == 1, "jenga_layer_score_qk: batch 1 only");
+  JENGA_CHECK_ARG(S >= 1, "jenga_layer_score_qk: S");
+  const size_t need = jenga_layer_score_qk_workspace_bytes(w, B, S);
+  if (!ws || ws_bytes < need) return fail(JENGA_EWORKSPACE, "jenga_layer_score_qk: workspace %zu < %zu", ws_bytes, need);
+  cudaStream_t st = (cudaStream_t)stream;
+  Carve pc((void*)packed);
+  Packed p;
+  carve_packed(pc, d, &p);
+  Carve c(ws, ws_bytes);
+  bf16* xn = c.take<bf16>((size_t)S * d.h);
+  float* t = c.take<float>((size_t)S * 2 * LORA_R);
+  bf16* tb = c.take<bf16>((size_t)S * LORA_PAD);
+  JENGA_TRY(rmsnorm((const bf16*)x, d.h, nullptr, 1, 0, nullptr, 1, S, d.h, w->rms_eps, (const bf16*)w->attn_norm,
+                    nullptr, xn, nullptr, st));
+  EpiParams e;
+  e.out = t;
+  e.ldo = 2 * LORA_R;
+  e.aux = tb;
+  e.ld_aux = LORA_PAD;
+  e.alpha = lora->scale;
+  e.beta = 1.f;
+  JENGA_TRY((launch_gemm<32, EPI_LORA_T>({xn, S, d.h}, {p.aqv, 2 * LORA_R, d.h}, d.h, nullptr, nullptr, 0, S,
+                                         2 * LORA_R, e, st, "gemm_lora_t_all")));
+  EpiParams q;
+  q.out = qk;
+  q.ldo = 2 * d.HD;
+  q.hd = d.HD;
+  q.inv_freq = p.inv_freq;
+  GemmOperand a2{tb, S, LORA_PAD}, b2{p.lorab, 2 * d.HD, LORA_PAD};
+  JENGA_TRY((launch_gemm<256, EPI_QKV_ROPE>({xn, S, d.h}, {p.wqkv, 2 * d.HD, d.h}, d.h, &a2, &b2, LORA_PAD, S,
+                                            2 * d.HD, q, st, "gemm_qk_rope_all")));
+  return JENGA_OK;
+}
+
+// ==================================================================== forward
+extern "C" size_t jenga_layer_saved_bytes(const jenga_layer_weights* w, int B, int blk, int n_kept_max) {
+  if (!w || B < 1 || blk < 1 || n_kept_max < 0) return 0;
+  Dims d{w->hidden, w->heads, w->head_dim, w->heads * w->head_dim, w->ffn};
+  Carve c(nullptr);
+  Saved s;
+  return carve_saved(c, d, n_kept_max * blk, &s);
+}
+
+extern "C" size_t jenga_layer_fwd_workspace_bytes(const jenga_layer_weights* w, int B, int blk, int n_kept_max) {
+  if (!w || B < 1 || blk < 1 || n_kept_max < 0) return 0;
+  Dims d{w->hidden, w->heads, w->head_dim, w->heads * w->head_dim, w->ffn};
+  Carve c(nullptr);
+  FwdWs f;
+  return carve_fwd_ws(c, d, n_kept_max * blk, &f);
+}
+
+extern "C" jenga_status jenga_sparse_layer_fwd(const jenga_layer_weights* w, const jenga_lora* lora,
+                                               const void* packed, void* x, int B, int S, int blk, const int32_t* idx,
+                                               const int32_t* n_kept, int n_kept_max, void* saved, size_t saved_bytes,
+                                               void* ws, size_t ws_bytes, jenga_stream_t stream) {
+  Dims d;
+  JENGA_TRY(check_weights(w, lora, &d));
+  JENGA_CHECK_ARG(packed && x && idx && n_kept, "jenga_sparse_layer_fwd: null pointer");
+  JENGA_CHECK_ARG(B == 1, "jenga_sparse_layer_fwd: batch 1 only");
+  JENGA_CHECK_ARG(blk >= 64 && blk % 64 == 0 && S % blk == 0, "jenga_sparse_layer_fwd: blk must be a multiple of 64 dividing S");
+  JENGA_CHECK_ARG(n_kept_max >= 0 && n_kept_max <= S / blk, "jenga_sparse_layer_fwd: n_kept_max");
+  const size_t need_s = jenga_layer_saved_bytes(w, B, blk, n_kept_max);
+  const size_t need_w = jenga_layer_fwd_workspace_bytes(w, B, blk, n_kept_max);
+  if (!saved || saved_bytes < need_s) return fail(JENGA_EWORKSPACE, "jenga_sparse_layer_fwd: saved %zu < %zu", saved_bytes, need_s);
+  if (!ws || ws_bytes < need_w) return fail(JENGA_EWORKSPACE, "jenga_sparse_layer_fwd: workspace %zu < %zu", ws_bytes, need_w);
+  const int nc = n_kept_max * blk;
+  if (nc == 0) return JENGA_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  Carve pc((void*)packed);
+  Packed p;
+  carve_packed(pc, d, &p);
+  Carve sc(saved, saved_bytes);
+  Saved s;
+  carve_saved(sc, d, nc, &s);
+  Carve wc(ws, ws_bytes);
+  FwdWs f;
+  carve_fwd_ws(wc, d, nc, &f);
+  bf16* X = (bf16*)x;
+  const int h = d.h, HD = d.HD, F = d.F;
+
+  // 1. permutation-free gather of the retained rows + RMSNorm
+  JENGA_TRY(rmsnorm(X, h, idx, blk, 0, n_kept, blk, nc, h, w->rms_eps, (const bf16*)w->attn_norm, s.xr, f.xn, s.rstd1, st,
+                    S));
+  // 2. LoRA down-projection t = xn [Aq; Av]^T (fp32 saved) and s * t (bf16, K-padded)
+  {
+    EpiParams e = epi_base(idx, blk, n_kept, 0);
+    e.out = s.t;
+    e.ldo = 2 * LORA_R;
+    e.aux = f.tb;
+    e.ld_aux = LORA_PAD;
+    e.alpha = lora->scale;
+    e.beta = 1.f;
+    JENGA_TRY((launch_gemm<32, EPI_LORA_T>({f.xn, nc, h}, {p.aqv, 2 * LORA_R, h}, h, nullptr, nullptr, 0, nc,
+                                           2 * LORA_R, e, st, "gemm_lora_t")));
+  }
+  // 3. QKV (+ LoRA up-projection as a second K phase) with RoPE at original positions
+  {
+    EpiParams e = epi_base(idx, blk, n_kept, 0);
+    e.out = s.qkv;
+    e.ldo = 3 * HD;
+    e.hd = HD;
+    e.inv_freq = p.inv_freq;
+    GemmOperand a2{f.tb, nc, LORA_PAD}, b2{p.lorab, 3 * HD, LORA_PAD};
+    JENGA_TRY((launch_gemm<256, EPI_QKV_ROPE>({f.xn, nc, h}, {p.wqkv, 3 * HD, h}, h, &a2, &b2, LORA_PAD, nc, 3 * HD,
+                                              e, st, "gemm_qkv_rope")));
+  }
+  // 4. causal attention among retained tokens
+  JENGA_TRY(attn_forward(s.qkv, s.qkv + HD, s.qkv + 2 * HD, 3 * HD, s.o, HD, s.lse, nc, d.H, n_kept, blk, nc, st));
+  // 5. o_proj with the in-place residual add into X (and a compact copy of h)
+  {
+    EpiParams e = epi_base(idx, blk, n_kept, 0);
+    e.x = X;
+    e.ldx = h;
+    e.x_rows = S;
+    e.aux = s.hres;
+    e.ld_aux = h;
+    JENGA_TRY((launch_gemm<256, EPI_SCATTER_ADD>({s.o, nc, HD}, {w->wo, h, HD}, HD, nullptr, nullptr, 0, nc, h, e, st, "gemm_o_scatter")));
+  }
+  // 6. RMSNorm before the MLP
+  JENGA_TRY(rmsnorm(s.hres, h, nullptr, 1, 0, n_kept, blk, nc, h, w->rms_eps, (const bf16*)w->mlp_norm, nullptr, f.xn,
+                    s.rstd2, st));
+  // 7. gate/up with SiLU(g) * u
+  {
+    EpiParams e = epi_base(idx, blk, n_kept, 0);
+    e.out = f.a;
+    e.ldo = F;
+    JENGA_TRY((launch_gemm<256, EPI_SWIGLU>({f.xn, nc, h}, {p.wgu, 2 * F, h}, h, nullptr, nullptr, 0, nc, 2 * F, e, st, "gemm_gateup_swiglu")));
+  }
+  // 8. down_proj with the in-place residual add into X
+  {
+    EpiParams e = epi_base(idx, blk, n_kept, 0);
+    e.x = X;
+    e.ldx = h;
+    e.x_rows = S;
+    JENGA_TRY((launch_gemm<256, EPI_SCATTER_ADD>({f.a, nc, F}, {w->wd, h, F}, F, nullptr, nullptr, 0, nc, h, e, st, "gemm_down_scatter")));
+  }
+  return JENGA_OK;
+}
+
+// ==================================================================== backward
+extern "C" size_t jenga_layer_bwd_workspace_bytes(const jenga_layer_weights* w, int B, int blk, int n_kept_max,
+                                                  int segment_tokens) {
+  if (!w || B < 1 || blk < 1 || n_kept_max < 0 || segment_tokens < 1) return 0;
+  Dims d{w->hidden, w->heads, w->head_dim, w->heads * w->head_dim, w->ffn};
+  const int nc = n_kept_max * blk;
+  const int T = segment_tokens < nc ? segment_tokens : (nc > 0 ? nc : 1);
+  Carve c(nullptr);
+  BwdWs b;
+  return carve_bwd_ws(c, d, nc, T, &b);
+}
+
+extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, const jenga_lora* lora,
+                                               const void* packed, void* dx, int B, int S, int blk, const int32_t* idx,
+                                               const int32_t* n_kept, int n_kept_max, const void* saved,
+                                               size_t saved_bytes, jenga_lora_grads* grads, int segment_tokens,
+                                               void* ws, size_t ws_bytes, jenga_stream_t stream) {
+  Dims d;
+  JENGA_TRY(check_weights(w, lora, &d));
+  JENGA_CHECK_ARG(packed && dx && idx && n_kept && saved && grads, "jenga_sparse_layer_bwd: null pointer");
+  JENGA_CHECK_ARG(grads->daq && grads->dbq && grads->dav && grads->dbv, "jenga_sparse_layer_bwd: null gradient");
+  JENGA_CHECK_ARG(B == 1, "jenga_sparse_layer_bwd: batch 1 only");
+  JENGA_CHECK_ARG(blk >= 64 && blk % 64 == 0 && S % blk == 0, "jenga_sparse_layer_bwd: blk");
+  JENGA_CHECK_ARG(n_kept_max >= 0 && n_kept_max <= S / blk, "jenga_sparse_layer_bwd: n_kept_max");
+  JENGA_CHECK_ARG(segment_tokens >= 128 && segment_tokens % 128 == 0 && segment_tokens % blk == 0,
+                  "jenga_sparse_layer_bwd: segment_tokens must be a multiple of 128 and of blk");
+  const size_t need_s = jenga_layer_saved_bytes(w, B, blk, n_kept_max);
+  const size_t need_w = jenga_layer_bwd_workspace_bytes(w, B, blk, n_kept_max, segment_tokens);
+  if (saved_bytes < need_s) return fail(JENGA_EWORKSPACE, "jenga_sparse_layer_bwd: saved %zu < %zu", saved_bytes, need_s);
+  if (!ws || ws_bytes < need_w) return fail(JENGA_EWORKSPACE, "jenga_sparse_layer_bwd: workspace %zu < %zu", ws_bytes, need_w);
+  const int nc = n_kept_max * blk;
+  if (nc == 0) return JENGA_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int h = d.h, HD = d.HD, F = d.F, H = d.H;
+  const float ls = lora->scale;
+  Carve pc((void*)packed);
+  Packed p;
+  carve_packed(pc, d, &p);
+  Carve sc((void*)saved, saved_bytes);
+  Saved s;
+  carve_saved(sc, d, nc, &s);
+  const int Tmax = segment_tokens < nc ? segment_tokens : nc;
+  Carve wc(ws, ws_bytes);
+  BwdWs b;
+  carve_bwd_ws(wc, d, nc, Tmax, &b);
+  bf16* dX = (bf16*)dx;
+
+  JENGA_CUDA_TRY(cudaMemsetAsync(b.dk_acc, 0, (size_t)nc * HD * sizeof(float), st));
+  JENGA_CUDA_TRY(cudaMemsetAsync(b.dv_acc, 0, (size_t)nc * HD * sizeof(float), st));
+  const int nseg = (nc + segment_tokens - 1) / segment_tokens;
+  for (int sg = nseg - 1; sg >= 0; --sg) {
+    const int s0 = sg * segment_tokens;
+    const int s1 = (s0 + segment_tokens < nc) ? s0 + segment_tokens : nc;
+    const int T = s1 - s0;
+    // --- MLP block (recomputed): hn, (g, u)
+    JENGA_TRY(rmsnorm(s.hres + (size_t)s0 * h, h, nullptr, 1, s0, n_kept, blk, T, h, w->rms_eps,
+                      (const bf16*)w->mlp_norm, nullptr, b.xn, nullptr, st));
+    {
+      EpiParams e = epi_base(idx, blk, n_kept, s0);
+      e.out = b.gu;
+      e.ldo = 2 * F;
+      JENGA_TRY((launch_gemm<256, EPI_STORE_BF16>({b.xn, T, h}, {p.wgu, 2 * F, h}, h, nullptr, nullptr, 0, T, 2 * F, e, st, "gemm_gateup_recompute")));
+    }
+    // upstream gradient rows of this segment
+    {
+    const int _ps = ::jenga::prof_begin("gather_seg", st);
+    gather_seg_kernel<<<grid_cap((int64_t)T * (h / 8), 256), 256, 0, st>>>(dX, h, b.g, h, idx, blk, s0, n_kept, blk, T, h,
+                                                                         S);
+    ::jenga::prof_end(_ps, st);
+    }
+    JENGA_LAUNCH_CHECK();
+    // dA = G Wd ; (dg, du) from SiLU(g) * u
+    {
+      EpiParams e = epi_base(idx, blk, n_kept, s0);
+      e.out = b.dgu;
+      e.ldo = 2 * F;
+      e.aux = b.gu;
+      e.ld_aux = 2 * F;
+      JENGA_TRY((launch_gemm<256, EPI_SWIGLU_BWD>({b.g, T, h}, {p.wdT, F, h}, h, nullptr, nullptr, 0, T, F, e, st, "gemm_da_swiglu_bwd")));
+    }
+    // dhn = [dg, du] [Wg; Wu]
+    {
+      EpiParams e = epi_base(idx, blk, n_kept, s0);
+      e.out = b.dhn;
+      e.ldo = h;
+      JENGA_TRY((launch_gemm<256, EPI_STORE_F32>({b.dgu, T, 2 * F}, {p.wguT, h, 2 * F}, 2 * F, nullptr, nullptr, 0, T, h, e, st, "gemm_dhn")));
+    }
+    // dh = G + RMSNorm_bwd(dhn)
+    {
+    const int _ps = ::jenga::prof_begin("rmsnorm_bwd_rows", st);
+    rmsnorm_bwd_rows_kernel<<<T, ROW_THREADS, 0, st>>>(b.dhn, h, s.hres + (size_t)s0 * h, h, s.rstd2 + s0,
+                                                        (const bf16*)w->mlp_norm, nullptr, b.g, h, b.dh, b.dhb, h,
+                                                        nullptr, 0, idx, blk, s0, n_kept, blk, h, S);
+    ::jenga::prof_end(_ps, st);
+    }
+    JENGA_LAUNCH_CHECK();
+    // --- attention block: dO = dh Wo
+    {
+      EpiParams e = epi_base(idx, blk, n_kept, s0);
+      e.out = b.dO;
+      e.ldo = HD;
+      JENGA_TRY((launch_gemm<256, EPI_STORE_BF16>({b.dhb, T, h}, {p.woT, HD, h}, h, nullptr, nullptr, 0, T, HD, e, st, "gemm_do")));
+    }
+    JENGA_TRY(attn_backward_segment(s.qkv, s.qkv + HD, s.qkv + 2 * HD, 3 * HD, s.o, HD, s.lse, nc, b.dO, HD, b.delta, T,
+                                    b.dq, HD, b.dk_acc, b.dv_acc, HD, H, s0, s1, n_kept, blk, nc, st));
+    // keys of this segment are complete: RoPE^T and pack dQKV (bf16)
+    {
+    const int _ps = ::jenga::prof_begin("rope_bwd_pack", st);
+    rope_bwd_pack_kernel<<<grid_cap((int64_t)T * H * 64, 256), 256, 0, st>>>(
+        b.dq, HD, b.dk_acc, b.dv_acc, HD, s0, b.dqkv, 3 * HD, idx, blk, n_kept, blk, T, H, p.inv_freq);
+    ::jenga::prof_end(_ps, st);
+    }
+    JENGA_LAUNCH_CHECK();
+    // dt = s [dq Bq, dv Bv]  (fp32, and bf16 K-padded for the dX GEMM)
+    {
+      EpiParams e = epi_base(idx, blk, n_kept, s0);
+      e.out = b.dt;
+      e.ldo = 2 * LORA_R;
+      e.aux = b.dtb;
+      e.ld_aux = LORA_PAD;
+      e.alpha = ls;
+      e.beta = ls;
+      JENGA_TRY((launch_gemm<32, EPI_LORA_T>({b.dqkv, T, 3 * HD}, {p.bcat, 2 * LORA_R, 3 * HD}, 3 * HD, nullptr, nullptr,
+                                             0, T, 2 * LORA_R, e, st, "gemm_dt")));
+    }
+    // xn of the segment (recomputed from the saved gathered input)
+    JENGA_TRY(rmsnorm(s.xr + (size_t)s0 * h, h, nullptr, 1, s0, n_kept, blk, T, h, w->rms_eps,
+                      (const bf16*)w->attn_norm, nullptr, b.xn, nullptr, st));
+    // LoRA gradients (deterministic split over rows)
+    {
+      const int chunks = (T + LG_CHUNK - 1) / LG_CHUNK;
+      struct G {
+        const bf16* X;
+        int64_t ldx;
+        const float* Y;
+        int C;
+        float scale;
+        float* out;
+        int64_t so_c, so_r;
+      } jobs[4] = {
+          {b.dqkv, 3 * HD, s.t + (size_t)s0 * 2 * LORA_R, HD, ls, grads->dbq, LORA_R, 1},
+          {b.dqkv + 2 * HD, 3 * HD, s.t + (size_t)s0 * 2 * LORA_R + LORA_R, HD, ls, grads->dbv, LORA_R, 1},
+          {b.xn, h, b.dt, h, 1.f, grads->daq, 1, h},
+          {b.xn, h, b.dt + LORA_R, h, 1.f, grads->dav, 1, h},
+      };
+      for (auto& j : jobs) {
+        {
+        const int _ps = ::jenga::prof_begin("lora_grad_partial", st);
+        lora_grad_partial_kernel<<<dim3(j.C / 64, chunks), 256, 0, st>>>(j.X, j.ldx, j.Y, 2 * LORA_R, j.C, T, n_kept,
+                                                                          blk, s0, b.part);
+        ::jenga::prof_end(_ps, st);
+        }
+        JENGA_LAUNCH_CHECK();
+        {
+        const int _ps = ::jenga::prof_begin("lora_grad_reduce", st);
+        lora_grad_reduce_kernel<<<(j.C * 16 + 255) / 256, 256, 0, st>>>(b.part, chunks, j.C, j.scale, j.out, j.so_c,
+                                                                          j.so_r);
+        ::jenga::prof_end(_ps, st);
+        }
+        JENGA_LAUNCH_CHECK();
+      }
+    }
+    // dxn = dQKV [Wq; Wk; Wv] + dt [Aq; Av]
+    {
+      EpiParams e = epi_base(idx, blk, n_kept, s0);
+      e.out = b.dhn;
+      e.ldo = h;
+      GemmOperand a2{b.dtb, T, LORA_PAD}, b2{p.aqvT, h, LORA_PAD};
+      JENGA_TRY((launch_gemm<256, EPI_STORE_F32>({b.dqkv, T, 3 * HD}, {p.wqkvT, h, 3 * HD}, 3 * HD, &a2, &b2, LORA_PAD, T,
+                                                 h, e, st, "gemm_dxn")));
+    }
+    // dX[rows] = dh + RMSNorm_bwd(dxn)  (written in place into the gradient buffer)
+    {
+    const int _ps = ::jenga::prof_begin("rmsnorm_bwd_rows", st);
+    rmsnorm_bwd_rows_kernel<<<T, ROW_THREADS, 0, st>>>(b.dhn, h, s.xr + (size_t)s0 * h, h, s.rstd1 + s0,
+                                                        (const bf16*)w->attn_norm, b.dh, nullptr, h, nullptr, nullptr,
+                                                        h, dX, h, idx, blk, s0, n_kept, blk, h, S);
+    ::jenga::prof_end(_ps, st);
+    }
+    JENGA_LAUNCH_CHECK();
+  }
+  return JENGA_OK;
+}
+
+// ==================================================================== test hook
+// C[M, N] = A[M, K] B[N, K]^T (bf16 in, fp32 accumulate), stored bf16 or fp32.
+extern "C" jenga_status jenga_test_gemm(const void* A, int64_t lda, const void* B, int64_t ldb, int M, int N, int K,
+                                        void* C, int64_t ldc, int out_f32, int bn, jenga_stream_t stream) {
+  JENGA_CHECK_ARG(A && B && C && M > 0 && N > 0 && K > 0 && K % 64 == 0, "jenga_test_gemm: bad args");
+  EpiParams e;
+  e.out = C;
+  e.ldo = ldc;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (bn == 256) {
+    if (out_f32) return launch_gemm<256, EPI_STORE_F32>({A, M, lda}, {B, N, ldb}, K, nullptr, nullptr, 0, M, N, e, st);
+    return launch_gemm<256, EPI_STORE_BF16>({A, M, lda}, {B, N, ldb}, K, nullptr, nullptr, 0, M, N, e, st);
+  }
+  if (bn == 32) return launch_gemm<32, EPI_STORE_F32>({A, M, lda}, {B, N, ldb}, K, nullptr, nullptr, 0, M, N, e, st);
+  return fail(JENGA_EINVAL, "jenga_test_gemm: bn must be 256 or 32");
+}

@@ -1,0 +1,305 @@
+// Row kernels of the retained-token layer: RMSNorm (with the permutation-free
+// gather of the retained rows), RMSNorm backward (with the in-place scatter of dX),
+// segment gather, RoPE backward + dQKV packing, LoRA gradient reductions, and the
+// weight re-layout used by jenga_layer_pack.
+#pragma once
+
+#include "common.cuh"
+
+namespace jenga {
+
+constexpr int ROW_THREADS = 256;
+constexpr int ROW_MAX_CHUNKS = 4;  // 8-element chunks per thread: hidden <= 8192
+
+__device__ __forceinline__ float block_sum_256(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int w = 0; w < ROW_THREADS / 32; ++w) t += red[w];
+  return t;
+}
+
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+__device__ __forceinline__ uint4 pack8(const float* f) {
+  uint4 u;
+  uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  return u;
+}
+
+__device__ __forceinline__ int valid_rows(const int32_t* n_valid, int mult, int row_offset, int cap) {
+  if (!n_valid) return cap;
+  int v = (*n_valid) * mult - row_offset;
+  return v < 0 ? 0 : (v < cap ? v : cap);
+}
+
+__device__ __forceinline__ int64_t seq_row(const int32_t* idx, int blk, int c) {
+  if (!idx) return c;
+  const int b = c / blk;
+  return (int64_t)__ldg(idx + b) * blk + (c - b * blk);
+}
+
+// xn[m] = bf16(x[row(m)] * rstd * gain); rstd[m]; optionally xr[m] = x[row(m)] (gathered copy).
+// One CTA per compact row m in [0, rows); row(m) = seq_row(idx, blk, row_offset + m).
+__global__ void __launch_bounds__(ROW_THREADS) rmsnorm_rows_kernel(
+    const bf16* __restrict__ x, int64_t ldx, const int32_t* __restrict__ idx, int blk, int row_offset,
+    const int32_t* __restrict__ n_valid, int valid_mult, int h, float eps, const bf16* __restrict__ gain,
+    bf16* __restrict__ xr, int64_t ldr, bf16* __restrict__ xn, int64_t ldn, float* __restrict__ rstd_out,
+    int64_t x_rows) {
+  __shared__ float red[ROW_THREADS / 32];
+  const int m = blockIdx.x;
+  if (m >= valid_rows(n_valid, valid_mult, row_offset, gridDim.x)) return;
+  // with a kept-block list, x is the full sequence; without one, x is already compact
+  const int64_t row = idx ? seq_row(idx, blk, row_offset + m) : m;
+  if (row < 0 || row >= x_rows) {
+    if (threadIdx.x == 0) record_device_error(JENGA_EINTERNAL, SITE_INDEX_RANGE, (unsigned)row);
+    return;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(x + row * ldx);
+  const int nch = h >> 3;
+  float v[ROW_MAX_CHUNKS][8];
+  uint4 raw[ROW_MAX_CHUNKS];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < ROW_MAX_CHUNKS; ++i) {
+    const int c = threadIdx.x + i * ROW_THREADS;
+    if (c < nch) {
+      raw[i] = src[c];
+      unpack8(raw[i], v[i]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss = fmaf(v[i][e], v[i][e], ss);
+    }
+  }
+  ss = block_sum_256(ss, red);
+  const float r = rsqrtf(ss / (float)h + eps);
+  if (threadIdx.x == 0 && rstd_out) rstd_out[m] = r;
+  const uint4* gp = reinterpret_cast<const uint4*>(gain);
+#pragma unroll
+  for (int i = 0; i < ROW_MAX_CHUNKS; ++i) {
+    const int c = threadIdx.x + i * ROW_THREADS;
+    if (c < nch) {
+      if (xr) reinterpret_cast<uint4*>(xr + (int64_t)m * ldr)[c] = raw[i];
+      float gv[8], o[8];
+      unpack8(gp[c], gv);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = v[i][e] * r * gv[e];
+      reinterpret_cast<uint4*>(xn + (int64_t)m * ldn)[c] = pack8(o);
+    }
+  }
+}
+
+// RMSNorm backward fused with the residual:
+//   out[m] = base[m] + r g dy - x r^3 / h * sum(dy g x)
+// base: fp32 (base_f) or bf16 (base_b); outputs: fp32 out_f, bf16 out_b, and/or the
+// bf16 scatter into dst[row(m)] (in place, pitch ldd).
+__global__ void __launch_bounds__(ROW_THREADS) rmsnorm_bwd_rows_kernel(
+    const float* __restrict__ dy, int64_t lddy, const bf16* __restrict__ x, int64_t ldx,
+    const float* __restrict__ rstd, const bf16* __restrict__ gain, const float* __restrict__ base_f,
+    const bf16* __restrict__ base_b, int64_t ldb, float* __restrict__ out_f, bf16* __restrict__ out_b,
+    int64_t ldo, bf16* __restrict__ dst, int64_t ldd, const int32_t* __restrict__ idx, int blk, int row_offset,
+    const int32_t* __restrict__ n_valid, int valid_mult, int h, int64_t dst_rows) {
+  __shared__ float red[ROW_THREADS / 32];
+  const int m = blockIdx.x;
+  if (m >= valid_rows(n_valid, valid_mult, row_offset, gridDim.x)) return;
+  const int nch = h >> 3;
+  const float r = rstd[m];
+  float dyg[ROW_MAX_CHUNKS][8], xv[ROW_MAX_CHUNKS][8];
+  float dot = 0.f;
+#pragma unroll
+  for (int i = 0; i < ROW_MAX_CHUNKS; ++i) {
+    const int c = threadIdx.x + i * ROW_THREADS;
+    if (c < nch) {
+      const float4* dp = reinterpret_cast<const float4*>(dy + (int64_t)m * lddy) + 2 * c;
+      float4 a = dp[0], b = dp[1];
+      float gv[8];
+      unpack8(reinterpret_cast<const uint4*>(gain)[c], gv);
+      unpack8(reinterpret_cast<const uint4*>(x + (int64_t)m * ldx)[c], xv[i]);
+      const float d[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        dyg[i][e] = d[e] * gv[e];
+        dot = fmaf(dyg[i][e], xv[i][e], dot);
+      }
+    }
+  }
+  dot = block_sum_256(dot, red);
+  const float k = r * r * r * dot / (float)h;
+  const int64_t drow = dst ? seq_row(idx, blk, row_offset + m) : 0;
+  if (dst && (drow < 0 || drow >= dst_rows)) {
+    if (threadIdx.x == 0) record_device_error(JENGA_EINTERNAL, SITE_INDEX_RANGE, (unsigned)drow);
+    return;
+  }
+#pragma unroll
+  for (int i = 0; i < ROW_MAX_CHUNKS; ++i) {
+    const int c = threadIdx.x + i * ROW_THREADS;
+    if (c < nch) {
+      float bv[8];
+      if (base_f) {
+        const float4* bp = reinterpret_cast<const float4*>(base_f + (int64_t)m * ldb) + 2 * c;
+        float4 a = bp[0], b = bp[1];
+        bv[0] = a.x; bv[1] = a.y; bv[2] = a.z; bv[3] = a.w;
+        bv[4] = b.x; bv[5] = b.y; bv[6] = b.z; bv[7] = b.w;
+      } else {
+        unpack8(reinterpret_cast<const uint4*>(base_b + (int64_t)m * ldb)[c], bv);
+      }
+      float o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = bv[e] + r * dyg[i][e] - xv[i][e] * k;
+      if (out_f) {
+        float4* op = reinterpret_cast<float4*>(out_f + (int64_t)m * ldo) + 2 * c;
+        op[0] = make_float4(o[0], o[1], o[2], o[3]);
+        op[1] = make_float4(o[4], o[5], o[6], o[7]);
+      }
+      if (out_b) reinterpret_cast<uint4*>(out_b + (int64_t)m * ldo)[c] = pack8(o);
+      if (dst) reinterpret_cast<uint4*>(dst + drow * ldd)[c] = pack8(o);
+    }
+  }
+}
+
+// out[m] = src[row(row_offset + m)] for m in [0, rows) (bf16 rows, 16-byte vectors)
+__global__ void gather_seg_kernel(const bf16* __restrict__ src, int64_t lds, bf16* __restrict__ out, int64_t ldo,
+                                  const int32_t* __restrict__ idx, int blk, int row_offset,
+                                  const int32_t* __restrict__ n_valid, int valid_mult, int rows, int h,
+                                  int64_t src_rows) {
+  const int vpr = h >> 3;
+  const int nv = valid_rows(n_valid, valid_mult, row_offset, rows);
+  const int64_t total = (int64_t)nv * vpr;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int m = (int)(e / vpr), c = (int)(e - (int64_t)m * vpr);
+    const int64_t r = seq_row(idx, blk, row_offset + m);
+    if (r < 0 || r >= src_rows) {
+      record_device_error(JENGA_EINTERNAL, SITE_INDEX_RANGE, (unsigned)r);
+      continue;
+    }
+    reinterpret_cast<uint4*>(out + (int64_t)m * ldo)[c] = reinterpret_cast<const uint4*>(src + r * lds)[c];
+  }
+}
+
+// dqkv[m] = [rope^T(dq[m]) | rope^T(dk[s0+m]) | dv[s0+m]] in bf16; positions row(s0 + m).
+// One thread per (row, head, pair i < 64).
+__global__ void rope_bwd_pack_kernel(const float* __restrict__ dq, int64_t ld_dq, const float* __restrict__ dk,
+                                     const float* __restrict__ dv, int64_t ld_acc, int s0, bf16* __restrict__ dqkv,
+                                     int64_t ld_out, const int32_t* __restrict__ idx, int blk,
+                                     const int32_t* __restrict__ n_valid, int valid_mult, int rows, int H,
+                                     const double* __restrict__ inv_freq) {
+  const int nv = valid_rows(n_valid, valid_mult, s0, rows);
+  const int64_t total = (int64_t)nv * H * 64;
+  const int HD = H * 128;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int i = (int)(e & 63);
+    const int64_t mh = e >> 6;
+    const int hh = (int)(mh % H);
+    const int m = (int)(mh / H);
+    const int64_t pos = seq_row(idx, blk, s0 + m);
+    const double ang = (double)pos * inv_freq[i];
+    const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
+    float sn, cs;
+    sincosf((float)red, &sn, &cs);
+    const int c1 = hh * 128 + i, c2 = c1 + 64;
+    const float* q = dq + (int64_t)m * ld_dq;
+    const float* kk = dk + (int64_t)(s0 + m) * ld_acc;
+    const float* vv = dv + (int64_t)(s0 + m) * ld_acc;
+    bf16* o = dqkv + (int64_t)m * ld_out;
+    const float a1 = q[c1], a2 = q[c2];
+    o[c1] = __float2bfloat16_rn(a1 * cs + a2 * sn);
+    o[c2] = __float2bfloat16_rn(a2 * cs - a1 * sn);
+    const float b1 = kk[c1], b2 = kk[c2];
+    o[HD + c1] = __float2bfloat16_rn(b1 * cs + b2 * sn);
+    o[HD + c2] = __float2bfloat16_rn(b2 * cs - b1 * sn);
+    o[2 * HD + c1] = __float2bfloat16_rn(vv[c1]);
+    o[2 * HD + c2] = __float2bfloat16_rn(vv[c2]);
+  }
+}
+
+// Split-K partials of  P[chunk][c][r] = sum_{m in chunk} X[m, c] * Y[m, r]   (r < 16)
+// X bf16 [rows, ldx] (columns [0, C)), Y fp32 [rows, ldy] (columns [0, 16)).
+// grid (C / 64, chunks), 256 threads = 64 columns x 4 groups of 4 r.
+constexpr int LG_CHUNK = 256;
+__global__ void __launch_bounds__(256) lora_grad_partial_kernel(const bf16* __restrict__ X, int64_t ldx,
+                                                                const float* __restrict__ Y, int64_t ldy, int C,
+                                                                int rows, const int32_t* __restrict__ n_valid,
+                                                                int valid_mult, int row_offset,
+                                                                float* __restrict__ part) {
+  const int c = blockIdx.x * 64 + (threadIdx.x & 63);
+  const int rg = threadIdx.x >> 6;
+  const int nv = valid_rows(n_valid, valid_mult, row_offset, rows);
+  const int m0 = blockIdx.y * LG_CHUNK, m1 = min(nv, m0 + LG_CHUNK);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int m = m0; m < m1; ++m) {
+    const float xv = __bfloat162float(X[(int64_t)m * ldx + c]);
+    const float4 y = *reinterpret_cast<const float4*>(Y + (int64_t)m * ldy + rg * 4);
+    acc[0] = fmaf(xv, y.x, acc[0]);
+    acc[1] = fmaf(xv, y.y, acc[1]);
+    acc[2] = fmaf(xv, y.z, acc[2]);
+    acc[3] = fmaf(xv, y.w, acc[3]);
+  }
+  float* p = part + ((int64_t)blockIdx.y * C + c) * 16 + rg * 4;
+  *reinterpret_cast<float4*>(p) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+}
+
+// out[c * so_c + r * so_r] += scale * sum_chunk part[chunk][c][r]   (fixed chunk order)
+__global__ void lora_grad_reduce_kernel(const float* __restrict__ part, int chunks, int C, float scale,
+                                        float* __restrict__ out, int64_t so_c, int64_t so_r) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= C * 16) return;
+  const int c = e >> 4, r = e & 15;
+  float s = 0.f;
+  for (int k = 0; k < chunks; ++k) s += part[((int64_t)k * C + c) * 16 + r];
+  out[c * so_c + r * so_r] += scale * s;
+}
+
+// ---- weight re-layout (pack)
+// dst[(dr0 + c) * ldd + dc0 + r] = src[(sr0 + r) * lds + sc0 + c] for r < R, c < C   (transpose)
+__global__ void transpose_bf16_kernel(const bf16* __restrict__ src, int64_t lds, bf16* __restrict__ dst,
+                                      int64_t ldd, int R, int C) {
+  __shared__ bf16 tile[32][33];
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < R && c < C) tile[i][threadIdx.x] = src[(int64_t)r * lds + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < R && c < C) dst[(int64_t)c * ldd + r] = tile[threadIdx.x][i];
+  }
+}
+
+// dst[r * ldd + c] = src[r * lds + c]
+__global__ void copy_bf16_kernel(const bf16* __restrict__ src, int64_t lds, bf16* __restrict__ dst, int64_t ldd,
+                                 int R, int C) {
+  const int64_t total = (int64_t)R * C;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int r = (int)(e / C), c = (int)(e - (int64_t)r * C);
+    dst[(int64_t)r * ldd + c] = src[(int64_t)r * lds + c];
+  }
+}
+
+__global__ void zero_bf16_kernel(bf16* __restrict__ dst, int64_t n) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
+    dst[e] = __float2bfloat16_rn(0.f);
+}
+
+__global__ void inv_freq_kernel(double* __restrict__ out, int D, double log2_theta) {
+  const int i = threadIdx.x;
+  if (i < D / 2) out[i] = exp2(-(double)(2 * i) / (double)D * log2_theta);
+}
+
+}  // namespace jenga

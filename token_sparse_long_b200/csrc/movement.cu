@@ -1,0 +1,256 @@
+// Permutation-free token movement: gather of retained rows, in-place residual
+// scatter-add, row scaling.  Jenga notes §4.4 / Jenga summary §4.4.1 (Fig. 9):
+// retained rows are read straight from the original input and results are added
+// back in place, so the sequence is never permuted in global memory.
+//
+// All three are HBM-bound row moves: 128-bit loads/stores, several independent
+// vectors in flight per thread, grid sized to a multiple of the SM count.
+#include "common.cuh"
+
+namespace jenga {
+
+// One vector = 16 bytes.  Row r of the compact output maps to sequence row
+// idx[r / blk] * blk + r % blk.
+template <int UNROLL>
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x, int64_t ldx_v,
+                                                          int64_t bsx_v, uint4* __restrict__ out, int64_t ldo_v,
+                                                          int64_t bso_v, int vpr, int blk, int nb,
+                                                          const int32_t* __restrict__ idx,
+                                                          const int32_t* __restrict__ n_kept, int n_cap) {
+  const int b = blockIdx.y;
+  int nk = n_kept[b];
+  if (nk < 0 || (int64_t)nk * blk > n_cap || nk > nb) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) record_device_error(JENGA_EINTERNAL, SITE_NKEPT_RANGE, nk);
+    return;
+  }
+  const int32_t* ib = idx + (int64_t)b * nb;
+  const int64_t total = (int64_t)nk * blk * vpr;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t e0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e0 < total; e0 += stride * UNROLL) {
+    uint4 v[UNROLL];
+    int64_t dst[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      int64_t e = e0 + (int64_t)u * stride;
+      dst[u] = -1;
+      if (e < total) {
+        int64_t r = e / vpr;
+        int c = (int)(e - r * vpr);
+        int blk_i = (int)(r / blk);
+        int t = (int)(r - (int64_t)blk_i * blk);
+        int src_blk = __ldg(ib + blk_i);
+        if (src_blk < 0 || src_blk >= nb) {
+          record_device_error(JENGA_EINTERNAL, SITE_INDEX_RANGE, (unsigned)src_blk);
+          continue;
+        }
+        v[u] = __ldcs(x + b * bsx_v + ((int64_t)src_blk * blk + t) * ldx_v + c);
+        dst[u] = b * bso_v + r * ldo_v + c;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u)
+      if (dst[u] >= 0) out[dst[u]] = v[u];
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
+  __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
+  return __bfloat1622float2(h);
+}
+
+// x = round(x + alpha * y): one fp32 FMA, then (bf16) one more rounding.
+template <bool BF16>
+__device__ __forceinline__ uint4 axpy_vec(uint4 xv, uint4 yv, float alpha) {
+  uint4 o;
+  if (BF16) {
+    uint32_t* xs = reinterpret_cast<uint32_t*>(&xv);
+    uint32_t* ys = reinterpret_cast<uint32_t*>(&yv);
+    uint32_t* os = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 a = unpack_bf16x2(xs[i]), b = unpack_bf16x2(ys[i]);
+      os[i] = pack_bf16x2(fmaf(alpha, b.x, a.x), fmaf(alpha, b.y, a.y));
+    }
+  } else {
+    o.x = __float_as_uint(fmaf(alpha, __uint_as_float(yv.x), __uint_as_float(xv.x)));
+    o.y = __float_as_uint(fmaf(alpha, __uint_as_float(yv.y), __uint_as_float(xv.y)));
+    o.z = __float_as_uint(fmaf(alpha, __uint_as_float(yv.z), __uint_as_float(xv.z)));
+    o.w = __float_as_uint(fmaf(alpha, __uint_as_float(yv.w), __uint_as_float(xv.w)));
+  }
+  return o;
+}
+
+template <bool BF16, int UNROLL>
+__global__ void __launch_bounds__(256) scatter_add_kernel(uint4* __restrict__ x, int64_t ldx_v, int64_t bsx_v,
+                                                          const uint4* __restrict__ y, int64_t ldy_v,
+                                                          int64_t bsy_v, int vpr, int blk, int nb,
+                                                          const int32_t* __restrict__ idx,
+                                                          const int32_t* __restrict__ n_kept, int n_cap,
+                                                          float alpha) {
+  const int b = blockIdx.y;
+  int nk = n_kept[b];
+  if (nk < 0 || (int64_t)nk * blk > n_cap || nk > nb) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) record_device_error(JENGA_EINTERNAL, SITE_NKEPT_RANGE, nk);
+    return;
+  }
+  const int32_t* ib = idx + (int64_t)b * nb;
+  const int64_t total = (int64_t)nk * blk * vpr;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t e0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e0 < total; e0 += stride * UNROLL) {
+    uint4 xv[UNROLL], yv[UNROLL];
+    int64_t dst[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      int64_t e = e0 + (int64_t)u * stride;
+      dst[u] = -1;
+      if (e < total) {
+        int64_t r = e / vpr;
+        int c = (int)(e - r * vpr);
+        int blk_i = (int)(r / blk);
+        int t = (int)(r - (int64_t)blk_i * blk);
+        int dst_blk = __ldg(ib + blk_i);
+        if (dst_blk < 0 || dst_blk >= nb) {
+          record_device_error(JENGA_EINTERNAL, SITE_INDEX_RANGE, (unsigned)dst_blk);
+          continue;
+        }
+        dst[u] = b * bsx_v + ((int64_t)dst_blk * blk + t) * ldx_v + c;
+        yv[u] = __ldcs(y + b * bsy_v + r * ldy_v + c);
+        xv[u] = x[dst[u]];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u)
+      if (dst[u] >= 0) x[dst[u]] = axpy_vec<BF16>(xv[u], yv[u], alpha);
+  }
+}
+
+template <bool BF16>
+__global__ void scale_rows_kernel(uint4* __restrict__ x, int64_t ldx_v, int64_t bsx_v, int vpr, int S,
+                                  const int32_t* __restrict__ rows, int n_rows, float f) {
+  const int b = blockIdx.y;
+  const int64_t total = (int64_t)n_rows * vpr;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    int i = (int)(e / vpr);
+    int c = (int)(e - (int64_t)i * vpr);
+    int r = rows[(int64_t)b * n_rows + i];
+    if (r < 0 || r >= S) {
+      record_device_error(JENGA_EINTERNAL, SITE_INDEX_RANGE, (unsigned)r);
+      continue;
+    }
+    uint4* p = x + b * bsx_v + (int64_t)r * ldx_v + c;
+    uint4 v = *p;
+    uint4 z = make_uint4(0, 0, 0, 0);
+    *p = axpy_vec<BF16>(z, v, f);
+  }
+}
+
+static int grid_for(int64_t vectors, int unroll) {
+  int64_t want = (vectors + 256LL * unroll - 1) / (256LL * unroll);
+  int cap = sm_count() * 8;  // 8 resident 256-thread CTAs per SM
+  if (want < 1) want = 1;
+  return (int)(want < cap ? want : cap);
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace jenga
+
+using namespace jenga;
+
+extern "C" jenga_status jenga_gather(const void* x, int64_t ldx, int B, int S, int h, int blk, const int32_t* idx,
+                                     const int32_t* n_kept, jenga_dtype dt, void* out, int64_t ldo, int n_cap,
+                                     jenga_stream_t stream) {
+  JENGA_CHECK_ARG(x && idx && n_kept && (out || n_cap == 0), "jenga_gather: null pointer");
+  JENGA_CHECK_ARG(B >= 1 && S >= 1 && h >= 1 && blk >= 1 && S % blk == 0 && n_cap >= 0,
+                  "jenga_gather: bad sizes B=%d S=%d h=%d blk=%d", B, S, h, blk);
+  JENGA_CHECK_ARG(dt == JENGA_F32 || dt == JENGA_BF16, "jenga_gather: dtype");
+  const int es = dt == JENGA_F32 ? 4 : 2;
+  JENGA_CHECK_ARG(ldx >= h && ldo >= h, "jenga_gather: row pitch smaller than h");
+  JENGA_CHECK_ARG((h * es) % 16 == 0 && (ldx * es) % 16 == 0 && (ldo * es) % 16 == 0 && aligned16(x) &&
+                      (n_cap == 0 || aligned16(out)),
+                  "jenga_gather: rows must be 16-byte aligned multiples of 16 bytes");
+  if (n_cap == 0) return JENGA_OK;
+  const int vpr = h * es / 16;
+  const int64_t ldx_v = ldx * es / 16, ldo_v = ldo * es / 16;
+  dim3 grid(grid_for((int64_t)n_cap * vpr, 4), B);
+  {
+  const int _ps = ::jenga::prof_begin("gather_rows", (cudaStream_t)stream);
+  gather_rows_kernel<4><<<grid, 256, 0, (cudaStream_t)stream>>>(
+      (const uint4*)x, ldx_v, (int64_t)S * ldx_v, (uint4*)out, ldo_v, (int64_t)n_cap * ldo_v, vpr, blk, S / blk,
+      idx, n_kept, n_cap);
+  ::jenga::prof_end(_ps, (cudaStream_t)stream);
+  }
+  JENGA_LAUNCH_CHECK();
+  return JENGA_OK;
+}
+
+extern "C" jenga_status jenga_scatter_add(void* x, int64_t ldx, const void* y, int64_t ldy, int B, int S, int h,
+                                          int blk, const int32_t* idx, const int32_t* n_kept, float alpha,
+                                          jenga_dtype dt, int n_cap, jenga_stream_t stream) {
+  JENGA_CHECK_ARG(x && idx && n_kept && (y || n_cap == 0), "jenga_scatter_add: null pointer");
+  JENGA_CHECK_ARG(B >= 1 && S >= 1 && h >= 1 && blk >= 1 && S % blk == 0 && n_cap >= 0,
+                  "jenga_scatter_add: bad sizes B=%d S=%d h=%d blk=%d", B, S, h, blk);
+  JENGA_CHECK_ARG(dt == JENGA_F32 || dt == JENGA_BF16, "jenga_scatter_add: dtype");
+  const int es = dt == JENGA_F32 ? 4 : 2;
+  JENGA_CHECK_ARG(ldx >= h && ldy >= h, "jenga_scatter_add: row pitch smaller than h");
+  JENGA_CHECK_ARG((h * es) % 16 == 0 && (ldx * es) % 16 == 0 && (ldy * es) % 16 == 0 && aligned16(x) &&
+                      (n_cap == 0 || aligned16(y)),
+                  "jenga_scatter_add: rows must be 16-byte aligned multiples of 16 bytes");
+  if (n_cap == 0) return JENGA_OK;
+  const int vpr = h * es / 16;
+  const int64_t ldx_v = ldx * es / 16, ldy_v = ldy * es / 16;
+  dim3 grid(grid_for((int64_t)n_cap * vpr, 4), B);
+  if (dt == JENGA_BF16)
+    {
+    const int _ps = ::jenga::prof_begin("scatter_add", (cudaStream_t)stream);
+    scatter_add_kernel<true, 4><<<grid, 256, 0, (cudaStream_t)stream>>>(
+        (uint4*)x, ldx_v, (int64_t)S * ldx_v, (const uint4*)y, ldy_v, (int64_t)n_cap * ldy_v, vpr, blk, S / blk,
+        idx, n_kept, n_cap, alpha);
+    ::jenga::prof_end(_ps, (cudaStream_t)stream);
+    }
+  else
+    {
+    const int _ps = ::jenga::prof_begin("scatter_add", (cudaStream_t)stream);
+    scatter_add_kernel<false, 4><<<grid, 256, 0, (cudaStream_t)stream>>>(
+        (uint4*)x, ldx_v, (int64_t)S * ldx_v, (const uint4*)y, ldy_v, (int64_t)n_cap * ldy_v, vpr, blk, S / blk,
+        idx, n_kept, n_cap, alpha);
+    ::jenga::prof_end(_ps, (cudaStream_t)stream);
+    }
+  JENGA_LAUNCH_CHECK();
+  return JENGA_OK;
+}
+
+extern "C" jenga_status jenga_scale_rows(void* x, int64_t ldx, int B, int S, int h, const int32_t* rows,
+                                         int n_rows, float factor, jenga_dtype dt, jenga_stream_t stream) {
+  JENGA_CHECK_ARG(x && (rows || n_rows == 0), "jenga_scale_rows: null pointer");
+  JENGA_CHECK_ARG(B >= 1 && S >= 1 && h >= 1 && n_rows >= 0 && ldx >= h, "jenga_scale_rows: bad sizes");
+  const int es = dt == JENGA_F32 ? 4 : 2;
+  JENGA_CHECK_ARG((h * es) % 16 == 0 && (ldx * es) % 16 == 0 && aligned16(x),
+                  "jenga_scale_rows: rows must be 16-byte aligned multiples of 16 bytes");
+  if (n_rows == 0) return JENGA_OK;
+  const int vpr = h * es / 16;
+  const int64_t ldx_v = ldx * es / 16;
+  dim3 grid(grid_for((int64_t)n_rows * vpr, 1), B);
+  if (dt == JENGA_BF16)
+    {
+    const int _ps = ::jenga::prof_begin("scale_rows", (cudaStream_t)stream);
+    scale_rows_kernel<true><<<grid, 256, 0, (cudaStream_t)stream>>>((uint4*)x, ldx_v, (int64_t)S * ldx_v, vpr, S,
+                                                                     rows, n_rows, factor);
+    ::jenga::prof_end(_ps, (cudaStream_t)stream);
+    }
+  else
+    {
+    const int _ps = ::jenga::prof_begin("scale_rows", (cudaStream_t)stream);
+    scale_rows_kernel<false><<<grid, 256, 0, (cudaStream_t)stream>>>((uint4*)x, ldx_v, (int64_t)S * ldx_v, vpr,
+                                                                      S, rows, n_rows, factor);
+    ::jenga::prof_end(_ps, (cudaStream_t)stream);
+    }
+  JENGA_LAUNCH_CHECK();
+  return JENGA_OK;
+}
