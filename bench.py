@@ -1,0 +1,477 @@
+#!/usr/bin/env python3
+"""Token-sparse layer benchmark: fwd+bwd tokens/s at S=32K.
+
+Workload (default ``llama7b_x4_s32k``): four stacked Llama-2-7B-shaped layers (hidden
+4096, 32 heads x 128, SwiGLU FFN 11008), bf16 storage / fp32 accumulation, S=32768,
+batch 1, token blocks of 128, per-layer top-k keep fractions 80/60/50/40 %, 4% salient
+rows x3 redrawn per layer, LoRA rank 16 on q/v, segment-wise backward over 4096
+retained tokens.  One step = for each layer: q/k projection of all S tokens, two-pass
+block scoring, top-k selection, retained-token forward (in place); then the backward
+of the four layers in reverse (upstream gradient G, loss = sum(out * G)).
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle instead on a
+bounded sample of the same workload.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "token-sparse layer fwd+bwd tokens/s at S=32K; score/select/gather % roofline"
+REF_TOKENS = 1024        # oracle sample per reference-arm step
+BASELINE_TOKENS = 2048   # oracle sample of the cpu_baseline leg
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="jenga", choices=["jenga", "reference"])
+    ap.add_argument("--workload", default="llama7b_x4_s32k")
+    ap.add_argument("--no-dense", action="store_true", help="skip the keep-all comparison")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained", p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------------------- work model
+def causal_pairs(n):
+    return n * (n + 1) / 2.0
+
+
+def work_model(case, ks, seg):
+    """Algorithmic work per step for each kernel name: (kind, amount) with kind
+    'flop' or 'byte'.  GEMM: 2 M N K.  Attention fwd: 2 matmuls per causal pair
+    (4 D H pairs); backward: 5 matmul-equivalents per pair (10 D H pairs), shared
+    3 : 4 between the dQ and dK/dV kernels in proportion to the matmuls each runs.
+    Scoring: one QK^T product per causal pair per pass (2 D H pairs)."""
+    sh = case.shape
+    S, h, H, D, F = case.S, sh.hidden, sh.heads, sh.head_dim, sh.ffn
+    HD = H * D
+    w = {}
+
+    def add(name, kind, v):
+        k0, v0 = w.get(name, (kind, 0.0))
+        w[name] = (kind, v0 + v)
+
+    for k in ks:
+        n = k * case.blk
+        add("gemm_lora_t_all", "flop", 2.0 * S * 32 * h)
+        add("gemm_qk_rope_all", "flop", 2.0 * S * 2 * HD * h)
+        add("score_lse_bf16", "flop", 2.0 * D * H * causal_pairs(S))
+        add("score_mass_bf16", "flop", 2.0 * D * H * causal_pairs(S))
+        add("gemm_lora_t", "flop", 2.0 * n * 32 * h)
+        add("gemm_qkv_rope", "flop", 2.0 * n * 3 * HD * h)
+        add("attn_fwd", "flop", 4.0 * D * H * causal_pairs(n))
+        add("gemm_o_scatter", "flop", 2.0 * n * h * HD)
+        add("gemm_gateup_swiglu", "flop", 2.0 * n * 2 * F * h)
+        add("gemm_down_scatter", "flop", 2.0 * n * h * F)
+        add("gemm_gateup_recompute", "flop", 2.0 * n * 2 * F * h)
+        add("gemm_da_swiglu_bwd", "flop", 2.0 * n * F * h)
+        add("gemm_dhn", "flop", 2.0 * n * h * 2 * F)
+        add("gemm_do", "flop", 2.0 * n * HD * h)
+        add("attn_bwd_dq", "flop", 10.0 * D * H * causal_pairs(n) * 3 / 7)
+        add("attn_bwd_dkdv", "flop", 10.0 * D * H * causal_pairs(n) * 4 / 7)
+        add("gemm_dt", "flop", 2.0 * n * 32 * 3 * HD)
+        add("gemm_dxn", "flop", 2.0 * n * h * 3 * HD)
+        add("rmsnorm_rows", "byte", 2.0 * (S * h * 2) + 3.0 * n * h * 2 * 2)
+        add("select_small", "byte", 9.0 * (S // case.blk))
+    return w
+
+
+def step_flops(case, ks):
+    return sum(v for k, v in work_model(case, ks, 4096).values() if k == "flop")
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+                for nm, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(nm)
+            except Exception:
+                pass
+        if not sm:
+            return None
+        busy = [s for s in sm if s > 0.5 * (mx or 1)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- oracle timing
+def oracle_sample(case, n_tok=256, layer=0):
+    """Time the CPU oracle on a bounded sample of the workload: the first n_tok tokens'
+    blocks of one layer run through the oracle's scoring (those tokens' q/k), selection,
+    and retained-token forward+backward.  Returns (seconds, algorithmic flops)."""
+    from oracle import layer as oly
+    from oracle import scores as osc
+    from oracle import select as osel
+    from oracle.bf16 import from_bits
+    W = oly.Weights.from_bits(case.layers[layer], case.shape)
+    X = from_bits(case.x[:n_tok])
+    G = from_bits(case.g[:n_tok])
+    sh = case.shape
+    blk = min(case.blk, n_tok)
+    t0 = time.perf_counter()
+    # a1-a3: q/k of the sample (keep-all forward gives q, k), then block scores
+    idx_all = np.arange(n_tok // blk, dtype=np.int32)
+    _, ctx0 = oly.sparse_layer_fwd(X, idx_all, n_tok // blk, blk, W, rnd=True)
+    sc = osc.block_scores_softmax_mass(ctx0["q"], ctx0["k"], blk)
+    idx, n, _ = osel.select_topk(sc, max(1, osel.topk_count(0.5, n_tok // blk)))
+    Xo, ctx = oly.sparse_layer_fwd(X, idx, n, blk, W, rnd=True)
+    oly.sparse_layer_bwd(ctx, G, W, 4096)
+    dt = time.perf_counter() - t0
+    HD = sh.heads * sh.head_dim
+    P = 4 * sh.hidden * HD + 3 * sh.hidden * sh.ffn
+    nr = n * blk
+    flops = (2.0 * P * n_tok + 4.0 * sh.head_dim * sh.heads * causal_pairs(n_tok)      # keep-all fwd for q/k
+             + 4.0 * sh.head_dim * sh.heads * causal_pairs(n_tok)                    # scoring (2 passes)
+             + 4.0 * P * nr + 14.0 * sh.head_dim * sh.heads * causal_pairs(nr))      # sparse fwd + bwd
+    return dt, flops
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        return max(int(i.get("num_threads", 1)) for i in threadpool_info()) or os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    case = synth.gen_workload(args.workload, seed=0, n_layers=1)
+    keep = list(w.keep) if len(w.keep) == w.n_layers else [w.keep[0]] * w.n_layers
+    ks = [synth_k(p, w.S // w.blk) for p in keep]
+    full = full_step_flops(w, ks)
+    for _ in range(args.warmup):
+        oracle_sample(case, REF_TOKENS)
+    ts, fs = [], []
+    for _ in range(args.steps):
+        dt, fl = oracle_sample(case, REF_TOKENS)
+        ts.append(dt)
+        fs.append(fl)
+    rate = sum(fs) / sum(ts)
+    value = w.S / (full / rate)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * full / rate,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "seq_len": w.S, "global_batch": 1, "layers": w.n_layers},
+            "cpu_baseline": {"kind": "oracle", "value": value, "unit": "tokens/s", "cores": cpu_cores(),
+                             "sample": f"per step: oracle scoring + top-50% selection + retained-token fwd+bwd of "
+                                       f"one layer on the first {REF_TOKENS} tokens; tokens/s = S / (full-step "
+                                       f"algorithmic flops / the oracle's measured flop rate)"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def synth_k(p, nb):
+    from math import ceil
+    return max(0, min(nb, ceil(p * nb - 1e-6)))
+
+
+def full_step_flops(w, ks):
+    class C:
+        pass
+    c = C()
+    c.shape, c.S, c.blk = w.shape, w.S, w.blk
+    return step_flops(c, ks)
+
+
+# ---------------------------------------------------------------------------- GPU arm
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=torch.device("cuda", local))
+
+    import token_sparse_long_b200 as J
+
+    def bits_to_torch(u16, device):
+        return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(torch.bfloat16).to(device)
+
+    def layer_handle(p, shape):
+        t = {k: bits_to_torch(getattr(p, k), dev) for k in ("wq", "wk", "wv", "wo", "wg", "wu", "wd", "attn_norm",
+                                                             "mlp_norm", "aq", "bq", "av", "bv")}
+        return J.LayerHandle(**t, heads=shape.heads, head_dim=shape.head_dim, rms_eps=shape.rms_eps,
+                             rope_theta=shape.rope_theta, lora_scale=shape.lora_scale)
+
+    J._lib.load()
+    w = synth.WORKLOADS[args.workload]
+    case = synth.gen_workload(args.workload, seed=0)
+    sh = case.shape
+    S, blk, nb, HD = case.S, case.blk, case.S // case.blk, sh.heads * sh.head_dim
+    keep = list(w.keep) if len(w.keep) == w.n_layers else [w.keep[0]] * w.n_layers
+    ks = [synth_k(p, nb) for p in keep]
+    dev = torch.device("cuda", local)
+
+    layers = [layer_handle(p, sh) for p in case.layers]
+    X0 = bits_to_torch(case.x, dev)
+    G0 = bits_to_torch(case.g, dev)
+    sal = [torch.from_numpy(s.astype(np.int32)).to(dev) for s in case.salient]
+    X = torch.empty_like(X0)
+    dX = torch.empty_like(G0)
+    seg = case.segment_tokens
+
+    def buffers(kmaxes):
+        b = {}
+        b["qk"] = torch.empty(S, 2 * HD, dtype=torch.bfloat16, device=dev)
+        b["qk_ws"] = torch.empty(layers[0].qk_ws_bytes(S), dtype=torch.uint8, device=dev)
+        lib = J._lib.load()
+        b["sc_ws"] = torch.empty(lib.jenga_score_workspace_bytes(1, S, sh.heads, sh.head_dim, blk),
+                                 dtype=torch.uint8, device=dev)
+        b["scores"] = [torch.empty(1, nb, dtype=torch.float32, device=dev) for _ in kmaxes]
+        b["sel"] = [(torch.empty(1, nb, dtype=torch.int32, device=dev), torch.empty(1, dtype=torch.int32, device=dev),
+                     torch.empty(1, nb, dtype=torch.uint8, device=dev)) for _ in kmaxes]
+        b["saved"] = [torch.empty(L.saved_bytes(blk, k), dtype=torch.uint8, device=dev) for L, k in zip(layers, kmaxes)]
+        b["fws"] = torch.empty(max(L.fwd_ws_bytes(blk, k) for L, k in zip(layers, kmaxes)), dtype=torch.uint8,
+                               device=dev)
+        b["bws"] = torch.empty(max(L.bwd_ws_bytes(blk, k, seg) for L, k in zip(layers, kmaxes)), dtype=torch.uint8,
+                               device=dev)
+        b["grads"] = [J.new_lora_grads(L) for L in layers]
+        return b
+
+    def step(b, kmaxes, sparse=True):
+        for l, L in enumerate(layers):
+            if l > 0 and len(case.salient[l]):
+                J.jenga_scale_rows(X, sal[l], case.salient_scale)
+            idx, nk, mask = b["sel"][l]
+            if sparse:
+                J.jenga_layer_score_qk(L, X, out=b["qk"], ws=b["qk_ws"])
+                J.jenga_score_blocks(b["qk"][:, :HD], b["qk"][:, HD:], sh.heads, sh.head_dim, blk, out=b["scores"][l],
+                                     ws=b["sc_ws"])
+                J.jenga_select(b["scores"][l], "topk_frac", keep[l], out=(idx, nk, mask))
+            J.jenga_sparse_layer_fwd(L, X, idx, nk, blk, kmaxes[l], saved=b["saved"][l], ws=b["fws"])
+        for l in reversed(range(len(layers))):
+            idx, nk, _ = b["sel"][l]
+            J.jenga_sparse_layer_bwd(layers[l], dX, idx, nk, blk, kmaxes[l], b["saved"][l], b["grads"][l],
+                                     segment_tokens=seg, ws=b["bws"])
+            if l > 0 and len(case.salient[l]):
+                J.jenga_scale_rows(dX, sal[l], case.salient_scale)
+
+    def zero_grads(b):
+        for g in b["grads"]:
+            for t in g.values():
+                t.zero_()
+
+    def device_step(b, kmaxes, sparse=True):
+        X.copy_(X0)
+        dX.copy_(G0)
+        zero_grads(b)
+        step(b, kmaxes, sparse)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def timed(fn, K, Wu):
+        for _ in range(Wu):
+            fn()
+        torch.cuda.synchronize()
+        barrier()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(K):
+            fn()
+        e.record()
+        torch.cuda.synchronize()
+        barrier()
+        ms = s.elapsed_time(e) / K
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    # ---------------- sparse step (headline)
+    torch.cuda.reset_peak_memory_stats(dev)
+    b = buffers(ks)
+    J.jenga_check_device_status()
+    for _ in range(args.warmup):
+        device_step(b, ks)
+    torch.cuda.synchronize()
+    J.jenga_check_device_status()
+    clocks = ClockSampler(local)
+    clocks.start()
+    J.jenga_profile_enable(True)
+    ms = timed(lambda: device_step(b, ks), args.steps, 0)
+    prof = J.jenga_profile_report()
+    J.jenga_profile_enable(False)
+    clk = clocks.stop()
+    J.jenga_check_device_status()
+    peak_sparse = torch.cuda.max_memory_allocated(dev) / 2 ** 30
+    n_kept = [int(b["sel"][l][1].item()) for l in range(len(layers))]
+
+    # ---------------- roofline of the dominant kernel (live per-launch events, timed region)
+    hbm, tf_burst, tf_sus, peak_src = load_peaks()
+    wm = work_model(case, ks, seg)
+    top = max(prof.items(), key=lambda kv: kv[1]["ms"])
+    tname, tstat = top
+    launches = sum(v["launches"] for v in prof.values())
+    roof = None
+    if tname in wm:
+        kind, amount = wm[tname]
+        sec = tstat["ms"] / 1e3 / args.steps
+        if kind == "flop":
+            ach = amount / sec / 1e12
+            roof = {"kernel": tname, "bound": "tensor", "achieved": ach, "peak": tf_sus, "unit": "TFLOP/s",
+                    "frac": ach / tf_sus, "traffic": None, "peak_source": f"{peak_src} bf16 sustained",
+                    "launches_per_step": tstat["launches"] / args.steps, "share": tstat["ms"] / sum(
+                        v["ms"] for v in prof.values())}
+        else:
+            ach = amount / sec / 1e9
+            roof = {"kernel": tname, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
+                    "frac": ach / hbm, "traffic": None, "peak_source": f"{peak_src} HBM copy"}
+    kernels = {}
+    for k, v in sorted(prof.items(), key=lambda kv: -kv[1]["ms"]):
+        e = {"ms_per_step": v["ms"] / args.steps, "launches_per_step": v["launches"] / args.steps}
+        if k in wm:
+            kind, amount = wm[k]
+            sec = v["ms"] / 1e3 / args.steps
+            if kind == "flop":
+                e["tflops"] = amount / sec / 1e12
+                e["frac_bf16_sustained"] = e["tflops"] / tf_sus
+            else:
+                e["gbs"] = amount / sec / 1e9
+        kernels[k] = e
+
+    # ---------------- dense comparison (keep-all, no scoring)
+    dense = None
+    if not args.no_dense:
+        del b
+        torch.cuda.empty_cache()
+        torch.cuda.reset_peak_memory_stats(dev)
+        kd = [nb] * len(layers)
+        bd = buffers(kd)
+        for l in range(len(layers)):
+            idx, nk, _ = bd["sel"][l]
+            idx.copy_(torch.arange(nb, dtype=torch.int32, device=dev)[None])
+            nk.fill_(nb)
+        ms_d = timed(lambda: device_step(bd, kd, sparse=False), max(1, min(2, args.steps)), 1)
+        dense = {"tokens_per_s": S * world / (ms_d / 1e3), "ms_per_step": ms_d,
+                 "peak_mem_gib": torch.cuda.max_memory_allocated(dev) / 2 ** 30,
+                 "note": "keep-all retained-token layers without scoring (same kernels)"}
+        del bd
+        torch.cuda.empty_cache()
+
+    # ---------------- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        b = buffers(ks)
+        hX = torch.empty(X0.shape, dtype=X0.dtype, pin_memory=True)
+        hX.copy_(X0.cpu())
+        hG = torch.empty(G0.shape, dtype=G0.dtype, pin_memory=True)
+        hG.copy_(G0.cpu())
+        hgrads = [{k: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for k, t in g.items()} for g in b["grads"]]
+
+        def e2e_step():
+            X.copy_(hX, non_blocking=True)
+            dX.copy_(hG, non_blocking=True)
+            zero_grads(b)
+            step(b, ks)
+            for hg, g in zip(hgrads, b["grads"]):
+                for k in g:
+                    hg[k].copy_(g[k], non_blocking=True)
+
+        ms_e = timed(e2e_step, args.steps, 1)
+        h2d = hX.numel() * 2 + hG.numel() * 2
+        d2h = sum(t.numel() * 4 for g in hgrads for t in g.values())
+        e2e = {"value": S * world / (ms_e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ms_e}
+        del b
+
+    # ---------------- CPU baseline (oracle, rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, fl = oracle_sample(case, BASELINE_TOKENS)
+        rate = fl / dt
+        full = step_flops(case, ks)
+        cpu = {"value": S / (full / rate), "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": f"oracle scoring + top-50% selection + retained-token fwd+bwd of layer 0 on the first "
+                         f"{BASELINE_TOKENS} tokens ({dt:.1f} s, {fl / 1e9:.0f} GFLOP); scaled by the full step's "
+                         f"algorithmic flops ({full / 1e12:.1f} TFLOP)"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": S * world / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": args.workload, "seq_len": S, "global_batch": world, "layers": len(layers),
+                           "hidden": sh.hidden, "heads": sh.heads, "ffn": sh.ffn, "block": blk, "keep": keep,
+                           "n_kept_blocks": n_kept, "segment_tokens": seg, "parallelism": f"replicas{world}",
+                           "l2": "inputs larger than L2 (X 256 MiB, weights 1.6 GiB)"},
+                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+                "clocks": clk, "peak_mem_gib": peak_sparse, "dense": dense,
+                "step_tflop": step_flops(case, ks) / 1e12, "kernels": kernels}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

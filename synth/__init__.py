@@ -38,14 +38,16 @@ import numpy as np
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """Round fp32 values to bf16 (round-to-nearest-even); return the uint16 bit patterns."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    r = ((u + 0x7FFF + lsb) >> 16) & 0xFFFF
-    # keep NaN a NaN
-    nan = np.isnan(a)
+    u = a.view(np.uint32)
+    r = (u >> 16) & np.uint32(1)
+    r += np.uint32(0x7FFF)
+    r += u                      # finite values cannot overflow 32 bits here
+    r >>= 16
+    out = r.astype(np.uint16)
+    nan = np.isnan(a)           # keep NaN a NaN
     if nan.any():
-        r = np.where(nan, 0x7FC0, r)
-    return r.astype(np.uint16)
+        out[nan] = 0x7FC0
+    return out
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:

@@ -58,6 +58,19 @@ def jenga_version():
     return load().jenga_version().decode()
 
 
+def jenga_profile_enable(on=True):
+    check(load().jenga_profile_enable(1 if on else 0))
+
+
+def jenga_profile_report():
+    """Per-kernel launch counts and milliseconds recorded since jenga_profile_enable."""
+    import json
+    lib = load()
+    buf = ctypes.create_string_buffer(1 << 16)
+    lib.jenga_profile_report(buf, 1 << 16)
+    return json.loads(buf.value.decode())
+
+
 # ------------------------------------------------------------------ scoring / selection / movement
 def jenga_score_blocks(q, k, heads, head_dim, blk, causal=True, mode="softmax_mass", out=None, ws=None,
                        stream=None):
@@ -80,18 +93,23 @@ def jenga_score_blocks(q, k, heads, head_dim, blk, causal=True, mode="softmax_ma
     return out if q.dim() == 3 else out[0]
 
 
-def jenga_select(scores, mode, param=0.0, stream=None):
-    """scores [B, nb] fp32 -> (idx int32 [B, nb], n_kept int32 [B], mask uint8 [B, nb])."""
+def jenga_select(scores, mode, param=0.0, out=None, ws=None, stream=None):
+    """scores [B, nb] fp32 -> (idx int32 [B, nb], n_kept int32 [B], mask uint8 [B, nb]).
+    out: optional preallocated (idx, n_kept, mask)."""
     _need_cuda(scores)
     s2 = scores if scores.dim() == 2 else scores.unsqueeze(0)
     s2 = s2.contiguous()
     B, nb = s2.shape
     lib = load()
-    idx = torch.empty(B, nb, dtype=torch.int32, device=scores.device)
-    nk = torch.empty(B, dtype=torch.int32, device=scores.device)
-    mask = torch.empty(B, nb, dtype=torch.uint8, device=scores.device)
+    if out is not None:
+        idx, nk, mask = out
+    else:
+        idx = torch.empty(B, nb, dtype=torch.int32, device=scores.device)
+        nk = torch.empty(B, dtype=torch.int32, device=scores.device)
+        mask = torch.empty(B, nb, dtype=torch.uint8, device=scores.device)
     need = lib.jenga_select_workspace_bytes(B, nb)
-    ws = _ws(need, scores.device)
+    if ws is None or ws.numel() < need:
+        ws = _ws(need, scores.device)
     check(lib.jenga_select(_p(s2), B, nb, SELECT_MODES[mode], float(param), _p(idx), _p(nk), _p(mask), _p(ws),
                            ws.numel(), _stream(stream)))
     if scores.dim() == 1:

@@ -235,10 +235,12 @@ extern "C" jenga_status jenga_layer_pack(const jenga_layer_weights* w, const jen
   JENGA_TRY(copy2d((const bf16*)lora->aq, h, p.aqv, h, LORA_R, h, st));
   JENGA_TRY(copy2d((const bf16*)lora->av, h, p.aqv + (size_t)LORA_R * h, h, LORA_R, h, st));
   // gate/up interleaved in groups of 64 rows: [g 0..63, u 0..63, g 64..127, u 64..127, ...]
-  for (int grp = 0; grp < F / 64; ++grp) {
-    JENGA_TRY(copy2d(wg + (size_t)grp * 64 * h, h, p.wgu + (size_t)grp * 128 * h, h, 64, h, st));
-    JENGA_TRY(copy2d(wu + (size_t)grp * 64 * h, h, p.wgu + (size_t)(grp * 128 + 64) * h, h, 64, h, st));
+  {
+    const int _ps = ::jenga::prof_begin("interleave_gate_up", st);
+    interleave_gate_up_kernel<<<grid_cap((int64_t)2 * F * h, 256), 256, 0, st>>>(wg, wu, p.wgu, F, h);
+    ::jenga::prof_end(_ps, st);
   }
+  JENGA_LAUNCH_CHECK();
   // transposes for the backward
   JENGA_TRY(transpose((const bf16*)w->wo, HD, p.woT, h, h, HD, st));          // Wo [h, HD] -> [HD, h]
   JENGA_TRY(transpose((const bf16*)w->wd, F, p.wdT, h, h, F, st));            // Wd [h, F]  -> [F, h]

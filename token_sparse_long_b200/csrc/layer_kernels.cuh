@@ -292,6 +292,18 @@ __global__ void copy_bf16_kernel(const bf16* __restrict__ src, int64_t lds, bf16
   }
 }
 
+// wgu row r: group g = r / 128; rows 0..63 of a group are gate rows 64g.., 64..127 up rows 64g..
+__global__ void interleave_gate_up_kernel(const bf16* __restrict__ wg, const bf16* __restrict__ wu,
+                                          bf16* __restrict__ wgu, int F, int h) {
+  const int64_t total = (int64_t)2 * F * h;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / h, c = e - r * h;
+    const int g = (int)(r >> 7), j = (int)(r & 127);
+    const bf16* src = (j < 64) ? wg + ((int64_t)g * 64 + j) * h : wu + ((int64_t)g * 64 + j - 64) * h;
+    wgu[e] = src[c];
+  }
+}
+
 __global__ void zero_bf16_kernel(bf16* __restrict__ dst, int64_t n) {
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
     dst[e] = __float2bfloat16_rn(0.f);
