@@ -31,7 +31,7 @@ enum GemmEpi : int {
   EPI_SCATTER_ADD = 2,  // x[row(m), n] = bf16(x + acc); aux[m, n] = same value (optional)
   EPI_SWIGLU = 3,       // 64-col groups (gate, up) -> out[m, n/2 + j] = bf16(silu(g) * u)
   EPI_QKV_ROPE = 4,     // q/k/v sections of width hd; RoPE(pos(m)) on q and k -> bf16
-  EPI_SWIGLU_BWD = 5,   // acc = dA; aux = (g, u) interleaved bf16 -> out = (dg, du) interleaved bf16
+  EPI_SWIGLU_BWD = 5,   // acc = dA; aux = (g, u) interleaved fp32 -> out = (dg, du) interleaved bf16
   EPI_LORA_T = 6,       // out fp32 [m, 0:N] = beta * acc ; aux bf16 [m, 0:64] = bf16(alpha * acc), zero padded
 };
 
@@ -260,10 +260,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const int j = n0 + c * 32;
           if (!row_ok || j >= N) continue;
           const int64_t col = (int64_t)(j >> 6) * 128 + (j & 63);
-          const bf16* gu = reinterpret_cast<const bf16*>(ep.aux) + (int64_t)m * ep.ld_aux + col;
+          const float* gu = reinterpret_cast<const float*>(ep.aux) + (int64_t)m * ep.ld_aux + col;
           float gv[32], uv[32], dg[32];
-          load_bf16x32(gu, gv);
-          load_bf16x32(gu + 64, uv);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 a = reinterpret_cast<const float4*>(gu)[q];
+            const float4 b = reinterpret_cast<const float4*>(gu + 64)[q];
+            gv[4 * q] = a.x; gv[4 * q + 1] = a.y; gv[4 * q + 2] = a.z; gv[4 * q + 3] = a.w;
+            uv[4 * q] = b.x; uv[4 * q + 1] = b.y; uv[4 * q + 2] = b.z; uv[4 * q + 3] = b.w;
+          }
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float sg = 1.f / (1.f + __expf(-gv[i]));

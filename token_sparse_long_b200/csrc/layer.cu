@@ -103,14 +103,14 @@ static size_t carve_fwd_ws(Carve& c, const Dims& d, int nc, FwdWs* w) {
 
 struct BwdWs {
   float *dk_acc, *dv_acc;
-  bf16 *xn, *gu, *g, *dgu, *dhb, *dO, *dqkv, *dtb;
-  float *dhn, *dh, *delta, *dq, *dt, *part;
+  bf16 *xn, *g, *dgu, *dhb, *dO, *dqkv, *dtb;
+  float *gu, *dhn, *dh, *delta, *dq, *dt, *part;
 };
 static size_t carve_bwd_ws(Carve& c, const Dims& d, int nc, int T, BwdWs* w) {
   w->dk_acc = c.take<float>((size_t)nc * d.HD);
   w->dv_acc = c.take<float>((size_t)nc * d.HD);
   w->xn = c.take<bf16>((size_t)T * d.h);
-  w->gu = c.take<bf16>((size_t)T * 2 * d.F);
+  w->gu = c.take<float>((size_t)T * 2 * d.F);
   w->g = c.take<bf16>((size_t)T * d.h);
   w->dgu = c.take<bf16>((size_t)T * 2 * d.F);
   w->dhb = c.take<bf16>((size_t)T * d.h);
@@ -478,7 +478,7 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
       EpiParams e = epi_base(idx, blk, n_kept, s0);
       e.out = b.gu;
       e.ldo = 2 * F;
-      JENGA_TRY((launch_gemm<256, EPI_STORE_BF16>({b.xn, T, h}, {p.wgu, 2 * F, h}, h, nullptr, nullptr, 0, T, 2 * F, e, st, "gemm_gateup_recompute")));
+      JENGA_TRY((launch_gemm<256, EPI_STORE_F32>({b.xn, T, h}, {p.wgu, 2 * F, h}, h, nullptr, nullptr, 0, T, 2 * F, e, st, "gemm_gateup_recompute")));
     }
     // upstream gradient rows of this segment
     {
