@@ -118,6 +118,25 @@ JENGA_API jenga_status jenga_score_blocks(const void* q, int64_t ldq, const void
                                 int D, int blk, int causal, jenga_dtype dt, jenga_score_mode mode,
                                 float* scores, void* ws, size_t ws_bytes, jenga_stream_t stream);
 
+/* jenga_score_blocks_noalloc -- jenga_score_blocks without a workspace argument.
+ * (The paper has no counterpart: this is an interface convenience.)  For callers that
+ * cannot hand the library device scratch memory -- hosts that own all device memory and
+ * allow no allocation outside their own pool, or latency-critical code that cannot
+ * afford cudaMalloc / cudaFree and the device synchronisation they may cause.  The
+ * scratch is one fixed 16 MiB array inside the library image (every GPU that loads the
+ * library holds it until the process exits), so B * H * S must stay below about 2M
+ * (two fp32 values per (batch, head, token)); larger sizes return JENGA_EWORKSPACE.
+ * Arguments and results are those of jenga_score_blocks.  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress, that device current):
+ * make that first call before any stream capture.  All calls share the array and each
+ * call overwrites what it reads, so nothing needs clearing, but calls whose kernels
+ * overlap on the GPU (for example on two streams) race on it.  Allocates nothing.
+ * jenga_score_blocks_noalloc_max_bytes() returns the array size in bytes. */
+JENGA_API size_t jenga_score_blocks_noalloc_max_bytes(void);
+JENGA_API jenga_status jenga_score_blocks_noalloc(const void* q, int64_t ldq, const void* k, int64_t ldk, int B,
+                                                  int S, int H, int D, int blk, int causal, jenga_dtype dt,
+                                                  jenga_score_mode mode, float* scores, jenga_stream_t stream);
+
 /* ------------------------------------------------------------------ selection
  * jenga_select -- threshold / top-k selection and compaction (a4).
  *   scores : [B, nb] fp32 (NaN compares as -inf).

@@ -54,6 +54,9 @@ _SIGS = {
     "jenga_score_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int, c_int]),
     "jenga_score_blocks": (c_int, [c_void_p, c_int64, c_void_p, c_int64, c_int, c_int, c_int, c_int, c_int, c_int,
                                    c_int, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "jenga_score_blocks_noalloc_max_bytes": (c_size_t, []),
+    "jenga_score_blocks_noalloc": (c_int, [c_void_p, c_int64, c_void_p, c_int64, c_int, c_int, c_int, c_int, c_int,
+                                           c_int, c_int, c_int, c_void_p, c_void_p]),
     "jenga_select_workspace_bytes": (c_size_t, [c_int, c_int]),
     "jenga_select": (c_int, [c_void_p, c_int, c_int, c_int, c_float, c_void_p, c_void_p, c_void_p, c_void_p,
                              c_size_t, c_void_p]),

@@ -8,3 +8,4 @@
 #include "attention.cu"
 #include "layer.cu"
 #include "predictor.cu"
+#include "score_noalloc.cu"
