@@ -79,8 +79,8 @@ def work_model(case, ks, seg):
         n = k * case.blk
         add("gemm_lora_t_all", "flop", 2.0 * S * 32 * h)
         add("gemm_qk_rope_all", "flop", 2.0 * S * 2 * HD * h)
-        add("score_lse_bf16", "flop", 2.0 * D * H * causal_pairs(S))
-        add("score_mass_bf16", "flop", 2.0 * D * H * causal_pairs(S))
+        add("score_lse_tc", "flop", 2.0 * D * H * causal_pairs(S))
+        add("score_mass_tc", "flop", 2.0 * D * H * causal_pairs(S))
         add("gemm_lora_t", "flop", 2.0 * n * 32 * h)
         add("gemm_qkv_rope", "flop", 2.0 * n * 3 * HD * h)
         add("attn_fwd", "flop", 4.0 * D * H * causal_pairs(n))

@@ -117,8 +117,9 @@ struct GemmSmem {
 template <int BN, int EPI>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
-                   const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, int nkb1,
-                   int nkb2, int N, EpiParams ep) {
+                   const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+                   const __grid_constant__ CUtensorMap tmA3, const __grid_constant__ CUtensorMap tmB3, int nkb1,
+                   int nkb2, int nkb3, int N, EpiParams ep) {
   using L = GemmSmem<BN>;
   constexpr int STAGES = L::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const int m0 = blockIdx.y * GEMM_BM;
   const int valid = epi_valid_rows(ep);
   if (m0 >= valid) return;  // whole tile past the valid rows (uniform per CTA)
-  const int nkb = nkb1 + nkb2;
+  const int nkb = nkb1 + nkb2 + nkb3;
 
   if (EPI == EPI_QKV_ROPE) {
     if (threadIdx.x < 64) s_inv_freq[threadIdx.x] = ep.inv_freq[threadIdx.x];
@@ -169,9 +170,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       if (kb < nkb1) {
         tma_load_2d(sa, &tmA1, &full[s], kb * GEMM_BK, m0);
         tma_load_2d(sb, &tmB1, &full[s], kb * GEMM_BK, n0);
-      } else {
+      } else if (kb < nkb1 + nkb2) {
         tma_load_2d(sa, &tmA2, &full[s], (kb - nkb1) * GEMM_BK, m0);
         tma_load_2d(sb, &tmB2, &full[s], (kb - nkb1) * GEMM_BK, n0);
+      } else {
+        tma_load_2d(sa, &tmA3, &full[s], (kb - nkb1 - nkb2) * GEMM_BK, m0);
+        tma_load_2d(sb, &tmB3, &full[s], (kb - nkb1 - nkb2) * GEMM_BK, n0);
       }
     }
   } else if (warp == 1 && lane == 0) {
@@ -348,7 +352,8 @@ struct GemmOperand {
 template <int BN, int EPI>
 jenga_status launch_gemm(const GemmOperand& A1, const GemmOperand& B1, int K1, const GemmOperand* A2,
                          const GemmOperand* B2, int K2, int M, int N, const EpiParams& ep, cudaStream_t st,
-                         const char* name = "gemm") {
+                         const char* name = "gemm", const GemmOperand* A3 = nullptr,
+                         const GemmOperand* B3 = nullptr, int K3 = 0) {
   using L = GemmSmem<BN>;
   if (M <= 0 || N <= 0) return JENGA_OK;
   if (K1 % GEMM_BK || K2 % GEMM_BK || K1 <= 0) return fail(JENGA_EINVAL, "gemm: K must be a multiple of 64");
@@ -363,14 +368,20 @@ jenga_status launch_gemm(const GemmOperand& A1, const GemmOperand& B1, int K1, c
     ta2 = ta1;
     tb2 = tb1;
   }
+  CUtensorMap ta3 = ta1, tb3 = tb1;
+  if (K3 % GEMM_BK) return fail(JENGA_EINVAL, "gemm: K must be a multiple of 64");
+  if (K3 > 0) {
+    if ((s = make_tmap_bf16(&ta3, A3->ptr, A3->rows, K3, A3->ld, GEMM_BM)) != JENGA_OK) return s;
+    if ((s = make_tmap_bf16(&tb3, B3->ptr, B3->rows, K3, B3->ld, BN)) != JENGA_OK) return s;
+  }
   JENGA_CUDA_TRY(
       cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL));
   EpiParams p = ep;
   p.m_host = M;
   dim3 grid((N + BN - 1) / BN, (M + GEMM_BM - 1) / GEMM_BM);
   const int ps = prof_begin(name, st);
-  gemm_tc_kernel<BN, EPI><<<grid, GEMM_THREADS, L::TOTAL, st>>>(ta1, tb1, ta2, tb2, K1 / GEMM_BK, K2 / GEMM_BK,
-                                                                 N, p);
+  gemm_tc_kernel<BN, EPI><<<grid, GEMM_THREADS, L::TOTAL, st>>>(ta1, tb1, ta2, tb2, ta3, tb3, K1 / GEMM_BK,
+                                                                 K2 / GEMM_BK, K3 / GEMM_BK, N, p);
   prof_end(ps, st);
   JENGA_LAUNCH_CHECK();
   return JENGA_OK;

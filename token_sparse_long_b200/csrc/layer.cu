@@ -103,7 +103,7 @@ static size_t carve_fwd_ws(Carve& c, const Dims& d, int nc, FwdWs* w) {
 
 struct BwdWs {
   float *dk_acc, *dv_acc;
-  bf16 *xn, *g, *dgu, *dhb, *dO, *dqkv, *dtb;
+  bf16 *xn, *g, *dgu, *dhb, *dhlo, *dO, *dqkv, *dqkvlo, *dtb;
   float *gu, *dhn, *dh, *delta, *dq, *dt, *part;
 };
 static size_t carve_bwd_ws(Carve& c, const Dims& d, int nc, int T, BwdWs* w) {
@@ -117,6 +117,8 @@ static size_t carve_bwd_ws(Carve& c, const Dims& d, int nc, int T, BwdWs* w) {
   w->dO = c.take<bf16>((size_t)T * d.HD);
   w->dqkv = c.take<bf16>((size_t)T * 3 * d.HD);
   w->dtb = c.take<bf16>((size_t)T * LORA_PAD);
+  w->dhlo = c.take<bf16>((size_t)T * d.h);
+  w->dqkvlo = c.take<bf16>((size_t)T * 3 * d.HD);
   w->dhn = c.take<float>((size_t)T * d.h);
   w->dh = c.take<float>((size_t)T * d.h);
   w->delta = c.take<float>((size_t)d.H * T);
@@ -508,8 +510,8 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
     {
     const int _ps = ::jenga::prof_begin("rmsnorm_bwd_rows", st);
     rmsnorm_bwd_rows_kernel<<<T, ROW_THREADS, 0, st>>>(b.dhn, h, s.hres + (size_t)s0 * h, h, s.rstd2 + s0,
-                                                        (const bf16*)w->mlp_norm, nullptr, b.g, h, b.dh, b.dhb, h,
-                                                        nullptr, 0, idx, blk, s0, n_kept, blk, h, S);
+                                                        (const bf16*)w->mlp_norm, nullptr, b.g, h, b.dh, b.dhb,
+                                                        b.dhlo, h, nullptr, 0, idx, blk, s0, n_kept, blk, h, S);
     ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();
@@ -518,7 +520,10 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
       EpiParams e = epi_base(idx, blk, n_kept, s0);
       e.out = b.dO;
       e.ldo = HD;
-      JENGA_TRY((launch_gemm<256, EPI_STORE_BF16>({b.dhb, T, h}, {p.woT, HD, h}, h, nullptr, nullptr, 0, T, HD, e, st, "gemm_do")));
+      // dh enters as a bf16 hi + lo pair (two K phases over the same weights)
+      GemmOperand a2{b.dhlo, T, h}, b2{p.woT, HD, h};
+      JENGA_TRY((launch_gemm<256, EPI_STORE_BF16>({b.dhb, T, h}, {p.woT, HD, h}, h, &a2, &b2, h, T, HD, e, st,
+                                                  "gemm_do")));
     }
     JENGA_TRY(attn_backward_segment(s.qkv, s.qkv + HD, s.qkv + 2 * HD, 3 * HD, s.o, HD, s.lse, nc, b.dO, HD, b.delta, T,
                                     b.dq, HD, b.dk_acc, b.dv_acc, HD, H, s0, s1, n_kept, blk, nc, st));
@@ -526,7 +531,7 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
     {
     const int _ps = ::jenga::prof_begin("rope_bwd_pack", st);
     rope_bwd_pack_kernel<<<grid_cap((int64_t)T * H * 64, 256), 256, 0, st>>>(
-        b.dq, HD, b.dk_acc, b.dv_acc, HD, s0, b.dqkv, 3 * HD, idx, blk, n_kept, blk, T, H, p.inv_freq);
+        b.dq, HD, b.dk_acc, b.dv_acc, HD, s0, b.dqkv, b.dqkvlo, 3 * HD, idx, blk, n_kept, blk, T, H, p.inv_freq);
     ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();
@@ -584,16 +589,18 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
       EpiParams e = epi_base(idx, blk, n_kept, s0);
       e.out = b.dhn;
       e.ldo = h;
-      GemmOperand a2{b.dtb, T, LORA_PAD}, b2{p.aqvT, h, LORA_PAD};
-      JENGA_TRY((launch_gemm<256, EPI_STORE_F32>({b.dqkv, T, 3 * HD}, {p.wqkvT, h, 3 * HD}, 3 * HD, &a2, &b2, LORA_PAD, T,
-                                                 h, e, st, "gemm_dxn")));
+      // dQKV enters as a bf16 hi + lo pair; the third K phase adds dt [Aq; Av]
+      GemmOperand a2{b.dqkvlo, T, 3 * HD}, b2{p.wqkvT, h, 3 * HD};
+      GemmOperand a3{b.dtb, T, LORA_PAD}, b3{p.aqvT, h, LORA_PAD};
+      JENGA_TRY((launch_gemm<256, EPI_STORE_F32>({b.dqkv, T, 3 * HD}, {p.wqkvT, h, 3 * HD}, 3 * HD, &a2, &b2, 3 * HD,
+                                                 T, h, e, st, "gemm_dxn", &a3, &b3, LORA_PAD)));
     }
     // dX[rows] = dh + RMSNorm_bwd(dxn)  (written in place into the gradient buffer)
     {
     const int _ps = ::jenga::prof_begin("rmsnorm_bwd_rows", st);
     rmsnorm_bwd_rows_kernel<<<T, ROW_THREADS, 0, st>>>(b.dhn, h, s.xr + (size_t)s0 * h, h, s.rstd1 + s0,
                                                         (const bf16*)w->attn_norm, b.dh, nullptr, h, nullptr, nullptr,
-                                                        h, dX, h, idx, blk, s0, n_kept, blk, h, S);
+                                                        nullptr, h, dX, h, idx, blk, s0, n_kept, blk, h, S);
     ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();

@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_bwd_rows_kernel(
     const float* __restrict__ dy, int64_t lddy, const bf16* __restrict__ x, int64_t ldx,
     const float* __restrict__ rstd, const bf16* __restrict__ gain, const float* __restrict__ base_f,
     const bf16* __restrict__ base_b, int64_t ldb, float* __restrict__ out_f, bf16* __restrict__ out_b,
-    int64_t ldo, bf16* __restrict__ dst, int64_t ldd, const int32_t* __restrict__ idx, int blk, int row_offset,
+    bf16* __restrict__ out_lo, int64_t ldo, bf16* __restrict__ dst, int64_t ldd, const int32_t* __restrict__ idx, int blk, int row_offset,
     const int32_t* __restrict__ n_valid, int valid_mult, int h, int64_t dst_rows) {
   __shared__ float red[ROW_THREADS / 32];
   const int m = blockIdx.x;
@@ -167,7 +167,17 @@ __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_bwd_rows_kernel(
         op[0] = make_float4(o[0], o[1], o[2], o[3]);
         op[1] = make_float4(o[4], o[5], o[6], o[7]);
       }
-      if (out_b) reinterpret_cast<uint4*>(out_b + (int64_t)m * ldo)[c] = pack8(o);
+      if (out_b) {
+        const uint4 hi = pack8(o);
+        reinterpret_cast<uint4*>(out_b + (int64_t)m * ldo)[c] = hi;
+        if (out_lo) {  // residual o - bf16(o), so that hi + lo carries ~16 mantissa bits
+          float hv[8], lo[8];
+          unpack8(hi, hv);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) lo[e] = o[e] - hv[e];
+          reinterpret_cast<uint4*>(out_lo + (int64_t)m * ldo)[c] = pack8(lo);
+        }
+      }
       if (dst) reinterpret_cast<uint4*>(dst + drow * ldd)[c] = pack8(o);
     }
   }
@@ -192,11 +202,12 @@ __global__ void gather_seg_kernel(const bf16* __restrict__ src, int64_t lds, bf1
   }
 }
 
-// dqkv[m] = [rope^T(dq[m]) | rope^T(dk[s0+m]) | dv[s0+m]] in bf16; positions row(s0 + m).
+// dqkv[m] = [rope^T(dq[m]) | rope^T(dk[s0+m]) | dv[s0+m]] as a bf16 hi part (dqkv) and the
+// bf16 residual (dqkv_lo); positions row(s0 + m).
 // One thread per (row, head, pair i < 64).
 __global__ void rope_bwd_pack_kernel(const float* __restrict__ dq, int64_t ld_dq, const float* __restrict__ dk,
                                      const float* __restrict__ dv, int64_t ld_acc, int s0, bf16* __restrict__ dqkv,
-                                     int64_t ld_out, const int32_t* __restrict__ idx, int blk,
+                                     bf16* __restrict__ dqkv_lo, int64_t ld_out, const int32_t* __restrict__ idx, int blk,
                                      const int32_t* __restrict__ n_valid, int valid_mult, int rows, int H,
                                      const double* __restrict__ inv_freq) {
   const int nv = valid_rows(n_valid, valid_mult, s0, rows);
@@ -217,14 +228,17 @@ __global__ void rope_bwd_pack_kernel(const float* __restrict__ dq, int64_t ld_dq
     const float* kk = dk + (int64_t)(s0 + m) * ld_acc;
     const float* vv = dv + (int64_t)(s0 + m) * ld_acc;
     bf16* o = dqkv + (int64_t)m * ld_out;
+    bf16* ol = dqkv_lo + (int64_t)m * ld_out;
     const float a1 = q[c1], a2 = q[c2];
-    o[c1] = __float2bfloat16_rn(a1 * cs + a2 * sn);
-    o[c2] = __float2bfloat16_rn(a2 * cs - a1 * sn);
     const float b1 = kk[c1], b2 = kk[c2];
-    o[HD + c1] = __float2bfloat16_rn(b1 * cs + b2 * sn);
-    o[HD + c2] = __float2bfloat16_rn(b2 * cs - b1 * sn);
-    o[2 * HD + c1] = __float2bfloat16_rn(vv[c1]);
-    o[2 * HD + c2] = __float2bfloat16_rn(vv[c2]);
+    const float val[6] = {a1 * cs + a2 * sn, a2 * cs - a1 * sn, b1 * cs + b2 * sn, b2 * cs - b1 * sn, vv[c1], vv[c2]};
+    const int col[6] = {c1, c2, HD + c1, HD + c2, 2 * HD + c1, 2 * HD + c2};
+#pragma unroll
+    for (int e = 0; e < 6; ++e) {
+      const bf16 hi = __float2bfloat16_rn(val[e]);
+      o[col[e]] = hi;
+      ol[col[e]] = __float2bfloat16_rn(val[e] - __bfloat162float(hi));
+    }
   }
 }
 

@@ -9,6 +9,7 @@
 // fp32 inputs: exact fp32 SIMT dot products.  bf16 inputs (head_dim 128): tensor-core
 // tiles of 64 queries x 64 keys.
 #include "attn_frag.cuh"
+#include "score_tc.cuh"
 
 namespace jenga {
 
@@ -383,6 +384,36 @@ extern "C" jenga_status jenga_score_blocks(const void* q, int64_t ldq, const voi
     if (D != AT_D || S % AT_ROWS || ldq % 8 || ldk % 8 || ((uintptr_t)q & 15) || ((uintptr_t)k & 15))
       return fail(JENGA_EUNSUPPORTED, "jenga_score_blocks: bf16 path needs D == 128, S % 64 == 0, aligned rows");
     const float sl2 = SC_LOG2E * scale;
+    if (S % SCT_ROWS == 0) {
+      // tcgen05 path: 128-token tiles, TMA-fed, accumulators in tensor memory
+      CUtensorMap tq, tk;
+      jenga_status s1 = make_tmap_bf16(&tq, q, (uint64_t)B * S, (uint64_t)H * D, ldq, SCT_ROWS);
+      if (s1 != JENGA_OK) return s1;
+      s1 = make_tmap_bf16(&tk, k, (uint64_t)B * S, (uint64_t)H * D, ldk, SCT_ROWS);
+      if (s1 != JENGA_OK) return s1;
+      JENGA_CUDA_TRY(cudaFuncSetAttribute(score_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, SCT_SMEM));
+      JENGA_CUDA_TRY(cudaFuncSetAttribute(score_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, SCT_SMEM));
+      dim3 gt(S / SCT_ROWS, H, B);
+      {
+        const int _ps = ::jenga::prof_begin("score_lse_tc", st);
+        score_tc_kernel<0><<<gt, SCT_THREADS, SCT_SMEM, st>>>(tq, tk, S, H, causal ? 1 : 0, sl2, nullptr, lse);
+        ::jenga::prof_end(_ps, st);
+      }
+      JENGA_LAUNCH_CHECK();
+      {
+        const int _ps = ::jenga::prof_begin("score_mass_tc", st);
+        score_tc_kernel<1><<<gt, SCT_THREADS, SCT_SMEM, st>>>(tq, tk, S, H, causal ? 1 : 0, sl2, lse, mass);
+        ::jenga::prof_end(_ps, st);
+      }
+      JENGA_LAUNCH_CHECK();
+      {
+        const int _ps = ::jenga::prof_begin("score_reduce", st);
+        score_reduce_kernel<<<dim3(nb, B), 1024, 0, st>>>(mass, S, H, blk, scores);
+        ::jenga::prof_end(_ps, st);
+      }
+      JENGA_LAUNCH_CHECK();
+      return JENGA_OK;
+    }
     dim3 g(S / AT_ROWS, H, B);
     JENGA_CUDA_TRY(
         cudaFuncSetAttribute(score_lse_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 3 * AT_TILE_BYTES));

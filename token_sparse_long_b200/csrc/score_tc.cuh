@@ -1,0 +1,184 @@
+// tcgen05 block-scoring passes (head_dim 128, 128-token tiles).
+//
+//   pass 1 (ROWS = queries): L_i = log2 sum_{j <= i} 2^(log2(e) q_i . k_j / sqrt(D))
+//   pass 2 (ROWS = keys):    mass_j = sum_{i >= j} 2^(log2(e) q_i . k_j / sqrt(D) - L_i)
+//
+// One CTA per (128-row tile, head, sequence), 192 threads:
+//   warp 0      TMA: the CTA's fixed 128 x 128 tile (two 64-column swizzled boxes), then
+//               the streamed tiles through a 4-stage shared-memory ring
+//   warp 1      TMEM allocation; one lane issues tcgen05.mma (M 128, N 128, K 16) x 8 per
+//               streamed tile into one of two 128-column TMEM accumulators
+//   warps 2..5  one TMEM lane (= one row of the tile) per thread: tcgen05.ld the 128 scores,
+//               release the accumulator, then exponentials and sums in registers, which
+//               overlaps the next tile's MMA
+// Causal diagonal tiles are masked in the epilogue.  All waits are bounded.
+#pragma once
+
+#include "common.cuh"
+
+namespace jenga {
+
+constexpr int SCT_ROWS = 128;
+constexpr int SCT_STAGES = 4;
+constexpr int SCT_BOX_BYTES = 128 * 64 * 2;          // one 128 x 64 bf16 box
+constexpr int SCT_TILE_BYTES = 2 * SCT_BOX_BYTES;     // 128 x 128 tile
+constexpr int SCT_SMEM = (1 + SCT_STAGES) * SCT_TILE_BYTES + 256 + 1024;
+constexpr int SCT_THREADS = 192;
+
+template <int MODE>  // 0: row LSE (rows = queries), 1: column mass (rows = keys)
+__global__ void __launch_bounds__(SCT_THREADS, 1)
+    score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, int S,
+                    int H, int causal, float scale_log2, const float* __restrict__ lse_in,
+                    float* __restrict__ out) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* fix = smem;
+  uint8_t* ring = smem + SCT_TILE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (1 + SCT_STAGES) * SCT_TILE_BYTES);
+  uint64_t* full = bars;                       // [STAGES]
+  uint64_t* empty = full + SCT_STAGES;         // [STAGES]
+  uint64_t* s_full = empty + SCT_STAGES;       // [2]
+  uint64_t* s_empty = s_full + 2;              // [2]
+  uint64_t* fix_full = s_empty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(fix_full + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntile = S / SCT_ROWS;
+  const int h = blockIdx.y, b = blockIdx.z;
+  // pass 1: longest query tiles first; pass 2: key tile 0 sees the most queries
+  const int t = (MODE == 0) ? (ntile - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+  const int j0 = (MODE == 0) ? 0 : (causal ? t : 0);
+  const int j1 = (MODE == 0) ? (causal ? t + 1 : ntile) : ntile;
+  const int nj = j1 - j0;
+  const int col0 = h * 128;
+  const int rowbase = b * S;
+  const CUtensorMap* tm_fix = (MODE == 0) ? &tmQ : &tmK;
+  const CUtensorMap* tm_str = (MODE == 0) ? &tmK : &tmQ;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SCT_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], 4);
+    }
+    mbar_init(fix_full, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(tm_fix);
+    prefetch_tmap(tm_str);
+    mbar_arrive_expect_tx(fix_full, SCT_TILE_BYTES);
+    tma_load_2d(fix, tm_fix, fix_full, col0, rowbase + t * SCT_ROWS);
+    tma_load_2d(fix + SCT_BOX_BYTES, tm_fix, fix_full, col0 + 64, rowbase + t * SCT_ROWS);
+    for (int i = 0; i < nj; ++i) {
+      const int s = i % SCT_STAGES;
+      if (i >= SCT_STAGES && !mbar_wait(&empty[s], ((i / SCT_STAGES) - 1) & 1, SITE_SCORE_TC)) break;
+      uint8_t* dst = ring + s * SCT_TILE_BYTES;
+      const int row = rowbase + (j0 + i) * SCT_ROWS;
+      mbar_arrive_expect_tx(&full[s], SCT_TILE_BYTES);
+      tma_load_2d(dst, tm_str, &full[s], col0, row);
+      tma_load_2d(dst + SCT_BOX_BYTES, tm_str, &full[s], col0 + 64, row);
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc = umma_idesc_bf16(128, 128);
+    bool ok = mbar_wait(fix_full, 0, SITE_SCORE_TC);
+    const uint32_t fa = smem_u32(fix);
+    for (int i = 0; ok && i < nj; ++i) {
+      const int s = i % SCT_STAGES, buf = i & 1;
+      if (!mbar_wait(&full[s], (i / SCT_STAGES) & 1, SITE_SCORE_TC)) break;
+      if (i >= 2 && !mbar_wait(&s_empty[buf], ((i >> 1) - 1) & 1, SITE_SCORE_TC)) break;
+      tc_fence_after();
+      const uint32_t sb = smem_u32(ring + s * SCT_TILE_BYTES);
+#pragma unroll
+      for (int kc = 0; kc < 2; ++kc)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_bf16(tmem + buf * 128, umma_desc_k_sw128(fa + kc * SCT_BOX_BYTES + k * 32),
+                    umma_desc_k_sw128(sb + kc * SCT_BOX_BYTES + k * 32), idesc, (kc | k) ? 1u : 0u);
+      umma_commit(&empty[s]);
+      umma_commit(&s_full[buf]);
+    }
+  } else if (warp >= 2) {
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    float m = -INFINITY, l = 0.f, acc = 0.f;
+    bool ok = true;
+    const float* lb = (MODE == 1) ? lse_in + ((int64_t)b * H + h) * S : nullptr;
+    for (int i = 0; i < nj; ++i) {
+      const int buf = i & 1, j = j0 + i;
+      if (!mbar_wait(&s_full[buf], (i >> 1) & 1, SITE_SCORE_TC)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t v[128];
+      tmem_ld32_nowait(tl + buf * 128 + 0, v);
+      tmem_ld32_nowait(tl + buf * 128 + 32, v + 32);
+      tmem_ld32_nowait(tl + buf * 128 + 64, v + 64);
+      tmem_ld32_nowait(tl + buf * 128 + 96, v + 96);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[buf]);
+      const bool diag = causal && (j == t);
+      if (MODE == 0) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          float x = __uint_as_float(v[c]) * scale_log2;
+          if (diag && c > r) x = -INFINITY;
+          v[c] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+        const float mn = fmaxf(m, mx);
+        float sum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) sum += fast_exp2(__uint_as_float(v[c]) - mn);
+        l = l * fast_exp2(m - mn) + sum;
+        m = mn;
+      } else {
+        const float4* L4 = reinterpret_cast<const float4*>(lb + (int64_t)j * SCT_ROWS);
+        float sum = 0.f;
+#pragma unroll
+        for (int c4 = 0; c4 < 32; ++c4) {
+          const float4 L = __ldg(L4 + c4);
+          const float Ls[4] = {L.x, L.y, L.z, L.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * c4 + e;
+            const float p = fast_exp2(fmaf(__uint_as_float(v[c]), scale_log2, -Ls[e]));
+            sum += (diag && c < r) ? 0.f : p;
+          }
+        }
+        acc += sum;
+      }
+    }
+    if (ok) {
+      if (MODE == 0)  // log-sum-exp in log2 units (pass 2 consumes it directly)
+        out[((int64_t)b * H + h) * S + t * SCT_ROWS + r] = m + __log2f(l);
+      else
+        out[((int64_t)b * H + h) * S + t * SCT_ROWS + r] = acc;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace jenga
