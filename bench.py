@@ -83,7 +83,7 @@ def work_model(case, ks, seg):
         add("score_mass_tc", "flop", 2.0 * D * H * causal_pairs(S))
         add("gemm_lora_t", "flop", 2.0 * n * 32 * h)
         add("gemm_qkv_rope", "flop", 2.0 * n * 3 * HD * h)
-        add("attn_fwd", "flop", 4.0 * D * H * causal_pairs(n))
+        add("attn_fwd_tc", "flop", 4.0 * D * H * causal_pairs(n))
         add("gemm_o_scatter", "flop", 2.0 * n * h * HD)
         add("gemm_gateup_swiglu", "flop", 2.0 * n * 2 * F * h)
         add("gemm_down_scatter", "flop", 2.0 * n * h * F)

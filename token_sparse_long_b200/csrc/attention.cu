@@ -11,6 +11,7 @@
 // accumulators for keys [0, segment end).  Processing segments last-first completes
 // a segment's key gradients exactly when its own queries have been processed.
 #include "attn_frag.cuh"
+#include "attn_tc.cuh"
 
 namespace jenga {
 
@@ -336,8 +337,24 @@ jenga_status attn_forward(const bf16* q, const bf16* k, const bf16* v, int64_t l
                           int64_t lse_ld, int H, const int32_t* n_valid, int valid_mult, int n_cap, cudaStream_t st) {
   if (n_cap <= 0) return JENGA_OK;
   if (n_cap % AT_ROWS) return fail(JENGA_EINVAL, "attention: rows must be a multiple of 64");
-  JENGA_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATTN_FWD_SMEM));
   const float scale_log2 = LOG2E / sqrtf((float)AT_D);
+  {
+    // tcgen05 path: TMA-fed 128-row tiles (rows of q/k/v past the valid count must be
+    // finite: the layer zeroes them before this call)
+    CUtensorMap tq, tk, tv;
+    jenga_status s1;
+    if ((s1 = make_tmap_bf16(&tq, q, n_cap, (uint64_t)H * AT_D, ld, ATC_ROWS)) != JENGA_OK) return s1;
+    if ((s1 = make_tmap_bf16(&tk, k, n_cap, (uint64_t)H * AT_D, ld, ATC_ROWS)) != JENGA_OK) return s1;
+    if ((s1 = make_tmap_bf16(&tv, v, n_cap, (uint64_t)H * AT_D, ld, ATC_ROWS)) != JENGA_OK) return s1;
+    JENGA_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATC_SMEM));
+    const int _ps = ::jenga::prof_begin("attn_fwd_tc", st);
+    attn_fwd_tc_kernel<<<dim3((n_cap + ATC_ROWS - 1) / ATC_ROWS, H), ATC_THREADS, ATC_SMEM, st>>>(
+        tq, tk, tv, o, ldo, lse, lse_ld, n_valid, valid_mult, n_cap, scale_log2);
+    ::jenga::prof_end(_ps, st);
+    JENGA_LAUNCH_CHECK();
+    return JENGA_OK;
+  }
+  JENGA_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATTN_FWD_SMEM));
   {
   const int _ps = ::jenga::prof_begin("attn_fwd", st);
   attn_fwd_kernel<<<dim3(n_cap / AT_ROWS, H), 128, ATTN_FWD_SMEM, st>>>(q, k, v, ld, o, ldo, lse, lse_ld, n_valid,

@@ -1,10 +1,11 @@
 // tcgen05 GEMM for the retained-token layer projections (sm_100a).
 //
-//   C[M, N] = A1[M, K1] * B1[N, K1]^T  (+ A2[M, K2] * B2[N, K2]^T)     bf16 in, fp32 accumulate
+//   C[M, N] = A1 B1^T (+ A2 B2^T (+ A3 B3^T))     bf16 (or fp16) in, fp32 accumulate
 //
-// Both operands are K-major bf16 (row-major [rows, K]).  The optional second
-// operand pair extends the reduction (used to fold the LoRA up-projection into the
-// QKV projection, and the LoRA down-projection's input gradient into the dX GEMM).
+// All operands are K-major (row-major [rows, K]).  The optional second and third
+// operand pairs extend the reduction: they fold the LoRA up-projection into the QKV
+// projection, carry the low half of a bf16 hi + lo split operand, and fold the LoRA
+// down-projection's input gradient into the dX GEMM.
 //
 // Structure (one 128 x BN output tile per CTA, 192 threads):
 //   warp 0      TMA producer: 128 x 64 A box + BN x 64 B box per stage into a
@@ -31,7 +32,7 @@ enum GemmEpi : int {
   EPI_SCATTER_ADD = 2,  // x[row(m), n] = bf16(x + acc); aux[m, n] = same value (optional)
   EPI_SWIGLU = 3,       // 64-col groups (gate, up) -> out[m, n/2 + j] = bf16(silu(g) * u)
   EPI_QKV_ROPE = 4,     // q/k/v sections of width hd; RoPE(pos(m)) on q and k -> bf16
-  EPI_SWIGLU_BWD = 5,   // acc = dA; aux = (g, u) interleaved fp32 -> out = (dg, du) interleaved bf16
+  EPI_SWIGLU_BWD = 5,   // acc = dA; aux = (g, u) interleaved fp32 -> out = (dg, du) interleaved fp16
   EPI_LORA_T = 6,       // out fp32 [m, 0:N] = beta * acc ; aux bf16 [m, 0:64] = bf16(alpha * acc), zero padded
 };
 
@@ -86,6 +87,21 @@ __device__ __forceinline__ void store_bf16x32(bf16* dst, const float* v) {
   }
 }
 
+__device__ __forceinline__ void store_f16x32(__half* dst, const float* v) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    uint32_t* ws = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half2 h = __floats2half2_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
+      ws[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    d[q] = w;
+  }
+}
+
 __device__ __forceinline__ void load_bf16x32(const bf16* src, float* v) {
   const uint4* s = reinterpret_cast<const uint4*>(src);
 #pragma unroll
@@ -119,7 +135,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                    const __grid_constant__ CUtensorMap tmA3, const __grid_constant__ CUtensorMap tmB3, int nkb1,
-                   int nkb2, int nkb3, int N, EpiParams ep) {
+                   int nkb2, int nkb3, int N, uint32_t idesc, EpiParams ep) {
   using L = GemmSmem<BN>;
   constexpr int STAGES = L::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -180,7 +196,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
-    constexpr uint32_t idesc = umma_idesc_bf16(GEMM_BM, BN);
+    // idesc: kind::f16 instruction descriptor (bf16 or fp16 operands, fp32 accumulate)
     bool ok = true;
     for (int kb = 0; kb < nkb; ++kb) {
       const int s = kb % STAGES;
@@ -204,7 +220,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const int m = m0 + r;
-    const bool ok = mbar_wait(accum, 0, SITE_GEMM_EPILOGUE);
+    // warp vote: the tcgen05.ld calls below are collective, so all lanes take one path
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(accum, 0, SITE_GEMM_EPILOGUE));
     tc_fence_after();
     if (ok) {
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -280,9 +297,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             dg[i] = da * uv[i] * sg * (1.f + gv[i] * (1.f - sg));
             v[i] = da * gv[i] * sg;  // du = dA * silu(g)
           }
-          bf16* o = reinterpret_cast<bf16*>(ep.out) + (int64_t)m * ep.ldo + col;
-          store_bf16x32(o, dg);
-          store_bf16x32(o + 64, v);
+          __half* o = reinterpret_cast<__half*>(ep.out) + (int64_t)m * ep.ldo + col;
+          store_f16x32(o, dg);
+          store_f16x32(o + 64, v);
         }
       } else if (EPI == EPI_LORA_T) {
         // N <= 32 (t_q, t_v): fp32 copy + scaled bf16 copy padded to 64 columns
@@ -353,7 +370,7 @@ template <int BN, int EPI>
 jenga_status launch_gemm(const GemmOperand& A1, const GemmOperand& B1, int K1, const GemmOperand* A2,
                          const GemmOperand* B2, int K2, int M, int N, const EpiParams& ep, cudaStream_t st,
                          const char* name = "gemm", const GemmOperand* A3 = nullptr,
-                         const GemmOperand* B3 = nullptr, int K3 = 0) {
+                         const GemmOperand* B3 = nullptr, int K3 = 0, bool f16_inputs = false) {
   using L = GemmSmem<BN>;
   if (M <= 0 || N <= 0) return JENGA_OK;
   if (K1 % GEMM_BK || K2 % GEMM_BK || K1 <= 0) return fail(JENGA_EINVAL, "gemm: K must be a multiple of 64");
@@ -379,9 +396,12 @@ jenga_status launch_gemm(const GemmOperand& A1, const GemmOperand& B1, int K1, c
   EpiParams p = ep;
   p.m_host = M;
   dim3 grid((N + BN - 1) / BN, (M + GEMM_BM - 1) / GEMM_BM);
+  // operand format fields (bits 7-9: A, 10-12: B) are 1 for bf16 and 0 for fp16
+  const uint32_t idesc = f16_inputs ? (umma_idesc_bf16(GEMM_BM, BN) & ~((7u << 7) | (7u << 10)))
+                                    : umma_idesc_bf16(GEMM_BM, BN);
   const int ps = prof_begin(name, st);
   gemm_tc_kernel<BN, EPI><<<grid, GEMM_THREADS, L::TOTAL, st>>>(ta1, tb1, ta2, tb2, ta3, tb3, K1 / GEMM_BK,
-                                                                 K2 / GEMM_BK, K3 / GEMM_BK, N, p);
+                                                                 K2 / GEMM_BK, K3 / GEMM_BK, N, idesc, p);
   prof_end(ps, st);
   JENGA_LAUNCH_CHECK();
   return JENGA_OK;

@@ -247,6 +247,13 @@ extern "C" jenga_status jenga_layer_pack(const jenga_layer_weights* w, const jen
   JENGA_TRY(transpose((const bf16*)w->wo, HD, p.woT, h, h, HD, st));          // Wo [h, HD] -> [HD, h]
   JENGA_TRY(transpose((const bf16*)w->wd, F, p.wdT, h, h, F, st));            // Wd [h, F]  -> [F, h]
   JENGA_TRY(transpose(p.wgu, h, p.wguT, 2 * F, 2 * F, h, st));                // [2F, h]    -> [h, 2F]
+  {  // the dhn product runs on fp16 operands (dg, du carry 3 more mantissa bits than bf16)
+    const int _ps = ::jenga::prof_begin("bf16_to_f16_inplace", st);
+    bf16_to_f16_inplace_kernel<<<grid_cap((int64_t)h * 2 * F, 256), 256, 0, st>>>((uint16_t*)p.wguT,
+                                                                                (int64_t)h * 2 * F);
+    ::jenga::prof_end(_ps, st);
+  }
+  JENGA_LAUNCH_CHECK();
   JENGA_TRY(transpose(p.wqkv, h, p.wqkvT, 3 * HD, 3 * HD, h, st));            // [3HD, h]   -> [h, 3HD]
   // dt = dqkv * bcat^T : rows 0..15 = [Bq^T | 0 | 0], rows 16..31 = [0 | 0 | Bv^T]
   JENGA_TRY(zero(p.bcat, (int64_t)2 * LORA_R * 3 * HD, st));
@@ -386,7 +393,14 @@ extern "C" jenga_status jenga_sparse_layer_fwd(const jenga_layer_weights* w, con
     JENGA_TRY((launch_gemm<256, EPI_QKV_ROPE>({f.xn, nc, h}, {p.wqkv, 3 * HD, h}, h, &a2, &b2, LORA_PAD, nc, 3 * HD,
                                               e, st, "gemm_qkv_rope")));
   }
-  // 4. causal attention among retained tokens
+  // 4. causal attention among retained tokens (q/k/v rows past the device count are
+  //    zeroed first: the tensor-core tiles read them and multiply them by zero weights)
+  {
+    const int _ps = ::jenga::prof_begin("zero_tail_rows", st);
+    zero_tail_rows_kernel<<<sm_count(), 256, 0, st>>>(s.qkv, 3 * HD, 3 * HD, n_kept, blk, nc);
+    ::jenga::prof_end(_ps, st);
+  }
+  JENGA_LAUNCH_CHECK();
   JENGA_TRY(attn_forward(s.qkv, s.qkv + HD, s.qkv + 2 * HD, 3 * HD, s.o, HD, s.lse, nc, d.H, n_kept, blk, nc, st));
   // 5. o_proj with the in-place residual add into X (and a compact copy of h)
   {
@@ -504,7 +518,8 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
       EpiParams e = epi_base(idx, blk, n_kept, s0);
       e.out = b.dhn;
       e.ldo = h;
-      JENGA_TRY((launch_gemm<256, EPI_STORE_F32>({b.dgu, T, 2 * F}, {p.wguT, h, 2 * F}, 2 * F, nullptr, nullptr, 0, T, h, e, st, "gemm_dhn")));
+      JENGA_TRY((launch_gemm<256, EPI_STORE_F32>({b.dgu, T, 2 * F}, {p.wguT, h, 2 * F}, 2 * F, nullptr, nullptr, 0, T,
+                                                 h, e, st, "gemm_dhn", nullptr, nullptr, 0, /*f16_inputs=*/true)));
     }
     // dh = G + RMSNorm_bwd(dhn)
     {

@@ -318,6 +318,30 @@ __global__ void interleave_gate_up_kernel(const bf16* __restrict__ wg, const bf1
   }
 }
 
+// Rows [valid, cap) of a bf16 [cap, cols] buffer set to zero (valid read on the device).
+__global__ void zero_tail_rows_kernel(bf16* __restrict__ x, int64_t ld, int cols, const int32_t* __restrict__ n_valid,
+                                      int valid_mult, int cap) {
+  int v = n_valid ? (*n_valid) * valid_mult : cap;
+  v = v < 0 ? 0 : (v < cap ? v : cap);
+  const int vpr = cols >> 3;
+  const int64_t total = (int64_t)(cap - v) * vpr;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = v + e / vpr;
+    const int c = (int)(e % vpr);
+    reinterpret_cast<uint4*>(x + r * ld)[c] = make_uint4(0, 0, 0, 0);
+  }
+}
+
+// In-place bf16 -> fp16 re-encoding (exact for magnitudes in [2^-14, 65504]; the frozen
+// gate/up weights used by the fp16 dhn product are well inside that range).
+__global__ void bf16_to_f16_inplace_kernel(uint16_t* __restrict__ x, int64_t n) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const float f = __uint_as_float((uint32_t)x[e] << 16);
+    const __half hv = __float2half_rn(f);
+    x[e] = *reinterpret_cast<const uint16_t*>(&hv);
+  }
+}
+
 __global__ void zero_bf16_kernel(bf16* __restrict__ dst, int64_t n) {
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
     dst[e] = __float2bfloat16_rn(0.f);

@@ -3,14 +3,16 @@
 //   pass 1 (ROWS = queries): L_i = log2 sum_{j <= i} 2^(log2(e) q_i . k_j / sqrt(D))
 //   pass 2 (ROWS = keys):    mass_j = sum_{i >= j} 2^(log2(e) q_i . k_j / sqrt(D) - L_i)
 //
-// One CTA per (128-row tile, head, sequence), 192 threads:
+// One CTA per (128-row tile, head, sequence), 320 threads:
 //   warp 0      TMA: the CTA's fixed 128 x 128 tile (two 64-column swizzled boxes), then
 //               the streamed tiles through a 4-stage shared-memory ring
 //   warp 1      TMEM allocation; one lane issues tcgen05.mma (M 128, N 128, K 16) x 8 per
 //               streamed tile into one of two 128-column TMEM accumulators
-//   warps 2..5  one TMEM lane (= one row of the tile) per thread: tcgen05.ld the 128 scores,
-//               release the accumulator, then exponentials and sums in registers, which
-//               overlaps the next tile's MMA
+//   warps 2..9  two quads; in each quad one TMEM lane (= one row of the tile) per thread,
+//               quad 0 taking columns 0..63 and quad 1 columns 64..127: tcgen05.ld, release
+//               the accumulator, then exponentials and sums in registers (8 independent
+//               partial sums), which overlaps the next tile's MMA; the two halves of each
+//               row are merged in shared memory at the end
 // Causal diagonal tiles are masked in the epilogue.  All waits are bounded.
 #pragma once
 
@@ -22,8 +24,8 @@ constexpr int SCT_ROWS = 128;
 constexpr int SCT_STAGES = 4;
 constexpr int SCT_BOX_BYTES = 128 * 64 * 2;          // one 128 x 64 bf16 box
 constexpr int SCT_TILE_BYTES = 2 * SCT_BOX_BYTES;     // 128 x 128 tile
-constexpr int SCT_SMEM = (1 + SCT_STAGES) * SCT_TILE_BYTES + 256 + 1024;
-constexpr int SCT_THREADS = 192;
+constexpr int SCT_SMEM = (1 + SCT_STAGES) * SCT_TILE_BYTES + 2048 + 1024;  // + barriers, row exchange, align
+constexpr int SCT_THREADS = 320;
 
 template <int MODE>  // 0: row LSE (rows = queries), 1: column mass (rows = keys)
 __global__ void __launch_bounds__(SCT_THREADS, 1)
@@ -62,7 +64,7 @@ __global__ void __launch_bounds__(SCT_THREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], 4);
+      mbar_init(&s_empty[s], 8);
     }
     mbar_init(fix_full, 1);
     fence_barrier_init();
@@ -111,66 +113,89 @@ __global__ void __launch_bounds__(SCT_THREADS, 1)
       umma_commit(&s_full[buf]);
     }
   } else if (warp >= 2) {
+    // two quads of epilogue warps: quad 0 (warps 2-5) takes columns 0..63 of every row,
+    // quad 1 (warps 6-9) columns 64..127; warp w reads TMEM lanes 32 * (w % 4) ..
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
-    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + half * 64;
     float m = -INFINITY, l = 0.f, acc = 0.f;
     bool ok = true;
     const float* lb = (MODE == 1) ? lse_in + ((int64_t)b * H + h) * S : nullptr;
     for (int i = 0; i < nj; ++i) {
       const int buf = i & 1, j = j0 + i;
-      if (!mbar_wait(&s_full[buf], (i >> 1) & 1, SITE_SCORE_TC)) {
+      // warp vote: the tcgen05.ld below is collective, so all lanes leave together
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[buf], (i >> 1) & 1, SITE_SCORE_TC))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t v[128];
+      uint32_t v[64];
       tmem_ld32_nowait(tl + buf * 128 + 0, v);
       tmem_ld32_nowait(tl + buf * 128 + 32, v + 32);
-      tmem_ld32_nowait(tl + buf * 128 + 64, v + 64);
-      tmem_ld32_nowait(tl + buf * 128 + 96, v + 96);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[buf]);
       const bool diag = causal && (j == t);
+      const int cbase = half * 64;
       if (MODE == 0) {
-        float mx = -INFINITY;
+        float mx[8];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
+        for (int a = 0; a < 8; ++a) mx[a] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
           float x = __uint_as_float(v[c]) * scale_log2;
-          if (diag && c > r) x = -INFINITY;
+          if (diag && cbase + c > r) x = -INFINITY;
           v[c] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
+          mx[c & 7] = fmaxf(mx[c & 7], x);
         }
-        const float mn = fmaxf(m, mx);
-        float sum = 0.f;
+        const float mxa = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float mn = fmaxf(m, mxa);
+        if (mn != -INFINITY) {  // a half row of the diagonal tile can be fully masked
+          float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 128; ++c) sum += fast_exp2(__uint_as_float(v[c]) - mn);
-        l = l * fast_exp2(m - mn) + sum;
-        m = mn;
+          for (int c = 0; c < 64; ++c) sm[c & 7] += fast_exp2(__uint_as_float(v[c]) - mn);
+          const float sum = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
+          l = l * fast_exp2(m - mn) + sum;
+          m = mn;
+        }
       } else {
-        const float4* L4 = reinterpret_cast<const float4*>(lb + (int64_t)j * SCT_ROWS);
-        float sum = 0.f;
+        const float4* L4 = reinterpret_cast<const float4*>(lb + (int64_t)j * SCT_ROWS + cbase);
+        float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c4 = 0; c4 < 32; ++c4) {
+        for (int c4 = 0; c4 < 16; ++c4) {
           const float4 L = __ldg(L4 + c4);
           const float Ls[4] = {L.x, L.y, L.z, L.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = 4 * c4 + e;
             const float p = fast_exp2(fmaf(__uint_as_float(v[c]), scale_log2, -Ls[e]));
-            sum += (diag && c < r) ? 0.f : p;
+            sm[c & 7] += (diag && cbase + c < r) ? 0.f : p;
           }
         }
-        acc += sum;
+        acc += ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
       }
     }
-    if (ok) {
-      if (MODE == 0)  // log-sum-exp in log2 units (pass 2 consumes it directly)
-        out[((int64_t)b * H + h) * S + t * SCT_ROWS + r] = m + __log2f(l);
-      else
-        out[((int64_t)b * H + h) * S + t * SCT_ROWS + r] = acc;
+    // merge the two column halves of each row (fixed order: half 0 then half 1)
+    float* xch = reinterpret_cast<float*>(tmem_holder + 4);  // 2 x 128 floats after the barriers
+    if (half == 1) {
+      xch[r] = (MODE == 0) ? m : acc;
+      xch[128 + r] = l;
+    }
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (half == 0 && ok) {
+      float res;
+      if (MODE == 0) {
+        const float m2 = xch[r], l2 = xch[128 + r];
+        const float mm = fmaxf(m, m2);
+        const float ll = l * fast_exp2(m - mm) + l2 * fast_exp2(m2 - mm);
+        res = mm + __log2f(ll);  // log-sum-exp in log2 units (pass 2 consumes it directly)
+      } else {
+        res = acc + xch[r];
+      }
+      out[((int64_t)b * H + h) * S + t * SCT_ROWS + r] = res;
     }
   }
   tc_fence_before();
