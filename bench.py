@@ -91,8 +91,8 @@ def work_model(case, ks, seg):
         add("gemm_da_swiglu_bwd", "flop", 2.0 * n * F * h)
         add("gemm_dhn", "flop", 2.0 * n * h * 2 * F)
         add("gemm_do", "flop", 2.0 * n * HD * h)
-        add("attn_bwd_dq", "flop", 10.0 * D * H * causal_pairs(n) * 3 / 7)
-        add("attn_bwd_dkdv", "flop", 10.0 * D * H * causal_pairs(n) * 4 / 7)
+        add("attn_bwd_dq_tc", "flop", 10.0 * D * H * causal_pairs(n) * 3 / 7)
+        add("attn_bwd_dkdv_tc", "flop", 10.0 * D * H * causal_pairs(n) * 4 / 7)
         add("gemm_dt", "flop", 2.0 * n * 32 * 3 * HD)
         add("gemm_dxn", "flop", 2.0 * n * h * 3 * HD)
         add("rmsnorm_rows", "byte", 2.0 * (S * h * 2) + 3.0 * n * h * 2 * 2)

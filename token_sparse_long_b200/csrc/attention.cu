@@ -12,6 +12,7 @@
 // a segment's key gradients exactly when its own queries have been processed.
 #include "attn_frag.cuh"
 #include "attn_tc.cuh"
+#include "attn_bwd_tc.cuh"
 
 namespace jenga {
 
@@ -383,6 +384,40 @@ jenga_status attn_backward_segment(const bf16* q, const bf16* k, const bf16* v, 
     ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();
+  }
+  if (s0 % 128 == 0) {
+    // tcgen05 path (segment starts are multiples of 128 tokens)
+    CUtensorMap tk128, tv128, tq64, tdo64, tq128, tdo128, tk64, tv64;
+    jenga_status e;
+    const uint64_t HDc = (uint64_t)H * AT_D;
+    if ((e = make_tmap_bf16(&tk128, k, n_cap, HDc, ld, 128)) != JENGA_OK) return e;
+    if ((e = make_tmap_bf16(&tv128, v, n_cap, HDc, ld, 128)) != JENGA_OK) return e;
+    if ((e = make_tmap_bf16(&tq64, q, n_cap, HDc, ld, 64)) != JENGA_OK) return e;
+    if ((e = make_tmap_bf16(&tdo64, dO, T, HDc, ld_do, 64)) != JENGA_OK) return e;
+    if ((e = make_tmap_bf16(&tq128, q, n_cap, HDc, ld, 128)) != JENGA_OK) return e;
+    if ((e = make_tmap_bf16(&tdo128, dO, T, HDc, ld_do, 128)) != JENGA_OK) return e;
+    if ((e = make_tmap_bf16(&tk64, k, n_cap, HDc, ld, 64)) != JENGA_OK) return e;
+    if ((e = make_tmap_bf16(&tv64, v, n_cap, HDc, ld, 64)) != JENGA_OK) return e;
+    JENGA_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DQ_SMEM));
+    JENGA_CUDA_TRY(
+        cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DKV_SMEM));
+    {
+      const int _ps = ::jenga::prof_begin("attn_bwd_dq_tc", st);
+      attn_bwd_dq_tc_kernel<<<dim3((T + 127) / 128, H), ABT_THREADS, DQ_SMEM, st>>>(
+          tq128, tdo128, tk64, tv64, lse, lse_ld, delta, delta_ld, dq, ld_dq, s0, n_valid, valid_mult, n_cap,
+          scale_log2, scale);
+      ::jenga::prof_end(_ps, st);
+    }
+    JENGA_LAUNCH_CHECK();
+    {
+      const int _ps = ::jenga::prof_begin("attn_bwd_dkdv_tc", st);
+      attn_bwd_dkdv_tc_kernel<<<dim3((s1 + 127) / 128, H), ABT_THREADS, DKV_SMEM, st>>>(
+          tk128, tv128, tq64, tdo64, lse, lse_ld, delta, delta_ld, dk_acc, dv_acc, ld_acc, s0, s1, n_valid,
+          valid_mult, n_cap, scale_log2, scale);
+      ::jenga::prof_end(_ps, st);
+    }
+    JENGA_LAUNCH_CHECK();
+    return JENGA_OK;
   }
   JENGA_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATTN_BWD_SMEM));
   JENGA_CUDA_TRY(

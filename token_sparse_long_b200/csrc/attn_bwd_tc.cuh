@@ -1,0 +1,488 @@
+// tcgen05 causal attention backward over the retained tokens (head_dim 128), one query
+// segment [s0, s1) at a time (the segment-wise gradient schedule of the layer backward).
+//
+//   dK/dV pass  one CTA per (128-key tile, head).  K and V resident in smem; the segment's
+//               64-query tiles of Q and dO stream through a 2-stage TMA ring.  Per tile:
+//                 S^T  = K Q^T        dP^T = V dO^T           (TMEM, double-buffered)
+//                 P^T  = 2^(S^T log2e/sqrt(D) - L_q),  dS^T = P^T (dP^T - Delta_q)   (epilogue)
+//                 dV  += P^T dO       dK  += dS^T Q           (A: smem K-major, B: MN-major)
+//               and at the end dV, dK (x 1/sqrt(D)) are added into fp32 accumulators.
+//   dQ pass     one CTA per (128-query tile of the segment, head).  Q and dO resident; the
+//               64-key tiles of K and V stream.  S = Q K^T, dP = dO V^T, dS = P (dP - Delta),
+//               dQ += dS K; dQ (x 1/sqrt(D)) stored fp32.
+// Warp roles: 0 TMA, 1 TMEM allocation + MMA issue, 2..9 epilogue in two quads: each quad
+// covers all 128 TMEM lanes (one row per thread), quad 0 the first 32 columns of a tile and
+// quad 1 the last 32.  P / dS tiles are double-buffered in shared memory so the epilogue of
+// tile i overlaps the gradient products of tile i-1 and the score products of tile i+1.
+// Causal masking, keys / queries past the valid count, and the segment bounds are applied
+// in the epilogue.  Every wait is bounded; waits that guard collective TMEM loads are voted.
+#pragma once
+
+#include "common.cuh"
+
+namespace jenga {
+
+constexpr int ABT_BOX128 = 128 * 64 * 2;   // 16 KB box: 128 rows x 64 bf16
+constexpr int ABT_BOX64 = 64 * 64 * 2;     // 8 KB box: 64 rows x 64 bf16
+constexpr int ABT_THREADS = 320;
+
+// smem layout of the dK/dV pass
+constexpr int DKV_K_OFF = 0;                               // 2 x 16 KB
+constexpr int DKV_V_OFF = 2 * ABT_BOX128;                  // 2 x 16 KB
+constexpr int DKV_RING_OFF = 4 * ABT_BOX128;               // stage s: Q (2 x 8 KB), dO (2 x 8 KB)
+constexpr int DKV_STAGE = 4 * ABT_BOX64;
+constexpr int DKV_PT_OFF = DKV_RING_OFF + 2 * DKV_STAGE;  // [2] x 128 x 64 bf16
+constexpr int DKV_DST_OFF = DKV_PT_OFF + 2 * ABT_BOX128;  // [2] x 128 x 64 bf16
+constexpr int DKV_BAR_OFF = DKV_DST_OFF + 2 * ABT_BOX128;
+constexpr int DKV_SMEM = DKV_BAR_OFF + 256 + 1024;
+
+// smem layout of the dQ pass
+constexpr int DQ_Q_OFF = 0;
+constexpr int DQ_DO_OFF = 2 * ABT_BOX128;
+constexpr int DQ_RING_OFF = 4 * ABT_BOX128;                // stage s: K (2 x 8 KB), V (2 x 8 KB)
+constexpr int DQ_STAGE = 4 * ABT_BOX64;
+constexpr int DQ_DS_OFF = DQ_RING_OFF + 2 * DQ_STAGE;      // [2] x 128 x 64 bf16
+constexpr int DQ_BAR_OFF = DQ_DS_OFF + 2 * ABT_BOX128;
+constexpr int DQ_SMEM = DQ_BAR_OFF + 256 + 1024;
+
+// Write 32 bf16 values (packed pairs pk[0..15]) as columns [32 * half, 32 * half + 32) of
+// row r of a 128 x 64 K-major tile with the 128-byte swizzle (row = 8 chunks of 16 bytes).
+__device__ __forceinline__ void st_row32_sw128(uint8_t* tile, int r, int half, const uint32_t* pk) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int ch = half * 4 + c;
+    *reinterpret_cast<uint4*>(tile + r * 128 + ((ch ^ (r & 7)) << 4)) =
+        make_uint4(pk[c * 4], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// ------------------------------------------------------------------ dK / dV
+__global__ void __launch_bounds__(ABT_THREADS, 1)
+    attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                            const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                            const float* __restrict__ lse, int64_t lse_ld, const float* __restrict__ delta,
+                            int64_t delta_ld, float* __restrict__ dk_acc, float* __restrict__ dv_acc, int64_t ld_acc,
+                            int s0, int s1, const int32_t* __restrict__ n_valid, int valid_mult, int n_cap,
+                            float scale_log2, float scale) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DKV_BAR_OFF);
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = bars + 1;      // [2]
+  uint64_t* q_empty = q_full + 2;   // [2]
+  uint64_t* s_full = q_empty + 2;   // [2]
+  uint64_t* s_free = s_full + 2;    // [2]
+  uint64_t* pd_full = s_free + 2;   // [2]
+  uint64_t* pd_free = pd_full + 2;  // [2]
+  uint64_t* done = pd_free + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  int n = n_valid ? (*n_valid) * valid_mult : n_cap;
+  n = n < n_cap ? n : n_cap;
+  const int send = min(s1, n);
+  const int k0 = blockIdx.x * 128;
+  if (k0 >= send || s0 >= send) return;
+  const int qa0 = max(k0, s0) >> 6;  // first 64-query tile
+  const int qa1 = (send + 63) >> 6;  // one past the last
+  const int nq = qa1 - qa0;
+  if (nq <= 0) return;
+  const int col = h * 128;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], 8);
+      mbar_init(&pd_full[s], 8);
+      mbar_init(&pd_free[s], 1);
+    }
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  // TMEM columns: S^T[2] at 0, 64; dP^T[2] at 128, 192; dV at 256; dK at 384
+  const uint32_t tdV = tmem + 256, tdK = tmem + 384;
+
+  if (warp == 0 && lane == 0) {
+    mbar_arrive_expect_tx(kv_full, 4 * ABT_BOX128);
+    tma_load_2d(smem + DKV_K_OFF, &tmK, kv_full, col, k0);
+    tma_load_2d(smem + DKV_K_OFF + ABT_BOX128, &tmK, kv_full, col + 64, k0);
+    tma_load_2d(smem + DKV_V_OFF, &tmV, kv_full, col, k0);
+    tma_load_2d(smem + DKV_V_OFF + ABT_BOX128, &tmV, kv_full, col + 64, k0);
+    for (int i = 0; i < nq; ++i) {
+      const int s = i & 1;
+      if (i >= 2 && !mbar_wait_at(&q_empty[s], ((i >> 1) - 1) & 1, 121, i)) break;
+      uint8_t* st = smem + DKV_RING_OFF + s * DKV_STAGE;
+      const int qrow = (qa0 + i) * 64;
+      mbar_arrive_expect_tx(&q_full[s], DKV_STAGE);
+      tma_load_2d(st, &tmQ, &q_full[s], col, qrow);
+      tma_load_2d(st + ABT_BOX64, &tmQ, &q_full[s], col + 64, qrow);
+      tma_load_2d(st + 2 * ABT_BOX64, &tmDO, &q_full[s], col, qrow - s0);
+      tma_load_2d(st + 3 * ABT_BOX64, &tmDO, &q_full[s], col + 64, qrow - s0);
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64);
+    constexpr uint32_t idesc_g = umma_idesc_bf16_bmn(128, 128);
+    const uint32_t ka = smem_u32(smem + DKV_K_OFF), va = smem_u32(smem + DKV_V_OFF);
+    bool ok = mbar_wait_at(kv_full, 0, 122, 0);
+    auto issue_grad = [&](int ii) -> bool {
+      const int b = ii & 1;
+      if (!mbar_wait_at(&pd_full[b], (ii >> 1) & 1, 123, ii)) return false;
+      tc_fence_after();
+      const uint32_t st = smem_u32(smem + DKV_RING_OFF + b * DKV_STAGE);
+      const uint32_t qs = st, dos = st + 2 * ABT_BOX64;
+      const uint32_t pta = smem_u32(smem + DKV_PT_OFF + b * ABT_BOX128);
+      const uint32_t dsa = smem_u32(smem + DKV_DST_OFF + b * ABT_BOX128);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {  // K = 64 queries in steps of 16
+        const uint32_t acc = (ii > 0 || ks > 0) ? 1u : 0u;
+        umma_bf16(tdV, umma_desc_k_sw128(pta + ks * 32), umma_desc_mn_sw128(dos + ks * 2048, ABT_BOX64), idesc_g,
+                  acc);
+        umma_bf16(tdK, umma_desc_k_sw128(dsa + ks * 32), umma_desc_mn_sw128(qs + ks * 2048, ABT_BOX64), idesc_g,
+                  acc);
+      }
+      umma_commit(&pd_free[b]);
+      umma_commit(&q_empty[b]);
+      return true;
+    };
+    for (int i = 0; ok && i < nq; ++i) {
+      const int s = i & 1;
+      if (!mbar_wait_at(&q_full[s], (i >> 1) & 1, 124, i)) {
+        ok = false;
+        break;
+      }
+      if (i >= 2 && !mbar_wait_at(&s_free[s], ((i >> 1) - 1) & 1, 125, i)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t st = smem_u32(smem + DKV_RING_OFF + s * DKV_STAGE);
+#pragma unroll
+      for (int kc = 0; kc < 2; ++kc)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t acc = (kc | k) ? 1u : 0u;
+          umma_bf16(tmem + s * 64, umma_desc_k_sw128(ka + kc * ABT_BOX128 + k * 32),
+                    umma_desc_k_sw128(st + kc * ABT_BOX64 + k * 32), idesc_s, acc);
+          umma_bf16(tmem + 128 + s * 64, umma_desc_k_sw128(va + kc * ABT_BOX128 + k * 32),
+                    umma_desc_k_sw128(st + 2 * ABT_BOX64 + kc * ABT_BOX64 + k * 32), idesc_s, acc);
+        }
+      umma_commit(&s_full[s]);
+      if (i >= 1 && !issue_grad(i - 1)) {
+        ok = false;
+        break;
+      }
+    }
+    if (ok && issue_grad(nq - 1)) umma_commit(done);
+  } else if (warp >= 2) {
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int r = quarter * 32 + lane;
+    const int key = k0 + r;
+    const uint32_t lo = (uint32_t)(quarter * 32) << 16;
+    const float* lb = lse + (int64_t)h * lse_ld;
+    const float* db = delta + (int64_t)h * delta_ld - s0;
+    bool ok = true;
+    for (int i = 0; i < nq; ++i) {
+      const int s = i & 1;
+      const int qbase = (qa0 + i) * 64 + half * 32;
+      // this half's 32 query log-sum-exps and Delta values (L1-resident: shared by all rows)
+      float4 L4[8], D4[8];
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4) {
+        L4[c4] = *reinterpret_cast<const float4*>(lb + qbase + 4 * c4);
+        D4[c4] = *reinterpret_cast<const float4*>(db + qbase + 4 * c4);
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait_at(&s_full[s], (i >> 1) & 1, 126, i))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sv[32], dp[32];
+      tmem_ld32_nowait(tmem + lo + s * 64 + half * 32, sv);
+      tmem_ld32_nowait(tmem + lo + 128 + s * 64 + half * 32, dp);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[s]);
+      uint32_t pk[16], dk[16];
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4) {
+        const float Ls[4] = {L4[c4].x, L4[c4].y, L4[c4].z, L4[c4].w};
+        const float Ds[4] = {D4[c4].x, D4[c4].y, D4[c4].z, D4[c4].w};
+        float p[4], d[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = 4 * c4 + e, q = qbase + c;
+          const bool valid = (q >= key) && (q < send);
+          const float pe =
+              valid ? fast_exp2(fmaf(__uint_as_float(sv[c]), scale_log2, -Ls[e] * 1.4426950408889634f)) : 0.f;
+          p[e] = pe;
+          d[e] = valid ? pe * (__uint_as_float(dp[c]) - Ds[e]) : 0.f;  // Delta past n is unset
+        }
+        pk[2 * c4] = pack_bf2(p[0], p[1]);
+        pk[2 * c4 + 1] = pack_bf2(p[2], p[3]);
+        dk[2 * c4] = pack_bf2(d[0], d[1]);
+        dk[2 * c4 + 1] = pack_bf2(d[2], d[3]);
+      }
+      // buffer s was last read by the gradient products of tile i-2
+      if (i >= 2 && !__all_sync(0xffffffffu, mbar_wait_at(&pd_free[s], ((i >> 1) - 1) & 1, 127, i))) {
+        ok = false;
+        break;
+      }
+      st_row32_sw128(smem + DKV_PT_OFF + s * ABT_BOX128, r, half, pk);
+      st_row32_sw128(smem + DKV_DST_OFF + s * ABT_BOX128, r, half, dk);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pd_full[s]);
+    }
+    if (__all_sync(0xffffffffu, ok && mbar_wait_at(done, 0, 128, nq))) {
+      tc_fence_after();
+      const bool row_ok = key < n;
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c0 = half * 64 + cc * 32;
+        uint32_t a[32], b[32];
+        tmem_ld32_nowait(tdV + lo + c0, a);
+        tmem_ld32_nowait(tdK + lo + c0, b);
+        tmem_wait_ld();
+        if (row_ok) {
+          float4* pv = reinterpret_cast<float4*>(dv_acc + (int64_t)key * ld_acc + col + c0);
+          float4* pk4 = reinterpret_cast<float4*>(dk_acc + (int64_t)key * ld_acc + col + c0);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            float4 x = pv[q4];
+            x.x += __uint_as_float(a[4 * q4]);
+            x.y += __uint_as_float(a[4 * q4 + 1]);
+            x.z += __uint_as_float(a[4 * q4 + 2]);
+            x.w += __uint_as_float(a[4 * q4 + 3]);
+            pv[q4] = x;
+            float4 y = pk4[q4];
+            y.x += __uint_as_float(b[4 * q4]) * scale;
+            y.y += __uint_as_float(b[4 * q4 + 1]) * scale;
+            y.z += __uint_as_float(b[4 * q4 + 2]) * scale;
+            y.w += __uint_as_float(b[4 * q4 + 3]) * scale;
+            pk4[q4] = y;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ dQ
+__global__ void __launch_bounds__(ABT_THREADS, 1)
+    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                          const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                          const float* __restrict__ lse, int64_t lse_ld, const float* __restrict__ delta,
+                          int64_t delta_ld, float* __restrict__ dq_out, int64_t ld_dq, int s0,
+                          const int32_t* __restrict__ n_valid, int valid_mult, int n_cap, float scale_log2,
+                          float scale) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DQ_BAR_OFF);
+  uint64_t* qd_full = bars;
+  uint64_t* kv_full = bars + 1;      // [2]
+  uint64_t* kv_empty = kv_full + 2;  // [2]
+  uint64_t* s_full = kv_empty + 2;   // [2]
+  uint64_t* s_free = s_full + 2;     // [2]
+  uint64_t* ds_full = s_free + 2;    // [2]
+  uint64_t* ds_free = ds_full + 2;   // [2]
+  uint64_t* done = ds_free + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  int n = n_valid ? (*n_valid) * valid_mult : n_cap;
+  n = n < n_cap ? n : n_cap;
+  const int qt = s0 / 128 + (gridDim.x - 1 - blockIdx.x);  // longest first
+  const int q0 = qt * 128;
+  if (q0 >= n) return;
+  const int kend = min(q0 + 128, n);
+  const int nk = (kend + 63) >> 6;
+  const int col = h * 128;
+
+  if (threadIdx.x == 0) {
+    mbar_init(qd_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], 8);
+      mbar_init(&ds_full[s], 8);
+      mbar_init(&ds_free[s], 1);
+    }
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t tdQ = tmem + 256;  // S[2] at 0, 64; dP[2] at 128, 192; dQ at 256
+
+  if (warp == 0 && lane == 0) {
+    mbar_arrive_expect_tx(qd_full, 4 * ABT_BOX128);
+    tma_load_2d(smem + DQ_Q_OFF, &tmQ, qd_full, col, q0);
+    tma_load_2d(smem + DQ_Q_OFF + ABT_BOX128, &tmQ, qd_full, col + 64, q0);
+    tma_load_2d(smem + DQ_DO_OFF, &tmDO, qd_full, col, q0 - s0);
+    tma_load_2d(smem + DQ_DO_OFF + ABT_BOX128, &tmDO, qd_full, col + 64, q0 - s0);
+    for (int j = 0; j < nk; ++j) {
+      const int s = j & 1;
+      if (j >= 2 && !mbar_wait_at(&kv_empty[s], ((j >> 1) - 1) & 1, 131, j)) break;
+      uint8_t* st = smem + DQ_RING_OFF + s * DQ_STAGE;
+      mbar_arrive_expect_tx(&kv_full[s], DQ_STAGE);
+      tma_load_2d(st, &tmK, &kv_full[s], col, j * 64);
+      tma_load_2d(st + ABT_BOX64, &tmK, &kv_full[s], col + 64, j * 64);
+      tma_load_2d(st + 2 * ABT_BOX64, &tmV, &kv_full[s], col, j * 64);
+      tma_load_2d(st + 3 * ABT_BOX64, &tmV, &kv_full[s], col + 64, j * 64);
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64);
+    constexpr uint32_t idesc_g = umma_idesc_bf16_bmn(128, 128);
+    const uint32_t qa = smem_u32(smem + DQ_Q_OFF), da = smem_u32(smem + DQ_DO_OFF);
+    bool ok = mbar_wait_at(qd_full, 0, 132, 0);
+    auto issue_dq = [&](int jj) -> bool {
+      const int b = jj & 1;
+      if (!mbar_wait_at(&ds_full[b], (jj >> 1) & 1, 133, jj)) return false;
+      tc_fence_after();
+      const uint32_t ks_ = smem_u32(smem + DQ_RING_OFF + b * DQ_STAGE);
+      const uint32_t dsa = smem_u32(smem + DQ_DS_OFF + b * ABT_BOX128);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        umma_bf16(tdQ, umma_desc_k_sw128(dsa + ks * 32), umma_desc_mn_sw128(ks_ + ks * 2048, ABT_BOX64), idesc_g,
+                  (jj > 0 || ks > 0) ? 1u : 0u);
+      umma_commit(&ds_free[b]);
+      umma_commit(&kv_empty[b]);
+      return true;
+    };
+    for (int j = 0; ok && j < nk; ++j) {
+      const int s = j & 1;
+      if (!mbar_wait_at(&kv_full[s], (j >> 1) & 1, 134, j)) {
+        ok = false;
+        break;
+      }
+      if (j >= 2 && !mbar_wait_at(&s_free[s], ((j >> 1) - 1) & 1, 135, j)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t st = smem_u32(smem + DQ_RING_OFF + s * DQ_STAGE);
+#pragma unroll
+      for (int kc = 0; kc < 2; ++kc)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t acc = (kc | k) ? 1u : 0u;
+          umma_bf16(tmem + s * 64, umma_desc_k_sw128(qa + kc * ABT_BOX128 + k * 32),
+                    umma_desc_k_sw128(st + kc * ABT_BOX64 + k * 32), idesc_s, acc);
+          umma_bf16(tmem + 128 + s * 64, umma_desc_k_sw128(da + kc * ABT_BOX128 + k * 32),
+                    umma_desc_k_sw128(st + 2 * ABT_BOX64 + kc * ABT_BOX64 + k * 32), idesc_s, acc);
+        }
+      umma_commit(&s_full[s]);
+      if (j >= 1 && !issue_dq(j - 1)) {
+        ok = false;
+        break;
+      }
+    }
+    if (ok && issue_dq(nk - 1)) umma_commit(done);
+  } else if (warp >= 2) {
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int r = quarter * 32 + lane;
+    const int q = q0 + r;
+    const uint32_t lo = (uint32_t)(quarter * 32) << 16;
+    const bool qvalid = q < n;
+    const float L = qvalid ? lse[(int64_t)h * lse_ld + q] * 1.4426950408889634f : 0.f;
+    const float Dq = qvalid ? delta[(int64_t)h * delta_ld + q - s0] : 0.f;
+    bool ok = true;
+    for (int j = 0; j < nk; ++j) {
+      const int s = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait_at(&s_full[s], (j >> 1) & 1, 136, j))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sv[32], dp[32];
+      tmem_ld32_nowait(tmem + lo + s * 64 + half * 32, sv);
+      tmem_ld32_nowait(tmem + lo + 128 + s * 64 + half * 32, dp);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[s]);
+      const int lim = qvalid ? min(q + 1, n) - j * 64 - half * 32 : 0;  // valid keys of this half: c < lim
+      uint32_t dk[16];
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) {
+        float d2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const bool valid = c + e < lim;
+          const float pe = valid ? fast_exp2(fmaf(__uint_as_float(sv[c + e]), scale_log2, -L)) : 0.f;
+          d2[e] = valid ? pe * (__uint_as_float(dp[c + e]) - Dq) : 0.f;
+        }
+        dk[c >> 1] = pack_bf2(d2[0], d2[1]);
+      }
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait_at(&ds_free[s], ((j >> 1) - 1) & 1, 137, j))) {
+        ok = false;
+        break;
+      }
+      st_row32_sw128(smem + DQ_DS_OFF + s * ABT_BOX128, r, half, dk);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ds_full[s]);
+    }
+    if (__all_sync(0xffffffffu, ok && mbar_wait_at(done, 0, 138, nk))) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c0 = half * 64 + cc * 32;
+        uint32_t a[32];
+        tmem_ld32_nowait(tdQ + lo + c0, a);
+        tmem_wait_ld();
+        if (qvalid) {
+          float4* dst = reinterpret_cast<float4*>(dq_out + (int64_t)(q - s0) * ld_dq + col + c0);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            dst[q4] = make_float4(__uint_as_float(a[4 * q4]) * scale, __uint_as_float(a[4 * q4 + 1]) * scale,
+                                  __uint_as_float(a[4 * q4 + 2]) * scale, __uint_as_float(a[4 * q4 + 3]) * scale);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace jenga
