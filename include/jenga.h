@@ -269,6 +269,13 @@ JENGA_API jenga_status jenga_predict_blocks(const void* x, int B, int S, int h, 
 JENGA_API jenga_status jenga_test_gemm(const void* A, int64_t lda, const void* B, int64_t ldb, int M, int N, int K,
                                        void* C, int64_t ldc, int out_f32, int bn, jenga_stream_t stream);
 
+/**
+ * jenga_test_exp2 -- y_fma[i] = 2^x[i] by the FMA-pipe exponential the scoring kernel uses
+ * for part of its columns (cubic on [-1/2, 1/2] after a binary split of x, inputs clamped
+ * to [-125, 64]), and y_mufu[i] = 2^x[i] by the hardware approximation (ex2.approx.ftz).
+ * x, y_fma, y_mufu: device fp32 arrays of n elements.  For accuracy tests only. */
+JENGA_API jenga_status jenga_test_exp2(const float* x, float* y_fma, float* y_mufu, int n, jenga_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -22,7 +22,9 @@ def J():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     import token_sparse_long_b200 as J
+    from token_sparse_long_b200 import api
     J._lib.load()
+    J._api_test_exp2 = api.jenga_test_exp2
     return J
 
 
@@ -85,6 +87,51 @@ def test_score_bf16_against_oracle(J, S, H, causal):
     got = sc.cpu().numpy().astype(np.float64)
     assert np.all(np.abs(got - ref) / np.abs(ref) < 2e-2), np.abs(got - ref).max()
     assert abs(got.sum() - H * S) < 2e-3 * H * S
+
+
+def test_score_bf16_large_logit_jump(J):
+    # one key far along the sequence whose logit exceeds every earlier one by > 60 (log2
+    # units): rows that reach it must leave the pass-1 fast path and rescale exactly
+    S, H, D = 1024, 2, 128
+    g = torch.Generator(device="cuda").manual_seed(21)
+    u = torch.randn(H * D, device="cuda", generator=g)
+    q = (u + 0.5 * torch.randn(S, H * D, device="cuda", generator=g)).to(torch.bfloat16)
+    k = (0.25 * torch.randn(S, H * D, device="cuda", generator=g))
+    k[700] = 8.0 * u
+    k = k.to(torch.bfloat16)
+    sc = J.jenga_score_blocks(q, k, H, D, 64)
+    J.jenga_check_device_status()
+    ref = osc.block_scores_softmax_mass(torch_to_f64(q).reshape(S, H, D), torch_to_f64(k).reshape(S, H, D), 64)
+    got = sc.cpu().numpy().astype(np.float64)
+    assert ref[700 // 64] > 0.5 * H * (S - 700)  # the salient key's block takes most of the mass
+    # blocks past the salient key score ~1e-33: their pairs sit below the fp32 normal range
+    # (2^-126), where ex2 flushes and the FMA-pipe exponential floors at 2^-125, so the
+    # relative bar gets an absolute allowance of 2^-124 per (query, key, head) pair
+    floor = H * S * 64 * 2.0 ** -124
+    assert np.all(np.abs(got - ref) <= 2e-2 * np.abs(ref) + floor), np.abs(got - ref).max()
+    big = ref > 1e-20
+    assert np.all(np.abs(got - ref)[big] / ref[big] < 2e-2)
+    assert abs(got.sum() - H * S) < 2e-3 * H * S
+
+
+def test_exp2_fma_against_float64(J):
+    # the FMA-pipe exponential (cubic after a binary split) that scoring uses for part of
+    # its columns: relative error of the fitted cubic is 7.5e-5; clamped outside [-125, 64]
+    g = torch.Generator(device="cuda").manual_seed(3)
+    x = torch.cat([torch.linspace(-125.0, 64.0, 1 << 20, device="cuda"),
+                   torch.rand(1 << 20, device="cuda", generator=g) * 40.0 - 30.0,
+                   torch.tensor([0.0, -0.5, 0.5, -1.0, 1.0, -124.75, 63.5], device="cuda")])
+    y_fma, y_mufu = J._api_test_exp2(x)
+    xd = x.double().cpu()
+    ref = torch.exp2(xd)
+    rel = ((y_fma.double().cpu() - ref).abs() / ref).max().item()
+    assert rel < 1e-4, rel
+    rel_mufu = ((y_fma.double() - y_mufu.double()).abs() / y_mufu.double()).max().item()
+    assert rel_mufu < 2e-4, rel_mufu
+    lo = J._api_test_exp2(torch.tensor([-200.0, -1e30, -float("inf")], device="cuda"))[0].double().cpu()
+    assert torch.all(lo <= 2.0 ** -125 * 1.5) and torch.all(lo > 0)
+    hi = J._api_test_exp2(torch.tensor([100.0, 1e30], device="cuda"))[0].double().cpu()
+    assert torch.all(torch.isfinite(hi)) and torch.all(hi >= 2.0 ** 63)
 
 
 def test_score_bf16_fused_qk_buffer_and_batch(J):

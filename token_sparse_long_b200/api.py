@@ -262,3 +262,12 @@ def jenga_test_gemm(a, b, out_f32=True, bn=256, stream=None):
     check(load().jenga_test_gemm(_p(a), a.stride(0), _p(b), b.stride(0), M, N, K, _p(c), c.stride(0),
                                  1 if out_f32 else 0, bn, _stream(stream)))
     return c
+
+
+def jenga_test_exp2(x, stream=None):
+    """(2^x by the FMA-pipe exponential, 2^x by ex2.approx) for fp32 device x (test hook)."""
+    x = x.contiguous()
+    y_fma = torch.empty_like(x)
+    y_mufu = torch.empty_like(x)
+    check(load().jenga_test_exp2(_p(x), _p(y_fma), _p(y_mufu), x.numel(), _stream(stream)))
+    return y_fma, y_mufu

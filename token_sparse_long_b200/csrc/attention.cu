@@ -17,118 +17,10 @@
 namespace jenga {
 
 constexpr float LOG2E = 1.4426950408889634f;
-constexpr float LN2 = 0.6931471805599453f;
 
 __device__ __forceinline__ int attn_rows(const int32_t* n_valid, int mult, int cap) {
   int n = n_valid ? (*n_valid) * mult : cap;
   return n < cap ? n : cap;
-}
-
-// ------------------------------------------------------------------ forward
-__global__ void __launch_bounds__(128) attn_fwd_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
-                                                       const bf16* __restrict__ v, int64_t ld, bf16* __restrict__ o,
-                                                       int64_t ldo, float* __restrict__ lse, int64_t lse_ld,
-                                                       const int32_t* __restrict__ n_valid, int valid_mult,
-                                                       int n_cap, float scale_log2) {
-  extern __shared__ __align__(128) uint8_t sm[];
-  const int h = blockIdx.y;
-  const int n = attn_rows(n_valid, valid_mult, n_cap);
-  const int qt = gridDim.x - 1 - blockIdx.x;  // longest rows first
-  const int q0 = qt * AT_ROWS;
-  if (q0 >= n) return;
-  const bf16* qh = q + h * AT_D;
-  const bf16* kh = k + h * AT_D;
-  const bf16* vh = v + h * AT_D;
-  uint8_t* sQ = sm;
-  uint8_t* sK[2] = {sm + AT_TILE_BYTES, sm + 3 * AT_TILE_BYTES};
-  uint8_t* sV[2] = {sm + 2 * AT_TILE_BYTES, sm + 4 * AT_TILE_BYTES};
-  load_tile_async(sQ, qh, ld, q0, n);
-  load_tile_async(sK[0], kh, ld, 0, n);
-  load_tile_async(sV[0], vh, ld, 0, n);
-  cp_async_commit();
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int row0 = q0 + warp * 16 + g, row1 = row0 + 8;
-  float acc[16][4];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  uint32_t qa[8][4];
-  const int nkt = qt + 1;
-  for (int kt = 0; kt < nkt; ++kt) {
-    if (kt + 1 < nkt) {
-      load_tile_async(sK[(kt + 1) & 1], kh, ld, (kt + 1) * AT_ROWS, n);
-      load_tile_async(sV[(kt + 1) & 1], vh, ld, (kt + 1) * AT_ROWS, n);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    if (kt == 0) {
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) ld_a(sQ, warp * 16, ks * 16, qa[ks]);
-    }
-    float s[8][4];
-    mm_regs_x_rowsT(qa, sK[kt & 1], s);
-    const bool diag = (kt == qt);
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int col = kt * AT_ROWS + j * 8 + 2 * t + e;
-        s[j][e] = (!diag || col <= row0) ? s[j][e] * scale_log2 : -INFINITY;
-        s[j][2 + e] = (!diag || col <= row1) ? s[j][2 + e] * scale_log2 : -INFINITY;
-        mx0 = fmaxf(mx0, s[j][e]);
-        mx1 = fmaxf(mx1, s[j][2 + e]);
-      }
-    }
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float c0 = exp2f(m0 - mn0), c1 = exp2f(m1 - mn1);
-    l0 *= c0;
-    l1 *= c1;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      acc[i][0] *= c0;
-      acc[i][1] *= c0;
-      acc[i][2] *= c1;
-      acc[i][3] *= c1;
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      s[j][0] = exp2f(s[j][0] - mn0);
-      s[j][1] = exp2f(s[j][1] - mn0);
-      s[j][2] = exp2f(s[j][2] - mn1);
-      s[j][3] = exp2f(s[j][3] - mn1);
-      l0 += s[j][0] + s[j][1];
-      l1 += s[j][2] + s[j][3];
-    }
-    m0 = mn0;
-    m1 = mn1;
-    mm_p_x_cols(s, sV[kt & 1], acc);
-    __syncthreads();
-  }
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  const float i0 = 1.f / l0, i1 = 1.f / l1;
-  bf16* o0 = o + (int64_t)row0 * ldo + h * AT_D;
-  bf16* o1 = o + (int64_t)row1 * ldo + h * AT_D;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    *reinterpret_cast<uint32_t*>(o0 + i * 8 + 2 * t) = pack2(acc[i][0] * i0, acc[i][1] * i0);
-    *reinterpret_cast<uint32_t*>(o1 + i * 8 + 2 * t) = pack2(acc[i][2] * i1, acc[i][3] * i1);
-  }
-  if (t == 0) {
-    lse[(int64_t)h * lse_ld + row0] = (m0 + log2f(l0)) * LN2;
-    lse[(int64_t)h * lse_ld + row1] = (m1 + log2f(l1)) * LN2;
-  }
 }
 
 // ------------------------------------------------------------------ backward helpers
@@ -177,7 +69,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(
   cp_async_commit();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int row0 = q0 + warp * 16 + g, row1 = row0 + 8;
-  const float L0 = lse[(int64_t)h * lse_ld + row0] * LOG2E, L1 = lse[(int64_t)h * lse_ld + row1] * LOG2E;
+  const float L0 = lse[(int64_t)h * lse_ld + row0], L1 = lse[(int64_t)h * lse_ld + row1];  // log2 units
   const float D0 = delta[(int64_t)h * delta_ld + row0 - s0], D1 = delta[(int64_t)h * delta_ld + row1 - s0];
   float dq[16][4];
 #pragma unroll
@@ -259,7 +151,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(
     load_tile_async(sO[buf], dO + h * AT_D, ld_do, qt * AT_ROWS - s0, n - s0);
     if (threadIdx.x < AT_ROWS) {
       const int r = qt * AT_ROWS + threadIdx.x;
-      sL[buf][threadIdx.x] = (r < n) ? lse[(int64_t)h * lse_ld + r] * LOG2E : 0.f;
+      sL[buf][threadIdx.x] = (r < n) ? lse[(int64_t)h * lse_ld + r] : 0.f;  // log2 units
       sD[buf][threadIdx.x] = (r < n) ? delta[(int64_t)h * delta_ld + r - s0] : 0.f;
     }
   };
@@ -331,7 +223,6 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(
 }
 
 // ------------------------------------------------------------------ host launchers
-constexpr int ATTN_FWD_SMEM = 5 * AT_TILE_BYTES;
 constexpr int ATTN_BWD_SMEM = 6 * AT_TILE_BYTES;
 
 jenga_status attn_forward(const bf16* q, const bf16* k, const bf16* v, int64_t ld, bf16* o, int64_t ldo, float* lse,
@@ -340,8 +231,8 @@ jenga_status attn_forward(const bf16* q, const bf16* k, const bf16* v, int64_t l
   if (n_cap % AT_ROWS) return fail(JENGA_EINVAL, "attention: rows must be a multiple of 64");
   const float scale_log2 = LOG2E / sqrtf((float)AT_D);
   {
-    // tcgen05 path: TMA-fed 128-row tiles (rows of q/k/v past the valid count must be
-    // finite: the layer zeroes them before this call)
+    // TMA-fed 128-row tiles (rows of q/k/v past the valid count must be finite: the layer
+    // zeroes them before this call)
     CUtensorMap tq, tk, tv;
     jenga_status s1;
     if ((s1 = make_tmap_bf16(&tq, q, n_cap, (uint64_t)H * AT_D, ld, ATC_ROWS)) != JENGA_OK) return s1;
@@ -355,15 +246,6 @@ jenga_status attn_forward(const bf16* q, const bf16* k, const bf16* v, int64_t l
     JENGA_LAUNCH_CHECK();
     return JENGA_OK;
   }
-  JENGA_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATTN_FWD_SMEM));
-  {
-  const int _ps = ::jenga::prof_begin("attn_fwd", st);
-  attn_fwd_kernel<<<dim3(n_cap / AT_ROWS, H), 128, ATTN_FWD_SMEM, st>>>(q, k, v, ld, o, ldo, lse, lse_ld, n_valid,
-                                                                       valid_mult, n_cap, scale_log2);
-  ::jenga::prof_end(_ps, st);
-  }
-  JENGA_LAUNCH_CHECK();
-  return JENGA_OK;
 }
 
 jenga_status attn_backward_segment(const bf16* q, const bf16* k, const bf16* v, int64_t ld, const bf16* o,
@@ -385,8 +267,11 @@ jenga_status attn_backward_segment(const bf16* q, const bf16* k, const bf16* v, 
     }
     JENGA_LAUNCH_CHECK();
   }
-  if (s0 % 128 == 0) {
-    // tcgen05 path (segment starts are multiples of 128 tokens)
+  const bool bulk_ok = lse_ld % 4 == 0 && delta_ld % 4 == 0 && ((uintptr_t)lse & 15) == 0 &&
+                       ((uintptr_t)delta & 15) == 0;
+  if (s0 % 128 == 0 && bulk_ok) {
+    // tcgen05 path (segment starts are multiples of 128 tokens; L and Delta rows are
+    // bulk-copied, so their pitches and bases must be 16-byte multiples)
     CUtensorMap tk128, tv128, tq64, tdo64, tq128, tdo128, tk64, tv64;
     jenga_status e;
     const uint64_t HDc = (uint64_t)H * AT_D;

@@ -2,14 +2,19 @@
 // segment [s0, s1) at a time (the segment-wise gradient schedule of the layer backward).
 //
 //   dK/dV pass  one CTA per (128-key tile, head).  K and V resident in smem; the segment's
-//               64-query tiles of Q and dO stream through a 2-stage TMA ring.  Per tile:
+//               64-query tiles of Q and dO stream through a 3-stage TMA ring.  Per tile:
 //                 S^T  = K Q^T        dP^T = V dO^T           (TMEM, double-buffered)
-//                 P^T  = 2^(S^T log2e/sqrt(D) - L_q),  dS^T = P^T (dP^T - Delta_q)   (epilogue)
+//                 P^T  = 2^(S^T log2e/sqrt(D) - L_q),  dS^T = P^T (dP^T - Delta_q)   (epilogue;
+//                 L_q, the forward's row log-sum-exp in log2 units, and Delta_q ride in the
+//                 Q / dO stage as two 256-byte bulk copies)
 //                 dV  += P^T dO       dK  += dS^T Q           (A: smem K-major, B: MN-major)
 //               and at the end dV, dK (x 1/sqrt(D)) are added into fp32 accumulators.
 //   dQ pass     one CTA per (128-query tile of the segment, head).  Q and dO resident; the
 //               64-key tiles of K and V stream.  S = Q K^T, dP = dO V^T, dS = P (dP - Delta),
 //               dQ += dS K; dQ (x 1/sqrt(D)) stored fp32.
+// The Q/dO (K/V) ring is 3 (4) stages deep: a stage is read by both products of its tile,
+// so with 2 stages the next tile's load could only start once the gradient product that
+// immediately precedes that tile's score product had finished.
 // Warp roles: 0 TMA, 1 TMEM allocation + MMA issue, 2..9 epilogue in two quads: each quad
 // covers all 128 TMEM lanes (one row per thread), quad 0 the first 32 columns of a tile and
 // quad 1 the last 32.  P / dS tiles are double-buffered in shared memory so the epilogue of
@@ -31,9 +36,12 @@ constexpr int DKV_K_OFF = 0;                               // 2 x 16 KB
 constexpr int DKV_V_OFF = 2 * ABT_BOX128;                  // 2 x 16 KB
 constexpr int DKV_RING_OFF = 4 * ABT_BOX128;               // stage s: Q (2 x 8 KB), dO (2 x 8 KB)
 constexpr int DKV_STAGE = 4 * ABT_BOX64;
-constexpr int DKV_PT_OFF = DKV_RING_OFF + 2 * DKV_STAGE;  // [2] x 128 x 64 bf16
+constexpr int DKV_STAGES = 3;  // a stage lives from S^T(i) to the gradient products of tile i
+constexpr int DKV_PT_OFF = DKV_RING_OFF + DKV_STAGES * DKV_STAGE;  // [2] x 128 x 64 bf16
 constexpr int DKV_DST_OFF = DKV_PT_OFF + 2 * ABT_BOX128;  // [2] x 128 x 64 bf16
-constexpr int DKV_BAR_OFF = DKV_DST_OFF + 2 * ABT_BOX128;
+constexpr int DKV_LD_OFF = DKV_DST_OFF + 2 * ABT_BOX128;  // stage s: L (64 fp32), Delta (64 fp32)
+constexpr int DKV_LD_BYTES = 512;
+constexpr int DKV_BAR_OFF = DKV_LD_OFF + DKV_STAGES * DKV_LD_BYTES;
 constexpr int DKV_SMEM = DKV_BAR_OFF + 256 + 1024;
 
 // smem layout of the dQ pass
@@ -41,7 +49,8 @@ constexpr int DQ_Q_OFF = 0;
 constexpr int DQ_DO_OFF = 2 * ABT_BOX128;
 constexpr int DQ_RING_OFF = 4 * ABT_BOX128;                // stage s: K (2 x 8 KB), V (2 x 8 KB)
 constexpr int DQ_STAGE = 4 * ABT_BOX64;
-constexpr int DQ_DS_OFF = DQ_RING_OFF + 2 * DQ_STAGE;      // [2] x 128 x 64 bf16
+constexpr int DQ_STAGES = 4;  // a stage lives from S(j) to the dQ product of tile j
+constexpr int DQ_DS_OFF = DQ_RING_OFF + DQ_STAGES * DQ_STAGE;  // [2] x 128 x 64 bf16
 constexpr int DQ_BAR_OFF = DQ_DS_OFF + 2 * ABT_BOX128;
 constexpr int DQ_SMEM = DQ_BAR_OFF + 256 + 1024;
 
@@ -56,11 +65,6 @@ __device__ __forceinline__ void st_row32_sw128(uint8_t* tile, int r, int half, c
   }
 }
 
-__device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
 // ------------------------------------------------------------------ dK / dV
 __global__ void __launch_bounds__(ABT_THREADS, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -73,9 +77,9 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DKV_BAR_OFF);
   uint64_t* kv_full = bars;
-  uint64_t* q_full = bars + 1;      // [2]
-  uint64_t* q_empty = q_full + 2;   // [2]
-  uint64_t* s_full = q_empty + 2;   // [2]
+  uint64_t* q_full = bars + 1;                // [DKV_STAGES]
+  uint64_t* q_empty = q_full + DKV_STAGES;    // [DKV_STAGES]
+  uint64_t* s_full = q_empty + DKV_STAGES;    // [2]
   uint64_t* s_free = s_full + 2;    // [2]
   uint64_t* pd_full = s_free + 2;   // [2]
   uint64_t* pd_free = pd_full + 2;  // [2]
@@ -97,9 +101,11 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < DKV_STAGES; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&s_free[s], 8);
       mbar_init(&pd_full[s], 8);
@@ -126,15 +132,19 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     tma_load_2d(smem + DKV_V_OFF, &tmV, kv_full, col, k0);
     tma_load_2d(smem + DKV_V_OFF + ABT_BOX128, &tmV, kv_full, col + 64, k0);
     for (int i = 0; i < nq; ++i) {
-      const int s = i & 1;
-      if (i >= 2 && !mbar_wait_at(&q_empty[s], ((i >> 1) - 1) & 1, 121, i)) break;
+      const int s = i % DKV_STAGES;
+      if (i >= DKV_STAGES && !mbar_wait_at(&q_empty[s], ((i / DKV_STAGES) - 1) & 1, 121, i)) break;
       uint8_t* st = smem + DKV_RING_OFF + s * DKV_STAGE;
       const int qrow = (qa0 + i) * 64;
-      mbar_arrive_expect_tx(&q_full[s], DKV_STAGE);
+      uint8_t* ldst = smem + DKV_LD_OFF + s * DKV_LD_BYTES;
+      mbar_arrive_expect_tx(&q_full[s], DKV_STAGE + DKV_LD_BYTES);
       tma_load_2d(st, &tmQ, &q_full[s], col, qrow);
       tma_load_2d(st + ABT_BOX64, &tmQ, &q_full[s], col + 64, qrow);
       tma_load_2d(st + 2 * ABT_BOX64, &tmDO, &q_full[s], col, qrow - s0);
       tma_load_2d(st + 3 * ABT_BOX64, &tmDO, &q_full[s], col + 64, qrow - s0);
+      // the tile's 64 query log-sum-exps (log2 units) and Delta values
+      bulk_load_1d(ldst, lse + (int64_t)h * lse_ld + qrow, 256, &q_full[s]);
+      bulk_load_1d(ldst + 256, delta + (int64_t)h * delta_ld + (qrow - s0), 256, &q_full[s]);
     }
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64);
@@ -142,10 +152,10 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     const uint32_t ka = smem_u32(smem + DKV_K_OFF), va = smem_u32(smem + DKV_V_OFF);
     bool ok = mbar_wait_at(kv_full, 0, 122, 0);
     auto issue_grad = [&](int ii) -> bool {
-      const int b = ii & 1;
+      const int b = ii & 1, rs = ii % DKV_STAGES;
       if (!mbar_wait_at(&pd_full[b], (ii >> 1) & 1, 123, ii)) return false;
       tc_fence_after();
-      const uint32_t st = smem_u32(smem + DKV_RING_OFF + b * DKV_STAGE);
+      const uint32_t st = smem_u32(smem + DKV_RING_OFF + rs * DKV_STAGE);
       const uint32_t qs = st, dos = st + 2 * ABT_BOX64;
       const uint32_t pta = smem_u32(smem + DKV_PT_OFF + b * ABT_BOX128);
       const uint32_t dsa = smem_u32(smem + DKV_DST_OFF + b * ABT_BOX128);
@@ -158,12 +168,12 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
                   acc);
       }
       umma_commit(&pd_free[b]);
-      umma_commit(&q_empty[b]);
+      umma_commit(&q_empty[rs]);
       return true;
     };
     for (int i = 0; ok && i < nq; ++i) {
-      const int s = i & 1;
-      if (!mbar_wait_at(&q_full[s], (i >> 1) & 1, 124, i)) {
+      const int s = i & 1, rs = i % DKV_STAGES;
+      if (!mbar_wait_at(&q_full[rs], (i / DKV_STAGES) & 1, 124, i)) {
         ok = false;
         break;
       }
@@ -172,7 +182,7 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t st = smem_u32(smem + DKV_RING_OFF + s * DKV_STAGE);
+      const uint32_t st = smem_u32(smem + DKV_RING_OFF + rs * DKV_STAGE);
 #pragma unroll
       for (int kc = 0; kc < 2; ++kc)
 #pragma unroll
@@ -196,20 +206,14 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     const int r = quarter * 32 + lane;
     const int key = k0 + r;
     const uint32_t lo = (uint32_t)(quarter * 32) << 16;
-    const float* lb = lse + (int64_t)h * lse_ld;
-    const float* db = delta + (int64_t)h * delta_ld - s0;
     bool ok = true;
     for (int i = 0; i < nq; ++i) {
-      const int s = i & 1;
+      const int s = i & 1, rs = i % DKV_STAGES;
       const int qbase = (qa0 + i) * 64 + half * 32;
-      // this half's 32 query log-sum-exps and Delta values (L1-resident: shared by all rows)
-      float4 L4[8], D4[8];
-#pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
-        L4[c4] = *reinterpret_cast<const float4*>(lb + qbase + 4 * c4);
-        D4[c4] = *reinterpret_cast<const float4*>(db + qbase + 4 * c4);
-      }
-      if (!__all_sync(0xffffffffu, mbar_wait_at(&s_full[s], (i >> 1) & 1, 126, i))) {
+      // S^T(i) done implies the stage landed; the second wait makes the bulk-copied L and
+      // Delta visible to these threads (the stage cannot be refilled before pd_full(i))
+      if (!__all_sync(0xffffffffu, mbar_wait_at(&s_full[s], (i >> 1) & 1, 126, i) &&
+                                       mbar_wait_at(&q_full[rs], (i / DKV_STAGES) & 1, 129, i))) {
         ok = false;
         break;
       }
@@ -217,29 +221,51 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
       uint32_t sv[32], dp[32];
       tmem_ld32_nowait(tmem + lo + s * 64 + half * 32, sv);
       tmem_ld32_nowait(tmem + lo + 128 + s * 64 + half * 32, dp);
+      const float4* L4 = reinterpret_cast<const float4*>(smem + DKV_LD_OFF + rs * DKV_LD_BYTES) + half * 8;
+      const float4* D4 = L4 + 16;
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[s]);
       uint32_t pk[16], dk[16];
+      if (qbase >= key && qbase + 32 <= send) {  // every (query, key) pair of this row is live
 #pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
-        const float Ls[4] = {L4[c4].x, L4[c4].y, L4[c4].z, L4[c4].w};
-        const float Ds[4] = {D4[c4].x, D4[c4].y, D4[c4].z, D4[c4].w};
-        float p[4], d[4];
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 Lq = L4[c4], Dq = D4[c4];
+          const float Ls[4] = {Lq.x, Lq.y, Lq.z, Lq.w};
+          const float Ds[4] = {Dq.x, Dq.y, Dq.z, Dq.w};
+          float p[4], d[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = 4 * c4 + e, q = qbase + c;
-          const bool valid = (q >= key) && (q < send);
-          const float pe =
-              valid ? fast_exp2(fmaf(__uint_as_float(sv[c]), scale_log2, -Ls[e] * 1.4426950408889634f)) : 0.f;
-          p[e] = pe;
-          d[e] = valid ? pe * (__uint_as_float(dp[c]) - Ds[e]) : 0.f;  // Delta past n is unset
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * c4 + e;
+            p[e] = fast_exp2(fmaf(__uint_as_float(sv[c]), scale_log2, -Ls[e]));
+            d[e] = p[e] * (__uint_as_float(dp[c]) - Ds[e]);
+          }
+          pk[2 * c4] = pack_bf2(p[0], p[1]);
+          pk[2 * c4 + 1] = pack_bf2(p[2], p[3]);
+          dk[2 * c4] = pack_bf2(d[0], d[1]);
+          dk[2 * c4 + 1] = pack_bf2(d[2], d[3]);
         }
-        pk[2 * c4] = pack_bf2(p[0], p[1]);
-        pk[2 * c4 + 1] = pack_bf2(p[2], p[3]);
-        dk[2 * c4] = pack_bf2(d[0], d[1]);
-        dk[2 * c4 + 1] = pack_bf2(d[2], d[3]);
+      } else {  // causal diagonal or the segment's ragged end
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 Lq = L4[c4], Dq = D4[c4];
+          const float Ls[4] = {Lq.x, Lq.y, Lq.z, Lq.w};
+          const float Ds[4] = {Dq.x, Dq.y, Dq.z, Dq.w};
+          float p[4], d[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * c4 + e, q = qbase + c;
+            const bool valid = (q >= key) && (q < send);
+            const float pe = valid ? fast_exp2(fmaf(__uint_as_float(sv[c]), scale_log2, -Ls[e])) : 0.f;
+            p[e] = pe;
+            d[e] = valid ? pe * (__uint_as_float(dp[c]) - Ds[e]) : 0.f;  // L, Delta past n are unset
+          }
+          pk[2 * c4] = pack_bf2(p[0], p[1]);
+          pk[2 * c4 + 1] = pack_bf2(p[2], p[3]);
+          dk[2 * c4] = pack_bf2(d[0], d[1]);
+          dk[2 * c4 + 1] = pack_bf2(d[2], d[3]);
+        }
       }
       // buffer s was last read by the gradient products of tile i-2
       if (i >= 2 && !__all_sync(0xffffffffu, mbar_wait_at(&pd_free[s], ((i >> 1) - 1) & 1, 127, i))) {
@@ -305,9 +331,9 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DQ_BAR_OFF);
   uint64_t* qd_full = bars;
-  uint64_t* kv_full = bars + 1;      // [2]
-  uint64_t* kv_empty = kv_full + 2;  // [2]
-  uint64_t* s_full = kv_empty + 2;   // [2]
+  uint64_t* kv_full = bars + 1;               // [DQ_STAGES]
+  uint64_t* kv_empty = kv_full + DQ_STAGES;   // [DQ_STAGES]
+  uint64_t* s_full = kv_empty + DQ_STAGES;    // [2]
   uint64_t* s_free = s_full + 2;     // [2]
   uint64_t* ds_full = s_free + 2;    // [2]
   uint64_t* ds_free = ds_full + 2;   // [2]
@@ -327,9 +353,11 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(qd_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < DQ_STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&s_free[s], 8);
       mbar_init(&ds_full[s], 8);
@@ -355,8 +383,8 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     tma_load_2d(smem + DQ_DO_OFF, &tmDO, qd_full, col, q0 - s0);
     tma_load_2d(smem + DQ_DO_OFF + ABT_BOX128, &tmDO, qd_full, col + 64, q0 - s0);
     for (int j = 0; j < nk; ++j) {
-      const int s = j & 1;
-      if (j >= 2 && !mbar_wait_at(&kv_empty[s], ((j >> 1) - 1) & 1, 131, j)) break;
+      const int s = j % DQ_STAGES;
+      if (j >= DQ_STAGES && !mbar_wait_at(&kv_empty[s], ((j / DQ_STAGES) - 1) & 1, 131, j)) break;
       uint8_t* st = smem + DQ_RING_OFF + s * DQ_STAGE;
       mbar_arrive_expect_tx(&kv_full[s], DQ_STAGE);
       tma_load_2d(st, &tmK, &kv_full[s], col, j * 64);
@@ -370,22 +398,22 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     const uint32_t qa = smem_u32(smem + DQ_Q_OFF), da = smem_u32(smem + DQ_DO_OFF);
     bool ok = mbar_wait_at(qd_full, 0, 132, 0);
     auto issue_dq = [&](int jj) -> bool {
-      const int b = jj & 1;
+      const int b = jj & 1, rs = jj % DQ_STAGES;
       if (!mbar_wait_at(&ds_full[b], (jj >> 1) & 1, 133, jj)) return false;
       tc_fence_after();
-      const uint32_t ks_ = smem_u32(smem + DQ_RING_OFF + b * DQ_STAGE);
+      const uint32_t ks_ = smem_u32(smem + DQ_RING_OFF + rs * DQ_STAGE);
       const uint32_t dsa = smem_u32(smem + DQ_DS_OFF + b * ABT_BOX128);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
         umma_bf16(tdQ, umma_desc_k_sw128(dsa + ks * 32), umma_desc_mn_sw128(ks_ + ks * 2048, ABT_BOX64), idesc_g,
                   (jj > 0 || ks > 0) ? 1u : 0u);
       umma_commit(&ds_free[b]);
-      umma_commit(&kv_empty[b]);
+      umma_commit(&kv_empty[rs]);
       return true;
     };
     for (int j = 0; ok && j < nk; ++j) {
-      const int s = j & 1;
-      if (!mbar_wait_at(&kv_full[s], (j >> 1) & 1, 134, j)) {
+      const int s = j & 1, rs = j % DQ_STAGES;
+      if (!mbar_wait_at(&kv_full[rs], (j / DQ_STAGES) & 1, 134, j)) {
         ok = false;
         break;
       }
@@ -394,7 +422,7 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t st = smem_u32(smem + DQ_RING_OFF + s * DQ_STAGE);
+      const uint32_t st = smem_u32(smem + DQ_RING_OFF + rs * DQ_STAGE);
 #pragma unroll
       for (int kc = 0; kc < 2; ++kc)
 #pragma unroll
@@ -419,7 +447,7 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     const int q = q0 + r;
     const uint32_t lo = (uint32_t)(quarter * 32) << 16;
     const bool qvalid = q < n;
-    const float L = qvalid ? lse[(int64_t)h * lse_ld + q] * 1.4426950408889634f : 0.f;
+    const float L = qvalid ? lse[(int64_t)h * lse_ld + q] : 0.f;  // log2 units
     const float Dq = qvalid ? delta[(int64_t)h * delta_ld + q - s0] : 0.f;
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
@@ -438,16 +466,25 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
       if (lane == 0) mbar_arrive(&s_free[s]);
       const int lim = qvalid ? min(q + 1, n) - j * 64 - half * 32 : 0;  // valid keys of this half: c < lim
       uint32_t dk[16];
+      if (lim >= 32) {  // every key of this half is live for this row
 #pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        float d2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const bool valid = c + e < lim;
-          const float pe = valid ? fast_exp2(fmaf(__uint_as_float(sv[c + e]), scale_log2, -L)) : 0.f;
-          d2[e] = valid ? pe * (__uint_as_float(dp[c + e]) - Dq) : 0.f;
+        for (int c = 0; c < 32; c += 2) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c]), scale_log2, -L));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), scale_log2, -L));
+          dk[c >> 1] = pack_bf2(p0 * (__uint_as_float(dp[c]) - Dq), p1 * (__uint_as_float(dp[c + 1]) - Dq));
         }
-        dk[c >> 1] = pack_bf2(d2[0], d2[1]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          float d2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const bool valid = c + e < lim;
+            const float pe = valid ? fast_exp2(fmaf(__uint_as_float(sv[c + e]), scale_log2, -L)) : 0.f;
+            d2[e] = valid ? pe * (__uint_as_float(dp[c + e]) - Dq) : 0.f;
+          }
+          dk[c >> 1] = pack_bf2(d2[0], d2[1]);
+        }
       }
       if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait_at(&ds_free[s], ((j >> 1) - 1) & 1, 137, j))) {
         ok = false;

@@ -148,6 +148,31 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Named barrier over `threads` threads (a multiple of 32) that also returns the AND of
+// every participant's predicate: warps that must leave a loop together use it.
+__device__ __forceinline__ bool bar_and(bool v, int bar_id, int threads) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(bar_id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ bool pair_all(bool v, int bar_id) { return bar_and(v, bar_id, 64); }
+
+// 1D bulk copy global -> shared (both addresses and the size multiples of 16 bytes),
+// completion counted on an mbarrier.
+__device__ __forceinline__ void bulk_load_1d(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(smem_dst)),
+               "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -263,6 +288,24 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// 2^x on the FMA / integer pipes, for kernels whose exponentials would otherwise queue on
+// the multi-function unit (16 results per clock per SM).  Binary split x = j + f with j the
+// integer nearest x (the 1.5 * 2^23 shifter rounds x into the low mantissa bits) and
+// |f| <= 1/2; 2^f is a cubic whose relative error is equal-ripple on [-1/2, 1/2]
+// (coefficients from token_sparse_long_b200/exp2_fit.py, max relative error 7.5e-5);
+// 2^j is added into the exponent field.  Inputs are clamped to [-125, HI], so the result
+// is >= 2^-125.5 for very negative x and finite for large x.
+template <int HI = 64>
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fminf(fmaxf(x, -125.f), (float)HI);
+  const float t = __fadd_rn(x, 12582912.f);
+  const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
+  float p = fmaf(0x1.c3f760p-5f, f, 0x1.f0de1ap-3f);
+  p = fmaf(p, f, 0x1.62f31ap-1f);
+  p = fmaf(p, f, 0x1.fff692p-1f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 // Shared-memory matrix descriptor for a K-major tile whose rows are 128 bytes
 // (64 bf16), stored with the 128-byte swizzle in 1024-byte groups of 8 rows.
 __device__ __forceinline__ uint64_t umma_desc_k_sw128(uint32_t smem_addr) {
@@ -281,6 +324,12 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
 }
 
 __device__ __forceinline__ float bf16_to_f(bf16 v) { return __bfloat162float(v); }
+
+// two floats -> packed bf16 pair (round to nearest even), a in the low half
+__device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
 
 // ------------------------------------------------------------------ host helpers
 // Encode a 2D row-major bf16 tensor map (rows x cols, row pitch ld elements) with a

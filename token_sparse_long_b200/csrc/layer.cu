@@ -639,3 +639,22 @@ extern "C" jenga_status jenga_test_gemm(const void* A, int64_t lda, const void* 
   if (bn == 32) return launch_gemm<32, EPI_STORE_F32>({A, M, lda}, {B, N, ldb}, K, nullptr, nullptr, 0, M, N, e, st);
   return fail(JENGA_EINVAL, "jenga_test_gemm: bn must be 256 or 32");
 }
+
+// 2^x through exp2_fma (FMA-pipe exponential) and through the multi-function unit, for
+// accuracy tests of the former.
+__global__ void test_exp2_kernel(const float* __restrict__ x, float* __restrict__ y_fma, float* __restrict__ y_mufu,
+                                 int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    y_fma[i] = exp2_fma<64>(x[i]);
+    y_mufu[i] = fast_exp2(x[i]);
+  }
+}
+
+extern "C" jenga_status jenga_test_exp2(const float* x, float* y_fma, float* y_mufu, int n, jenga_stream_t stream) {
+  JENGA_CHECK_ARG(x && y_fma && y_mufu && n >= 0, "jenga_test_exp2: bad args");
+  if (n == 0) return JENGA_OK;
+  test_exp2_kernel<<<(n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024, 256, 0, (cudaStream_t)stream>>>(x, y_fma,
+                                                                                                     y_mufu, n);
+  JENGA_LAUNCH_CHECK();
+  return JENGA_OK;
+}
