@@ -15,7 +15,9 @@
 // The Q/dO (K/V) ring is 3 (4) stages deep: a stage is read by both products of its tile,
 // so with 2 stages the next tile's load could only start once the gradient product that
 // immediately precedes that tile's score product had finished.
-// Warp roles: 0 TMA, 1 TMEM allocation + MMA issue, 2..9 epilogue in two quads: each quad
+// Warp roles: 0 TMA, 1 and 2 MMA issue (1 also allocates TMEM; a warp can issue a
+// tcgen05.mma only every ~100 clocks, so one issuer would cap these M 128 x N 64 / N 128
+// products well below the tensor peak), 3..10 epilogue in two quads: each quad
 // covers all 128 TMEM lanes (one row per thread), quad 0 the first 32 columns of a tile and
 // quad 1 the last 32.  P / dS tiles are double-buffered in shared memory so the epilogue of
 // tile i overlaps the gradient products of tile i-1 and the score products of tile i+1.
@@ -29,7 +31,7 @@ namespace jenga {
 
 constexpr int ABT_BOX128 = 128 * 64 * 2;   // 16 KB box: 128 rows x 64 bf16
 constexpr int ABT_BOX64 = 64 * 64 * 2;     // 8 KB box: 64 rows x 64 bf16
-constexpr int ABT_THREADS = 320;
+constexpr int ABT_THREADS = 352;  // warps 0 TMA, 1 and 2 MMA issue, 3 .. 10 epilogue
 
 // smem layout of the dK/dV pass
 constexpr int DKV_K_OFF = 0;                               // 2 x 16 KB
@@ -103,15 +105,15 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     mbar_init(kv_full, 1);
     for (int s = 0; s < DKV_STAGES; ++s) {
       mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1);
+      mbar_init(&q_empty[s], 2);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
+      mbar_init(&s_full[s], 2);
       mbar_init(&s_free[s], 8);
       mbar_init(&pd_full[s], 8);
-      mbar_init(&pd_free[s], 1);
+      mbar_init(&pd_free[s], 2);
     }
-    mbar_init(done, 1);
+    mbar_init(done, 2);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -146,27 +148,30 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
       bulk_load_1d(ldst, lse + (int64_t)h * lse_ld + qrow, 256, &q_full[s]);
       bulk_load_1d(ldst + 256, delta + (int64_t)h * delta_ld + (qrow - s0), 256, &q_full[s]);
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if ((warp == 1 || warp == 2) && lane == 0) {
+    // two issuing warps (a warp can issue a tcgen05.mma only every ~100 clocks): warp 1
+    // issues S^T and dV (the P chain), warp 2 dP^T and dK (the dS chain); the barriers that
+    // both chains feed (s_full, pd_free, q_empty, done) count two commits
+    const bool pchain = (warp == 1);
     constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64);
     constexpr uint32_t idesc_g = umma_idesc_bf16_bmn(128, 128);
-    const uint32_t ka = smem_u32(smem + DKV_K_OFF), va = smem_u32(smem + DKV_V_OFF);
+    const uint32_t aa = smem_u32(smem + (pchain ? DKV_K_OFF : DKV_V_OFF));  // K or V: A of S^T / dP^T
+    const uint32_t acc_s = tmem + (pchain ? 0 : 128);                       // S^T[2] or dP^T[2]
+    const uint32_t acc_g = pchain ? tdV : tdK;
+    const int gbuf_off = pchain ? DKV_PT_OFF : DKV_DST_OFF;                 // P^T or dS^T tiles
+    const int b_g_off = pchain ? 2 * ABT_BOX64 : 0;                          // dO or Q: B of dV / dK
+    const int b_s_off = pchain ? 0 : 2 * ABT_BOX64;                          // Q or dO: B of S^T / dP^T
     bool ok = mbar_wait_at(kv_full, 0, 122, 0);
     auto issue_grad = [&](int ii) -> bool {
       const int b = ii & 1, rs = ii % DKV_STAGES;
       if (!mbar_wait_at(&pd_full[b], (ii >> 1) & 1, 123, ii)) return false;
       tc_fence_after();
-      const uint32_t st = smem_u32(smem + DKV_RING_OFF + rs * DKV_STAGE);
-      const uint32_t qs = st, dos = st + 2 * ABT_BOX64;
-      const uint32_t pta = smem_u32(smem + DKV_PT_OFF + b * ABT_BOX128);
-      const uint32_t dsa = smem_u32(smem + DKV_DST_OFF + b * ABT_BOX128);
+      const uint32_t bs = smem_u32(smem + DKV_RING_OFF + rs * DKV_STAGE + b_g_off);
+      const uint32_t ga = smem_u32(smem + gbuf_off + b * ABT_BOX128);
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {  // K = 64 queries in steps of 16
-        const uint32_t acc = (ii > 0 || ks > 0) ? 1u : 0u;
-        umma_bf16(tdV, umma_desc_k_sw128(pta + ks * 32), umma_desc_mn_sw128(dos + ks * 2048, ABT_BOX64), idesc_g,
-                  acc);
-        umma_bf16(tdK, umma_desc_k_sw128(dsa + ks * 32), umma_desc_mn_sw128(qs + ks * 2048, ABT_BOX64), idesc_g,
-                  acc);
-      }
+      for (int ks = 0; ks < 4; ++ks)  // K = 64 queries in steps of 16
+        umma_bf16(acc_g, umma_desc_k_sw128(ga + ks * 32), umma_desc_mn_sw128(bs + ks * 2048, ABT_BOX64), idesc_g,
+                  (ii > 0 || ks > 0) ? 1u : 0u);
       umma_commit(&pd_free[b]);
       umma_commit(&q_empty[rs]);
       return true;
@@ -182,17 +187,13 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t st = smem_u32(smem + DKV_RING_OFF + rs * DKV_STAGE);
+      const uint32_t st = smem_u32(smem + DKV_RING_OFF + rs * DKV_STAGE + b_s_off);
 #pragma unroll
       for (int kc = 0; kc < 2; ++kc)
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t acc = (kc | k) ? 1u : 0u;
-          umma_bf16(tmem + s * 64, umma_desc_k_sw128(ka + kc * ABT_BOX128 + k * 32),
-                    umma_desc_k_sw128(st + kc * ABT_BOX64 + k * 32), idesc_s, acc);
-          umma_bf16(tmem + 128 + s * 64, umma_desc_k_sw128(va + kc * ABT_BOX128 + k * 32),
-                    umma_desc_k_sw128(st + 2 * ABT_BOX64 + kc * ABT_BOX64 + k * 32), idesc_s, acc);
-        }
+        for (int k = 0; k < 4; ++k)
+          umma_bf16(acc_s + s * 64, umma_desc_k_sw128(aa + kc * ABT_BOX128 + k * 32),
+                    umma_desc_k_sw128(st + kc * ABT_BOX64 + k * 32), idesc_s, (kc | k) ? 1u : 0u);
       umma_commit(&s_full[s]);
       if (i >= 1 && !issue_grad(i - 1)) {
         ok = false;
@@ -200,9 +201,9 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
       }
     }
     if (ok && issue_grad(nq - 1)) umma_commit(done);
-  } else if (warp >= 2) {
+  } else if (warp >= 3) {
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int half = (warp - 3) >> 2;
     const int r = quarter * 32 + lane;
     const int key = k0 + r;
     const uint32_t lo = (uint32_t)(quarter * 32) << 16;
@@ -355,10 +356,10 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     mbar_init(qd_full, 1);
     for (int s = 0; s < DQ_STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], 2);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
+      mbar_init(&s_full[s], 2);
       mbar_init(&s_free[s], 8);
       mbar_init(&ds_full[s], 8);
       mbar_init(&ds_free[s], 1);
@@ -393,9 +394,10 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
       tma_load_2d(st + 3 * ABT_BOX64, &tmV, &kv_full[s], col + 64, j * 64);
     }
   } else if (warp == 1 && lane == 0) {
+    // warp 1 issues S and dQ; warp 2 issues dP (two issuers: see the dK/dV pass)
     constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64);
     constexpr uint32_t idesc_g = umma_idesc_bf16_bmn(128, 128);
-    const uint32_t qa = smem_u32(smem + DQ_Q_OFF), da = smem_u32(smem + DQ_DO_OFF);
+    const uint32_t qa = smem_u32(smem + DQ_Q_OFF);
     bool ok = mbar_wait_at(qd_full, 0, 132, 0);
     auto issue_dq = [&](int jj) -> bool {
       const int b = jj & 1, rs = jj % DQ_STAGES;
@@ -426,13 +428,9 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
 #pragma unroll
       for (int kc = 0; kc < 2; ++kc)
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t acc = (kc | k) ? 1u : 0u;
+        for (int k = 0; k < 4; ++k)
           umma_bf16(tmem + s * 64, umma_desc_k_sw128(qa + kc * ABT_BOX128 + k * 32),
-                    umma_desc_k_sw128(st + kc * ABT_BOX64 + k * 32), idesc_s, acc);
-          umma_bf16(tmem + 128 + s * 64, umma_desc_k_sw128(da + kc * ABT_BOX128 + k * 32),
-                    umma_desc_k_sw128(st + 2 * ABT_BOX64 + kc * ABT_BOX64 + k * 32), idesc_s, acc);
-        }
+                    umma_desc_k_sw128(st + kc * ABT_BOX64 + k * 32), idesc_s, (kc | k) ? 1u : 0u);
       umma_commit(&s_full[s]);
       if (j >= 1 && !issue_dq(j - 1)) {
         ok = false;
@@ -440,9 +438,28 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
       }
     }
     if (ok && issue_dq(nk - 1)) umma_commit(done);
-  } else if (warp >= 2) {
+  } else if (warp == 2 && lane == 0) {
+    constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64);
+    const uint32_t da = smem_u32(smem + DQ_DO_OFF);
+    bool ok = mbar_wait_at(qd_full, 0, 139, 0);
+    for (int j = 0; ok && j < nk; ++j) {
+      const int s = j & 1, rs = j % DQ_STAGES;
+      if (!mbar_wait_at(&kv_full[rs], (j / DQ_STAGES) & 1, 140, j)) break;
+      if (j >= 2 && !mbar_wait_at(&s_free[s], ((j >> 1) - 1) & 1, 141, j)) break;
+      tc_fence_after();
+      const uint32_t st = smem_u32(smem + DQ_RING_OFF + rs * DQ_STAGE);
+#pragma unroll
+      for (int kc = 0; kc < 2; ++kc)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_bf16(tmem + 128 + s * 64, umma_desc_k_sw128(da + kc * ABT_BOX128 + k * 32),
+                    umma_desc_k_sw128(st + 2 * ABT_BOX64 + kc * ABT_BOX64 + k * 32), idesc_s, (kc | k) ? 1u : 0u);
+      umma_commit(&s_full[s]);
+      umma_commit(&kv_empty[rs]);
+    }
+  } else if (warp >= 3) {
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int half = (warp - 3) >> 2;
     const int r = quarter * 32 + lane;
     const int q = q0 + r;
     const uint32_t lo = (uint32_t)(quarter * 32) << 16;

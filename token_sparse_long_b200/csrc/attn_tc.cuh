@@ -1,13 +1,13 @@
 // tcgen05 causal attention forward over the retained tokens (head_dim 128).
 //
-// One CTA per (128-query tile, head), 320 threads:
+// One CTA per (128-query tile, head), 352 threads:
 //   warp 0      TMA: the Q tile once, then K_j through a 2-stage ring and V_j through a
 //               3-stage ring (K_j is free once S_j is computed, V_j only after the PV
 //               product, so separate rings let each load start as early as it can)
 //   warp 1      TMEM allocation (S0 | S1 | O, 384 of 512 columns); one lane issues
 //                 S_j = Q K_j^T            (A = Q smem K-major, B = K_j smem K-major) into S[j % 2]
-//                 O  += P_{j-1} V_{j-1}    (A = P smem K-major, B = V smem MN-major) into O
-//   warps 2..9  softmax, one TMEM lane (= one query row) per thread and one half of the
+//   warp 2      one lane issues O += P_j V_j (A = P smem K-major, B = V smem MN-major) into O
+//   warps 3..10 softmax, one TMEM lane (= one query row) per thread and one half of the
 //               key columns per warp (warps w and w + 4 share rows and exchange their
 //               half-row maxima): load S_j, mask (causal diagonal, keys past n; only on
 //               those tiles), online max with lazy rescaling (O and l are rescaled in TMEM
@@ -35,7 +35,7 @@ constexpr int ATC_P_OFF = ATC_V_OFF + ATC_V_STAGES * ATC_TILE;
 constexpr int ATC_XM_OFF = ATC_P_OFF + ATC_TILE;           // [2 halves][128 rows] fp32 exchange
 constexpr int ATC_BAR_OFF = ATC_XM_OFF + 2 * 128 * 4;
 constexpr int ATC_SMEM = ATC_BAR_OFF + 256 + 1024;
-constexpr int ATC_THREADS = 320;
+constexpr int ATC_THREADS = 352;
 
 __global__ void __launch_bounds__(ATC_THREADS, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -117,35 +117,15 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
       tma_load_2d(vd + ATC_BOX, &tmV, &v_full[sv], col + 64, j * ATC_ROWS);
     }
   } else if (warp == 1 && lane == 0) {
+    // S_j = Q K_j^T (warp 2 issues the PV products: a warp can issue a tcgen05.mma only
+    // every ~100 clocks, so one issuer would cap these M 128 x N 128 products near 60%)
     constexpr uint32_t idesc_s = umma_idesc_bf16(128, 128);
-    constexpr uint32_t idesc_o = umma_idesc_bf16_bmn(128, 128);
     const uint32_t qa = smem_u32(smem + ATC_Q_OFF);
-    const uint32_t pa = smem_u32(smem + ATC_P_OFF);
     bool ok = mbar_wait_at(q_full, 0, 102, qt << 16);
-    auto issue_pv = [&](int jj) -> bool {
-      const int sv = jj % ATC_V_STAGES;
-      if (!mbar_wait_at(p_full, jj & 1, 103, (qt << 16) | jj)) return false;
-      if (!mbar_wait_at(&v_full[sv], (jj / ATC_V_STAGES) & 1, 111, (qt << 16) | jj)) return false;
-      tc_fence_after();
-      const uint32_t va = smem_u32(smem + ATC_V_OFF + sv * ATC_TILE);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        umma_bf16(tO, umma_desc_k_sw128(pa + (ks >> 2) * ATC_BOX + (ks & 3) * 32),
-                  umma_desc_mn_sw128(va + ks * 2048, ATC_BOX), idesc_o, (jj > 0 || ks > 0) ? 1u : 0u);
-      umma_commit(&v_empty[sv]);
-      umma_commit(pv_done);
-      return true;
-    };
     for (int j = 0; ok && j < nj; ++j) {
       const int s = j % ATC_K_STAGES, sb = j & 1;
-      if (!mbar_wait_at(&k_full[s], (j / ATC_K_STAGES) & 1, 104, (qt << 16) | j)) {
-        ok = false;
-        break;
-      }
-      if (j >= 2 && !mbar_wait_at(&s_free[sb], ((j >> 1) - 1) & 1, 105, (qt << 16) | j)) {
-        ok = false;
-        break;
-      }
+      if (!mbar_wait_at(&k_full[s], (j / ATC_K_STAGES) & 1, 104, (qt << 16) | j)) break;
+      if (j >= 2 && !mbar_wait_at(&s_free[sb], ((j >> 1) - 1) & 1, 105, (qt << 16) | j)) break;
       tc_fence_after();
       const uint32_t ka = smem_u32(smem + ATC_K_OFF + s * ATC_TILE);
 #pragma unroll
@@ -156,18 +136,30 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     umma_desc_k_sw128(ka + kc * ATC_BOX + k * 32), idesc_s, (kc | k) ? 1u : 0u);
       umma_commit(&k_empty[s]);
       umma_commit(&s_full[sb]);
-      if (j >= 1 && !issue_pv(j - 1)) {
-        ok = false;
-        break;
-      }
     }
-    if (ok) issue_pv(nj - 1);
-  } else if (warp >= 2) {
+  } else if (warp == 2 && lane == 0) {
+    // O += P_j V_j once the softmax has written P_j
+    constexpr uint32_t idesc_o = umma_idesc_bf16_bmn(128, 128);
+    const uint32_t pa = smem_u32(smem + ATC_P_OFF);
+    for (int j = 0; j < nj; ++j) {
+      const int sv = j % ATC_V_STAGES;
+      if (!mbar_wait_at(p_full, j & 1, 103, (qt << 16) | j)) break;
+      if (!mbar_wait_at(&v_full[sv], (j / ATC_V_STAGES) & 1, 111, (qt << 16) | j)) break;
+      tc_fence_after();
+      const uint32_t va = smem_u32(smem + ATC_V_OFF + sv * ATC_TILE);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        umma_bf16(tO, umma_desc_k_sw128(pa + (ks >> 2) * ATC_BOX + (ks & 3) * 32),
+                  umma_desc_mn_sw128(va + ks * 2048, ATC_BOX), idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
+      umma_commit(&v_empty[sv]);
+      umma_commit(pv_done);
+    }
+  } else if (warp >= 3) {
     // eight softmax warps: warp w reads TMEM lanes 32 * (w % 4) (its 32 query rows) and
-    // half hf = (w - 2) / 4 of every tile's 128 key columns; the two warps of a pair
+    // half hf = (w - 3) / 4 of every tile's 128 key columns; the two warps of a pair
     // (w, w + 4) exchange their half-row maxima through shared memory each tile
     const int quarter = warp & 3;
-    const int hf = (warp - 2) >> 2;
+    const int hf = (warp - 3) >> 2;
     const int r = quarter * 32 + lane;
     const int qrow = q0 + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;

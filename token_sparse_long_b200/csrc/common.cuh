@@ -207,6 +207,21 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 inputs, fp32 accumulate (kind::f16).  A sits in
+// tensor memory with row i in lane i and element k of the row in column k / 2 (bf16 pairs,
+// even k in the low half), so one K = 16 step spans 8 columns.  Reading A from tensor
+// memory instead of shared memory halves the shared-memory traffic of an M 128 x N 128 MMA,
+// which otherwise saturates shared-memory bandwidth before the tensor core.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on an mbarrier once all previously issued tcgen05.mma of this thread complete.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -258,6 +273,25 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Copy row r of a 128 x 128 bf16 tile held in shared memory as two 64-column boxes with the
+// 128-byte swizzle (the TMA layout) into tensor-memory columns [col, col + 64) of lane r,
+// in the A-operand layout of umma_bf16_ts.  Warp-collective (tcgen05.st).
+__device__ __forceinline__ void tile_row_to_tmem(const uint8_t* tile, int r, uint32_t taddr_lane_col) {
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    uint32_t w[32];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 q = *reinterpret_cast<const uint4*>(tile + b * 16384 + r * 128 + ((c ^ (r & 7)) << 4));
+      w[4 * c] = q.x;
+      w[4 * c + 1] = q.y;
+      w[4 * c + 2] = q.z;
+      w[4 * c + 3] = q.w;
+    }
+    tmem_st32(taddr_lane_col + b * 32, w);
+  }
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy
 // (tensor-core operand reads, TMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -288,6 +322,31 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction for two lanes' worth)
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // 2^x on the FMA / integer pipes, for kernels whose exponentials would otherwise queue on
 // the multi-function unit (16 results per clock per SM).  Binary split x = j + f with j the
 // integer nearest x (the 1.5 * 2^23 shifter rounds x into the low mantissa bits) and
@@ -304,6 +363,39 @@ __device__ __forceinline__ float exp2_fma(float x) {
   p = fmaf(p, f, 0x1.62f31ap-1f);
   p = fmaf(p, f, 0x1.fff692p-1f);
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Pair form of exp2_fma (same arithmetic, f32x2 instructions for the split and the cubic);
+// HI < 0 skips the upper clamp (callers whose inputs are known to be <= 0).
+template <int HI = 64>
+__device__ __forceinline__ uint64_t exp2_fma_x2(uint64_t x2) {
+  float x0, x1;
+  f2unpack(x2, x0, x1);
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  if constexpr (HI >= 0) {
+    x0 = fminf(x0, (float)HI);
+    x1 = fminf(x1, (float)HI);
+  }
+  const uint64_t x = f2pack(x0, x1);
+  const uint64_t t = fadd2(x, f2pack(12582912.f, 12582912.f));
+  const uint64_t j = fadd2(t, f2pack(-12582912.f, -12582912.f));
+  const uint64_t f = ffma2(j, f2pack(-1.f, -1.f), x);
+  uint64_t p = ffma2(f2pack(0x1.c3f760p-5f, 0x1.c3f760p-5f), f, f2pack(0x1.f0de1ap-3f, 0x1.f0de1ap-3f));
+  p = ffma2(p, f, f2pack(0x1.62f31ap-1f, 0x1.62f31ap-1f));
+  p = ffma2(p, f, f2pack(0x1.fff692p-1f, 0x1.fff692p-1f));
+  float p0, p1, t0, t1;
+  f2unpack(p, p0, p1);
+  f2unpack(t, t0, t1);
+  return f2pack(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
+                __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
+}
+
+// 2^x for both halves of a pair on the multi-function unit
+__device__ __forceinline__ uint64_t exp2_mufu_x2(uint64_t x2) {
+  float x0, x1;
+  f2unpack(x2, x0, x1);
+  return f2pack(fast_exp2(x0), fast_exp2(x1));
 }
 
 // Shared-memory matrix descriptor for a K-major tile whose rows are 128 bytes

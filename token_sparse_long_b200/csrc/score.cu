@@ -10,6 +10,7 @@
 // tiles of 64 queries x 64 keys.
 #include "attn_frag.cuh"
 #include "score_tc.cuh"
+#include "score_mass_tc.cuh"
 
 namespace jenga {
 
@@ -391,18 +392,18 @@ extern "C" jenga_status jenga_score_blocks(const void* q, int64_t ldq, const voi
       if (s1 != JENGA_OK) return s1;
       s1 = make_tmap_bf16(&tk, k, (uint64_t)B * S, (uint64_t)H * D, ldk, SCT_ROWS);
       if (s1 != JENGA_OK) return s1;
-      JENGA_CUDA_TRY(cudaFuncSetAttribute(score_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, SCT_SMEM));
-      JENGA_CUDA_TRY(cudaFuncSetAttribute(score_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, SCT_SMEM));
+      JENGA_CUDA_TRY(cudaFuncSetAttribute(score_lse_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SCT_SMEM));
+      JENGA_CUDA_TRY(cudaFuncSetAttribute(score_mass_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMT_SMEM));
       dim3 gt(S / SCT_ROWS, H, B);
       {
         const int _ps = ::jenga::prof_begin("score_lse_tc", st);
-        score_tc_kernel<0><<<gt, SCT_THREADS, SCT_SMEM, st>>>(tq, tk, S, H, causal ? 1 : 0, sl2, nullptr, lse);
+        score_lse_tc_kernel<<<gt, SCT_THREADS, SCT_SMEM, st>>>(tq, tk, S, H, causal ? 1 : 0, sl2, lse);
         ::jenga::prof_end(_ps, st);
       }
       JENGA_LAUNCH_CHECK();
       {
         const int _ps = ::jenga::prof_begin("score_mass_tc", st);
-        score_tc_kernel<1><<<gt, SCT_THREADS, SCT_SMEM, st>>>(tq, tk, S, H, causal ? 1 : 0, sl2, lse, mass);
+        score_mass_tc_kernel<<<gt, SMT_THREADS, SMT_SMEM, st>>>(tq, tk, S, H, causal ? 1 : 0, sl2, lse, mass);
         ::jenga::prof_end(_ps, st);
       }
       JENGA_LAUNCH_CHECK();
