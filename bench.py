@@ -43,6 +43,7 @@ def parse():
     ap.add_argument("--no-dense", action="store_true", help="skip the keep-all comparison")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-movement", action="store_true", help="skip the standalone gather/scatter/select timing")
     return ap.parse_args()
 
 
@@ -98,6 +99,25 @@ def work_model(case, ks, seg):
         add("rmsnorm_rows", "byte", 2.0 * (S * h * 2) + 3.0 * n * h * 2 * 2)
         add("select_small", "byte", 9.0 * (S // case.blk))
     return w
+
+
+# DRAM bytes per unit of work of a kernel, from one ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum; the capture and its command are in profiles/).  attn_bwd_dkdv_tc:
+# its traffic is dominated by the fp32 dK / dV accumulator read-modify-write and the K / V
+# reads, both proportional to the keys [0, segment end) a launch covers, so the unit is a key
+# row; captured on llama7b_s16k (one launch over 4096 keys: 269.5 MB read + 88.5 MB written).
+TRAFFIC_PER_UNIT = {"attn_bwd_dkdv_tc": ("key row", (269.52064e6 + 88.46208e6) / 4096)}
+
+
+def traffic_units(name, case, ks, seg):
+    """Units (as in TRAFFIC_PER_UNIT) a step's launches of kernel `name` process, summed."""
+    if name == "attn_bwd_dkdv_tc":
+        tot = 0
+        for k in ks:
+            n = k * case.blk
+            tot += sum(min(s0 + seg, n) for s0 in range(0, n, seg))
+        return tot
+    return None
 
 
 def step_flops(case, ks):
@@ -235,6 +255,57 @@ def full_step_flops(w, ks):
 
 
 # ---------------------------------------------------------------------------- GPU arm
+def measure_movement(J, torch, dev, X0, case, ks, hbm):
+    """Standalone timing of the HBM-bound entry points at the workload's sizes: gather and
+    scatter-add of layer 0's retained rows of X (bf16 [S, h]), and threshold selection
+    (ABS_GE) over 2^26 fp32 scores.  Algorithmic bytes: gather 2 n h e, scatter-add 3 n h e
+    (eliminated rows cost nothing), select 4 nb read + 4 n_kept + nb + 4 written.  Each
+    call moves more than the 126 MB L2; CUDA events, median of 10 after 3 warm-ups."""
+    blk, S, h = case.blk, case.S, X0.shape[1]
+    nb = S // blk
+    k0 = ks[0]
+    idx = torch.full((1, nb), -1, dtype=torch.int32, device=dev)
+    idx[0, :k0] = torch.arange(0, nb, nb / k0, device=dev).to(torch.int32)[:k0]  # spread over the sequence
+    nk = torch.tensor([k0], dtype=torch.int32, device=dev)
+    n = k0 * blk
+    xg = torch.empty(n, h, dtype=X0.dtype, device=dev)
+    x2 = X0.clone()
+
+    def med(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(10):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) / 1e3)
+        return sorted(ts)[len(ts) // 2]
+
+    out = {}
+    t = med(lambda: J.jenga_gather(X0, idx, nk, blk, n, out=xg))
+    by = 2.0 * n * h * X0.element_size()
+    out["gather"] = {"rows": n, "bytes": by, "us": t * 1e6, "gbs": by / t / 1e9, "frac_hbm": by / t / 1e9 / hbm}
+    t = med(lambda: J.jenga_scatter_add(x2, xg, idx, nk, blk, 1.0))
+    by = 3.0 * n * h * X0.element_size()
+    out["scatter_add"] = {"rows": n, "bytes": by, "us": t * 1e6, "gbs": by / t / 1e9, "frac_hbm": by / t / 1e9 / hbm}
+    del xg, x2
+    nsel = 1 << 26
+    g = torch.Generator(device=dev).manual_seed(0)
+    sc = torch.rand(1, nsel, device=dev, generator=g)
+    sel_out = (torch.empty(1, nsel, dtype=torch.int32, device=dev), torch.empty(1, dtype=torch.int32, device=dev),
+               torch.empty(1, nsel, dtype=torch.uint8, device=dev))
+    t = med(lambda: J.jenga_select(sc, "abs_ge", 0.5, out=sel_out))
+    kept = int(sel_out[1].item())
+    by = 4.0 * nsel + 4.0 * kept + nsel + 4
+    out["select_abs_ge"] = {"scores": nsel, "kept": kept, "bytes": by, "us": t * 1e6, "gbs": by / t / 1e9,
+                            "frac_hbm": by / t / 1e9 / hbm}
+    out["hbm_peak_gbs"] = hbm
+    return out
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -380,8 +451,12 @@ def main():
         sec = tstat["ms"] / 1e3 / args.steps
         if kind == "flop":
             ach = amount / sec / 1e12
+            traffic = None
+            if tname in TRAFFIC_PER_UNIT:
+                units = traffic_units(tname, case, ks, seg)
+                traffic = TRAFFIC_PER_UNIT[tname][1] * units / (tstat["launches"] / args.steps)
             roof = {"kernel": tname, "bound": "tensor", "achieved": ach, "peak": tf_sus, "unit": "TFLOP/s",
-                    "frac": ach / tf_sus, "traffic": None, "peak_source": f"{peak_src} bf16 sustained",
+                    "frac": ach / tf_sus, "traffic": traffic, "peak_source": f"{peak_src} bf16 sustained",
                     "launches_per_step": tstat["launches"] / args.steps, "share": tstat["ms"] / sum(
                         v["ms"] for v in prof.values())}
         else:
@@ -446,6 +521,11 @@ def main():
                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e}
         del b
 
+    # ---------------- standalone token movement and selection (HBM-bound kernels)
+    movement = None
+    if not args.no_movement:
+        movement = measure_movement(J, torch, dev, X0, case, ks, hbm)
+
     # ---------------- CPU baseline (oracle, rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -465,7 +545,7 @@ def main():
                            "hidden": sh.hidden, "heads": sh.heads, "ffn": sh.ffn, "block": blk, "keep": keep,
                            "n_kept_blocks": n_kept, "segment_tokens": seg, "parallelism": f"replicas{world}",
                            "l2": "inputs larger than L2 (X 256 MiB, weights 1.6 GiB)"},
-                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "movement": movement,
                 "clocks": clk, "peak_mem_gib": peak_sparse, "dense": dense,
                 "step_tflop": step_flops(case, ks) / 1e12, "kernels": kernels}
         print(json.dumps(line), flush=True)
