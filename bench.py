@@ -259,7 +259,8 @@ def measure_movement(J, torch, dev, X0, case, ks, hbm):
     """Standalone timing of the HBM-bound entry points at the workload's sizes: gather and
     scatter-add of layer 0's retained rows of X (bf16 [S, h]), and threshold selection
     (ABS_GE) over 2^26 fp32 scores.  Algorithmic bytes: gather 2 n h e, scatter-add 3 n h e
-    (eliminated rows cost nothing), select 4 nb read + 4 n_kept + nb + 4 written.  Each
+    (eliminated rows cost nothing), select 4 nb read + 4 nb (idx, -1 past n_kept) + nb + 4
+    written.  Each
     call moves more than the 126 MB L2; CUDA events, median of 10 after 3 warm-ups."""
     blk, S, h = case.blk, case.S, X0.shape[1]
     nb = S // blk
@@ -299,7 +300,7 @@ def measure_movement(J, torch, dev, X0, case, ks, hbm):
                torch.empty(1, nsel, dtype=torch.uint8, device=dev))
     t = med(lambda: J.jenga_select(sc, "abs_ge", 0.5, out=sel_out))
     kept = int(sel_out[1].item())
-    by = 4.0 * nsel + 4.0 * kept + nsel + 4
+    by = 4.0 * nsel + 4.0 * nsel + nsel + 4  # scores in; idx (kept, then -1 fill), mask, n_kept out
     out["select_abs_ge"] = {"scores": nsel, "kept": kept, "bytes": by, "us": t * 1e6, "gbs": by / t / 1e9,
                             "frac_hbm": by / t / 1e9 / hbm}
     out["hbm_peak_gbs"] = hbm

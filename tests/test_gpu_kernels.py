@@ -171,9 +171,11 @@ def test_select_bit_exact(J, nb, mode, param, dist):
     assert np.array_equal(mask.cpu().numpy(), om)
 
 
-@pytest.mark.parametrize("mode,param", [("abs_ge", 0.25), ("mean_ge", 0)])
-def test_select_large_multi_cta(J, mode, param):
-    nb = (1 << 20) + 777
+@pytest.mark.parametrize("mode,param,nb", [("abs_ge", 0.25, (1 << 20) + 777), ("mean_ge", 0, (1 << 20) + 777),
+                                           ("abs_ge", 0.5, 1 << 22), ("mean_ge", 0, (1 << 22) + 4)])
+def test_select_large_multi_cta(J, mode, param, nb):
+    # single-pass look-back compaction: ragged tails (scalar loads) and multiples of 4
+    # (vector loads, 16-byte mask stores)
     sc = synth.gen_scores(5, 2, nb)
     idx, nk, mask = J.jenga_select(torch.from_numpy(sc).cuda(), mode, param)
     J.jenga_check_device_status()
