@@ -7,13 +7,20 @@
 // projection, carry the low half of a bf16 hi + lo split operand, and fold the LoRA
 // down-projection's input gradient into the dX GEMM.
 //
-// Structure (one 128 x BN output tile per CTA, 192 threads):
+// Structure: persistent, one CTA per SM walking the 128 x BN output tiles in a fixed
+// stride (tile = blockIdx.x, + gridDim.x, ...; N tiles fastest), 192 threads:
 //   warp 0      TMA producer: 128 x 64 A box + BN x 64 B box per stage into a
-//               STAGES-deep shared-memory ring (128-byte swizzle), mbarrier tx counts
-//   warp 1      allocates BN TMEM columns; one lane issues tcgen05.mma (M=128, N=BN,
-//               K=16) x 4 per stage and tcgen05.commit to release the stage
+//               STAGES-deep shared-memory ring (128-byte swizzle) that runs on across
+//               tiles, mbarrier tx counts
+//   warp 1      allocates 2 x BN TMEM columns (two accumulators); one lane issues
+//               tcgen05.mma (M=128, N=BN, K=16) x 4 per stage into the accumulator of the
+//               tile's parity and tcgen05.commit to release the stage
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time of their TMEM lane quarter
-//               (row = 32 * (warp % 4) + lane), fused epilogue, global stores
+//               (row = 32 * (warp % 4) + lane), release the accumulator after its last
+//               load, fused epilogue, global stores -- overlapping the next tile's MMAs
+// With one tile per CTA the tensor core idled through every tile's prologue (barrier
+// set-up, TMEM allocation, first TMA round trip) and epilogue stores; K = 4096 projections
+// ran at about half the rate of the long-K ones.
 // Every wait is bounded (see mbar_wait); rows past the device-side valid count are
 // neither loaded usefully nor stored.
 #pragma once
@@ -142,15 +149,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint64_t* empty = full + STAGES;
-  uint64_t* accum = empty + STAGES;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 1);
+  uint64_t* acc_full = empty + STAGES;  // [2]
+  uint64_t* acc_empty = acc_full + 2;   // [2]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
   __shared__ double s_inv_freq[64];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN;
-  const int m0 = blockIdx.y * GEMM_BM;
   const int valid = epi_valid_rows(ep);
-  if (m0 >= valid) return;  // whole tile past the valid rows (uniform per CTA)
+  const int ntn = (N + BN - 1) / BN;
+  const int ntm = (min(valid, ep.m_host) + GEMM_BM - 1) / GEMM_BM;  // tiles past the valid rows are skipped
+  const int ntiles = ntn * ntm;
+  if ((int)blockIdx.x >= ntiles) return;  // uniform per CTA
   const int nkb = nkb1 + nkb2 + nkb3;
 
   if (EPI == EPI_QKV_ROPE) {
@@ -161,11 +170,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accum, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, BN < 32 ? 32 : BN);
+    tmem_alloc(tmem_holder, 2 * (BN < 32 ? 32 : BN));
     tmem_relinquish();
   }
   tc_fence_before();
@@ -177,9 +189,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // ---------------- TMA producer
     prefetch_tmap(&tmA1);
     prefetch_tmap(&tmB1);
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % STAGES;
-      if (kb >= STAGES && !mbar_wait(&empty[s], ((kb / STAGES) - 1) & 1, SITE_GEMM_PRODUCER)) break;
+    int g = 0;  // k-blocks issued by this CTA so far (ring position)
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+    const int n0 = (tile % ntn) * BN, m0 = (tile / ntn) * GEMM_BM;
+    for (int kb = 0; kb < nkb; ++kb, ++g) {
+      const int s = g % STAGES;
+      if (g >= STAGES && !mbar_wait(&empty[s], ((g / STAGES) - 1) & 1, SITE_GEMM_PRODUCER)) {
+        ok = false;
+        break;
+      }
       uint8_t* sa = smem + s * L::STAGE_BYTES;
       uint8_t* sb = sa + L::A_BYTES;
       mbar_arrive_expect_tx(&full[s], L::STAGE_BYTES);
@@ -194,37 +213,51 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         tma_load_2d(sb, &tmB3, &full[s], (kb - nkb1 - nkb2) * GEMM_BK, n0);
       }
     }
+    }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
     // idesc: kind::f16 instruction descriptor (bf16 or fp16 operands, fp32 accumulate)
     bool ok = true;
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % STAGES;
-      if (!mbar_wait(&full[s], (kb / STAGES) & 1, SITE_GEMM_MMA)) {
-        ok = false;
-        break;
-      }
+    int g = 0, it = 0;
+    for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
+      const int buf = it & 1;
+      // the epilogue must have read this accumulator's previous tile (two tiles ago)
+      if (it >= 2 && !mbar_wait(&acc_empty[buf], ((it >> 1) - 1) & 1, SITE_GEMM_MMA)) break;
       tc_fence_after();
-      const uint32_t sa = smem_u32(smem + s * L::STAGE_BYTES);
-      const uint32_t sb = sa + L::A_BYTES;
+      const uint32_t acc = tmem + buf * (BN < 32 ? 32 : BN);
+      for (int kb = 0; kb < nkb; ++kb, ++g) {
+        const int s = g % STAGES;
+        if (!mbar_wait(&full[s], (g / STAGES) & 1, SITE_GEMM_MMA)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + s * L::STAGE_BYTES);
+        const uint32_t sb = sa + L::A_BYTES;
 #pragma unroll
-      for (int k = 0; k < GEMM_BK / 16; ++k) {
-        umma_bf16(tmem, umma_desc_k_sw128(sa + k * 32), umma_desc_k_sw128(sb + k * 32), idesc,
-                  (kb > 0 || k > 0) ? 1u : 0u);
+        for (int k = 0; k < GEMM_BK / 16; ++k) {
+          umma_bf16(acc, umma_desc_k_sw128(sa + k * 32), umma_desc_k_sw128(sb + k * 32), idesc,
+                    (kb > 0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit(&empty[s]);
       }
-      umma_commit(&empty[s]);
+      if (ok) umma_commit(&acc_full[buf]);
     }
-    if (ok) umma_commit(accum);
   } else if (warp >= 2) {
     // ---------------- epilogue
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+    const int buf = it & 1;
+    const int n0 = (tile % ntn) * BN, m0 = (tile / ntn) * GEMM_BM;
     const int m = m0 + r;
     // warp vote: the tcgen05.ld calls below are collective, so all lanes take one path
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(accum, 0, SITE_GEMM_EPILOGUE));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (it >> 1) & 1, SITE_GEMM_EPILOGUE));
     tc_fence_after();
-    if (ok) {
-      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16);
+    if (!ok) break;
+    {
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * (BN < 32 ? 32 : BN);
       const bool row_ok = m < valid;
       float v[32];
       if (EPI == EPI_STORE_BF16 || EPI == EPI_STORE_F32 || EPI == EPI_SCATTER_ADD) {
@@ -350,12 +383,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
       }
     }
+    // every TMEM load of this accumulator is done: the MMAs of tile it + 2 may overwrite it
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, BN < 32 ? 32 : BN);
+    tmem_dealloc(tmem, 2 * (BN < 32 ? 32 : BN));
   }
 }
 
@@ -395,7 +433,9 @@ jenga_status launch_gemm(const GemmOperand& A1, const GemmOperand& B1, int K1, c
       cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL));
   EpiParams p = ep;
   p.m_host = M;
-  dim3 grid((N + BN - 1) / BN, (M + GEMM_BM - 1) / GEMM_BM);
+  // persistent: one CTA per SM (or per tile when there are fewer tiles)
+  const int ntiles = ((N + BN - 1) / BN) * ((M + GEMM_BM - 1) / GEMM_BM);
+  dim3 grid(ntiles < sm_count() ? ntiles : sm_count());
   // operand format fields (bits 7-9: A, 10-12: B) are 1 for bf16 and 0 for fp16
   const uint32_t idesc = f16_inputs ? (umma_idesc_bf16(GEMM_BM, BN) & ~((7u << 7) | (7u << 10)))
                                     : umma_idesc_bf16(GEMM_BM, BN);
