@@ -126,7 +126,7 @@ static size_t carve_bwd_ws(Carve& c, const Dims& d, int nc, int T, BwdWs* w) {
   w->dt = c.take<float>((size_t)T * 2 * LORA_R);
   const int chunks = (T + LG_CHUNK - 1) / LG_CHUNK;
   const int cmax = d.HD > d.h ? d.HD : d.h;
-  w->part = c.take<float>((size_t)chunks * cmax * 16);
+  w->part = c.take<float>((size_t)4 * chunks * cmax * 16);
   return c.used();
 }
 
@@ -565,39 +565,28 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
     // xn of the segment (recomputed from the saved gathered input)
     JENGA_TRY(rmsnorm(s.xr + (size_t)s0 * h, h, nullptr, 1, s0, n_kept, blk, T, h, w->rms_eps,
                       (const bf16*)w->attn_norm, nullptr, b.xn, nullptr, st));
-    // LoRA gradients (deterministic split over rows)
+    // LoRA gradients (deterministic split over rows), all four products in one launch
     {
       const int chunks = (T + LG_CHUNK - 1) / LG_CHUNK;
-      struct G {
-        const bf16* X;
-        int64_t ldx;
-        const float* Y;
-        int C;
-        float scale;
-        float* out;
-        int64_t so_c, so_r;
-      } jobs[4] = {
-          {b.dqkv, 3 * HD, s.t + (size_t)s0 * 2 * LORA_R, HD, ls, grads->dbq, LORA_R, 1},
-          {b.dqkv + 2 * HD, 3 * HD, s.t + (size_t)s0 * 2 * LORA_R + LORA_R, HD, ls, grads->dbv, LORA_R, 1},
-          {b.xn, h, b.dt, h, 1.f, grads->daq, 1, h},
-          {b.xn, h, b.dt + LORA_R, h, 1.f, grads->dav, 1, h},
-      };
-      for (auto& j : jobs) {
-        {
+      const int cmax = HD > h ? HD : h;
+      LoraGradJobs jobs;
+      jobs.j[0] = {b.dqkv, 3 * HD, s.t + (size_t)s0 * 2 * LORA_R, HD, ls, grads->dbq, LORA_R, 1};
+      jobs.j[1] = {b.dqkv + 2 * HD, 3 * HD, s.t + (size_t)s0 * 2 * LORA_R + LORA_R, HD, ls, grads->dbv, LORA_R, 1};
+      jobs.j[2] = {b.xn, h, b.dt, h, 1.f, grads->daq, 1, h};
+      jobs.j[3] = {b.xn, h, b.dt + LORA_R, h, 1.f, grads->dav, 1, h};
+      {
         const int _ps = ::jenga::prof_begin("lora_grad_partial", st);
-        lora_grad_partial_kernel<<<dim3(j.C / 64, chunks), 256, 0, st>>>(j.X, j.ldx, j.Y, 2 * LORA_R, j.C, T, n_kept,
-                                                                          blk, s0, b.part);
+        lora_grad_partial_kernel<<<dim3((cmax + LG_COLS - 1) / LG_COLS, chunks, 4), 256, 0, st>>>(
+            jobs, 2 * LORA_R, T, n_kept, blk, s0, cmax, b.part);
         ::jenga::prof_end(_ps, st);
-        }
-        JENGA_LAUNCH_CHECK();
-        {
-        const int _ps = ::jenga::prof_begin("lora_grad_reduce", st);
-        lora_grad_reduce_kernel<<<(j.C * 16 + 255) / 256, 256, 0, st>>>(b.part, chunks, j.C, j.scale, j.out, j.so_c,
-                                                                          j.so_r);
-        ::jenga::prof_end(_ps, st);
-        }
-        JENGA_LAUNCH_CHECK();
       }
+      JENGA_LAUNCH_CHECK();
+      {
+        const int _ps = ::jenga::prof_begin("lora_grad_reduce", st);
+        lora_grad_reduce_kernel<<<dim3((cmax * 16 + 255) / 256, 4), 256, 0, st>>>(jobs, b.part, chunks, cmax);
+        ::jenga::prof_end(_ps, st);
+      }
+      JENGA_LAUNCH_CHECK();
     }
     // dxn = dQKV [Wq; Wk; Wv] + dt [Aq; Av]
     {

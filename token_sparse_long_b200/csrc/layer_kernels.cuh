@@ -245,38 +245,83 @@ __global__ void rope_bwd_pack_kernel(const float* __restrict__ dq, int64_t ld_dq
 // Split-K partials of  P[chunk][c][r] = sum_{m in chunk} X[m, c] * Y[m, r]   (r < 16)
 // X bf16 [rows, ldx] (columns [0, C)), Y fp32 [rows, ldy] (columns [0, 16)).
 // grid (C / 64, chunks), 256 threads = 64 columns x 4 groups of 4 r.
-constexpr int LG_CHUNK = 256;
-__global__ void __launch_bounds__(256) lora_grad_partial_kernel(const bf16* __restrict__ X, int64_t ldx,
-                                                                const float* __restrict__ Y, int64_t ldy, int C,
-                                                                int rows, const int32_t* __restrict__ n_valid,
-                                                                int valid_mult, int row_offset,
-                                                                float* __restrict__ part) {
-  const int c = blockIdx.x * 64 + (threadIdx.x & 63);
-  const int rg = threadIdx.x >> 6;
+constexpr int LG_CHUNK = 512;   // rows per partial sum
+constexpr int LG_COLS = 512;    // columns per block (2 per thread)
+
+// One LoRA gradient product: out[c * so_c + r * so_r] += scale * sum_m X[m, c] Y[m, r]
+// (r < 16).  The four of a layer segment (dB_q, dB_v from dQ / dV and t; dA_q, dA_v from
+// xn and dt) run in one launch, blockIdx.z = job.
+struct LoraGradJob {
+  const bf16* X;
+  int64_t ldx;
+  const float* Y;  // 16 consecutive fp32 per row, row pitch ldy
+  int C;
+  float scale;
+  float* out;
+  int64_t so_c, so_r;
+};
+struct LoraGradJobs {
+  LoraGradJob j[4];
+};
+
+// part[job][chunk][c][16]: each thread owns 2 columns x 16 ranks of one 512-row chunk; the
+// chunk's Y rows are staged in shared memory (broadcast reads), X arrives as bf16 pairs
+// and the products accumulate as packed f32x2 FMAs.
+__global__ void __launch_bounds__(256) lora_grad_partial_kernel(LoraGradJobs jobs, int64_t ldy, int rows,
+                                                                const int32_t* __restrict__ n_valid, int valid_mult,
+                                                                int row_offset, int cmax, float* __restrict__ part) {
+  __shared__ __align__(16) float sY[LG_CHUNK * 16];
+  const LoraGradJob jb = jobs.j[blockIdx.z];
   const int nv = valid_rows(n_valid, valid_mult, row_offset, rows);
   const int m0 = blockIdx.y * LG_CHUNK, m1 = min(nv, m0 + LG_CHUNK);
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int m = m0; m < m1; ++m) {
-    const float xv = __bfloat162float(X[(int64_t)m * ldx + c]);
-    const float4 y = *reinterpret_cast<const float4*>(Y + (int64_t)m * ldy + rg * 4);
-    acc[0] = fmaf(xv, y.x, acc[0]);
-    acc[1] = fmaf(xv, y.y, acc[1]);
-    acc[2] = fmaf(xv, y.z, acc[2]);
-    acc[3] = fmaf(xv, y.w, acc[3]);
+  const int c = blockIdx.x * LG_COLS + threadIdx.x * 2;
+  if (blockIdx.x * LG_COLS >= jb.C) return;  // uniform per block
+  for (int e = threadIdx.x; e < LG_CHUNK * 4; e += 256) {
+    const int rr = e >> 2, q = e & 3;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (m0 + rr < m1) v = *reinterpret_cast<const float4*>(jb.Y + (int64_t)(m0 + rr) * ldy + 4 * q);
+    reinterpret_cast<float4*>(sY)[e] = v;
   }
-  float* p = part + ((int64_t)blockIdx.y * C + c) * 16 + rg * 4;
-  *reinterpret_cast<float4*>(p) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  __syncthreads();
+  uint64_t acc[16];  // acc[r] = (column c, column c + 1) pair of rank r
+#pragma unroll
+  for (int r = 0; r < 16; ++r) acc[r] = 0ull;
+  if (c < jb.C) {
+    const bf16* xp = jb.X + (int64_t)m0 * jb.ldx + c;
+    for (int m = m0; m < m1; ++m, xp += jb.ldx) {
+      const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(xp));
+      const uint64_t x2 = f2pack(x.x, x.y);
+      const float4* yr = reinterpret_cast<const float4*>(sY + (m - m0) * 16);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 y = yr[q];
+        acc[4 * q] = ffma2(x2, f2pack(y.x, y.x), acc[4 * q]);
+        acc[4 * q + 1] = ffma2(x2, f2pack(y.y, y.y), acc[4 * q + 1]);
+        acc[4 * q + 2] = ffma2(x2, f2pack(y.z, y.z), acc[4 * q + 2]);
+        acc[4 * q + 3] = ffma2(x2, f2pack(y.w, y.w), acc[4 * q + 3]);
+      }
+    }
+    float lo[16], hi[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) f2unpack(acc[r], lo[r], hi[r]);
+    float* p = part + (((int64_t)blockIdx.z * gridDim.y + blockIdx.y) * cmax + c) * 16;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      reinterpret_cast<float4*>(p)[q] = make_float4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
+      reinterpret_cast<float4*>(p + 16)[q] = make_float4(hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
+    }
+  }
 }
 
-// out[c * so_c + r * so_r] += scale * sum_chunk part[chunk][c][r]   (fixed chunk order)
-__global__ void lora_grad_reduce_kernel(const float* __restrict__ part, int chunks, int C, float scale,
-                                        float* __restrict__ out, int64_t so_c, int64_t so_r) {
+// out[c * so_c + r * so_r] += scale * sum_chunk part[job][chunk][c][r]   (fixed chunk order)
+__global__ void lora_grad_reduce_kernel(LoraGradJobs jobs, const float* __restrict__ part, int chunks, int cmax) {
+  const LoraGradJob jb = jobs.j[blockIdx.y];
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= C * 16) return;
+  if (e >= jb.C * 16) return;
   const int c = e >> 4, r = e & 15;
   float s = 0.f;
-  for (int k = 0; k < chunks; ++k) s += part[((int64_t)k * C + c) * 16 + r];
-  out[c * so_c + r * so_r] += scale * s;
+  for (int k = 0; k < chunks; ++k) s += part[(((int64_t)blockIdx.y * chunks + k) * cmax + c) * 16 + r];
+  jb.out[c * jb.so_c + r * jb.so_r] += jb.scale * s;
 }
 
 // ---- weight re-layout (pack)
