@@ -136,7 +136,7 @@ def split_saved(saved, nc, h, H, D=128, r=16):
     take("o", nc * HD, torch.bfloat16, (nc, HD))
     take("h", nc * h, torch.bfloat16, (nc, h))
     take("t", nc * 2 * r, torch.float32, (nc, 2 * r))
-    take("lse", H * nc, torch.float32, (H, nc))  # row log-sum-exp, log2 units
+    take("lse", H * nc, torch.float32, (H, nc))  # negated row log-sum-exp, log2 units
     take("rstd1", nc, torch.float32, (nc,))
     take("rstd2", nc, torch.float32, (nc,))
     return out

@@ -52,7 +52,7 @@ def test_forward_intermediates(J, keep_blocks):
     errs["q"] = rel_max_ulp(qkv[:, :HD], ctx["q"].reshape(nc, HD))
     errs["k"] = rel_max_ulp(qkv[:, HD:2 * HD], ctx["k"].reshape(nc, HD))
     errs["v"] = rel_max_ulp(qkv[:, 2 * HD:], ctx["v"].reshape(nc, HD))
-    errs["lse"] = rel_max(parts["lse"].cpu().numpy() * np.log(2.0), ctx["lse"])  # saved in log2 units
+    errs["lse"] = rel_max(-parts["lse"].cpu().numpy() * np.log(2.0), ctx["lse"])  # saved negated, log2 units
     errs["o"] = rel_max_ulp(torch_to_f64(parts["o"]), ctx["o"].reshape(nc, HD))
     errs["h"] = rel_delta_ulp(torch_to_f64(parts["h"]), ctx["h"], X[rows])
     errs["out"] = rel_delta_ulp(torch_to_f64(x)[rows], out, X[rows])

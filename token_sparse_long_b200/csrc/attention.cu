@@ -24,7 +24,8 @@ __device__ __forceinline__ int attn_rows(const int32_t* n_valid, int mult, int c
 }
 
 // ------------------------------------------------------------------ backward helpers
-// delta[h, r] = sum_d dO[r, h, d] * O[r, h, d] for rows r in [0, T)
+// delta[h, r] = -sum_d dO[r, h, d] * O[r, h, d] for rows r in [0, T) (negated: the
+// backward adds it to dP)
 __global__ void attn_delta_kernel(const bf16* __restrict__ dO, int64_t ld_do, const bf16* __restrict__ o,
                                   int64_t ldo, float* __restrict__ delta, int64_t delta_ld, int T, int H) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
@@ -39,7 +40,7 @@ __global__ void attn_delta_kernel(const bf16* __restrict__ dO, int64_t ld_do, co
   float s = x0.x * y0.x + x0.y * y0.y + x1.x * y1.x + x1.y * y1.y;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) delta[(int64_t)h * delta_ld + r] = s;
+  if (lane == 0) delta[(int64_t)h * delta_ld + r] = -s;
 }
 
 // dQ for the query rows [s0, s0 + gridDim.x*64) (segment), keys [0, q tile end).
@@ -69,8 +70,9 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(
   cp_async_commit();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int row0 = q0 + warp * 16 + g, row1 = row0 + 8;
-  const float L0 = lse[(int64_t)h * lse_ld + row0], L1 = lse[(int64_t)h * lse_ld + row1];  // log2 units
-  const float D0 = delta[(int64_t)h * delta_ld + row0 - s0], D1 = delta[(int64_t)h * delta_ld + row1 - s0];
+  // both stored negated (log2 units for the log-sum-exp)
+  const float L0 = -lse[(int64_t)h * lse_ld + row0], L1 = -lse[(int64_t)h * lse_ld + row1];
+  const float D0 = -delta[(int64_t)h * delta_ld + row0 - s0], D1 = -delta[(int64_t)h * delta_ld + row1 - s0];
   float dq[16][4];
 #pragma unroll
   for (int i = 0; i < 16; ++i) dq[i][0] = dq[i][1] = dq[i][2] = dq[i][3] = 0.f;
@@ -151,8 +153,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(
     load_tile_async(sO[buf], dO + h * AT_D, ld_do, qt * AT_ROWS - s0, n - s0);
     if (threadIdx.x < AT_ROWS) {
       const int r = qt * AT_ROWS + threadIdx.x;
-      sL[buf][threadIdx.x] = (r < n) ? lse[(int64_t)h * lse_ld + r] : 0.f;  // log2 units
-      sD[buf][threadIdx.x] = (r < n) ? delta[(int64_t)h * delta_ld + r - s0] : 0.f;
+      sL[buf][threadIdx.x] = (r < n) ? -lse[(int64_t)h * lse_ld + r] : 0.f;  // stored negated, log2 units
+      sD[buf][threadIdx.x] = (r < n) ? -delta[(int64_t)h * delta_ld + r - s0] : 0.f;
     }
   };
   load_q(qt_begin, 0);
@@ -296,7 +298,7 @@ jenga_status attn_backward_segment(const bf16* q, const bf16* k, const bf16* v, 
     JENGA_LAUNCH_CHECK();
     {
       const int _ps = ::jenga::prof_begin("attn_bwd_dkdv_tc", st);
-      attn_bwd_dkdv_tc_kernel<<<dim3((s1 + 127) / 128, H), ABT_THREADS, DKV_SMEM, st>>>(
+      attn_bwd_dkdv_tc_kernel<<<dim3((s1 + 127) / 128, H), DKV_THREADS, DKV_SMEM, st>>>(
           tk128, tv128, tq64, tdo64, lse, lse_ld, delta, delta_ld, dk_acc, dv_acc, ld_acc, s0, s1, n_valid,
           valid_mult, n_cap, scale_log2, scale);
       ::jenga::prof_end(_ps, st);

@@ -6,7 +6,8 @@
 //                 S^T  = K Q^T        dP^T = V dO^T           (TMEM, double-buffered)
 //                 P^T  = 2^(S^T log2e/sqrt(D) - L_q),  dS^T = P^T (dP^T - Delta_q)   (epilogue;
 //                 L_q, the forward's row log-sum-exp in log2 units, and Delta_q ride in the
-//                 Q / dO stage as two 256-byte bulk copies)
+//                 Q / dO stage as two 256-byte bulk copies; both are stored negated, so the
+//                 epilogue's packed f32x2 arithmetic adds them)
 //                 dV  += P^T dO       dK  += dS^T Q           (A: smem K-major, B: MN-major)
 //               and at the end dV, dK (x 1/sqrt(D)) are added into fp32 accumulators.
 //   dQ pass     one CTA per (128-query tile of the segment, head).  Q and dO resident; the
@@ -15,11 +16,15 @@
 // The Q/dO (K/V) ring is 3 (4) stages deep: a stage is read by both products of its tile,
 // so with 2 stages the next tile's load could only start once the gradient product that
 // immediately precedes that tile's score product had finished.
-// Warp roles: 0 TMA, 1 and 2 MMA issue (1 also allocates TMEM; a warp can issue a
-// tcgen05.mma only every ~100 clocks, so one issuer would cap these M 128 x N 64 / N 128
-// products well below the tensor peak), 3..10 epilogue in two quads: each quad
-// covers all 128 TMEM lanes (one row per thread), quad 0 the first 32 columns of a tile and
-// quad 1 the last 32.  P / dS tiles are double-buffered in shared memory so the epilogue of
+// Warp roles (a warp can issue a tcgen05.mma only every ~100 clocks, so one issuer would
+// cap these M 128 x N 64 / N 128 products well below the tensor peak, and an issuer that
+// also waits on the epilogue stalls the products queued behind that wait):
+//   dK/dV pass  0 TMA; 1 S^T, 2 dP^T, 3 dV, 4 dK issue (1 also allocates TMEM); 5..20
+//               epilogue in four quads, quad c taking columns 16c .. 16c + 15 of a tile (two
+//               epilogue warps per SMSP left the exponentials latency-bound)
+//   dQ pass     0 TMA; 1 S and dQ, 2 dP issue; 3..10 epilogue in two quads (first / last
+//               32 columns)
+// Each quad covers all 128 TMEM lanes, one row per thread.  P / dS tiles are double-buffered in shared memory so the epilogue of
 // tile i overlaps the gradient products of tile i-1 and the score products of tile i+1.
 // Causal masking, keys / queries past the valid count, and the segment bounds are applied
 // in the epilogue.  Every wait is bounded; waits that guard collective TMEM loads are voted.
@@ -31,17 +36,19 @@ namespace jenga {
 
 constexpr int ABT_BOX128 = 128 * 64 * 2;   // 16 KB box: 128 rows x 64 bf16
 constexpr int ABT_BOX64 = 64 * 64 * 2;     // 8 KB box: 64 rows x 64 bf16
-constexpr int ABT_THREADS = 352;  // warps 0 TMA, 1 and 2 MMA issue, 3 .. 10 epilogue
+constexpr int ABT_THREADS = 352;  // dQ pass: warps 0 TMA, 1 and 2 MMA issue, 3 .. 10 epilogue
+constexpr int DKV_EPI_WARPS = 16;
+constexpr int DKV_EPI_WARP0 = 5;  // dK/dV pass: warps 0 TMA, 1 .. 4 MMA issue, 5 .. 20 epilogue
+constexpr int DKV_THREADS = 32 * (DKV_EPI_WARP0 + DKV_EPI_WARPS);
 
-// smem layout of the dK/dV pass
-constexpr int DKV_K_OFF = 0;                               // 2 x 16 KB
-constexpr int DKV_V_OFF = 2 * ABT_BOX128;                  // 2 x 16 KB
-constexpr int DKV_RING_OFF = 4 * ABT_BOX128;               // stage s: Q (2 x 8 KB), dO (2 x 8 KB)
+// smem layout of the dK/dV pass.  K and V are staged through the P^T / dS^T buffers and
+// copied into tensor memory (the A operands of S^T and dP^T) before the first tile.
+constexpr int DKV_PT_OFF = 0;                              // [2] x 128 x 64 bf16 (first: K)
+constexpr int DKV_DST_OFF = DKV_PT_OFF + 2 * ABT_BOX128;   // [2] x 128 x 64 bf16 (first: V)
+constexpr int DKV_RING_OFF = DKV_DST_OFF + 2 * ABT_BOX128;  // stage s: Q (2 x 8 KB), dO (2 x 8 KB)
 constexpr int DKV_STAGE = 4 * ABT_BOX64;
-constexpr int DKV_STAGES = 3;  // a stage lives from S^T(i) to the gradient products of tile i
-constexpr int DKV_PT_OFF = DKV_RING_OFF + DKV_STAGES * DKV_STAGE;  // [2] x 128 x 64 bf16
-constexpr int DKV_DST_OFF = DKV_PT_OFF + 2 * ABT_BOX128;  // [2] x 128 x 64 bf16
-constexpr int DKV_LD_OFF = DKV_DST_OFF + 2 * ABT_BOX128;  // stage s: L (64 fp32), Delta (64 fp32)
+constexpr int DKV_STAGES = 4;  // a stage lives from its load to the gradient products of its tile
+constexpr int DKV_LD_OFF = DKV_RING_OFF + DKV_STAGES * DKV_STAGE;  // stage s: L (64 fp32), Delta (64 fp32)
 constexpr int DKV_LD_BYTES = 512;
 constexpr int DKV_BAR_OFF = DKV_LD_OFF + DKV_STAGES * DKV_LD_BYTES;
 constexpr int DKV_SMEM = DKV_BAR_OFF + 256 + 1024;
@@ -58,6 +65,19 @@ constexpr int DQ_SMEM = DQ_BAR_OFF + 256 + 1024;
 
 // Write 32 bf16 values (packed pairs pk[0..15]) as columns [32 * half, 32 * half + 32) of
 // row r of a 128 x 64 K-major tile with the 128-byte swizzle (row = 8 chunks of 16 bytes).
+__device__ __forceinline__ void st_row32_sw128(uint8_t* tile, int r, int half, const uint32_t* pk);
+
+// Write 16 bf16 values (packed pairs pk[0..7]) as columns [16 * quad, 16 * quad + 16) of row r
+// of a 128 x 64 K-major tile with the 128-byte swizzle.
+__device__ __forceinline__ void st_row16_sw128(uint8_t* tile, int r, int quad, const uint32_t* pk) {
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    const int ch = quad * 2 + c;
+    *reinterpret_cast<uint4*>(tile + r * 128 + ((ch ^ (r & 7)) << 4)) =
+        make_uint4(pk[c * 4], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
+  }
+}
+
 __device__ __forceinline__ void st_row32_sw128(uint8_t* tile, int r, int half, const uint32_t* pk) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
@@ -68,7 +88,7 @@ __device__ __forceinline__ void st_row32_sw128(uint8_t* tile, int r, int half, c
 }
 
 // ------------------------------------------------------------------ dK / dV
-__global__ void __launch_bounds__(ABT_THREADS, 1)
+__global__ void __launch_bounds__(DKV_THREADS, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                             const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                             const float* __restrict__ lse, int64_t lse_ld, const float* __restrict__ delta,
@@ -81,12 +101,13 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
   uint64_t* kv_full = bars;
   uint64_t* q_full = bars + 1;                // [DKV_STAGES]
   uint64_t* q_empty = q_full + DKV_STAGES;    // [DKV_STAGES]
-  uint64_t* s_full = q_empty + DKV_STAGES;    // [2]
-  uint64_t* s_free = s_full + 2;    // [2]
-  uint64_t* pd_full = s_free + 2;   // [2]
+  uint64_t* s_full = q_empty + DKV_STAGES;    // S^T / dP^T of the current tile written
+  uint64_t* s_free = s_full + 1;              // ... and read by the epilogue
+  uint64_t* pd_full = s_free + 1;   // [2]
   uint64_t* pd_free = pd_full + 2;  // [2]
   uint64_t* done = pd_free + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* kv_tmem = done + 1;     // K and V are in tensor memory
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(kv_tmem + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
@@ -105,15 +126,16 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     mbar_init(kv_full, 1);
     for (int s = 0; s < DKV_STAGES; ++s) {
       mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 2);
+      mbar_init(&q_empty[s], 4);  // all four products read the stage
     }
+    mbar_init(s_full, 2);
+    mbar_init(s_free, DKV_EPI_WARPS);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 2);
-      mbar_init(&s_free[s], 8);
-      mbar_init(&pd_full[s], 8);
+      mbar_init(&pd_full[s], DKV_EPI_WARPS);
       mbar_init(&pd_free[s], 2);
     }
     mbar_init(done, 2);
+    mbar_init(kv_tmem, 8);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -124,15 +146,16 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  // TMEM columns: S^T[2] at 0, 64; dP^T[2] at 128, 192; dV at 256; dK at 384
-  const uint32_t tdV = tmem + 256, tdK = tmem + 384;
+  // TMEM columns: dV 0..127, dK 128..255, K 256..319, V 320..383 (bf16 pairs, A operands),
+  // S^T 384..447, dP^T 448..511
+  const uint32_t tdV = tmem, tdK = tmem + 128, tK = tmem + 256, tV = tmem + 320, tS = tmem + 384, tP = tmem + 448;
 
   if (warp == 0 && lane == 0) {
     mbar_arrive_expect_tx(kv_full, 4 * ABT_BOX128);
-    tma_load_2d(smem + DKV_K_OFF, &tmK, kv_full, col, k0);
-    tma_load_2d(smem + DKV_K_OFF + ABT_BOX128, &tmK, kv_full, col + 64, k0);
-    tma_load_2d(smem + DKV_V_OFF, &tmV, kv_full, col, k0);
-    tma_load_2d(smem + DKV_V_OFF + ABT_BOX128, &tmV, kv_full, col + 64, k0);
+    tma_load_2d(smem + DKV_PT_OFF, &tmK, kv_full, col, k0);
+    tma_load_2d(smem + DKV_PT_OFF + ABT_BOX128, &tmK, kv_full, col + 64, k0);
+    tma_load_2d(smem + DKV_DST_OFF, &tmV, kv_full, col, k0);
+    tma_load_2d(smem + DKV_DST_OFF + ABT_BOX128, &tmV, kv_full, col + 64, k0);
     for (int i = 0; i < nq; ++i) {
       const int s = i % DKV_STAGES;
       if (i >= DKV_STAGES && !mbar_wait_at(&q_empty[s], ((i / DKV_STAGES) - 1) & 1, 121, i)) break;
@@ -149,107 +172,128 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
       bulk_load_1d(ldst + 256, delta + (int64_t)h * delta_ld + (qrow - s0), 256, &q_full[s]);
     }
   } else if ((warp == 1 || warp == 2) && lane == 0) {
-    // two issuing warps (a warp can issue a tcgen05.mma only every ~100 clocks): warp 1
-    // issues S^T and dV (the P chain), warp 2 dP^T and dK (the dS chain); the barriers that
-    // both chains feed (s_full, pd_free, q_empty, done) count two commits
-    const bool pchain = (warp == 1);
+    // score products, one issuing warp each (a warp can issue a tcgen05.mma only every ~100
+    // clocks): warp 1 S^T = K Q^T, warp 2 dP^T = V dO^T, A (K, V) from tensor memory and B
+    // (Q, dO) from the ring, independent of the gradient products.  One accumulator each:
+    // tile i + 1's product starts as soon as the epilogue has read tile i's.
+    const bool s_chain = (warp == 1);
     constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64);
-    constexpr uint32_t idesc_g = umma_idesc_bf16_bmn(128, 128);
-    const uint32_t aa = smem_u32(smem + (pchain ? DKV_K_OFF : DKV_V_OFF));  // K or V: A of S^T / dP^T
-    const uint32_t acc_s = tmem + (pchain ? 0 : 128);                       // S^T[2] or dP^T[2]
-    const uint32_t acc_g = pchain ? tdV : tdK;
-    const int gbuf_off = pchain ? DKV_PT_OFF : DKV_DST_OFF;                 // P^T or dS^T tiles
-    const int b_g_off = pchain ? 2 * ABT_BOX64 : 0;                          // dO or Q: B of dV / dK
-    const int b_s_off = pchain ? 0 : 2 * ABT_BOX64;                          // Q or dO: B of S^T / dP^T
-    bool ok = mbar_wait_at(kv_full, 0, 122, 0);
-    auto issue_grad = [&](int ii) -> bool {
-      const int b = ii & 1, rs = ii % DKV_STAGES;
-      if (!mbar_wait_at(&pd_full[b], (ii >> 1) & 1, 123, ii)) return false;
-      tc_fence_after();
-      const uint32_t bs = smem_u32(smem + DKV_RING_OFF + rs * DKV_STAGE + b_g_off);
-      const uint32_t ga = smem_u32(smem + gbuf_off + b * ABT_BOX128);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)  // K = 64 queries in steps of 16
-        umma_bf16(acc_g, umma_desc_k_sw128(ga + ks * 32), umma_desc_mn_sw128(bs + ks * 2048, ABT_BOX64), idesc_g,
-                  (ii > 0 || ks > 0) ? 1u : 0u);
-      umma_commit(&pd_free[b]);
-      umma_commit(&q_empty[rs]);
-      return true;
-    };
+    const uint32_t ta = s_chain ? tK : tV;
+    const uint32_t acc_s = s_chain ? tS : tP;
+    const int b_s_off = s_chain ? 0 : 2 * ABT_BOX64;  // Q or dO
+    bool ok = mbar_wait_at(kv_tmem, 0, 122, 0);
     for (int i = 0; ok && i < nq; ++i) {
-      const int s = i & 1, rs = i % DKV_STAGES;
-      if (!mbar_wait_at(&q_full[rs], (i / DKV_STAGES) & 1, 124, i)) {
-        ok = false;
-        break;
-      }
-      if (i >= 2 && !mbar_wait_at(&s_free[s], ((i >> 1) - 1) & 1, 125, i)) {
-        ok = false;
-        break;
-      }
+      const int rs = i % DKV_STAGES;
+      if (!mbar_wait_at(&q_full[rs], (i / DKV_STAGES) & 1, 124, i)) break;
+      if (i >= 1 && !mbar_wait_at(s_free, (i - 1) & 1, 125, i)) break;
       tc_fence_after();
       const uint32_t st = smem_u32(smem + DKV_RING_OFF + rs * DKV_STAGE + b_s_off);
 #pragma unroll
       for (int kc = 0; kc < 2; ++kc)
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          umma_bf16(acc_s + s * 64, umma_desc_k_sw128(aa + kc * ABT_BOX128 + k * 32),
-                    umma_desc_k_sw128(st + kc * ABT_BOX64 + k * 32), idesc_s, (kc | k) ? 1u : 0u);
-      umma_commit(&s_full[s]);
-      if (i >= 1 && !issue_grad(i - 1)) {
+          umma_bf16_ts(acc_s, ta + kc * 32 + k * 8, umma_desc_k_sw128(st + kc * ABT_BOX64 + k * 32), idesc_s,
+                       (kc | k) ? 1u : 0u);
+      umma_commit(s_full);
+      umma_commit(&q_empty[rs]);
+    }
+  } else if ((warp == 3 || warp == 4) && lane == 0) {
+    // gradient products: warp 3 dV += P^T dO, warp 4 dK += dS^T Q, each as soon as the
+    // epilogue has written tile i's P^T / dS^T
+    const bool p_chain = (warp == 3);
+    constexpr uint32_t idesc_g = umma_idesc_bf16_bmn(128, 128);
+    const uint32_t acc_g = p_chain ? tdV : tdK;
+    const int gbuf_off = p_chain ? DKV_PT_OFF : DKV_DST_OFF;  // P^T or dS^T tiles
+    const int b_g_off = p_chain ? 2 * ABT_BOX64 : 0;          // dO or Q
+    bool ok = true;
+    for (int i = 0; i < nq; ++i) {
+      const int b = i & 1, rs = i % DKV_STAGES;
+      if (!mbar_wait_at(&pd_full[b], (i >> 1) & 1, 123, i)) {
         ok = false;
         break;
       }
+      tc_fence_after();
+      const uint32_t bs = smem_u32(smem + DKV_RING_OFF + rs * DKV_STAGE + b_g_off);
+      const uint32_t ga = smem_u32(smem + gbuf_off + b * ABT_BOX128);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)  // K = 64 queries in steps of 16
+        umma_bf16(acc_g, umma_desc_k_sw128(ga + ks * 32), umma_desc_mn_sw128(bs + ks * 2048, ABT_BOX64), idesc_g,
+                  (i > 0 || ks > 0) ? 1u : 0u);
+      umma_commit(&pd_free[b]);
+      umma_commit(&q_empty[rs]);
     }
-    if (ok && issue_grad(nq - 1)) umma_commit(done);
-  } else if (warp >= 3) {
+    if (ok) umma_commit(done);
+  } else if (warp >= DKV_EPI_WARP0) {
+    // 16 epilogue warps in four quads: quad c takes query columns 16c .. 16c + 15 of every
+    // 64-query tile (four warps per SMSP hide the exponential and conversion latencies)
     const int quarter = warp & 3;
-    const int half = (warp - 3) >> 2;
+    const int quad = (warp - DKV_EPI_WARP0) >> 2;
     const int r = quarter * 32 + lane;
     const int key = k0 + r;
     const uint32_t lo = (uint32_t)(quarter * 32) << 16;
     bool ok = true;
-    for (int i = 0; i < nq; ++i) {
+    if (quad < 2) {
+      // quad 0 copies K, quad 1 V from their staging tiles into tensor memory
+      if (__all_sync(0xffffffffu, mbar_wait_at(kv_full, 0, 130, 0))) {
+        tile_row_to_tmem(smem + (quad == 0 ? DKV_PT_OFF : DKV_DST_OFF), r, (quad == 0 ? tK : tV) + lo);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(kv_tmem);
+      } else {
+        ok = false;
+      }
+    }
+    // the staging tiles become the P^T / dS^T buffers only after every copy is done
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * DKV_EPI_WARPS) : "memory");
+    const uint64_t sl2x2 = f2pack(scale_log2, scale_log2);
+    for (int i = 0; ok && i < nq; ++i) {
       const int s = i & 1, rs = i % DKV_STAGES;
-      const int qbase = (qa0 + i) * 64 + half * 32;
+      const int qbase = (qa0 + i) * 64 + quad * 16;
       // S^T(i) done implies the stage landed; the second wait makes the bulk-copied L and
       // Delta visible to these threads (the stage cannot be refilled before pd_full(i))
-      if (!__all_sync(0xffffffffu, mbar_wait_at(&s_full[s], (i >> 1) & 1, 126, i) &&
+      if (!__all_sync(0xffffffffu, mbar_wait_at(s_full, i & 1, 126, i) &&
                                        mbar_wait_at(&q_full[rs], (i / DKV_STAGES) & 1, 129, i))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sv[32], dp[32];
-      tmem_ld32_nowait(tmem + lo + s * 64 + half * 32, sv);
-      tmem_ld32_nowait(tmem + lo + 128 + s * 64 + half * 32, dp);
-      const float4* L4 = reinterpret_cast<const float4*>(smem + DKV_LD_OFF + rs * DKV_LD_BYTES) + half * 8;
+      uint32_t sv[16], dp[16];
+      tmem_ld16_nowait(tS + lo + quad * 16, sv);
+      tmem_ld16_nowait(tP + lo + quad * 16, dp);
+      const float4* L4 = reinterpret_cast<const float4*>(smem + DKV_LD_OFF + rs * DKV_LD_BYTES) + quad * 4;
       const float4* D4 = L4 + 16;
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[s]);
-      uint32_t pk[16], dk[16];
-      if (qbase >= key && qbase + 32 <= send) {  // every (query, key) pair of this row is live
+      if (lane == 0) mbar_arrive(s_free);
+      uint32_t pk[8], dk[8];
+      if (qbase >= key && qbase + 16 <= send) {  // every (query, key) pair of this row is live
+        // packed pairs: x = s log2(e)/sqrt(D) - L, p = 2^x, dS = p (dP - Delta)
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 Lq = L4[c4], Dq = D4[c4];
-          const float Ls[4] = {Lq.x, Lq.y, Lq.z, Lq.w};
-          const float Ds[4] = {Dq.x, Dq.y, Dq.z, Dq.w};
-          float p[4], d[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 4 * c4 + e;
-            p[e] = fast_exp2(fmaf(__uint_as_float(sv[c]), scale_log2, -Ls[e]));
-            d[e] = p[e] * (__uint_as_float(dp[c]) - Ds[e]);
-          }
-          pk[2 * c4] = pack_bf2(p[0], p[1]);
-          pk[2 * c4 + 1] = pack_bf2(p[2], p[3]);
-          dk[2 * c4] = pack_bf2(d[0], d[1]);
-          dk[2 * c4 + 1] = pack_bf2(d[2], d[3]);
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const float4 Lq = L4[c4], Dq = D4[c4];  // -L, -Delta
+          const uint64_t p01 = exp2_mufu_x2(
+              ffma2(f2pack(__uint_as_float(sv[4 * c4]), __uint_as_float(sv[4 * c4 + 1])), sl2x2, f2pack(Lq.x, Lq.y)));
+          const uint64_t p23 = exp2_mufu_x2(ffma2(f2pack(__uint_as_float(sv[4 * c4 + 2]), __uint_as_float(sv[4 * c4 + 3])),
+                                                  sl2x2, f2pack(Lq.z, Lq.w)));
+          const uint64_t d01 =
+              fmul2(p01, fadd2(f2pack(__uint_as_float(dp[4 * c4]), __uint_as_float(dp[4 * c4 + 1])), f2pack(Dq.x, Dq.y)));
+          const uint64_t d23 = fmul2(
+              p23, fadd2(f2pack(__uint_as_float(dp[4 * c4 + 2]), __uint_as_float(dp[4 * c4 + 3])), f2pack(Dq.z, Dq.w)));
+          float a, bb;
+          f2unpack(p01, a, bb);
+          pk[2 * c4] = pack_bf2(a, bb);
+          f2unpack(p23, a, bb);
+          pk[2 * c4 + 1] = pack_bf2(a, bb);
+          f2unpack(d01, a, bb);
+          dk[2 * c4] = pack_bf2(a, bb);
+          f2unpack(d23, a, bb);
+          dk[2 * c4 + 1] = pack_bf2(a, bb);
         }
       } else {  // causal diagonal or the segment's ragged end
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
+        for (int c4 = 0; c4 < 4; ++c4) {
           const float4 Lq = L4[c4], Dq = D4[c4];
           const float Ls[4] = {Lq.x, Lq.y, Lq.z, Lq.w};
           const float Ds[4] = {Dq.x, Dq.y, Dq.z, Dq.w};
@@ -258,9 +302,9 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
           for (int e = 0; e < 4; ++e) {
             const int c = 4 * c4 + e, q = qbase + c;
             const bool valid = (q >= key) && (q < send);
-            const float pe = valid ? fast_exp2(fmaf(__uint_as_float(sv[c]), scale_log2, -Ls[e])) : 0.f;
+            const float pe = valid ? fast_exp2(fmaf(__uint_as_float(sv[c]), scale_log2, Ls[e])) : 0.f;
             p[e] = pe;
-            d[e] = valid ? pe * (__uint_as_float(dp[c]) - Ds[e]) : 0.f;  // L, Delta past n are unset
+            d[e] = valid ? pe * (__uint_as_float(dp[c]) + Ds[e]) : 0.f;  // L, Delta past n are unset
           }
           pk[2 * c4] = pack_bf2(p[0], p[1]);
           pk[2 * c4 + 1] = pack_bf2(p[2], p[3]);
@@ -273,8 +317,8 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
         ok = false;
         break;
       }
-      st_row32_sw128(smem + DKV_PT_OFF + s * ABT_BOX128, r, half, pk);
-      st_row32_sw128(smem + DKV_DST_OFF + s * ABT_BOX128, r, half, dk);
+      st_row16_sw128(smem + DKV_PT_OFF + s * ABT_BOX128, r, quad, pk);
+      st_row16_sw128(smem + DKV_DST_OFF + s * ABT_BOX128, r, quad, dk);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -283,31 +327,28 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     if (__all_sync(0xffffffffu, ok && mbar_wait_at(done, 0, 128, nq))) {
       tc_fence_after();
       const bool row_ok = key < n;
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c0 = half * 64 + cc * 32;
-        uint32_t a[32], b[32];
-        tmem_ld32_nowait(tdV + lo + c0, a);
-        tmem_ld32_nowait(tdK + lo + c0, b);
-        tmem_wait_ld();
-        if (row_ok) {
-          float4* pv = reinterpret_cast<float4*>(dv_acc + (int64_t)key * ld_acc + col + c0);
-          float4* pk4 = reinterpret_cast<float4*>(dk_acc + (int64_t)key * ld_acc + col + c0);
+      const int c0 = quad * 32;  // this quad's 32 of the 128 head dimensions
+      uint32_t a[32], b[32];
+      tmem_ld32_nowait(tdV + lo + c0, a);
+      tmem_ld32_nowait(tdK + lo + c0, b);
+      tmem_wait_ld();
+      if (row_ok) {
+        float4* pv = reinterpret_cast<float4*>(dv_acc + (int64_t)key * ld_acc + col + c0);
+        float4* pk4 = reinterpret_cast<float4*>(dk_acc + (int64_t)key * ld_acc + col + c0);
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            float4 x = pv[q4];
-            x.x += __uint_as_float(a[4 * q4]);
-            x.y += __uint_as_float(a[4 * q4 + 1]);
-            x.z += __uint_as_float(a[4 * q4 + 2]);
-            x.w += __uint_as_float(a[4 * q4 + 3]);
-            pv[q4] = x;
-            float4 y = pk4[q4];
-            y.x += __uint_as_float(b[4 * q4]) * scale;
-            y.y += __uint_as_float(b[4 * q4 + 1]) * scale;
-            y.z += __uint_as_float(b[4 * q4 + 2]) * scale;
-            y.w += __uint_as_float(b[4 * q4 + 3]) * scale;
-            pk4[q4] = y;
-          }
+        for (int q4 = 0; q4 < 8; ++q4) {
+          float4 x = pv[q4];
+          x.x += __uint_as_float(a[4 * q4]);
+          x.y += __uint_as_float(a[4 * q4 + 1]);
+          x.z += __uint_as_float(a[4 * q4 + 2]);
+          x.w += __uint_as_float(a[4 * q4 + 3]);
+          pv[q4] = x;
+          float4 y = pk4[q4];
+          y.x += __uint_as_float(b[4 * q4]) * scale;
+          y.y += __uint_as_float(b[4 * q4 + 1]) * scale;
+          y.z += __uint_as_float(b[4 * q4 + 2]) * scale;
+          y.w += __uint_as_float(b[4 * q4 + 3]) * scale;
+          pk4[q4] = y;
         }
       }
     }
@@ -464,8 +505,9 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     const int q = q0 + r;
     const uint32_t lo = (uint32_t)(quarter * 32) << 16;
     const bool qvalid = q < n;
-    const float L = qvalid ? lse[(int64_t)h * lse_ld + q] : 0.f;  // log2 units
-    const float Dq = qvalid ? delta[(int64_t)h * delta_ld + q - s0] : 0.f;
+    const float L = qvalid ? lse[(int64_t)h * lse_ld + q] : 0.f;  // -L, log2 units
+    const float Dq = qvalid ? delta[(int64_t)h * delta_ld + q - s0] : 0.f;  // -Delta
+    const uint64_t sl2x2 = f2pack(scale_log2, scale_log2), nL2 = f2pack(L, L), nD2 = f2pack(Dq, Dq);
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
       const int s = j & 1;
@@ -486,9 +528,12 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
       if (lim >= 32) {  // every key of this half is live for this row
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c]), scale_log2, -L));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), scale_log2, -L));
-          dk[c >> 1] = pack_bf2(p0 * (__uint_as_float(dp[c]) - Dq), p1 * (__uint_as_float(dp[c + 1]) - Dq));
+          const uint64_t p2 =
+              exp2_mufu_x2(ffma2(f2pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, nL2));
+          const uint64_t d2 = fmul2(p2, fadd2(f2pack(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), nD2));
+          float a, bb;
+          f2unpack(d2, a, bb);
+          dk[c >> 1] = pack_bf2(a, bb);
         }
       } else {
 #pragma unroll
@@ -497,8 +542,8 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const bool valid = c + e < lim;
-            const float pe = valid ? fast_exp2(fmaf(__uint_as_float(sv[c + e]), scale_log2, -L)) : 0.f;
-            d2[e] = valid ? pe * (__uint_as_float(dp[c + e]) - Dq) : 0.f;
+            const float pe = valid ? fast_exp2(fmaf(__uint_as_float(sv[c + e]), scale_log2, L)) : 0.f;
+            d2[e] = valid ? pe * (__uint_as_float(dp[c + e]) + Dq) : 0.f;
           }
           dk[c >> 1] = pack_bf2(d2[0], d2[1]);
         }

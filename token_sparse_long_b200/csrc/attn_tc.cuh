@@ -15,8 +15,8 @@
 //               sqrt(D) - m) as bf16 into a 128-byte-swizzled smem tile (one exponential in
 //               four on the FMA pipe, exp2_fma), row sums in fp32
 // The softmax of tile j overlaps the PV product of tile j-1 and the QK^T product of
-// tile j+1.  Output o = O / l (bf16) and the row log-sum-exp in log2 units (the backward
-// uses it as the exponent offset directly).
+// tile j+1.  Output o = O / l (bf16) and the negated row log-sum-exp in log2 units (the
+// backward adds it to the scaled logits directly).
 #pragma once
 
 #include "common.cuh"
@@ -295,7 +295,8 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
           }
         }
       }
-      if (row_ok && hf == 0) lse[(int64_t)h * lse_ld + qrow] = m_used + __log2f(l_row);  // log2 units
+      // negated row log-sum-exp in log2 units: the backward's exponent addend
+      if (row_ok && hf == 0) lse[(int64_t)h * lse_ld + qrow] = -(m_used + __log2f(l_row));
     }
   }
   tc_fence_before();
