@@ -60,7 +60,7 @@ struct EpiParams {
   float alpha = 1.f;
   float beta = 1.f;              // LORA_T: scale of the fp32 copy
   int hd = 0;                    // QKV: H * D (section width)
-  const double* inv_freq = nullptr;  // QKV: RoPE inverse frequencies [64] (head_dim 128)
+  const float2* rope_tab = nullptr;  // QKV: (cos, sin) of position(m) x frequency j, [M rows][64]
 };
 
 __device__ __forceinline__ int epi_valid_rows(const EpiParams& p) {
@@ -152,7 +152,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint64_t* acc_full = empty + STAGES;  // [2]
   uint64_t* acc_empty = acc_full + 2;   // [2]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
-  __shared__ double s_inv_freq[64];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int valid = epi_valid_rows(ep);
@@ -162,9 +161,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   if ((int)blockIdx.x >= ntiles) return;  // uniform per CTA
   const int nkb = nkb1 + nkb2 + nkb3;
 
-  if (EPI == EPI_QKV_ROPE) {
-    if (threadIdx.x < 64) s_inv_freq[threadIdx.x] = ep.inv_freq[threadIdx.x];
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -352,8 +348,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           store_bf16x32(a + 32, w);
         }
       } else if (EPI == EPI_QKV_ROPE) {
-        // tile = BN/128 heads; section = (n / hd): 0 q, 1 k, 2 v; RoPE on q and k
-        const int64_t pos = row_ok ? map_row(ep, m + ep.row_offset) : 0;
+        // tile = BN/128 heads; section = (n / hd): 0 q, 1 k, 2 v; RoPE on q and k with this
+        // row's (cos, sin) from the table (rope_table_kernel: same angles, computed once)
+        const float4* tab = reinterpret_cast<const float4*>(ep.rope_tab + (int64_t)(row_ok ? m : 0) * 64);
 #pragma unroll 1
         for (int g = 0; g < BN / 128; ++g) {
           const int nh = n0 + g * 128;
@@ -365,15 +362,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             tmem_ld32(tbase + g * 128 + 64 + hh * 32, u);
             if (!row_ok || nh >= N) continue;
             if (rope) {
-#pragma unroll 4
-              for (int i = 0; i < 32; ++i) {
-                const double ang = (double)pos * s_inv_freq[hh * 32 + i];
-                const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
-                float sn, cs;
-                sincosf((float)red, &sn, &cs);
-                const float a = v[i], b = u[i];
-                v[i] = a * cs - b * sn;
-                u[i] = b * cs + a * sn;
+#pragma unroll
+              for (int i2 = 0; i2 < 16; ++i2) {
+                const float4 t = __ldg(tab + hh * 16 + i2);  // (cos, sin) of frequencies 2 i2, 2 i2 + 1
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  const int i = 2 * i2 + e;
+                  const float cs = e ? t.z : t.x, sn = e ? t.w : t.y;
+                  const float a = v[i], b = u[i];
+                  v[i] = a * cs - b * sn;
+                  u[i] = b * cs + a * sn;
+                }
               }
             }
             bf16* o = reinterpret_cast<bf16*>(ep.out) + (int64_t)m * ep.ldo + nh;

@@ -93,11 +93,13 @@ static size_t carve_saved(Carve& c, const Dims& d, int nc, Saved* s) {
 
 struct FwdWs {
   bf16 *xn, *tb, *a;
+  float2* rope;  // [nc][64] (cos, sin) of the retained rows' positions
 };
 static size_t carve_fwd_ws(Carve& c, const Dims& d, int nc, FwdWs* w) {
   w->xn = c.take<bf16>((size_t)nc * d.h);
   w->tb = c.take<bf16>((size_t)nc * LORA_PAD);
   w->a = c.take<bf16>((size_t)nc * d.F);
+  w->rope = c.take<float2>((size_t)nc * 64);
   return c.used();
 }
 
@@ -278,6 +280,7 @@ extern "C" size_t jenga_layer_score_qk_workspace_bytes(const jenga_layer_weights
   c.take<bf16>((size_t)S * w->hidden);
   c.take<float>((size_t)S * 2 * LORA_R);
   c.take<bf16>((size_t)S * LORA_PAD);
+  c.take<float2>((size_t)S * 64);
   return c.used();
 }
 
@@ -299,6 +302,13 @@ extern "C" jenga_status jenga_layer_score_qk(const jenga_layer_weights* w, const
   bf16* xn = c.take<bf16>((size_t)S * d.h);
   float* t = c.take<float>((size_t)S * 2 * LORA_R);
   bf16* tb = c.take<bf16>((size_t)S * LORA_PAD);
+  float2* rope = c.take<float2>((size_t)S * 64);
+  {
+    const int _ps = ::jenga::prof_begin("rope_table", st);
+    rope_table_kernel<<<grid_cap((int64_t)S * 64, 256), 256, 0, st>>>(rope, S, nullptr, 1, nullptr, 1, p.inv_freq);
+    ::jenga::prof_end(_ps, st);
+  }
+  JENGA_LAUNCH_CHECK();
   JENGA_TRY(rmsnorm((const bf16*)x, d.h, nullptr, 1, 0, nullptr, 1, S, d.h, w->rms_eps, (const bf16*)w->attn_norm,
                     nullptr, xn, nullptr, st));
   EpiParams e;
@@ -314,7 +324,7 @@ extern "C" jenga_status jenga_layer_score_qk(const jenga_layer_weights* w, const
   q.out = qk;
   q.ldo = 2 * d.HD;
   q.hd = d.HD;
-  q.inv_freq = p.inv_freq;
+  q.rope_tab = rope;
   GemmOperand a2{tb, S, LORA_PAD}, b2{p.lorab, 2 * d.HD, LORA_PAD};
   JENGA_TRY((launch_gemm<256, EPI_QKV_ROPE>({xn, S, d.h}, {p.wqkv, 2 * d.HD, d.h}, d.h, &a2, &b2, LORA_PAD, S,
                                             2 * d.HD, q, st, "gemm_qk_rope_all")));
@@ -388,7 +398,13 @@ extern "C" jenga_status jenga_sparse_layer_fwd(const jenga_layer_weights* w, con
     e.out = s.qkv;
     e.ldo = 3 * HD;
     e.hd = HD;
-    e.inv_freq = p.inv_freq;
+    e.rope_tab = f.rope;
+    {
+      const int _ps = ::jenga::prof_begin("rope_table", st);
+      rope_table_kernel<<<grid_cap((int64_t)nc * 64, 256), 256, 0, st>>>(f.rope, nc, idx, blk, n_kept, blk, p.inv_freq);
+      ::jenga::prof_end(_ps, st);
+    }
+    JENGA_LAUNCH_CHECK();
     GemmOperand a2{f.tb, nc, LORA_PAD}, b2{p.lorab, 3 * HD, LORA_PAD};
     JENGA_TRY((launch_gemm<256, EPI_QKV_ROPE>({f.xn, nc, h}, {p.wqkv, 3 * HD, h}, h, &a2, &b2, LORA_PAD, nc, 3 * HD,
                                               e, st, "gemm_qkv_rope")));

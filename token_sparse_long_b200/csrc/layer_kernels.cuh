@@ -324,6 +324,25 @@ __global__ void lora_grad_reduce_kernel(LoraGradJobs jobs, const float* __restri
   jb.out[c * jb.so_c + r * jb.so_r] += jb.scale * s;
 }
 
+// RoPE table: tab[m][j] = (cos, sin)(position(m) * inv_freq[j]) for the rows m of a QKV GEMM
+// (position through the kept-block list when idx is given), the angle reduced to [-pi, pi] in
+// float64 before a float sincos.  Rows past the device-side valid count get position 0.
+__global__ void rope_table_kernel(float2* __restrict__ tab, int rows, const int32_t* __restrict__ idx, int blk,
+                                  const int32_t* __restrict__ n_valid, int valid_mult,
+                                  const double* __restrict__ inv_freq) {
+  const int nv = valid_rows(n_valid, valid_mult, 0, rows);
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < (int64_t)rows * 64;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int m = (int)(e >> 6), j = (int)(e & 63);
+    const int64_t pos = (m < nv) ? (idx ? seq_row(idx, blk, m) : m) : 0;
+    const double ang = (double)pos * inv_freq[j];
+    const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
+    float sn, cs;
+    sincosf((float)red, &sn, &cs);
+    tab[e] = make_float2(cs, sn);
+  }
+}
+
 // ---- weight re-layout (pack)
 // dst[(dr0 + c) * ldd + dc0 + r] = src[(sr0 + r) * lds + sc0 + c] for r < R, c < C   (transpose)
 __global__ void transpose_bf16_kernel(const bf16* __restrict__ src, int64_t lds, bf16* __restrict__ dst,
