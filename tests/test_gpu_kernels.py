@@ -218,6 +218,31 @@ def test_gather_scatter_random(J, dtype):
     assert torch.equal(x3, x)
 
 
+def test_gather_scatter_batched_pitched(J):
+    # two sequences, rows 136 bf16 wide (17 vectors: an odd divisor for the row split) inside
+    # a 200-wide pitch, block 32 (544 vectors per block: one partial chunk per block)
+    B, S, h, W, blk = 2, 2048, 136, 200, 32
+    g = torch.Generator(device="cuda").manual_seed(13)
+    xw = torch.randn(B, S, W, device="cuda", generator=g).to(torch.bfloat16)
+    x = xw[:, :, :h]
+    sc = synth.gen_scores(14, B, S // blk)
+    idx, nk, _ = J.jenga_select(torch.from_numpy(sc).cuda(), "topk_frac", 0.3)
+    n_cap = (S // blk) * blk
+    out = J.jenga_gather(x, idx, nk, blk, n_cap)
+    yw = torch.randn(B, n_cap, W, device="cuda", generator=g).to(torch.bfloat16)
+    y = yw[:, :, :h]
+    xw2 = xw.clone()
+    J.jenga_scatter_add(xw2[:, :, :h], y, idx, nk, blk, 0.5)
+    for b in range(B):
+        xi = idx.cpu().numpy()[b]
+        n = int(nk[b])
+        assert np.array_equal(torch_to_f64(out[b, : n * blk]), omv.gather(torch_to_f64(x[b]), xi, n, blk))
+        ref = omv.scatter_add(torch_to_f64(x[b]), torch_to_f64(y[b, : n * blk]), xi, n, blk, 0.5, "bf16")
+        assert np.array_equal(torch_to_f64(xw2[b, :, :h]), ref)
+    assert torch.equal(xw2[:, :, h:], xw[:, :, h:]), "the pitch padding is never written"
+    J.jenga_check_device_status()
+
+
 def test_scale_rows(J):
     x = torch.randn(64, 256, device="cuda").to(torch.bfloat16)
     rows = torch.tensor([3, 17, 40], dtype=torch.int32, device="cuda")

@@ -9,47 +9,72 @@
 
 namespace jenga {
 
-// One vector = 16 bytes.  Row r of the compact output maps to sequence row
-// idx[r / blk] * blk + r % blk.
-template <int UNROLL>
+// Unsigned division by a runtime constant d >= 1 as a multiply-high and a shift (the
+// round-up method of Granlund and Montgomery, "Division by invariant integers using
+// multiplication", 1994): with s = ceil(log2 d) and m = floor(2^32 (2^s - d) / d) + 1,
+// n / d = (umulhi(n, m) + n) >> s for every n < 2^31.
+struct FastDiv {
+  uint32_t d, mul, shift;
+};
+
+static FastDiv make_fastdiv(uint32_t d) {
+  uint32_t s = 0;
+  while ((1ull << s) < d) ++s;
+  const uint64_t m = ((1ull << 32) * ((1ull << s) - d)) / d + 1;
+  return FastDiv{d, (uint32_t)m, s};
+}
+
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f) {
+  return (__umulhi(n, f.mul) + n) >> f.shift;
+}
+
+// Work decomposition shared by gather and scatter-add: item w is chunk j = w % cpb of
+// kept block i = w / cpb, a chunk being MV_CHUNK consecutive vectors (16 bytes each) of the
+// block's blk x vpr vectors; vector e of block i is row e / vpr, column e % vpr.  Compact
+// row i * blk + t maps to sequence row idx[i] * blk + t.  Divisions are by invariant
+// constants (FastDiv) on 32-bit values: the item count and blk * vpr stay below 2^31.
+constexpr int MV_UNROLL = 8;
+constexpr int MV_CHUNK = 256 * MV_UNROLL;
+
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x, int64_t ldx_v,
                                                           int64_t bsx_v, uint4* __restrict__ out, int64_t ldo_v,
-                                                          int64_t bso_v, int vpr, int blk, int nb,
+                                                          int64_t bso_v, FastDiv vpr, FastDiv cpb, int blk, int nb,
                                                           const int32_t* __restrict__ idx,
                                                           const int32_t* __restrict__ n_kept, int n_cap) {
   const int b = blockIdx.y;
-  int nk = n_kept[b];
+  const int nk = n_kept[b];
   if (nk < 0 || (int64_t)nk * blk > n_cap || nk > nb) {
     if (threadIdx.x == 0 && blockIdx.x == 0) record_device_error(JENGA_EINTERNAL, SITE_NKEPT_RANGE, nk);
     return;
   }
   const int32_t* ib = idx + (int64_t)b * nb;
-  const int64_t total = (int64_t)nk * blk * vpr;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t e0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e0 < total; e0 += stride * UNROLL) {
-    uint4 v[UNROLL];
-    int64_t dst[UNROLL];
+  const uint32_t per_blk = (uint32_t)blk * vpr.d;
+  const uint32_t items = (uint32_t)nk * cpb.d;
+  for (uint32_t w = blockIdx.x; w < items; w += gridDim.x) {
+    const uint32_t bi = fast_div(w, cpb), j = w - bi * cpb.d;
+    const int src_blk = __ldg(ib + bi);
+    if (src_blk < 0 || src_blk >= nb) {
+      if (threadIdx.x == 0) record_device_error(JENGA_EINTERNAL, SITE_INDEX_RANGE, (unsigned)src_blk);
+      continue;
+    }
+    const uint4* src = x + b * bsx_v + (int64_t)src_blk * blk * ldx_v;
+    uint4* dst = out + b * bso_v + (int64_t)bi * blk * ldo_v;
+    uint4 v[MV_UNROLL];
+    int64_t so[MV_UNROLL], dof[MV_UNROLL];
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      int64_t e = e0 + (int64_t)u * stride;
-      dst[u] = -1;
-      if (e < total) {
-        int64_t r = e / vpr;
-        int c = (int)(e - r * vpr);
-        int blk_i = (int)(r / blk);
-        int t = (int)(r - (int64_t)blk_i * blk);
-        int src_blk = __ldg(ib + blk_i);
-        if (src_blk < 0 || src_blk >= nb) {
-          record_device_error(JENGA_EINTERNAL, SITE_INDEX_RANGE, (unsigned)src_blk);
-          continue;
-        }
-        v[u] = __ldcs(x + b * bsx_v + ((int64_t)src_blk * blk + t) * ldx_v + c);
-        dst[u] = b * bso_v + r * ldo_v + c;
+    for (int u = 0; u < MV_UNROLL; ++u) {
+      const uint32_t e = j * MV_CHUNK + u * 256 + threadIdx.x;
+      so[u] = -1;
+      if (e < per_blk) {
+        const uint32_t t = fast_div(e, vpr), c = e - t * vpr.d;
+        so[u] = (int64_t)t * ldx_v + c;
+        dof[u] = (int64_t)t * ldo_v + c;
+        v[u] = __ldcs(src + so[u]);
       }
     }
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u)
-      if (dst[u] >= 0) out[dst[u]] = v[u];
+    for (int u = 0; u < MV_UNROLL; ++u)
+      if (so[u] >= 0) dst[dof[u]] = v[u];
   }
 }
 
@@ -85,47 +110,48 @@ __device__ __forceinline__ uint4 axpy_vec(uint4 xv, uint4 yv, float alpha) {
   return o;
 }
 
-template <bool BF16, int UNROLL>
+// x[seq row] = x + alpha * y[compact row] in place, same decomposition as the gather
+template <bool BF16>
 __global__ void __launch_bounds__(256) scatter_add_kernel(uint4* __restrict__ x, int64_t ldx_v, int64_t bsx_v,
                                                           const uint4* __restrict__ y, int64_t ldy_v,
-                                                          int64_t bsy_v, int vpr, int blk, int nb,
+                                                          int64_t bsy_v, FastDiv vpr, FastDiv cpb, int blk, int nb,
                                                           const int32_t* __restrict__ idx,
                                                           const int32_t* __restrict__ n_kept, int n_cap,
                                                           float alpha) {
   const int b = blockIdx.y;
-  int nk = n_kept[b];
+  const int nk = n_kept[b];
   if (nk < 0 || (int64_t)nk * blk > n_cap || nk > nb) {
     if (threadIdx.x == 0 && blockIdx.x == 0) record_device_error(JENGA_EINTERNAL, SITE_NKEPT_RANGE, nk);
     return;
   }
   const int32_t* ib = idx + (int64_t)b * nb;
-  const int64_t total = (int64_t)nk * blk * vpr;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t e0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e0 < total; e0 += stride * UNROLL) {
-    uint4 xv[UNROLL], yv[UNROLL];
-    int64_t dst[UNROLL];
+  const uint32_t per_blk = (uint32_t)blk * vpr.d;
+  const uint32_t items = (uint32_t)nk * cpb.d;
+  for (uint32_t w = blockIdx.x; w < items; w += gridDim.x) {
+    const uint32_t bi = fast_div(w, cpb), j = w - bi * cpb.d;
+    const int dst_blk = __ldg(ib + bi);
+    if (dst_blk < 0 || dst_blk >= nb) {
+      if (threadIdx.x == 0) record_device_error(JENGA_EINTERNAL, SITE_INDEX_RANGE, (unsigned)dst_blk);
+      continue;
+    }
+    uint4* xb = x + b * bsx_v + (int64_t)dst_blk * blk * ldx_v;
+    const uint4* yb = y + b * bsy_v + (int64_t)bi * blk * ldy_v;
+    uint4 xv[MV_UNROLL], yv[MV_UNROLL];
+    int64_t xo[MV_UNROLL];
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      int64_t e = e0 + (int64_t)u * stride;
-      dst[u] = -1;
-      if (e < total) {
-        int64_t r = e / vpr;
-        int c = (int)(e - r * vpr);
-        int blk_i = (int)(r / blk);
-        int t = (int)(r - (int64_t)blk_i * blk);
-        int dst_blk = __ldg(ib + blk_i);
-        if (dst_blk < 0 || dst_blk >= nb) {
-          record_device_error(JENGA_EINTERNAL, SITE_INDEX_RANGE, (unsigned)dst_blk);
-          continue;
-        }
-        dst[u] = b * bsx_v + ((int64_t)dst_blk * blk + t) * ldx_v + c;
-        yv[u] = __ldcs(y + b * bsy_v + r * ldy_v + c);
-        xv[u] = x[dst[u]];
+    for (int u = 0; u < MV_UNROLL; ++u) {
+      const uint32_t e = j * MV_CHUNK + u * 256 + threadIdx.x;
+      xo[u] = -1;
+      if (e < per_blk) {
+        const uint32_t t = fast_div(e, vpr), c = e - t * vpr.d;
+        xo[u] = (int64_t)t * ldx_v + c;
+        yv[u] = __ldcs(yb + (int64_t)t * ldy_v + c);
+        xv[u] = xb[xo[u]];
       }
     }
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u)
-      if (dst[u] >= 0) x[dst[u]] = axpy_vec<BF16>(xv[u], yv[u], alpha);
+    for (int u = 0; u < MV_UNROLL; ++u)
+      if (xo[u] >= 0) xb[xo[u]] = axpy_vec<BF16>(xv[u], yv[u], alpha);
   }
 }
 
@@ -178,12 +204,16 @@ extern "C" jenga_status jenga_gather(const void* x, int64_t ldx, int B, int S, i
   if (n_cap == 0) return JENGA_OK;
   const int vpr = h * es / 16;
   const int64_t ldx_v = ldx * es / 16, ldo_v = ldo * es / 16;
-  dim3 grid(grid_for((int64_t)n_cap * vpr, 4), B);
+  JENGA_CHECK_ARG((int64_t)blk * vpr < (1ll << 30) && (int64_t)n_cap * vpr < (1ll << 40),
+                  "jenga_gather: rows too long");
+  const int cpb = (int)(((int64_t)blk * vpr + MV_CHUNK - 1) / MV_CHUNK);
+  JENGA_CHECK_ARG((int64_t)(S / blk) * cpb < (1ll << 31), "jenga_gather: too many blocks");
+  dim3 grid(grid_for((int64_t)n_cap * vpr, MV_UNROLL), B);
   {
   const int _ps = ::jenga::prof_begin("gather_rows", (cudaStream_t)stream);
-  gather_rows_kernel<4><<<grid, 256, 0, (cudaStream_t)stream>>>(
-      (const uint4*)x, ldx_v, (int64_t)S * ldx_v, (uint4*)out, ldo_v, (int64_t)n_cap * ldo_v, vpr, blk, S / blk,
-      idx, n_kept, n_cap);
+  gather_rows_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(
+      (const uint4*)x, ldx_v, (int64_t)S * ldx_v, (uint4*)out, ldo_v, (int64_t)n_cap * ldo_v, make_fastdiv(vpr),
+      make_fastdiv(cpb), blk, S / blk, idx, n_kept, n_cap);
   ::jenga::prof_end(_ps, (cudaStream_t)stream);
   }
   JENGA_LAUNCH_CHECK();
@@ -205,20 +235,24 @@ extern "C" jenga_status jenga_scatter_add(void* x, int64_t ldx, const void* y, i
   if (n_cap == 0) return JENGA_OK;
   const int vpr = h * es / 16;
   const int64_t ldx_v = ldx * es / 16, ldy_v = ldy * es / 16;
-  dim3 grid(grid_for((int64_t)n_cap * vpr, 4), B);
+  JENGA_CHECK_ARG((int64_t)blk * vpr < (1ll << 30), "jenga_scatter_add: rows too long");
+  const int cpb = (int)(((int64_t)blk * vpr + MV_CHUNK - 1) / MV_CHUNK);
+  JENGA_CHECK_ARG((int64_t)(S / blk) * cpb < (1ll << 31), "jenga_scatter_add: too many blocks");
+  const FastDiv vd = make_fastdiv(vpr), cd = make_fastdiv(cpb);
+  dim3 grid(grid_for((int64_t)n_cap * vpr, MV_UNROLL), B);
   if (dt == JENGA_BF16)
     {
     const int _ps = ::jenga::prof_begin("scatter_add", (cudaStream_t)stream);
-    scatter_add_kernel<true, 4><<<grid, 256, 0, (cudaStream_t)stream>>>(
-        (uint4*)x, ldx_v, (int64_t)S * ldx_v, (const uint4*)y, ldy_v, (int64_t)n_cap * ldy_v, vpr, blk, S / blk,
+    scatter_add_kernel<true><<<grid, 256, 0, (cudaStream_t)stream>>>(
+        (uint4*)x, ldx_v, (int64_t)S * ldx_v, (const uint4*)y, ldy_v, (int64_t)n_cap * ldy_v, vd, cd, blk, S / blk,
         idx, n_kept, n_cap, alpha);
     ::jenga::prof_end(_ps, (cudaStream_t)stream);
     }
   else
     {
     const int _ps = ::jenga::prof_begin("scatter_add", (cudaStream_t)stream);
-    scatter_add_kernel<false, 4><<<grid, 256, 0, (cudaStream_t)stream>>>(
-        (uint4*)x, ldx_v, (int64_t)S * ldx_v, (const uint4*)y, ldy_v, (int64_t)n_cap * ldy_v, vpr, blk, S / blk,
+    scatter_add_kernel<false><<<grid, 256, 0, (cudaStream_t)stream>>>(
+        (uint4*)x, ldx_v, (int64_t)S * ldx_v, (const uint4*)y, ldy_v, (int64_t)n_cap * ldy_v, vd, cd, blk, S / blk,
         idx, n_kept, n_cap, alpha);
     ::jenga::prof_end(_ps, (cudaStream_t)stream);
     }
