@@ -261,7 +261,8 @@ def measure_movement(J, torch, dev, X0, case, ks, hbm):
     (ABS_GE) over 2^26 fp32 scores.  Algorithmic bytes: gather 2 n h e, scatter-add 3 n h e
     (eliminated rows cost nothing), select 4 nb read + 4 nb (idx, -1 past n_kept) + nb + 4
     written.  Each
-    call moves more than the 126 MB L2; CUDA events, median of 10 after 3 warm-ups."""
+    call moves more than the 126 MB L2; CUDA events around 10 back-to-back calls, median of 5
+    such groups after 3 warm-ups."""
     blk, S, h = case.blk, case.S, X0.shape[1]
     nb = S // blk
     k0 = ks[0]
@@ -272,17 +273,20 @@ def measure_movement(J, torch, dev, X0, case, ks, hbm):
     xg = torch.empty(n, h, dtype=X0.dtype, device=dev)
     x2 = X0.clone()
 
-    def med(fn):
+    def med(fn, reps=10):
+        # device time per call: `reps` calls back to back between two events (the host
+        # enqueues ahead of the device, so launch latency is not timed), median of 5
         for _ in range(3):
             fn()
         ts = []
-        for _ in range(10):
+        for _ in range(5):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
-            fn()
+            for _ in range(reps):
+                fn()
             b.record()
             torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b) / 1e3)
+            ts.append(a.elapsed_time(b) / 1e3 / reps)
         return sorted(ts)[len(ts) // 2]
 
     out = {}
