@@ -10,20 +10,20 @@
 //                 epilogue's packed f32x2 arithmetic adds them)
 //                 dV  += P^T dO       dK  += dS^T Q           (A: smem K-major, B: MN-major)
 //               and at the end dV, dK (x 1/sqrt(D)) are added into fp32 accumulators.
-//   dQ pass     one CTA per (128-query tile of the segment, head).  Q and dO resident; the
-//               64-key tiles of K and V stream.  S = Q K^T, dP = dO V^T, dS = P (dP - Delta),
-//               dQ += dS K; dQ (x 1/sqrt(D)) stored fp32.
-// The Q/dO (K/V) ring is 3 (4) stages deep: a stage is read by both products of its tile,
-// so with 2 stages the next tile's load could only start once the gradient product that
-// immediately precedes that tile's score product had finished.
+//   dQ pass     one CTA per (128-query tile of the segment, head).  Q and dO resident in
+//               tensor memory; the 64-key tiles of K and V stream through a 5-stage ring.
+//               S = Q K^T, dP = dO V^T (double-buffered), dS = P (dP - Delta), dQ += dS K;
+//               dQ (x 1/sqrt(D)) stored fp32.
+// A ring stage is read by the score products and the gradient product of its tile, which
+// runs an epilogue later, so the rings hold 4 (Q/dO) and 5 (K/V) tiles.
 // Warp roles (a warp can issue a tcgen05.mma only every ~100 clocks, so one issuer would
 // cap these M 128 x N 64 / N 128 products well below the tensor peak, and an issuer that
 // also waits on the epilogue stalls the products queued behind that wait):
 //   dK/dV pass  0 TMA; 1 S^T, 2 dP^T, 3 dV, 4 dK issue (1 also allocates TMEM); 5..20
 //               epilogue in four quads, quad c taking columns 16c .. 16c + 15 of a tile (two
 //               epilogue warps per SMSP left the exponentials latency-bound)
-//   dQ pass     0 TMA; 1 S and dQ, 2 dP issue; 3..10 epilogue in two quads (first / last
-//               32 columns)
+//   dQ pass     0 TMA; 1 S, 2 dP, 3 dQ issue (1 also allocates TMEM); 4..19 epilogue in four
+//               quads, quad c taking key columns 16c .. 16c + 15
 // Each quad covers all 128 TMEM lanes, one row per thread.  P / dS tiles are double-buffered in shared memory so the epilogue of
 // tile i overlaps the gradient products of tile i-1 and the score products of tile i+1.
 // Causal masking, keys / queries past the valid count, and the segment bounds are applied
@@ -36,7 +36,9 @@ namespace jenga {
 
 constexpr int ABT_BOX128 = 128 * 64 * 2;   // 16 KB box: 128 rows x 64 bf16
 constexpr int ABT_BOX64 = 64 * 64 * 2;     // 8 KB box: 64 rows x 64 bf16
-constexpr int ABT_THREADS = 352;  // dQ pass: warps 0 TMA, 1 and 2 MMA issue, 3 .. 10 epilogue
+constexpr int DQ_EPI_WARP0 = 4;   // dQ pass: warps 0 TMA, 1 S, 2 dP, 3 dQ issue, 4 .. 19 epilogue
+constexpr int DQ_EPI_WARPS = 16;
+constexpr int ABT_THREADS = 32 * (DQ_EPI_WARP0 + DQ_EPI_WARPS);
 constexpr int DKV_EPI_WARPS = 16;
 constexpr int DKV_EPI_WARP0 = 5;  // dK/dV pass: warps 0 TMA, 1 .. 4 MMA issue, 5 .. 20 epilogue
 constexpr int DKV_THREADS = 32 * (DKV_EPI_WARP0 + DKV_EPI_WARPS);
@@ -53,15 +55,17 @@ constexpr int DKV_LD_BYTES = 512;
 constexpr int DKV_BAR_OFF = DKV_LD_OFF + DKV_STAGES * DKV_LD_BYTES;
 constexpr int DKV_SMEM = DKV_BAR_OFF + 256 + 1024;
 
-// smem layout of the dQ pass
+// smem layout of the dQ pass.  Q and dO are staged and copied into tensor memory (the A
+// operands of S and dP) before the first tile; the Q staging then holds the dS buffers.
 constexpr int DQ_Q_OFF = 0;
 constexpr int DQ_DO_OFF = 2 * ABT_BOX128;
+constexpr int DQ_DS_OFF = DQ_Q_OFF;                        // [2] x 128 x 64 bf16, after the copy
 constexpr int DQ_RING_OFF = 4 * ABT_BOX128;                // stage s: K (2 x 8 KB), V (2 x 8 KB)
 constexpr int DQ_STAGE = 4 * ABT_BOX64;
-constexpr int DQ_STAGES = 4;  // a stage lives from S(j) to the dQ product of tile j
-constexpr int DQ_DS_OFF = DQ_RING_OFF + DQ_STAGES * DQ_STAGE;  // [2] x 128 x 64 bf16
-constexpr int DQ_BAR_OFF = DQ_DS_OFF + 2 * ABT_BOX128;
+constexpr int DQ_STAGES = 5;  // a stage lives from S(j) to the dQ product of tile j
+constexpr int DQ_BAR_OFF = DQ_RING_OFF + DQ_STAGES * DQ_STAGE;
 constexpr int DQ_SMEM = DQ_BAR_OFF + 256 + 1024;
+static_assert(DQ_SMEM <= 232448 && DKV_SMEM <= 232448, "shared memory per CTA");
 
 // Write 32 bf16 values (packed pairs pk[0..15]) as columns [32 * half, 32 * half + 32) of
 // row r of a 128 x 64 K-major tile with the 128-byte swizzle (row = 8 chunks of 16 bytes).
@@ -374,13 +378,14 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DQ_BAR_OFF);
   uint64_t* qd_full = bars;
   uint64_t* kv_full = bars + 1;               // [DQ_STAGES]
-  uint64_t* kv_empty = kv_full + DQ_STAGES;   // [DQ_STAGES]
+  uint64_t* kv_empty = kv_full + DQ_STAGES;   // [DQ_STAGES]: S, dP and dQ products read a stage
   uint64_t* s_full = kv_empty + DQ_STAGES;    // [2]
   uint64_t* s_free = s_full + 2;     // [2]
   uint64_t* ds_full = s_free + 2;    // [2]
   uint64_t* ds_free = ds_full + 2;   // [2]
   uint64_t* done = ds_free + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* qd_tmem = done + 1;      // Q and dO are in tensor memory
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qd_tmem + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
@@ -397,15 +402,16 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     mbar_init(qd_full, 1);
     for (int s = 0; s < DQ_STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 2);
+      mbar_init(&kv_empty[s], 3);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 2);
-      mbar_init(&s_free[s], 8);
-      mbar_init(&ds_full[s], 8);
+      mbar_init(&s_free[s], DQ_EPI_WARPS);
+      mbar_init(&ds_full[s], DQ_EPI_WARPS);
       mbar_init(&ds_free[s], 1);
     }
     mbar_init(done, 1);
+    mbar_init(qd_tmem, 8);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -416,7 +422,9 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tdQ = tmem + 256;  // S[2] at 0, 64; dP[2] at 128, 192; dQ at 256
+  // TMEM columns: S[2] 0, 64; dP[2] 128, 192; dQ 256..383; Q 384..447, dO 448..511 (bf16
+  // pairs, A operands)
+  const uint32_t tdQ = tmem + 256, tQ = tmem + 384, tDO = tmem + 448;
 
   if (warp == 0 && lane == 0) {
     mbar_arrive_expect_tx(qd_full, 4 * ABT_BOX128);
@@ -434,73 +442,57 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
       tma_load_2d(st + 2 * ABT_BOX64, &tmV, &kv_full[s], col, j * 64);
       tma_load_2d(st + 3 * ABT_BOX64, &tmV, &kv_full[s], col + 64, j * 64);
     }
-  } else if (warp == 1 && lane == 0) {
-    // warp 1 issues S and dQ; warp 2 issues dP (two issuers: see the dK/dV pass)
+  } else if ((warp == 1 || warp == 2) && lane == 0) {
+    // score products, one issuing warp each: warp 1 S = Q K^T, warp 2 dP = dO V^T, A (Q, dO)
+    // from tensor memory, B (K, V) from the ring, double-buffered accumulators
+    const bool s_chain = (warp == 1);
     constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64);
+    const uint32_t ta = s_chain ? tQ : tDO;
+    const uint32_t acc0 = tmem + (s_chain ? 0 : 128);
+    const int b_off = s_chain ? 0 : 2 * ABT_BOX64;  // K or V
+    bool ok = mbar_wait_at(qd_tmem, 0, 132, 0);
+    for (int j = 0; ok && j < nk; ++j) {
+      const int s = j & 1, rs = j % DQ_STAGES;
+      if (!mbar_wait_at(&kv_full[rs], (j / DQ_STAGES) & 1, 134, j)) break;
+      if (j >= 2 && !mbar_wait_at(&s_free[s], ((j >> 1) - 1) & 1, 135, j)) break;
+      tc_fence_after();
+      const uint32_t st = smem_u32(smem + DQ_RING_OFF + rs * DQ_STAGE + b_off);
+#pragma unroll
+      for (int kc = 0; kc < 2; ++kc)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_bf16_ts(acc0 + s * 64, ta + kc * 32 + k * 8, umma_desc_k_sw128(st + kc * ABT_BOX64 + k * 32), idesc_s,
+                       (kc | k) ? 1u : 0u);
+      umma_commit(&s_full[s]);
+      umma_commit(&kv_empty[rs]);
+    }
+  } else if (warp == 3 && lane == 0) {
+    // dQ += dS K as soon as the epilogue has written tile j's dS (A: smem K-major, B: the
+    // ring's K tile MN-major)
     constexpr uint32_t idesc_g = umma_idesc_bf16_bmn(128, 128);
-    const uint32_t qa = smem_u32(smem + DQ_Q_OFF);
-    bool ok = mbar_wait_at(qd_full, 0, 132, 0);
-    auto issue_dq = [&](int jj) -> bool {
-      const int b = jj & 1, rs = jj % DQ_STAGES;
-      if (!mbar_wait_at(&ds_full[b], (jj >> 1) & 1, 133, jj)) return false;
+    bool ok = true;
+    for (int j = 0; j < nk; ++j) {
+      const int b = j & 1, rs = j % DQ_STAGES;
+      if (!mbar_wait_at(&ds_full[b], (j >> 1) & 1, 133, j)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const uint32_t ks_ = smem_u32(smem + DQ_RING_OFF + rs * DQ_STAGE);
       const uint32_t dsa = smem_u32(smem + DQ_DS_OFF + b * ABT_BOX128);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
         umma_bf16(tdQ, umma_desc_k_sw128(dsa + ks * 32), umma_desc_mn_sw128(ks_ + ks * 2048, ABT_BOX64), idesc_g,
-                  (jj > 0 || ks > 0) ? 1u : 0u);
+                  (j > 0 || ks > 0) ? 1u : 0u);
       umma_commit(&ds_free[b]);
       umma_commit(&kv_empty[rs]);
-      return true;
-    };
-    for (int j = 0; ok && j < nk; ++j) {
-      const int s = j & 1, rs = j % DQ_STAGES;
-      if (!mbar_wait_at(&kv_full[rs], (j / DQ_STAGES) & 1, 134, j)) {
-        ok = false;
-        break;
-      }
-      if (j >= 2 && !mbar_wait_at(&s_free[s], ((j >> 1) - 1) & 1, 135, j)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t st = smem_u32(smem + DQ_RING_OFF + rs * DQ_STAGE);
-#pragma unroll
-      for (int kc = 0; kc < 2; ++kc)
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          umma_bf16(tmem + s * 64, umma_desc_k_sw128(qa + kc * ABT_BOX128 + k * 32),
-                    umma_desc_k_sw128(st + kc * ABT_BOX64 + k * 32), idesc_s, (kc | k) ? 1u : 0u);
-      umma_commit(&s_full[s]);
-      if (j >= 1 && !issue_dq(j - 1)) {
-        ok = false;
-        break;
-      }
     }
-    if (ok && issue_dq(nk - 1)) umma_commit(done);
-  } else if (warp == 2 && lane == 0) {
-    constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64);
-    const uint32_t da = smem_u32(smem + DQ_DO_OFF);
-    bool ok = mbar_wait_at(qd_full, 0, 139, 0);
-    for (int j = 0; ok && j < nk; ++j) {
-      const int s = j & 1, rs = j % DQ_STAGES;
-      if (!mbar_wait_at(&kv_full[rs], (j / DQ_STAGES) & 1, 140, j)) break;
-      if (j >= 2 && !mbar_wait_at(&s_free[s], ((j >> 1) - 1) & 1, 141, j)) break;
-      tc_fence_after();
-      const uint32_t st = smem_u32(smem + DQ_RING_OFF + rs * DQ_STAGE);
-#pragma unroll
-      for (int kc = 0; kc < 2; ++kc)
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          umma_bf16(tmem + 128 + s * 64, umma_desc_k_sw128(da + kc * ABT_BOX128 + k * 32),
-                    umma_desc_k_sw128(st + 2 * ABT_BOX64 + kc * ABT_BOX64 + k * 32), idesc_s, (kc | k) ? 1u : 0u);
-      umma_commit(&s_full[s]);
-      umma_commit(&kv_empty[rs]);
-    }
-  } else if (warp >= 3) {
+    if (ok) umma_commit(done);
+  } else if (warp >= DQ_EPI_WARP0) {
+    // 16 epilogue warps in four quads: quad c takes key columns 16c .. 16c + 15 of every
+    // 64-key tile, one query row per thread
     const int quarter = warp & 3;
-    const int half = (warp - 3) >> 2;
+    const int quad = (warp - DQ_EPI_WARP0) >> 2;
     const int r = quarter * 32 + lane;
     const int q = q0 + r;
     const uint32_t lo = (uint32_t)(quarter * 32) << 16;
@@ -509,25 +501,39 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     const float Dq = qvalid ? delta[(int64_t)h * delta_ld + q - s0] : 0.f;  // -Delta
     const uint64_t sl2x2 = f2pack(scale_log2, scale_log2), nL2 = f2pack(L, L), nD2 = f2pack(Dq, Dq);
     bool ok = true;
-    for (int j = 0; j < nk; ++j) {
+    if (quad < 2) {
+      // quad 0 copies Q, quad 1 dO from their staging tiles into tensor memory
+      if (__all_sync(0xffffffffu, mbar_wait_at(qd_full, 0, 139, 0))) {
+        tile_row_to_tmem(smem + (quad == 0 ? DQ_Q_OFF : DQ_DO_OFF), r, (quad == 0 ? tQ : tDO) + lo);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(qd_tmem);
+      } else {
+        ok = false;
+      }
+    }
+    // the Q staging tiles become the dS buffers only after every copy is done
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * DQ_EPI_WARPS) : "memory");
+    for (int j = 0; ok && j < nk; ++j) {
       const int s = j & 1;
       if (!__all_sync(0xffffffffu, mbar_wait_at(&s_full[s], (j >> 1) & 1, 136, j))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sv[32], dp[32];
-      tmem_ld32_nowait(tmem + lo + s * 64 + half * 32, sv);
-      tmem_ld32_nowait(tmem + lo + 128 + s * 64 + half * 32, dp);
+      uint32_t sv[16], dp[16];
+      tmem_ld16_nowait(tmem + lo + s * 64 + quad * 16, sv);
+      tmem_ld16_nowait(tmem + lo + 128 + s * 64 + quad * 16, dp);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[s]);
-      const int lim = qvalid ? min(q + 1, n) - j * 64 - half * 32 : 0;  // valid keys of this half: c < lim
-      uint32_t dk[16];
-      if (lim >= 32) {  // every key of this half is live for this row
+      const int lim = qvalid ? min(q + 1, n) - j * 64 - quad * 16 : 0;  // valid keys of this quad: c < lim
+      uint32_t dk[8];
+      if (lim >= 16) {  // every key of this quad is live for this row
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
+        for (int c = 0; c < 16; c += 2) {
           const uint64_t p2 =
               exp2_mufu_x2(ffma2(f2pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, nL2));
           const uint64_t d2 = fmul2(p2, fadd2(f2pack(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), nD2));
@@ -537,7 +543,7 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
+        for (int c = 0; c < 16; c += 2) {
           float d2[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
@@ -552,7 +558,7 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
         ok = false;
         break;
       }
-      st_row32_sw128(smem + DQ_DS_OFF + s * ABT_BOX128, r, half, dk);
+      st_row16_sw128(smem + DQ_DS_OFF + s * ABT_BOX128, r, quad, dk);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -560,19 +566,16 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     }
     if (__all_sync(0xffffffffu, ok && mbar_wait_at(done, 0, 138, nk))) {
       tc_fence_after();
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c0 = half * 64 + cc * 32;
-        uint32_t a[32];
-        tmem_ld32_nowait(tdQ + lo + c0, a);
-        tmem_wait_ld();
-        if (qvalid) {
-          float4* dst = reinterpret_cast<float4*>(dq_out + (int64_t)(q - s0) * ld_dq + col + c0);
+      const int c0 = quad * 32;  // this quad's 32 of the 128 head dimensions
+      uint32_t a[32];
+      tmem_ld32_nowait(tdQ + lo + c0, a);
+      tmem_wait_ld();
+      if (qvalid) {
+        float4* dst = reinterpret_cast<float4*>(dq_out + (int64_t)(q - s0) * ld_dq + col + c0);
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4)
-            dst[q4] = make_float4(__uint_as_float(a[4 * q4]) * scale, __uint_as_float(a[4 * q4 + 1]) * scale,
-                                  __uint_as_float(a[4 * q4 + 2]) * scale, __uint_as_float(a[4 * q4 + 3]) * scale);
-        }
+        for (int q4 = 0; q4 < 8; ++q4)
+          dst[q4] = make_float4(__uint_as_float(a[4 * q4]) * scale, __uint_as_float(a[4 * q4 + 1]) * scale,
+                                __uint_as_float(a[4 * q4 + 2]) * scale, __uint_as_float(a[4 * q4 + 3]) * scale);
       }
     }
   }
