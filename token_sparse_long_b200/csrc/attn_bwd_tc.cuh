@@ -22,8 +22,8 @@
 //   dK/dV pass  0 TMA; 1 S^T, 2 dP^T, 3 dV, 4 dK issue (1 also allocates TMEM); 5..20
 //               epilogue in four quads, quad c taking columns 16c .. 16c + 15 of a tile (two
 //               epilogue warps per SMSP left the exponentials latency-bound)
-//   dQ pass     0 TMA; 1 S, 2 dP, 3 dQ issue (1 also allocates TMEM); 4..19 epilogue in four
-//               quads, quad c taking key columns 16c .. 16c + 15
+//   dQ pass     0 TMA; 1-2 S, 3-4 dP (even / odd tiles), 5 dQ issue (1 also allocates TMEM);
+//               6..21 epilogue in four quads, quad c taking key columns 16c .. 16c + 15
 // Each quad covers all 128 TMEM lanes, one row per thread.  P / dS tiles are double-buffered in shared memory so the epilogue of
 // tile i overlaps the gradient products of tile i-1 and the score products of tile i+1.
 // Causal masking, keys / queries past the valid count, and the segment bounds are applied
@@ -36,7 +36,7 @@ namespace jenga {
 
 constexpr int ABT_BOX128 = 128 * 64 * 2;   // 16 KB box: 128 rows x 64 bf16
 constexpr int ABT_BOX64 = 64 * 64 * 2;     // 8 KB box: 64 rows x 64 bf16
-constexpr int DQ_EPI_WARP0 = 4;   // dQ pass: warps 0 TMA, 1 S, 2 dP, 3 dQ issue, 4 .. 19 epilogue
+constexpr int DQ_EPI_WARP0 = 6;   // dQ pass: warps 0 TMA, 1-2 S, 3-4 dP, 5 dQ issue, 6 .. 21 epilogue
 constexpr int DQ_EPI_WARPS = 16;
 constexpr int ABT_THREADS = 32 * (DQ_EPI_WARP0 + DQ_EPI_WARPS);
 constexpr int DKV_EPI_WARPS = 16;
@@ -442,16 +442,18 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
       tma_load_2d(st + 2 * ABT_BOX64, &tmV, &kv_full[s], col, j * 64);
       tma_load_2d(st + 3 * ABT_BOX64, &tmV, &kv_full[s], col + 64, j * 64);
     }
-  } else if ((warp == 1 || warp == 2) && lane == 0) {
-    // score products, one issuing warp each: warp 1 S = Q K^T, warp 2 dP = dO V^T, A (Q, dO)
-    // from tensor memory, B (K, V) from the ring, double-buffered accumulators
-    const bool s_chain = (warp == 1);
+  } else if (warp >= 1 && warp <= 4 && lane == 0) {
+    // score products: warps 1 and 2 S = Q K^T, warps 3 and 4 dP = dO V^T, each warp the
+    // tiles of one parity (its accumulator buffer), so the two buffers fill concurrently;
+    // A (Q, dO) from tensor memory, B (K, V) from the ring
+    const bool s_chain = (warp <= 2);
+    const int par = (warp - 1) & 1;
     constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64);
     const uint32_t ta = s_chain ? tQ : tDO;
     const uint32_t acc0 = tmem + (s_chain ? 0 : 128);
     const int b_off = s_chain ? 0 : 2 * ABT_BOX64;  // K or V
     bool ok = mbar_wait_at(qd_tmem, 0, 132, 0);
-    for (int j = 0; ok && j < nk; ++j) {
+    for (int j = par; ok && j < nk; j += 2) {
       const int s = j & 1, rs = j % DQ_STAGES;
       if (!mbar_wait_at(&kv_full[rs], (j / DQ_STAGES) & 1, 134, j)) break;
       if (j >= 2 && !mbar_wait_at(&s_free[s], ((j >> 1) - 1) & 1, 135, j)) break;
@@ -466,7 +468,7 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
       umma_commit(&s_full[s]);
       umma_commit(&kv_empty[rs]);
     }
-  } else if (warp == 3 && lane == 0) {
+  } else if (warp == 5 && lane == 0) {
     // dQ += dS K as soon as the epilogue has written tile j's dS (A: smem K-major, B: the
     // ring's K tile MN-major)
     constexpr uint32_t idesc_g = umma_idesc_bf16_bmn(128, 128);
