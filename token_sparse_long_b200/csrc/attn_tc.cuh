@@ -1,21 +1,21 @@
 // tcgen05 causal attention forward over the retained tokens (head_dim 128).
 //
 // One CTA per (128-query tile, head), 352 threads:
-//   warp 0      TMA: the Q tile once, then K_j through a 2-stage ring and V_j through a
-//               3-stage ring (K_j is free once S_j is computed, V_j only after the PV
-//               product, so separate rings let each load start as early as it can)
-//   warp 1      TMEM allocation (S0 | S1 | O, 384 of 512 columns); one lane issues
+//   warp 0      TMA: the Q tile once, then K_j and V_j through two 3-stage rings (K_j is
+//               free once S_j is computed, V_j only after the PV product, so separate rings
+//               let each load start as early as it can)
+//   warp 1      TMEM allocation (S0 | S1 | O | P0 | P1); one lane issues
 //                 S_j = Q K_j^T            (A = Q smem K-major, B = K_j smem K-major) into S[j % 2]
-//   warp 2      one lane issues O += P_j V_j (A = P smem K-major, B = V smem MN-major) into O
+//   warp 2      one lane issues O += P_j V_j (A = P_j from tensor memory, B = V smem MN-major)
 //   warps 3..10 softmax, one TMEM lane (= one query row) per thread and one half of the
 //               key columns per warp (warps w and w + 4 share rows and exchange their
 //               half-row maxima): load S_j, mask (causal diagonal, keys past n; only on
 //               those tiles), online max with lazy rescaling (O and l are rescaled in TMEM
 //               only when the running max grows by more than 2^8), P = 2^(s log2e /
-//               sqrt(D) - m) as bf16 into a 128-byte-swizzled smem tile (one exponential in
+//               sqrt(D) - m) as bf16 pairs into tensor memory P[j % 2] (one exponential in
 //               four on the FMA pipe, exp2_fma), row sums in fp32
 // The softmax of tile j overlaps the PV product of tile j-1 and the QK^T product of
-// tile j+1.  Output o = O / l (bf16) and the negated row log-sum-exp in log2 units (the
+// tile j+1; with P double-buffered it waits only for the PV product of tile j-2.  Output o = O / l (bf16) and the negated row log-sum-exp in log2 units (the
 // backward adds it to the scaled logits directly).
 #pragma once
 
@@ -24,17 +24,17 @@
 namespace jenga {
 
 constexpr int ATC_ROWS = 128;
-constexpr int ATC_K_STAGES = 2;
+constexpr int ATC_K_STAGES = 3;
 constexpr int ATC_V_STAGES = 3;
 constexpr int ATC_BOX = 128 * 64 * 2;     // 16 KB: 128 rows x 64 bf16
 constexpr int ATC_TILE = 2 * ATC_BOX;      // 32 KB: 128 x 128
 constexpr int ATC_Q_OFF = 0;
 constexpr int ATC_K_OFF = ATC_TILE;                             // K stage s at + s * TILE
 constexpr int ATC_V_OFF = ATC_K_OFF + ATC_K_STAGES * ATC_TILE;  // V stage s at + s * TILE
-constexpr int ATC_P_OFF = ATC_V_OFF + ATC_V_STAGES * ATC_TILE;
-constexpr int ATC_XM_OFF = ATC_P_OFF + ATC_TILE;           // [2 halves][128 rows] fp32 exchange
+constexpr int ATC_XM_OFF = ATC_V_OFF + ATC_V_STAGES * ATC_TILE;  // [2 halves][128 rows] fp32 exchange
 constexpr int ATC_BAR_OFF = ATC_XM_OFF + 2 * 128 * 4;
 constexpr int ATC_SMEM = ATC_BAR_OFF + 256 + 1024;
+static_assert(ATC_SMEM <= 232448, "shared memory per CTA");
 constexpr int ATC_THREADS = 352;
 
 __global__ void __launch_bounds__(ATC_THREADS, 1)
@@ -52,9 +52,9 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   uint64_t* v_empty = v_full + ATC_V_STAGES;          // [V_STAGES]
   uint64_t* s_full = v_empty + ATC_V_STAGES;          // [2]
   uint64_t* s_free = s_full + 2;                      // [2]
-  uint64_t* p_full = s_free + 2;
-  uint64_t* pv_done = p_full + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pv_done + 1);
+  uint64_t* p_full = s_free + 2;                      // [2] P_j written (8 softmax warps)
+  uint64_t* p_free = p_full + 2;                      // [2] PV product of P_j complete
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(p_free + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
@@ -80,8 +80,10 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
       mbar_init(&s_full[s], 1);
       mbar_init(&s_free[s], 8);
     }
-    mbar_init(p_full, 8);
-    mbar_init(pv_done, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&p_full[s], 8);
+      mbar_init(&p_free[s], 1);
+    }
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -92,7 +94,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tO = tmem + 256;
+  const uint32_t tO = tmem + 256, tP = tmem + 384;  // P[b] at tP + 64 b (bf16 pairs)
 
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmQ);
@@ -101,7 +103,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     mbar_arrive_expect_tx(q_full, ATC_TILE);
     tma_load_2d(smem + ATC_Q_OFF, &tmQ, q_full, col, q0);
     tma_load_2d(smem + ATC_Q_OFF + ATC_BOX, &tmQ, q_full, col + 64, q0);
-    // in order K_0 V_0 K_1 V_1 ...: K_j waits for S_{j-2}, V_j for the PV product of tile
+    // in order K_0 V_0 K_1 V_1 ...: K_j waits for S_{j-3}, V_j for the PV product of tile
     // j-3, both issued before anything that needs K_j or V_j
     for (int j = 0; j < nj; ++j) {
       const int sk = j % ATC_K_STAGES, sv = j % ATC_V_STAGES;
@@ -140,19 +142,18 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   } else if (warp == 2 && lane == 0) {
     // O += P_j V_j once the softmax has written P_j
     constexpr uint32_t idesc_o = umma_idesc_bf16_bmn(128, 128);
-    const uint32_t pa = smem_u32(smem + ATC_P_OFF);
     for (int j = 0; j < nj; ++j) {
-      const int sv = j % ATC_V_STAGES;
-      if (!mbar_wait_at(p_full, j & 1, 103, (qt << 16) | j)) break;
+      const int sv = j % ATC_V_STAGES, b = j & 1;
+      if (!mbar_wait_at(&p_full[b], (j >> 1) & 1, 103, (qt << 16) | j)) break;
       if (!mbar_wait_at(&v_full[sv], (j / ATC_V_STAGES) & 1, 111, (qt << 16) | j)) break;
       tc_fence_after();
       const uint32_t va = smem_u32(smem + ATC_V_OFF + sv * ATC_TILE);
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        umma_bf16(tO, umma_desc_k_sw128(pa + (ks >> 2) * ATC_BOX + (ks & 3) * 32),
-                  umma_desc_mn_sw128(va + ks * 2048, ATC_BOX), idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
+      for (int ks = 0; ks < 8; ++ks)  // K = 128 keys in steps of 16 (8 TMEM columns of P)
+        umma_bf16_ts(tO, tP + b * 64 + ks * 8, umma_desc_mn_sw128(va + ks * 2048, ATC_BOX), idesc_o,
+                     (j > 0 || ks > 0) ? 1u : 0u);
       umma_commit(&v_empty[sv]);
-      umma_commit(pv_done);
+      umma_commit(&p_free[b]);
     }
   } else if (warp >= 3) {
     // eight softmax warps: warp w reads TMEM lanes 32 * (w % 4) (its 32 query rows) and
@@ -163,7 +164,6 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     const int r = quarter * 32 + lane;
     const int qrow = q0 + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    uint8_t* P = smem + ATC_P_OFF + hf * ATC_BOX;  // this half's 64-key box of the P tile
     float* xm = reinterpret_cast<float*>(smem + ATC_XM_OFF);  // [2 halves][128 rows]
     const int pair_bar = 1 + quarter;
     float m_used = -INFINITY, l = 0.f;
@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         // rescale this half's 64 output columns: the PV product of tile j-1 must have landed
         // (a failed wait skips the TMEM access and ends the pair's loop at the next tile)
         waited = true;
-        if (__all_sync(0xffffffffu, mbar_wait_at(pv_done, (j - 1) & 1, 107, (qt << 16) | j))) {
+        if (__all_sync(0xffffffffu, mbar_wait_at(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, 107, (qt << 16) | j))) {
           tc_fence_after();
           const float m_new = fmaxf(m_used, mxs);
           const float f = fast_exp2(m_used - m_new);
@@ -254,20 +254,23 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         }
       }
       l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-      // P smem tile is free once the PV product of tile j-1 completed
-      if (j >= 1 && !waited && !__all_sync(0xffffffffu, mbar_wait_at(pv_done, (j - 1) & 1, 108, (qt << 16) | j)))
+      // P buffer j % 2 is free once the PV product of tile j-2 completed (implied by the
+      // wait for tile j-1 a rescale made); a failed wait skips the TMEM store and ends the
+      // pair's loop at the next tile
+      const int pb = j & 1;
+      if (j >= 2 && !waited &&
+          !__all_sync(0xffffffffu, mbar_wait_at(&p_free[pb], ((j >> 1) - 1) & 1, 108, (qt << 16) | j)))
         ok = false;
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        uint4 w = make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-        *reinterpret_cast<uint4*>(P + r * 128 + ((ch ^ (r & 7)) << 4)) = w;
+      if (ok) {
+        tmem_st32(tP + lane_off + pb * 64 + hf * 32, pk);  // keys 64 hf .. 64 hf + 63 as bf16 pairs
+        tmem_wait_st();
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[pb]);
     }
-    const bool fin = pair_all(ok && mbar_wait_at(pv_done, (nj - 1) & 1, 109, (qt << 16) | nj), pair_bar);
+    const bool fin =
+        pair_all(ok && mbar_wait_at(&p_free[(nj - 1) & 1], ((nj - 1) >> 1) & 1, 109, (qt << 16) | nj), pair_bar);
     // merge the two halves' row sums (same maxima history, so they add directly)
     asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
     xm[hf * 128 + r] = l;
