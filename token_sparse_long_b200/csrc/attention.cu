@@ -285,6 +285,9 @@ jenga_status attn_backward_segment(const bf16* q, const bf16* k, const bf16* v, 
     if ((e = make_tmap_bf16(&tdo128, dO, T, HDc, ld_do, 128)) != JENGA_OK) return e;
     if ((e = make_tmap_bf16(&tk64, k, n_cap, HDc, ld, 64)) != JENGA_OK) return e;
     if ((e = make_tmap_bf16(&tv64, v, n_cap, HDc, ld, 64)) != JENGA_OK) return e;
+    CUtensorMap tdk, tdv;  // fp32 accumulators [n_cap, H * 128], 128-row x 32-column boxes
+    if ((e = make_tmap_f32(&tdk, dk_acc, n_cap, HDc, ld_acc, 128)) != JENGA_OK) return e;
+    if ((e = make_tmap_f32(&tdv, dv_acc, n_cap, HDc, ld_acc, 128)) != JENGA_OK) return e;
     JENGA_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DQ_SMEM));
     JENGA_CUDA_TRY(
         cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DKV_SMEM));
@@ -299,8 +302,8 @@ jenga_status attn_backward_segment(const bf16* q, const bf16* k, const bf16* v, 
     {
       const int _ps = ::jenga::prof_begin("attn_bwd_dkdv_tc", st);
       attn_bwd_dkdv_tc_kernel<<<dim3((s1 + 127) / 128, H), DKV_THREADS, DKV_SMEM, st>>>(
-          tk128, tv128, tq64, tdo64, lse, lse_ld, delta, delta_ld, dk_acc, dv_acc, ld_acc, s0, s1, n_valid,
-          valid_mult, n_cap, scale_log2, scale);
+          tk128, tv128, tq64, tdo64, lse, lse_ld, delta, delta_ld, tdk, tdv, s0, s1, n_valid, valid_mult, n_cap,
+          scale_log2, scale);
       ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();

@@ -9,7 +9,8 @@
 //                 Q / dO stage as two 256-byte bulk copies; both are stored negated, so the
 //                 epilogue's packed f32x2 arithmetic adds them)
 //                 dV  += P^T dO       dK  += dS^T Q           (A: smem K-major, B: MN-major)
-//               and at the end dV, dK (x 1/sqrt(D)) are added into fp32 accumulators.
+//               and at the end dV, dK (x 1/sqrt(D)) are added into fp32 accumulators by TMA
+//               reduce-adds staged in the ring.
 //   dQ pass     one CTA per (128-query tile of the segment, head).  Q and dO resident in
 //               tensor memory; the 64-key tiles of K and V stream through a 5-stage ring.
 //               S = Q K^T, dP = dO V^T (double-buffered), dS = P (dP - Delta), dQ += dS K;
@@ -52,6 +53,8 @@ constexpr int DKV_STAGE = 4 * ABT_BOX64;
 constexpr int DKV_STAGES = 4;  // a stage lives from its load to the gradient products of its tile
 constexpr int DKV_LD_OFF = DKV_RING_OFF + DKV_STAGES * DKV_STAGE;  // stage s: L (64 fp32), Delta (64 fp32)
 constexpr int DKV_LD_BYTES = 512;
+constexpr int DKV_F32_BOX = 128 * 32 * 4;  // 16 KB: one quad's dV or dK columns, staged in the ring
+static_assert(8 * DKV_F32_BOX <= DKV_STAGES * DKV_STAGE, "final dV/dK staging fits in the ring");
 constexpr int DKV_BAR_OFF = DKV_LD_OFF + DKV_STAGES * DKV_LD_BYTES;
 constexpr int DKV_SMEM = DKV_BAR_OFF + 256 + 1024;
 
@@ -96,9 +99,10 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                             const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                             const float* __restrict__ lse, int64_t lse_ld, const float* __restrict__ delta,
-                            int64_t delta_ld, float* __restrict__ dk_acc, float* __restrict__ dv_acc, int64_t ld_acc,
-                            int s0, int s1, const int32_t* __restrict__ n_valid, int valid_mult, int n_cap,
-                            float scale_log2, float scale) {
+                            int64_t delta_ld, const __grid_constant__ CUtensorMap tmDK,
+                            const __grid_constant__ CUtensorMap tmDV, int s0, int s1,
+                            const int32_t* __restrict__ n_valid, int valid_mult, int n_cap, float scale_log2,
+                            float scale) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DKV_BAR_OFF);
@@ -328,33 +332,39 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&pd_full[s]);
     }
-    if (__all_sync(0xffffffffu, ok && mbar_wait_at(done, 0, 128, nq))) {
+    // dV and dK (x 1/sqrt(D)) are added into the fp32 accumulators by TMA reduce-adds
+    // (the L2 does the additions, so no read-modify-write round trips from this SM): each
+    // quad stages its 32 columns of both in the ring, free once every product is done.
+    // Keys past n carry exact zeros (no valid query reaches them); rows past n_cap are
+    // clipped by the tensor maps.
+    const bool fin = __all_sync(0xffffffffu, ok && mbar_wait_at(done, 0, 128, nq));
+    uint8_t* bv = smem + DKV_RING_OFF + quad * 2 * DKV_F32_BOX;  // [128 rows][32 fp32], 128-byte swizzle
+    uint8_t* bk = bv + DKV_F32_BOX;
+    if (fin) {
       tc_fence_after();
-      const bool row_ok = key < n;
       const int c0 = quad * 32;  // this quad's 32 of the 128 head dimensions
-      uint32_t a[32], b[32];
-      tmem_ld32_nowait(tdV + lo + c0, a);
-      tmem_ld32_nowait(tdK + lo + c0, b);
-      tmem_wait_ld();
-      if (row_ok) {
-        float4* pv = reinterpret_cast<float4*>(dv_acc + (int64_t)key * ld_acc + col + c0);
-        float4* pk4 = reinterpret_cast<float4*>(dk_acc + (int64_t)key * ld_acc + col + c0);
+#pragma unroll 1
+      for (int t = 0; t < 2; ++t) {  // dV, then dK
+        uint32_t a[32];
+        tmem_ld32_nowait((t ? tdK : tdV) + lo + c0, a);
+        tmem_wait_ld();
+        const float f = t ? scale : 1.f;
+        uint8_t* dst = t ? bk : bv;
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          float4 x = pv[q4];
-          x.x += __uint_as_float(a[4 * q4]);
-          x.y += __uint_as_float(a[4 * q4 + 1]);
-          x.z += __uint_as_float(a[4 * q4 + 2]);
-          x.w += __uint_as_float(a[4 * q4 + 3]);
-          pv[q4] = x;
-          float4 y = pk4[q4];
-          y.x += __uint_as_float(b[4 * q4]) * scale;
-          y.y += __uint_as_float(b[4 * q4 + 1]) * scale;
-          y.z += __uint_as_float(b[4 * q4 + 2]) * scale;
-          y.w += __uint_as_float(b[4 * q4 + 3]) * scale;
-          pk4[q4] = y;
-        }
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<float4*>(dst + r * 128 + ((c ^ (r & 7)) << 4)) =
+              make_float4(__uint_as_float(a[4 * c]) * f, __uint_as_float(a[4 * c + 1]) * f,
+                          __uint_as_float(a[4 * c + 2]) * f, __uint_as_float(a[4 * c + 3]) * f);
       }
+      fence_proxy_async_smem();
+    }
+    // every epilogue warp staged its rows (or none did: the vote is CTA-wide)
+    const bool all_fin = bar_and(fin, 1, 32 * DKV_EPI_WARPS);
+    if (all_fin && (warp - DKV_EPI_WARP0) % 4 == 0 && lane == 0) {
+      tma_reduce_add_2d(&tmDV, bv, col + quad * 32, k0);
+      tma_reduce_add_2d(&tmDK, bk, col + quad * 32, k0);
+      bulk_commit_group();
+      bulk_wait_group_read0();  // shared memory must outlive the reads
     }
   }
   tc_fence_before();

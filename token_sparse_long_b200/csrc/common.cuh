@@ -164,6 +164,21 @@ __device__ __forceinline__ bool bar_and(bool v, int bar_id, int threads) {
 }
 __device__ __forceinline__ bool pair_all(bool v, int bar_id) { return bar_and(v, bar_id, 64); }
 
+// Element-wise add of a shared-memory tile into global memory through a tensor map (the L2
+// performs the additions); the copy belongs to this thread's current bulk async-group.
+// Coordinates must be non-negative, x a multiple of 4 (fp32, 16 bytes).
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* smem_src, int x, int y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk group of this thread has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // 1D bulk copy global -> shared (both addresses and the size multiples of 16 bytes),
 // completion counted on an mbarrier.
 __device__ __forceinline__ void bulk_load_1d(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
@@ -437,6 +452,9 @@ __device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
 // box of box_rows x 64 columns and the 128-byte swizzle.
 jenga_status make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
                             uint32_t box_rows);
+// Same for an fp32 tensor: box of box_rows x 32 columns (128-byte rows), 128-byte swizzle.
+jenga_status make_tmap_f32(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                           uint32_t box_rows);
 
 int sm_count();
 unsigned long long host_wait_budget_ns();
