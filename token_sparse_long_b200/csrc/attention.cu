@@ -285,6 +285,8 @@ jenga_status attn_backward_segment(const bf16* q, const bf16* k, const bf16* v, 
     if ((e = make_tmap_bf16(&tdo128, dO, T, HDc, ld_do, 128)) != JENGA_OK) return e;
     if ((e = make_tmap_bf16(&tk64, k, n_cap, HDc, ld, 64)) != JENGA_OK) return e;
     if ((e = make_tmap_bf16(&tv64, v, n_cap, HDc, ld, 64)) != JENGA_OK) return e;
+    CUtensorMap tdq;  // fp32 dQ rows of the segment [T, H * 128]
+    if ((e = make_tmap_f32(&tdq, dq, T, HDc, ld_dq, 128)) != JENGA_OK) return e;
     CUtensorMap tdk, tdv;  // fp32 accumulators [n_cap, H * 128], 128-row x 32-column boxes
     if ((e = make_tmap_f32(&tdk, dk_acc, n_cap, HDc, ld_acc, 128)) != JENGA_OK) return e;
     if ((e = make_tmap_f32(&tdv, dv_acc, n_cap, HDc, ld_acc, 128)) != JENGA_OK) return e;
@@ -294,8 +296,8 @@ jenga_status attn_backward_segment(const bf16* q, const bf16* k, const bf16* v, 
     {
       const int _ps = ::jenga::prof_begin("attn_bwd_dq_tc", st);
       attn_bwd_dq_tc_kernel<<<dim3((T + 127) / 128, H), ABT_THREADS, DQ_SMEM, st>>>(
-          tq128, tdo128, tk64, tv64, lse, lse_ld, delta, delta_ld, dq, ld_dq, s0, n_valid, valid_mult, n_cap,
-          scale_log2, scale);
+          tq128, tdo128, tk64, tv64, lse, lse_ld, delta, delta_ld, tdq, s0, n_valid, valid_mult, n_cap, scale_log2,
+          scale);
       ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();

@@ -380,7 +380,7 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                           const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                           const float* __restrict__ lse, int64_t lse_ld, const float* __restrict__ delta,
-                          int64_t delta_ld, float* __restrict__ dq_out, int64_t ld_dq, int s0,
+                          int64_t delta_ld, const __grid_constant__ CUtensorMap tmDQ, int s0,
                           const int32_t* __restrict__ n_valid, int valid_mult, int n_cap, float scale_log2,
                           float scale) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -509,6 +509,7 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     const int q = q0 + r;
     const uint32_t lo = (uint32_t)(quarter * 32) << 16;
     const bool qvalid = q < n;
+    static_assert(4 * DKV_F32_BOX <= DQ_STAGES * DQ_STAGE, "final dQ staging fits in the ring");
     const float L = qvalid ? lse[(int64_t)h * lse_ld + q] : 0.f;  // -L, log2 units
     const float Dq = qvalid ? delta[(int64_t)h * delta_ld + q - s0] : 0.f;  // -Delta
     const uint64_t sl2x2 = f2pack(scale_log2, scale_log2), nL2 = f2pack(L, L), nD2 = f2pack(Dq, Dq);
@@ -576,19 +577,28 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ds_full[s]);
     }
-    if (__all_sync(0xffffffffu, ok && mbar_wait_at(done, 0, 138, nk))) {
+    // dQ (x 1/sqrt(D)) leaves through TMA stores: each quad stages its 32 columns in the
+    // ring (free once every product is done); rows past the segment are clipped by the
+    // tensor map, and rows of queries past n hold exact zeros
+    const bool fin = __all_sync(0xffffffffu, ok && mbar_wait_at(done, 0, 138, nk));
+    uint8_t* box = smem + DQ_RING_OFF + quad * DKV_F32_BOX;  // [128 rows][32 fp32], 128-byte swizzle
+    if (fin) {
       tc_fence_after();
-      const int c0 = quad * 32;  // this quad's 32 of the 128 head dimensions
       uint32_t a[32];
-      tmem_ld32_nowait(tdQ + lo + c0, a);
+      tmem_ld32_nowait(tdQ + lo + quad * 32, a);
       tmem_wait_ld();
-      if (qvalid) {
-        float4* dst = reinterpret_cast<float4*>(dq_out + (int64_t)(q - s0) * ld_dq + col + c0);
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4)
-          dst[q4] = make_float4(__uint_as_float(a[4 * q4]) * scale, __uint_as_float(a[4 * q4 + 1]) * scale,
-                                __uint_as_float(a[4 * q4 + 2]) * scale, __uint_as_float(a[4 * q4 + 3]) * scale);
-      }
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<float4*>(box + r * 128 + ((c ^ (r & 7)) << 4)) =
+            make_float4(__uint_as_float(a[4 * c]) * scale, __uint_as_float(a[4 * c + 1]) * scale,
+                        __uint_as_float(a[4 * c + 2]) * scale, __uint_as_float(a[4 * c + 3]) * scale);
+      fence_proxy_async_smem();
+    }
+    const bool all_fin = bar_and(fin, 1, 32 * DQ_EPI_WARPS);
+    if (all_fin && (warp - DQ_EPI_WARP0) % 4 == 0 && lane == 0) {
+      tma_store_2d(&tmDQ, box, col + quad * 32, q0 - s0);
+      bulk_commit_group();
+      bulk_wait_group_read0();  // shared memory must outlive the reads
     }
   }
   tc_fence_before();
