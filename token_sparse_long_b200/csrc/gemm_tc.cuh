@@ -129,20 +129,27 @@ __device__ __forceinline__ float silu_f(float z) { return z / (1.f + __expf(-z))
 
 template <int BN>
 struct GemmSmem {
+  // (the static_assert below keeps TOTAL within the 227 KB a CTA may use)
   static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
   static constexpr int A_BYTES = GEMM_BM * GEMM_BK * 2;
   static constexpr int B_BYTES = BN * GEMM_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  // fp32 output staging: per epilogue warp two 32-row x 32-column tiles (4 KB each) for
+  // TMA stores
+  static constexpr int STG_OFF = STAGES * STAGE_BYTES;
+  static constexpr int STG_BYTES = 4 * 2 * 4096;
+  static constexpr int BAR_OFF = STG_OFF + STG_BYTES;
   static constexpr int TOTAL = BAR_OFF + 256 + 1024;  // barriers + 1 KB alignment slack
+  static_assert(TOTAL <= 232448, "shared memory per CTA");
 };
 
 template <int BN, int EPI>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                   const __grid_constant__ CUtensorMap tmA3, const __grid_constant__ CUtensorMap tmB3, int nkb1,
-                   int nkb2, int nkb3, int N, uint32_t idesc, EpiParams ep) {
+                   const __grid_constant__ CUtensorMap tmA3, const __grid_constant__ CUtensorMap tmB3,
+                   const __grid_constant__ CUtensorMap tmOut, int nkb1, int nkb2, int nkb3, int N, uint32_t idesc,
+                   EpiParams ep) {
   using L = GemmSmem<BN>;
   constexpr int STAGES = L::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -243,6 +250,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // ---------------- epilogue
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
+    uint8_t* stg = smem + L::STG_OFF + quarter * 2 * 4096;  // this warp's two fp32 staging tiles
+    int nst = 0;  // TMA stores issued by this warp (lane 0)
     int it = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
     const int buf = it & 1;
@@ -261,6 +270,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         for (int c = 0; c < BN / 32; ++c) {
           tmem_ld32(tbase + c * 32, v);
           const int n = n0 + c * 32;
+          if (EPI == EPI_STORE_F32 && n < N && m0 + quarter * 32 + 32 <= valid) {
+            // the warp's 32 rows are all valid: stage them (128-byte swizzle) and write the
+            // 32 x 32 tile with one TMA store (full-line writes instead of 32 rows of 16-byte
+            // pieces per instruction); a staging tile is reused once its store has read it
+            uint8_t* sb = stg + (nst & 1) * 4096;
+            if (lane == 0 && nst >= 2) bulk_wait_group_read<1>();
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<float4*>(sb + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                  make_float4(v[4 * q] * ep.alpha, v[4 * q + 1] * ep.alpha, v[4 * q + 2] * ep.alpha,
+                              v[4 * q + 3] * ep.alpha);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmOut, sb, n, m0 + quarter * 32);
+              bulk_commit_group();
+            }
+            ++nst;
+            continue;
+          }
           if (!row_ok || n >= N) continue;
           if (EPI == EPI_STORE_BF16) {
 #pragma unroll
@@ -387,6 +417,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     __syncwarp();
     if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
+    if (EPI == EPI_STORE_F32 && lane == 0) bulk_wait_group_read<0>();  // staging outlives the stores' reads
   }
   tc_fence_before();
   __syncthreads();
@@ -428,6 +459,10 @@ jenga_status launch_gemm(const GemmOperand& A1, const GemmOperand& B1, int K1, c
     if ((s = make_tmap_bf16(&ta3, A3->ptr, A3->rows, K3, A3->ld, GEMM_BM)) != JENGA_OK) return s;
     if ((s = make_tmap_bf16(&tb3, B3->ptr, B3->rows, K3, B3->ld, BN)) != JENGA_OK) return s;
   }
+  CUtensorMap tout = ta1;  // fp32 output, 32 x 32 boxes (EPI_STORE_F32 only)
+  if (EPI == EPI_STORE_F32 &&
+      (s = make_tmap_f32(&tout, ep.out, (uint64_t)M, (uint64_t)N, (uint64_t)ep.ldo, 32)) != JENGA_OK)
+    return s;
   JENGA_CUDA_TRY(
       cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL));
   EpiParams p = ep;
@@ -439,7 +474,7 @@ jenga_status launch_gemm(const GemmOperand& A1, const GemmOperand& B1, int K1, c
   const uint32_t idesc = f16_inputs ? (umma_idesc_bf16(GEMM_BM, BN) & ~((7u << 7) | (7u << 10)))
                                     : umma_idesc_bf16(GEMM_BM, BN);
   const int ps = prof_begin(name, st);
-  gemm_tc_kernel<BN, EPI><<<grid, GEMM_THREADS, L::TOTAL, st>>>(ta1, tb1, ta2, tb2, ta3, tb3, K1 / GEMM_BK,
+  gemm_tc_kernel<BN, EPI><<<grid, GEMM_THREADS, L::TOTAL, st>>>(ta1, tb1, ta2, tb2, ta3, tb3, tout, K1 / GEMM_BK,
                                                                  K2 / GEMM_BK, K3 / GEMM_BK, N, idesc, p);
   prof_end(ps, st);
   JENGA_LAUNCH_CHECK();
