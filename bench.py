@@ -103,10 +103,11 @@ def work_model(case, ks, seg):
 
 # DRAM bytes per unit of work of a kernel, from one ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum; the capture and its command are in profiles/).  attn_bwd_dkdv_tc:
-# its traffic is dominated by the fp32 dK / dV accumulator read-modify-write and the K / V
-# reads, both proportional to the keys [0, segment end) a launch covers, so the unit is a key
-# row; captured on llama7b_s16k (one launch over 4096 keys: 269.5 MB read + 88.5 MB written).
-TRAFFIC_PER_UNIT = {"attn_bwd_dkdv_tc": ("key row", (269.52064e6 + 88.46208e6) / 4096)}
+# its traffic is dominated by the fp32 dK / dV accumulators (read and written back by the
+# L2's reduce-adds) and the K / V reads, both proportional to the keys [0, segment end) a
+# launch covers, so the unit is a key row; captured on llama7b_s16k (one launch over 4096
+# keys: 269.6 MB read + 85.9 MB written).
+TRAFFIC_PER_UNIT = {"attn_bwd_dkdv_tc": ("key row", (269.571584e6 + 85.910528e6) / 4096)}
 
 
 def traffic_units(name, case, ks, seg):
