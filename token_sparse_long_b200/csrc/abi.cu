@@ -103,6 +103,23 @@ jenga_status make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, u
   return JENGA_OK;
 }
 
+jenga_status make_tmap_f16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                           uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(JENGA_ECUDA, "cuTensorMapEncodeTiled entry point not available");
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (ld * 2) % 16 || rows == 0 || cols == 0)
+    return fail(JENGA_EINVAL, "tensor map: base must be 16-byte aligned and row pitch a multiple of 16 bytes");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(JENGA_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return JENGA_OK;
+}
+
 jenga_status make_tmap_f32(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
                            uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();

@@ -465,6 +465,9 @@ __device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
 // box of box_rows x 64 columns and the 128-byte swizzle.
 jenga_status make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
                             uint32_t box_rows);
+// Same for an fp16 tensor (box of box_rows x 64 columns).
+jenga_status make_tmap_f16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                           uint32_t box_rows);
 // Same for an fp32 tensor: box of box_rows x 32 columns (128-byte rows), 128-byte swizzle.
 jenga_status make_tmap_f32(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
                            uint32_t box_rows);

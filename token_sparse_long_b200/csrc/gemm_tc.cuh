@@ -61,6 +61,7 @@ struct EpiParams {
   float beta = 1.f;              // LORA_T: scale of the fp32 copy
   int hd = 0;                    // QKV: H * D (section width)
   const float2* rope_tab = nullptr;  // QKV: (cos, sin) of position(m) x frequency j, [M rows][64]
+  bool tma_out = false;          // set by the launcher: the output tensor map is valid
 };
 
 __device__ __forceinline__ int epi_valid_rows(const EpiParams& p) {
@@ -107,6 +108,30 @@ __device__ __forceinline__ void store_f16x32(__half* dst, const float* v) {
     }
     d[q] = w;
   }
+}
+
+// 32 floats -> 16 packed pairs (bf16, or fp16 with F16), round to nearest even
+template <bool F16>
+__device__ __forceinline__ void pack32(const float* v, uint32_t* w) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if (F16) {
+      __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&h);
+    } else {
+      __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+  }
+}
+
+// 16 packed words (32 two-byte values) as the 16-byte chunks ch0 .. ch0 + 3 of row `row` of
+// a 32 x 64 staging tile (128-byte rows, 128-byte swizzle)
+__device__ __forceinline__ void stage_row32(uint8_t* tile, int row, int ch0, const uint32_t* w) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<uint4*>(tile + row * 128 + (((ch0 + q) ^ (row & 7)) << 4)) =
+        make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
 }
 
 __device__ __forceinline__ void load_bf16x32(const bf16* src, float* v) {
@@ -250,8 +275,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // ---------------- epilogue
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    uint8_t* stg = smem + L::STG_OFF + quarter * 2 * 4096;  // this warp's two fp32 staging tiles
+    uint8_t* stg = smem + L::STG_OFF + quarter * 2 * 4096;  // this warp's two staging tiles
     int nst = 0;  // TMA stores issued by this warp (lane 0)
+    // Output tiles of 32 rows leave through TMA stores when all 32 rows of the warp are
+    // valid.  tile_wait(k): before staging into the next k tiles (k = 1: tile nst & 1;
+    // k = 2: both), wait until the stores that last read them are done.
+    auto tile_wait = [&](int k) {
+      if (lane == 0 && nst >= 3 - k) {
+        if (k == 1)
+          bulk_wait_group_read<1>();
+        else
+          bulk_wait_group_read<0>();
+      }
+      __syncwarp();
+    };
+    auto tile_store = [&](uint8_t* tile, int x, int y) {  // after the warp staged `tile`
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&tmOut, tile, x, y);
+        bulk_commit_group();
+      }
+      ++nst;
+    };
     int it = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
     const int buf = it & 1;
@@ -270,7 +316,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         for (int c = 0; c < BN / 32; ++c) {
           tmem_ld32(tbase + c * 32, v);
           const int n = n0 + c * 32;
-          if (EPI == EPI_STORE_F32 && n < N && m0 + quarter * 32 + 32 <= valid) {
+          if (EPI == EPI_STORE_F32 && ep.tma_out && n < N && m0 + quarter * 32 + 32 <= valid) {
             // the warp's 32 rows are all valid: stage them (128-byte swizzle) and write the
             // 32 x 32 tile with one TMA store (full-line writes instead of 32 rows of 16-byte
             // pieces per instruction); a staging tile is reused once its store has read it
@@ -289,6 +335,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               bulk_commit_group();
             }
             ++nst;
+            continue;
+          }
+          if (EPI == EPI_STORE_BF16 && ep.tma_out && n < N && m0 + quarter * 32 + 32 <= valid) {
+            // two 32-column chunks per 64-column bf16 tile
+            uint8_t* tb = stg + (nst & 1) * 4096;
+            if ((c & 1) == 0) tile_wait(1);
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= ep.alpha;
+            pack32<false>(v, w);
+            stage_row32(tb, lane, (c & 1) * 4, w);
+            if ((c & 1) || c + 1 == BN / 32 || n + 32 >= N) tile_store(tb, n0 + (c >> 1) * 64, m0 + quarter * 32);
             continue;
           }
           if (!row_ok || n >= N) continue;
@@ -326,9 +384,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             tmem_ld32(tbase + g * 128 + hh * 32, v);
             tmem_ld32(tbase + g * 128 + 64 + hh * 32, u);
             const int n = n0 + g * 128;
-            if (!row_ok || n >= N) continue;
+            if (n >= N) continue;
+            const bool tma = ep.tma_out && m0 + quarter * 32 + 32 <= valid;
+            if (!tma && !row_ok) continue;
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = silu_f(v[i]) * u[i];
+            if (tma) {  // the group's 64 outputs form one bf16 tile
+              uint8_t* tb = stg + (nst & 1) * 4096;
+              if (hh == 0) tile_wait(1);
+              uint32_t w[16];
+              pack32<false>(v, w);
+              stage_row32(tb, lane, hh * 4, w);
+              if (hh == 1) tile_store(tb, n >> 1, m0 + quarter * 32);
+              continue;
+            }
             store_bf16x32(reinterpret_cast<bf16*>(ep.out) + (int64_t)m * ep.ldo + (n >> 1) + hh * 32, v);
           }
         }
@@ -338,7 +407,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         for (int c = 0; c < BN / 32; ++c) {
           tmem_ld32(tbase + c * 32, v);
           const int j = n0 + c * 32;
-          if (!row_ok || j >= N) continue;
+          if (j >= N) continue;
+          const bool tma = ep.tma_out && m0 + quarter * 32 + 32 <= valid;
+          if (!tma && !row_ok) continue;
           const int64_t col = (int64_t)(j >> 6) * 128 + (j & 63);
           const float* gu = reinterpret_cast<const float*>(ep.aux) + (int64_t)m * ep.ld_aux + col;
           float gv[32], uv[32], dg[32];
@@ -355,6 +426,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const float da = v[i];
             dg[i] = da * uv[i] * sg * (1.f + gv[i] * (1.f - sg));
             v[i] = da * gv[i] * sg;  // du = dA * silu(g)
+          }
+          if (tma) {  // a 64-column group of dA gives one fp16 tile of dg and one of du
+            if ((j & 63) == 0) tile_wait(2);
+            uint32_t w[16];
+            pack32<true>(dg, w);
+            stage_row32(stg, lane, (j & 32) >> 3, w);
+            pack32<true>(v, w);
+            stage_row32(stg + 4096, lane, (j & 32) >> 3, w);
+            if ((j & 63) == 32 || j + 32 >= N) {
+              const int x = (j >> 6) * 128;
+              tile_store(stg, x, m0 + quarter * 32);
+              tile_store(stg + 4096, x + 64, m0 + quarter * 32);
+            }
+            continue;
           }
           __half* o = reinterpret_cast<__half*>(ep.out) + (int64_t)m * ep.ldo + col;
           store_f16x32(o, dg);
@@ -390,7 +475,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             float u[32];
             tmem_ld32(tbase + g * 128 + hh * 32, v);
             tmem_ld32(tbase + g * 128 + 64 + hh * 32, u);
-            if (!row_ok || nh >= N) continue;
+            if (nh >= N) continue;
+            const bool tma = ep.tma_out && m0 + quarter * 32 + 32 <= valid;
+            if (!tma && !row_ok) continue;
             if (rope) {
 #pragma unroll
               for (int i2 = 0; i2 < 16; ++i2) {
@@ -405,6 +492,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 }
               }
             }
+            if (tma) {  // the head's 128 outputs form two bf16 tiles (v: columns 0-63, u: 64-127)
+              if (hh == 0) tile_wait(2);
+              uint32_t w[16];
+              pack32<false>(v, w);
+              stage_row32(stg, lane, hh * 4, w);
+              pack32<false>(u, w);
+              stage_row32(stg + 4096, lane, hh * 4, w);
+              if (hh == 1) {
+                tile_store(stg, nh, m0 + quarter * 32);
+                tile_store(stg + 4096, nh + 64, m0 + quarter * 32);
+              }
+              continue;
+            }
             bf16* o = reinterpret_cast<bf16*>(ep.out) + (int64_t)m * ep.ldo + nh;
             store_bf16x32(o + hh * 32, v);
             store_bf16x32(o + 64 + hh * 32, u);
@@ -417,7 +517,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     __syncwarp();
     if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
-    if (EPI == EPI_STORE_F32 && lane == 0) bulk_wait_group_read<0>();  // staging outlives the stores' reads
+    if (lane == 0 && nst > 0) bulk_wait_group_read<0>();  // staging outlives the stores' reads
   }
   tc_fence_before();
   __syncthreads();
@@ -459,14 +559,27 @@ jenga_status launch_gemm(const GemmOperand& A1, const GemmOperand& B1, int K1, c
     if ((s = make_tmap_bf16(&ta3, A3->ptr, A3->rows, K3, A3->ld, GEMM_BM)) != JENGA_OK) return s;
     if ((s = make_tmap_bf16(&tb3, B3->ptr, B3->rows, K3, B3->ld, BN)) != JENGA_OK) return s;
   }
-  CUtensorMap tout = ta1;  // fp32 output, 32 x 32 boxes (EPI_STORE_F32 only)
-  if (EPI == EPI_STORE_F32 &&
-      (s = make_tmap_f32(&tout, ep.out, (uint64_t)M, (uint64_t)N, (uint64_t)ep.ldo, 32)) != JENGA_OK)
-    return s;
-  JENGA_CUDA_TRY(
-      cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL));
+  // output tensor map of the TMA-store epilogues (fp32 32 x 32 boxes, bf16 / fp16 32 x 64);
+  // an output the map cannot describe (alignment) keeps the per-thread stores
+  CUtensorMap tout = ta1;
   EpiParams p = ep;
   p.m_host = M;
+  {
+    jenga_status ts = JENGA_EUNSUPPORTED;
+    const bool al = ((reinterpret_cast<uintptr_t>(ep.out) & 15) == 0);
+    if (al && EPI == EPI_STORE_F32 && ep.ldo % 4 == 0)
+      ts = make_tmap_f32(&tout, ep.out, (uint64_t)M, (uint64_t)N, (uint64_t)ep.ldo, 32);
+    else if (al && (EPI == EPI_STORE_BF16 || EPI == EPI_QKV_ROPE) && ep.ldo % 8 == 0)
+      ts = make_tmap_bf16(&tout, ep.out, (uint64_t)M, (uint64_t)N, (uint64_t)ep.ldo, 32);
+    else if (al && EPI == EPI_SWIGLU && ep.ldo % 8 == 0)
+      ts = make_tmap_bf16(&tout, ep.out, (uint64_t)M, (uint64_t)N / 2, (uint64_t)ep.ldo, 32);
+    else if (al && EPI == EPI_SWIGLU_BWD && ep.ldo % 8 == 0)
+      ts = make_tmap_f16(&tout, ep.out, (uint64_t)M, 2 * (uint64_t)N, (uint64_t)ep.ldo, 32);
+    if (ts == JENGA_OK) p.tma_out = true;
+    else tout = ta1;
+  }
+  JENGA_CUDA_TRY(
+      cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL));
   // persistent: one CTA per SM (or per tile when there are fewer tiles)
   const int ntiles = ((N + BN - 1) / BN) * ((M + GEMM_BM - 1) / GEMM_BM);
   dim3 grid(ntiles < sm_count() ? ntiles : sm_count());
