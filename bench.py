@@ -355,6 +355,11 @@ def main():
     X = torch.empty_like(X0)
     dX = torch.empty_like(G0)
     seg = case.segment_tokens
+    pred = None  # (w1, b1, w2, b2) on the device when the workload scores blocks with the predictor
+    if case.predictor is not None:
+        pr = case.predictor
+        pred = (bits_to_torch(pr["w1"], dev), torch.from_numpy(pr["b1"]).to(dev),
+                bits_to_torch(pr["w2"], dev).reshape(-1), torch.from_numpy(pr["b2"]).to(dev))
 
     def buffers(kmaxes):
         b = {}
@@ -372,6 +377,9 @@ def main():
         b["bws"] = torch.empty(max(L.bwd_ws_bytes(blk, k, seg) for L, k in zip(layers, kmaxes)), dtype=torch.uint8,
                                device=dev)
         b["grads"] = [J.new_lora_grads(L) for L in layers]
+        if pred is not None:
+            b["pred_ws"] = torch.empty(lib.jenga_predict_workspace_bytes(1, S, sh.hidden, blk), dtype=torch.uint8,
+                                       device=dev)
         return b
 
     def step(b, kmaxes, sparse=True):
@@ -379,7 +387,10 @@ def main():
             if l > 0 and len(case.salient[l]):
                 J.jenga_scale_rows(X, sal[l], case.salient_scale)
             idx, nk, mask = b["sel"][l]
-            if sparse:
+            if sparse and pred is not None:  # block scores from the predictor MLP (a10)
+                J.jenga_predict_blocks(X, blk, *pred, out=b["scores"][l], ws=b["pred_ws"])
+                J.jenga_select(b["scores"][l], "topk_frac", keep[l], out=(idx, nk, mask))
+            elif sparse:
                 J.jenga_layer_score_qk(L, X, out=b["qk"], ws=b["qk_ws"])
                 J.jenga_score_blocks(b["qk"][:, :HD], b["qk"][:, HD:], sh.heads, sh.head_dim, blk, out=b["scores"][l],
                                      ws=b["sc_ws"])
@@ -482,6 +493,39 @@ def main():
                 e["gbs"] = amount / sec / 1e9
         kernels[k] = e
 
+    # ---------------- predictor path: agreement of predicted and exact block scores (layer 0
+    # input; outside the timed region) and the predictor kernels' HBM roofline
+    predictor = None
+    if pred is not None:
+        import scipy.stats
+        L0 = layers[0]
+        pws = torch.empty(J._lib.load().jenga_predict_workspace_bytes(1, S, sh.hidden, blk), dtype=torch.uint8,
+                          device=dev)
+        p_sc = J.jenga_predict_blocks(X0, blk, *pred, ws=pws)
+        J.jenga_layer_score_qk(L0, X0, out=b["qk"], ws=b["qk_ws"])
+        e_sc = J.jenga_score_blocks(b["qk"][:, :HD], b["qk"][:, HD:], sh.heads, sh.head_dim, blk, ws=b["sc_ws"])
+        ps, es = p_sc.reshape(-1).double().cpu().numpy(), e_sc.reshape(-1).double().cpu().numpy()
+        kk = ks[0]
+
+        def topk_set(v):  # (score desc, index asc), the selection's tie-break
+            return set(np.lexsort((np.arange(v.size), -v))[:kk].tolist())
+
+        for _ in range(3):
+            J.jenga_predict_blocks(X0, blk, *pred, out=p_sc, ws=pws)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
+        for _ in range(10):
+            J.jenga_predict_blocks(X0, blk, *pred, out=p_sc, ws=pws)
+        ev1.record()
+        torch.cuda.synchronize()
+        us = ev0.elapsed_time(ev1) * 100.0  # per call, 10 back to back
+        by = S * sh.hidden * X0.element_size()
+        predictor = {"rank_agreement": {"spearman": float(scipy.stats.spearmanr(ps, es).statistic),
+                                        "kendall_tau_b": float(scipy.stats.kendalltau(ps, es).statistic),
+                                        "topk_overlap": len(topk_set(ps) & topk_set(es)) / kk, "k": kk, "nb": nb},
+                     "us_per_call": us, "bytes": by, "gbs": by / us / 1e3, "frac_hbm": by / us / 1e3 / hbm,
+                     "note": "random-init predictor weights: agreement with exact scores is not expected"}
+
     # ---------------- dense comparison (keep-all, no scoring)
     dense = None
     if not args.no_dense:
@@ -550,9 +594,11 @@ def main():
                 "config": {"workload": args.workload, "seq_len": S, "global_batch": world, "layers": len(layers),
                            "hidden": sh.hidden, "heads": sh.heads, "ffn": sh.ffn, "block": blk, "keep": keep,
                            "n_kept_blocks": n_kept, "segment_tokens": seg, "parallelism": f"replicas{world}",
-                           "l2": "inputs larger than L2 (X 256 MiB, weights 1.6 GiB)"},
+                           "l2": f"inputs larger than L2 (X {X0.numel() * 2 / 2 ** 20:.0f} MiB, weights "
+                                 f"{len(layers) * (4 * sh.hidden ** 2 + 3 * sh.hidden * sh.ffn) * 2 / 2 ** 30:.1f} GiB)"},
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "movement": movement,
                 "clocks": clk, "peak_mem_gib": peak_sparse, "dense": dense,
+                **({"predictor": predictor} if predictor is not None else {}),
                 "step_tflop": step_flops(case, ks) / 1e12, "kernels": kernels}
         print(json.dumps(line), flush=True)
     if world > 1:
