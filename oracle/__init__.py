@@ -18,6 +18,7 @@ bf16       round-to-nearest-even float64 -> bf16 (storage rounding at stated poi
 scores     block informativeness (softmax column mass; Eq. 2 block-max form)
 select     threshold selection / top-k / compaction to ascending block indices
 movement   permutation-free gather and in-place scatter-add
+lm_loss    causal-LM cross-entropy over the vocabulary and its hidden-state gradient
 layer      retained-token Llama decoder layer forward and backward (+ segmented)
 predictor  block-score predictor MLP (mean pool -> Linear -> GELU -> Linear)
 rank       rank agreement statistics (Spearman, Kendall tau-b, top-k recall)
