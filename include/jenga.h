@@ -262,6 +262,28 @@ JENGA_API jenga_status jenga_predict_blocks(const void* x, int B, int S, int h, 
                                   const void* w2, const float* b2, int m, float* scores, void* ws,
                                   size_t ws_bytes, jenga_stream_t stream);
 
+/**
+ * jenga_lm_loss_segmented -- causal-LM cross-entropy over the vocabulary with its
+ * hidden-state gradient, computed segment by segment (Jenga summary §4.4.2, segment-based
+ * peak cutting, Fig. 10): the tokens are processed segment_tokens rows at a time, so the
+ * vocabulary-wide logits of only one segment exist at a time.
+ *   logits_t  = hidden_t . W^T                          (W [V, h]: frozen output embedding)
+ *   *loss     = (1/n) sum over valid t of (logsumexp(logits_t) - logits_t[labels[t]])
+ *   dhidden_t = (1/n) (softmax(logits_t) - onehot(labels[t])) . W for valid t, else 0
+ * where t is valid when 0 <= labels[t] < V (any other label, e.g. -100, is ignored) and n
+ * is the number of valid tokens (loss 0 and zero gradient when n == 0).
+ * hidden: device bf16 [S, h] (row pitch h); w: device bf16 [V, h]; labels: device int32
+ * [S] (already shifted to the next token); loss: device fp32 scalar; dhidden: device bf16
+ * [S, h] (written).  h and V multiples of 64; hidden, w, dhidden 16-byte aligned.  The
+ * result does not depend on segment_tokens (each row depends only on itself).
+ * ws: jenga_lm_loss_workspace_bytes(S, h, V, segment_tokens) bytes of device memory
+ * (transposed W, one segment's fp32 logits and bf16 gradient rows, per-row losses); all
+ * buffers are caller-owned.  Errors: JENGA_EINVAL (sizes, alignment, null), JENGA_EWORKSPACE. */
+JENGA_API size_t jenga_lm_loss_workspace_bytes(int S, int h, int V, int segment_tokens);
+JENGA_API jenga_status jenga_lm_loss_segmented(const void* hidden, const void* w, const int32_t* labels, int S, int h,
+                                               int V, int segment_tokens, float* loss, void* dhidden, void* ws,
+                                               size_t ws_bytes, jenga_stream_t stream);
+
 /* ------------------------------------------------------------------ test hook
  * jenga_test_gemm -- C[M, N] = A[M, K] * B[N, K]^T through the tcgen05 GEMM the layer
  * uses (bf16 inputs, fp32 accumulate; C fp32 if out_f32 else bf16).  bn: 256 or 32

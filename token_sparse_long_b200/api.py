@@ -254,6 +254,26 @@ def jenga_predict_blocks(x, blk, w1, b1, w2, b2, out=None, ws=None, stream=None)
     return out if x.dim() == 3 else out[0]
 
 
+def jenga_lm_loss_segmented(hidden, w, labels, segment_tokens=4096, dhidden=None, loss=None, ws=None, stream=None):
+    """hidden [S, h] bf16, w [V, h] bf16, labels [S] int32 -> (loss fp32 [1], dhidden [S, h] bf16).
+
+    Mean causal-LM cross-entropy over the tokens whose label is in [0, V) and its gradient
+    with respect to hidden, computed segment_tokens rows at a time."""
+    _need_cuda(hidden, w, labels)
+    S, h = hidden.shape
+    V = w.shape[0]
+    lib = load()
+    if ws is None:
+        ws = _ws(lib.jenga_lm_loss_workspace_bytes(S, h, V, segment_tokens), hidden.device)
+    if dhidden is None:
+        dhidden = torch.empty(S, h, dtype=torch.bfloat16, device=hidden.device)
+    if loss is None:
+        loss = torch.empty(1, dtype=torch.float32, device=hidden.device)
+    check(lib.jenga_lm_loss_segmented(_p(hidden), _p(w), _p(labels), S, h, V, segment_tokens, _p(loss), _p(dhidden),
+                                      _p(ws), ws.numel(), _stream(stream)))
+    return loss, dhidden
+
+
 def jenga_test_gemm(a, b, out_f32=True, bn=256, stream=None):
     """C = A B^T through the tcgen05 GEMM (test hook)."""
     M, K = a.shape

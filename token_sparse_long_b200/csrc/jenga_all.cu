@@ -7,5 +7,6 @@
 #include "score.cu"
 #include "attention.cu"
 #include "layer.cu"
+#include "lm_loss.cu"
 #include "predictor.cu"
 #include "score_noalloc.cu"
