@@ -44,6 +44,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-movement", action="store_true", help="skip the standalone gather/scatter/select timing")
+    ap.add_argument("--no-lm-loss", action="store_true", help="skip the segmented LM-head loss timing")
     return ap.parse_args()
 
 
@@ -256,6 +257,47 @@ def full_step_flops(w, ks):
 
 
 # ---------------------------------------------------------------------------- GPU arm
+def measure_lm_loss(J, torch, dev, S, h, tf_peak, V=32000, seg=4096):
+    """Segmented causal-LM loss (vocabulary cross-entropy and its hidden-state gradient) at
+    the workload's sequence length and hidden size with the Llama-2 vocabulary (32000),
+    4096-token segments: synthetic hidden states N(0,1), output embedding N(0,0.02),
+    uniform labels.  Algorithmic work 4 S V h flop (logits and gradient GEMMs); device
+    time per call over 3 back-to-back calls, median of 3.  Peak workspace against the
+    unsegmented form (segment = S)."""
+    g = torch.Generator(device=dev).manual_seed(0)
+    hid = torch.randn(S, h, device=dev, generator=g).to(torch.bfloat16)
+    w = (torch.randn(V, h, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+    lab = torch.randint(0, V, (S,), device=dev, generator=g, dtype=torch.int32)
+    lib = J._lib.load()
+    ws_b = lib.jenga_lm_loss_workspace_bytes(S, h, V, seg)
+    ws_full = lib.jenga_lm_loss_workspace_bytes(S, h, V, S)
+    ws = torch.empty(ws_b, dtype=torch.uint8, device=dev)
+    dh = torch.empty(S, h, dtype=torch.bfloat16, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    fn = lambda: J.jenga_lm_loss_segmented(hid, w, lab, segment_tokens=seg, dhidden=dh, loss=loss, ws=ws)
+    for _ in range(2):
+        fn()
+    ts = []
+    for _ in range(3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(3):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) / 3 / 1e3)
+    t = sorted(ts)[1]
+    J.jenga_check_device_status()
+    fl = 4.0 * S * V * h
+    out = {"S": S, "h": h, "V": V, "segment_tokens": seg, "ms": t * 1e3, "tokens_per_s": S / t,
+           "tflops": fl / t / 1e12, "frac_bf16_sustained": fl / t / 1e12 / tf_peak,
+           "workspace_gib": ws_b / 2 ** 30, "workspace_unsegmented_gib": ws_full / 2 ** 30,
+           "loss": float(loss.item()), "loss_uniform_reference": float(np.log(V))}
+    del hid, w, lab, ws, dh
+    torch.cuda.empty_cache()
+    return out
+
+
 def measure_movement(J, torch, dev, X0, case, ks, hbm):
     """Standalone timing of the HBM-bound entry points at the workload's sizes: gather and
     scatter-add of layer 0's retained rows of X (bf16 [S, h]), and threshold selection
@@ -576,6 +618,11 @@ def main():
     if not args.no_movement:
         movement = measure_movement(J, torch, dev, X0, case, ks, hbm)
 
+    # ---------------- segmented LM-head loss (segment-based peak cutting)
+    lm_loss = None
+    if not args.no_lm_loss:
+        lm_loss = measure_lm_loss(J, torch, dev, S, sh.hidden, tf_sus)
+
     # ---------------- CPU baseline (oracle, rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -598,7 +645,7 @@ def main():
                                  f"{len(layers) * (4 * sh.hidden ** 2 + 3 * sh.hidden * sh.ffn) * 2 / 2 ** 30:.1f} GiB)"},
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "movement": movement,
                 "clocks": clk, "peak_mem_gib": peak_sparse, "dense": dense,
-                **({"predictor": predictor} if predictor is not None else {}),
+                **({"predictor": predictor} if predictor is not None else {}), "lm_loss": lm_loss,
                 "step_tflop": step_flops(case, ks) / 1e12, "kernels": kernels}
         print(json.dumps(line), flush=True)
     if world > 1:
