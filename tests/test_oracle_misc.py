@@ -74,3 +74,64 @@ def test_topk_recall():
     assert ork.topk_recall(exact, exact, 5) == 1.0
     assert ork.topk_recall(-exact, exact, 5) == 0.0
     assert ork.topk_recall(np.array([9, 8, 0, 0, 0, 0, 0, 0, 0, 7.0]), exact, 3) == pytest.approx(1 / 3)
+
+
+# ------------------------------------------------------------------ Q/K predictor pair
+def _pair_case(seed, S=64, h=24, blk=8, r1=10, r2=6, d=3):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((S, h))
+    mk = lambda: (rng.standard_normal((r1, h)) * 0.3, rng.standard_normal((r2, r1)) * 0.3,
+                  rng.standard_normal((d, r2)) * 0.3)
+    return x, blk, mk(), mk()
+
+
+def test_predictor_pair_brute_force_loops():
+    x, blk, qw, kw = _pair_case(0)
+    nb = x.shape[0] // blk
+    want = np.zeros(nb)
+    for n in range(nb):
+        for m in range(n, nb):
+            xm = x[m * blk:(m + 1) * blk].sum(axis=0) / blk
+            xn = x[n * blk:(n + 1) * blk].sum(axis=0) / blk
+            qv = np.zeros(qw[2].shape[0])
+            kv = np.zeros(kw[2].shape[0])
+            for side, xv, out in ((qw, xm, qv), (kw, xn, kv)):
+                a1 = [max(0.0, sum(side[0][i, c] * xv[c] for c in range(xv.size))) for i in range(side[0].shape[0])]
+                a2 = [max(0.0, sum(side[1][i, c] * a1[c] for c in range(len(a1)))) for i in range(side[1].shape[0])]
+                for i in range(out.size):
+                    out[i] = sum(side[2][i, c] * a2[c] for c in range(len(a2)))
+            want[n] += sum(qv[i] * kv[i] for i in range(qv.size))
+    np.testing.assert_allclose(opr.predict_blocks_qk(x, blk, qw, kw), want, rtol=1e-12, atol=1e-13)
+
+
+def test_predictor_pair_matches_torch_modules():
+    x, blk, qw, kw = _pair_case(1)
+    xt = torch.tensor(x).reshape(-1, blk, x.shape[1]).mean(dim=1)
+
+    def side(w):
+        net = torch.nn.Sequential(torch.nn.Linear(w[0].shape[1], w[0].shape[0], bias=False), torch.nn.ReLU(),
+                                  torch.nn.Linear(w[1].shape[1], w[1].shape[0], bias=False), torch.nn.ReLU(),
+                                  torch.nn.Linear(w[2].shape[1], w[2].shape[0], bias=False)).double()
+        for lin, wi in zip([net[0], net[2], net[4]], w):
+            lin.weight.data = torch.tensor(wi)
+        return net(xt)
+
+    blocks = side(qw) @ side(kw).T
+    want = torch.tril(blocks).sum(dim=0).detach().numpy()
+    np.testing.assert_allclose(opr.predict_blocks_qk(x, blk, qw, kw), want, rtol=1e-12, atol=1e-13)
+    full = blocks.sum(dim=0).detach().numpy()
+    np.testing.assert_allclose(opr.predict_blocks_qk(x, blk, qw, kw, causal=False), full, rtol=1e-12, atol=1e-13)
+
+
+def test_predictor_pair_rank_one_closed_form():
+    # d = 1 and identical representative embeddings in every block: every query block has
+    # the same scalar q and every key block the same k, so key block n scores q k (nb - n)
+    rng = np.random.default_rng(2)
+    blk, h, nb = 4, 12, 9
+    row = rng.standard_normal(h)
+    x = np.tile(row, (nb * blk, 1))
+    qw = (np.abs(rng.standard_normal((5, h))), np.abs(rng.standard_normal((4, 5))), rng.standard_normal((1, 4)))
+    kw = (np.abs(rng.standard_normal((5, h))), np.abs(rng.standard_normal((4, 5))), rng.standard_normal((1, 4)))
+    q = opr.predictor_pair_side(row[None, :], *qw)[0, 0]
+    k = opr.predictor_pair_side(row[None, :], *kw)[0, 0]
+    np.testing.assert_allclose(opr.predict_blocks_qk(x, blk, qw, kw), q * k * (nb - np.arange(nb)), rtol=1e-12)
