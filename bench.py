@@ -562,10 +562,30 @@ def main():
         torch.cuda.synchronize()
         us = ev0.elapsed_time(ev1) * 100.0  # per call, 10 back to back
         by = S * sh.hidden * X0.element_size()
+        # the pages' Q/K predictor pair (Eq. 3) on the same input: ranks 128, 128, output 16
+        gq = torch.Generator(device=dev).manual_seed(1)
+        pw = lambda: tuple((torch.randn(*shp, device=dev, generator=gq) * sd).to(torch.bfloat16)
+                           for shp, sd in (((128, sh.hidden), 0.02), ((128, 128), 0.1), ((16, 128), 0.1)))
+        qw_, kw_ = pw(), pw()
+        pq = J.jenga_predict_blocks_qk(X0, blk, qw_, kw_)
+        for _ in range(3):
+            J.jenga_predict_blocks_qk(X0, blk, qw_, kw_, out=pq)
+        ev0.record()
+        for _ in range(10):
+            J.jenga_predict_blocks_qk(X0, blk, qw_, kw_, out=pq)
+        ev1.record()
+        torch.cuda.synchronize()
+        us_pair = ev0.elapsed_time(ev1) * 100.0
+        pqs = pq.reshape(-1).double().cpu().numpy()
+        predictor_pair = {"us_per_call": us_pair, "gbs": by / us_pair / 1e3, "frac_hbm": by / us_pair / 1e3 / hbm,
+                          "ranks": [128, 128, 16],
+                          "rank_agreement": {"spearman": float(scipy.stats.spearmanr(pqs, es).statistic),
+                                             "topk_overlap": len(topk_set(pqs) & topk_set(es)) / kk}}
         predictor = {"rank_agreement": {"spearman": float(scipy.stats.spearmanr(ps, es).statistic),
                                         "kendall_tau_b": float(scipy.stats.kendalltau(ps, es).statistic),
                                         "topk_overlap": len(topk_set(ps) & topk_set(es)) / kk, "k": kk, "nb": nb},
                      "us_per_call": us, "bytes": by, "gbs": by / us / 1e3, "frac_hbm": by / us / 1e3 / hbm,
+                     "pair_qk": predictor_pair,
                      "note": "random-init predictor weights: agreement with exact scores is not expected"}
 
     # ---------------- dense comparison (keep-all, no scoring)

@@ -263,6 +263,24 @@ JENGA_API jenga_status jenga_predict_blocks(const void* x, int B, int S, int h, 
                                   size_t ws_bytes, jenga_stream_t stream);
 
 /**
+ * jenga_predict_blocks_qk -- the pages' Q/K predictor pair (Jenga summary §4.3.1 Eq. (3),
+ * Fig. 8): a query-side and a key-side predictor, each three bias-free low-rank matrices
+ * with ReLU between them, map the mean of each block's raw layer-input rows to d-vectors
+ *   qhat_m = W3q ReLU(W2q ReLU(W1q xbar_m)),   khat_n = W3k ReLU(W2k ReLU(W1k xbar_n));
+ * the score block (m, n) is qhat_m . khat_n and scores[b, n] is the sum of column n over
+ * the query blocks m (m >= n when causal != 0).
+ * x: device bf16 [B, S, h] (row pitch h, 16-byte aligned); q_w1, k_w1: bf16 [r1, h]
+ * (16-byte aligned); q_w2, k_w2: bf16 [r2, r1]; q_w3, k_w3: bf16 [d, r2]; scores: device
+ * fp32 [B, S / blk].  h % 8 == 0, h <= 12288, r1 and r2 in [1, 1024], d in [1, 64].
+ * ws: jenga_predict_qk_workspace_bytes(B, S, h, blk, d) bytes (block means and the two
+ * sides' outputs, fp32).  Errors: JENGA_EINVAL, JENGA_EWORKSPACE. */
+JENGA_API size_t jenga_predict_qk_workspace_bytes(int B, int S, int h, int blk, int d);
+JENGA_API jenga_status jenga_predict_blocks_qk(const void* x, int B, int S, int h, int blk, const void* q_w1,
+                                               const void* q_w2, const void* q_w3, const void* k_w1,
+                                               const void* k_w2, const void* k_w3, int r1, int r2, int d, int causal,
+                                               float* scores, void* ws, size_t ws_bytes, jenga_stream_t stream);
+
+/**
  * jenga_lm_loss_segmented -- causal-LM cross-entropy over the vocabulary with its
  * hidden-state gradient, computed segment by segment (Jenga summary §4.4.2, segment-based
  * peak cutting, Fig. 10): the tokens are processed segment_tokens rows at a time, so the

@@ -268,3 +268,22 @@ def test_predictor_against_oracle(J):
     ref = opr.predict_blocks(from_bits(case.x), 128, from_bits(pr["w1"]), pr["b1"], from_bits(pr["w2"]), pr["b2"])
     got = s.cpu().numpy().astype(np.float64)
     assert rel_max(got, ref) < 1e-3
+
+
+# ------------------------------------------------------------------ Q/K predictor pair (Eq. 3)
+@pytest.mark.parametrize("S,h,blk,r1,r2,d,causal,B", [(2048, 512, 128, 128, 64, 16, True, 1),
+                                                      (1024, 264, 64, 40, 24, 1, True, 2),
+                                                      (4096, 5120, 128, 128, 128, 32, False, 1)])
+def test_predictor_pair_against_oracle(J, S, h, blk, r1, r2, d, causal, B):
+    g = torch.Generator(device="cpu").manual_seed(S + d)
+    x = torch.randn(B, S, h, generator=g).to(torch.bfloat16)
+    mk = lambda: tuple((torch.randn(*shp, generator=g) * sd).to(torch.bfloat16)
+                       for shp, sd in (((r1, h), 0.02), ((r2, r1), 0.1), ((d, r2), 0.1)))
+    qw, kw = mk(), mk()
+    got = J.jenga_predict_blocks_qk(x.cuda(), blk, tuple(t.cuda() for t in qw), tuple(t.cuda() for t in kw),
+                                    causal=causal)
+    J.jenga_check_device_status()
+    f64 = lambda t: t.to(torch.float64).numpy()
+    for b in range(B):
+        ref = opr.predict_blocks_qk(f64(x[b]), blk, tuple(f64(t) for t in qw), tuple(f64(t) for t in kw), causal)
+        assert rel_max(got[b].cpu().numpy().astype(np.float64), ref) < 1e-3

@@ -254,6 +254,23 @@ def jenga_predict_blocks(x, blk, w1, b1, w2, b2, out=None, ws=None, stream=None)
     return out if x.dim() == 3 else out[0]
 
 
+def jenga_predict_blocks_qk(x, blk, q_w, k_w, causal=True, out=None, ws=None, stream=None):
+    """x [S, h] or [B, S, h] bf16; q_w, k_w: (W1 [r1, h], W2 [r2, r1], W3 [d, r2]) bf16 ->
+    scores [nb] (or [B, nb]) fp32: column sums of the query-key score-block products."""
+    _need_cuda(x, *q_w, *k_w)
+    x3 = x if x.dim() == 3 else x.unsqueeze(0)
+    B, S, h = x3.shape
+    r1, r2, d = q_w[0].shape[0], q_w[1].shape[0], q_w[2].shape[0]
+    lib = load()
+    if ws is None:
+        ws = _ws(lib.jenga_predict_qk_workspace_bytes(B, S, h, blk, d), x.device)
+    if out is None:
+        out = torch.empty(B, S // blk, dtype=torch.float32, device=x.device)
+    check(lib.jenga_predict_blocks_qk(_p(x3), B, S, h, blk, *[_p(t) for t in q_w], *[_p(t) for t in k_w], r1, r2, d,
+                                      1 if causal else 0, _p(out), _p(ws), ws.numel(), _stream(stream)))
+    return out if x.dim() == 3 else out[0]
+
+
 def jenga_lm_loss_segmented(hidden, w, labels, segment_tokens=4096, dhidden=None, loss=None, ws=None, stream=None):
     """hidden [S, h] bf16, w [V, h] bf16, labels [S] int32 -> (loss fp32 [1], dhidden [S, h] bf16).
 
