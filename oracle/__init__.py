@@ -19,6 +19,7 @@ scores     block informativeness (softmax column mass; Eq. 2 block-max form)
 select     threshold selection / top-k / compaction to ascending block indices
 movement   permutation-free gather and in-place scatter-add
 lm_loss    causal-LM cross-entropy over the vocabulary and its hidden-state gradient
+mlp_blocks MLP-block elimination criterion (|SiLU(gate) * up| mass per block) and index composition
 layer      retained-token Llama decoder layer forward and backward (+ segmented)
 predictor  block-score predictor MLP (mean pool -> Linear -> GELU -> Linear)
 rank       rank agreement statistics (Spearman, Kendall tau-b, top-k recall)
