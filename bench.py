@@ -303,7 +303,7 @@ def measure_movement(J, torch, dev, X0, case, ks, hbm):
     scatter-add of layer 0's retained rows of X (bf16 [S, h]), and threshold selection
     (ABS_GE) over 2^26 fp32 scores.  Algorithmic bytes: gather 2 n h e, scatter-add 3 n h e
     (eliminated rows cost nothing), select 4 nb read + 4 nb (idx, -1 past n_kept) + nb + 4
-    written.  Each
+    written, MLP-block criterion 2 n F read (the retained rows' intermediate activation).  Each
     call moves more than the 126 MB L2; CUDA events around 10 back-to-back calls, median of 5
     such groups after 3 warm-ups."""
     blk, S, h = case.blk, case.S, X0.shape[1]
@@ -340,6 +340,15 @@ def measure_movement(J, torch, dev, X0, case, ks, hbm):
     by = 3.0 * n * h * X0.element_size()
     out["scatter_add"] = {"rows": n, "bytes": by, "us": t * 1e6, "gbs": by / t / 1e9, "frac_hbm": by / t / 1e9 / hbm}
     del xg, x2
+    # MLP-block criterion over the retained blocks' intermediate activation [n, F]
+    F = case.shape.ffn
+    act = torch.randn(n, F, device=dev, generator=torch.Generator(device=dev).manual_seed(1)).to(torch.bfloat16)
+    msc = torch.empty(k0, dtype=torch.float32, device=dev)
+    t = med(lambda: J.jenga_mlp_block_scores(act, blk, nk, out=msc))
+    by = 2.0 * n * F + 4.0 * k0
+    out["mlp_block_scores"] = {"rows": n, "ffn": F, "bytes": by, "us": t * 1e6, "gbs": by / t / 1e9,
+                               "frac_hbm": by / t / 1e9 / hbm}
+    del act
     nsel = 1 << 26
     g = torch.Generator(device=dev).manual_seed(0)
     sc = torch.rand(1, nsel, device=dev, generator=g)

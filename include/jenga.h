@@ -263,6 +263,27 @@ JENGA_API jenga_status jenga_predict_blocks(const void* x, int B, int S, int h, 
                                   size_t ws_bytes, jenga_stream_t stream);
 
 /**
+ * jenga_mlp_block_scores -- MLP-block elimination criterion (Jenga summary §4.2.4): the
+ * informativeness of a retained token block for the MLP sub-block from the block's
+ * intermediate activation a = SiLU(gate) * up:
+ *   scores[i] = sum over the blk rows of block i and the F neurons of |a|,   i < *n_kept,
+ *   scores[i] = -inf for n_kept <= i < n_cap (never selected).
+ * a: device bf16 [n_cap * blk, F] with row pitch lda (rows in compact retained order, as
+ * the layer forward forms them), 16-byte aligned, F and lda multiples of 8; n_kept:
+ * device int32 (retained blocks; null = n_cap); scores: device fp32 [n_cap].  Selecting
+ * on these scores (jenga_select) gives positions in the retained list; compose them with
+ * jenga_compose_block_indices for sequence block numbers.  Errors: JENGA_EINVAL. */
+JENGA_API jenga_status jenga_mlp_block_scores(const void* a, int64_t lda, int F, int blk, const int32_t* n_kept,
+                                              int n_cap, float* scores, jenga_stream_t stream);
+/* jenga_compose_block_indices -- out[i] = outer[pos[i]] for i < *n_pos, -1 for
+ * *n_pos <= i < n_cap: a list of positions in the outer index list (e.g. the MLP's kept
+ * positions among the attention-retained blocks) in the outer list's numbering.  All
+ * device int32; an out-of-range position records JENGA_EINTERNAL and writes -1. */
+JENGA_API jenga_status jenga_compose_block_indices(const int32_t* outer, int n_outer_cap, const int32_t* pos,
+                                                   const int32_t* n_pos, int n_cap, int32_t* out,
+                                                   jenga_stream_t stream);
+
+/**
  * jenga_predict_blocks_qk -- the pages' Q/K predictor pair (Jenga summary §4.3.1 Eq. (3),
  * Fig. 8): a query-side and a key-side predictor, each three bias-free low-rank matrices
  * with ReLU between them, map the mean of each block's raw layer-input rows to d-vectors

@@ -287,3 +287,31 @@ def test_predictor_pair_against_oracle(J, S, h, blk, r1, r2, d, causal, B):
     for b in range(B):
         ref = opr.predict_blocks_qk(f64(x[b]), blk, tuple(f64(t) for t in qw), tuple(f64(t) for t in kw), causal)
         assert rel_max(got[b].cpu().numpy().astype(np.float64), ref) < 1e-3
+
+
+# ------------------------------------------------------------------ MLP-block criterion (§4.2.4)
+@pytest.mark.parametrize("n_cap,n_kept,blk,F,pitch", [(64, 50, 64, 11008, 11008), (33, 33, 32, 520, 528),
+                                                      (16, 0, 128, 256, 256)])
+def test_mlp_block_scores_and_second_list(J, n_cap, n_kept, blk, F, pitch):
+    from oracle import mlp_blocks as omb
+    g = torch.Generator(device="cpu").manual_seed(n_cap + F)
+    aw = (torch.randn(n_cap * blk, pitch, generator=g) * torch.rand(n_cap * blk, 1, generator=g) * 3).to(torch.bfloat16)
+    a = aw.cuda()[:, :F]
+    nk = torch.tensor([n_kept], dtype=torch.int32, device="cuda")
+    sc = J.jenga_mlp_block_scores(a, blk, nk)
+    J.jenga_check_device_status()
+    ref = omb.mlp_block_scores(aw[:, :F].to(torch.float64).numpy(), blk, n_kept)
+    got = sc.cpu().numpy().astype(np.float64)
+    assert np.all(np.isneginf(got[n_kept:]))
+    if n_kept:
+        assert np.all(np.abs(got[:n_kept] - ref[:n_kept]) / ref[:n_kept] < 1e-5)
+    # second index list: the MLP keeps half of the attention-retained blocks (GPU scores
+    # through the oracle's selection, bit-exact), composed with an attention list
+    k = (n_kept + 1) // 2
+    pos, npos, _ = J.jenga_select(sc[None], "topk", float(k))
+    opos, onpos, _ = osel.select_topk(got, k)
+    assert int(npos[0]) == onpos and np.array_equal(pos.cpu().numpy()[0], opos)
+    outer = torch.arange(0, 2 * n_cap, 2, dtype=torch.int32, device="cuda")  # attention list: even blocks
+    inner = J.jenga_compose_block_indices(outer, pos[0], npos)
+    want = omb.compose_indices(outer.cpu().numpy(), opos, onpos)
+    assert np.array_equal(inner.cpu().numpy(), want)

@@ -80,6 +80,8 @@ _SIGS = {
                                        c_void_p, c_size_t, c_void_p]),
     "jenga_predict_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),
     "jenga_lm_loss_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),
+    "jenga_mlp_block_scores": (c_int, [c_void_p, c_int64, c_int, c_int, c_void_p, c_int, c_void_p, c_void_p]),
+    "jenga_compose_block_indices": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p]),
     "jenga_predict_qk_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int, c_int]),
     "jenga_predict_blocks_qk": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                         c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_size_t,

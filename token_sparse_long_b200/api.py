@@ -254,6 +254,27 @@ def jenga_predict_blocks(x, blk, w1, b1, w2, b2, out=None, ws=None, stream=None)
     return out if x.dim() == 3 else out[0]
 
 
+def jenga_mlp_block_scores(a, blk, n_kept=None, out=None, stream=None):
+    """a [n_cap * blk, F] bf16 (compact retained rows) -> scores [n_cap] fp32 (-inf past n_kept)."""
+    _need_cuda(a)
+    n_cap = a.shape[0] // blk
+    if out is None:
+        out = torch.empty(n_cap, dtype=torch.float32, device=a.device)
+    check(load().jenga_mlp_block_scores(_p(a), a.stride(0), a.shape[1], blk, _p(n_kept) if n_kept is not None else None,
+                                        n_cap, _p(out), _stream(stream)))
+    return out
+
+
+def jenga_compose_block_indices(outer, pos, n_pos, out=None, stream=None):
+    """out[i] = outer[pos[i]] for i < n_pos, -1 after (int32 device tensors)."""
+    _need_cuda(outer, pos, n_pos)
+    if out is None:
+        out = torch.empty(pos.numel(), dtype=torch.int32, device=pos.device)
+    check(load().jenga_compose_block_indices(_p(outer), outer.numel(), _p(pos), _p(n_pos), pos.numel(), _p(out),
+                                             _stream(stream)))
+    return out
+
+
 def jenga_predict_blocks_qk(x, blk, q_w, k_w, causal=True, out=None, ws=None, stream=None):
     """x [S, h] or [B, S, h] bf16; q_w, k_w: (W1 [r1, h], W2 [r2, r1], W3 [d, r2]) bf16 ->
     scores [nb] (or [B, nb]) fp32: column sums of the query-key score-block products."""

@@ -176,6 +176,74 @@ __global__ void scale_rows_kernel(uint4* __restrict__ x, int64_t ldx_v, int64_t 
   }
 }
 
+// MLP-block elimination criterion (Jenga summary §4.2.4): block i's score is the sum of
+// |a| over its blk rows and the F intermediate neurons, a = SiLU(gate) * up the MLP's
+// intermediate activation (bf16, compact retained rows).  One CTA per block; 16-byte
+// loads, fp32 sums, fixed-order reduction; blocks at or past the device count n_kept
+// score -inf.
+__global__ void __launch_bounds__(256) mlp_block_scores_kernel(const bf16* __restrict__ a, int64_t lda, int F,
+                                                               int blk, const int32_t* __restrict__ n_kept,
+                                                               int n_cap, float* __restrict__ scores) {
+  const int i = blockIdx.x;
+  int nk = n_kept ? *n_kept : n_cap;
+  nk = nk < 0 ? 0 : (nk > n_cap ? n_cap : nk);
+  if (i >= nk) {
+    if (threadIdx.x == 0) scores[i] = -INFINITY;
+    return;
+  }
+  __shared__ float s_w[8];
+  float acc = 0.f;
+  const int vpr = F / 8;  // 16-byte vectors per row
+  const int total = blk * vpr;
+  const bf16* ab = a + (int64_t)i * blk * lda;
+  for (int e0 = threadIdx.x; e0 < total; e0 += 4 * 256) {  // 4 vectors in flight per thread
+    uint4 u[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = e0 + q * 256;
+      const int r = e / vpr, c = e - r * vpr;
+      u[q] = (e < total) ? __ldcs(reinterpret_cast<const uint4*>(ab + (int64_t)r * lda) + c) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u[q]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __bfloat1622float2(p[k]);
+        acc += fabsf(f.x) + fabsf(f.y);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < 8; ++w) t += s_w[w];
+    scores[i] = t;
+  }
+}
+
+// out[i] = outer[pos[i]] for i < *n_pos, -1 after (pos indexes the outer list)
+__global__ void compose_indices_kernel(const int32_t* __restrict__ outer, int n_outer_cap,
+                                       const int32_t* __restrict__ pos, const int32_t* __restrict__ n_pos, int n_cap,
+                                       int32_t* __restrict__ out) {
+  const int np = *n_pos;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_cap; i += gridDim.x * blockDim.x) {
+    int v = -1;
+    if (i < np) {
+      const int p = pos[i];
+      if (p < 0 || p >= n_outer_cap) {
+        record_device_error(JENGA_EINTERNAL, SITE_INDEX_RANGE, (unsigned)p);
+      } else {
+        v = outer[p];
+      }
+    }
+    out[i] = v;
+  }
+}
+
 static int grid_for(int64_t vectors, int unroll) {
   int64_t want = (vectors + 256LL * unroll - 1) / (256LL * unroll);
   int cap = sm_count() * 8;  // 8 resident 256-thread CTAs per SM
@@ -285,6 +353,37 @@ extern "C" jenga_status jenga_scale_rows(void* x, int64_t ldx, int B, int S, int
                                                                       S, rows, n_rows, factor);
     ::jenga::prof_end(_ps, (cudaStream_t)stream);
     }
+  JENGA_LAUNCH_CHECK();
+  return JENGA_OK;
+}
+
+extern "C" jenga_status jenga_mlp_block_scores(const void* a, int64_t lda, int F, int blk, const int32_t* n_kept,
+                                               int n_cap, float* scores, jenga_stream_t stream) {
+  JENGA_CHECK_ARG(a && scores, "jenga_mlp_block_scores: null pointer");
+  JENGA_CHECK_ARG(F >= 8 && F % 8 == 0 && lda >= F && lda % 8 == 0 && blk >= 1 && n_cap >= 0 &&
+                      (int64_t)blk * (F / 8) < (1ll << 30) &&
+                      ((uintptr_t)a & 15) == 0,
+                  "jenga_mlp_block_scores: F and lda multiples of 8, 16-byte aligned rows");
+  if (n_cap == 0) return JENGA_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  {
+    const int _ps = ::jenga::prof_begin("mlp_block_scores", st);
+    mlp_block_scores_kernel<<<n_cap, 256, 0, st>>>((const bf16*)a, lda, F, blk, n_kept, n_cap, scores);
+    ::jenga::prof_end(_ps, st);
+  }
+  JENGA_LAUNCH_CHECK();
+  return JENGA_OK;
+}
+
+extern "C" jenga_status jenga_compose_block_indices(const int32_t* outer, int n_outer_cap, const int32_t* pos,
+                                                    const int32_t* n_pos, int n_cap, int32_t* out,
+                                                    jenga_stream_t stream) {
+  JENGA_CHECK_ARG(outer && pos && n_pos && out && n_outer_cap >= 0 && n_cap >= 0,
+                  "jenga_compose_block_indices: bad arguments");
+  if (n_cap == 0) return JENGA_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  compose_indices_kernel<<<(n_cap + 255) / 256 < 1024 ? (n_cap + 255) / 256 : 1024, 256, 0, st>>>(
+      outer, n_outer_cap, pos, n_pos, n_cap, out);
   JENGA_LAUNCH_CHECK();
   return JENGA_OK;
 }
