@@ -5,6 +5,8 @@
 //
 // All three are HBM-bound row moves: 128-bit loads/stores, several independent
 // vectors in flight per thread, grid sized to a multiple of the SM count.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 
 namespace jenga {
@@ -178,31 +180,38 @@ __global__ void scale_rows_kernel(uint4* __restrict__ x, int64_t ldx_v, int64_t 
 
 // MLP-block elimination criterion (Jenga summary §4.2.4): block i's score is the sum of
 // |a| over its blk rows and the F intermediate neurons, a = SiLU(gate) * up the MLP's
-// intermediate activation (bf16, compact retained rows).  One CTA per block; 16-byte
-// loads, fp32 sums, fixed-order reduction; blocks at or past the device count n_kept
-// score -inf.
-__global__ void __launch_bounds__(256) mlp_block_scores_kernel(const bf16* __restrict__ a, int64_t lda, int F,
-                                                               int blk, const int32_t* __restrict__ n_kept,
-                                                               int n_cap, float* __restrict__ scores) {
-  const int i = blockIdx.x;
+// intermediate activation (bf16, compact retained rows).  A cluster of MLP_SPLIT CTAs per
+// block (CTA p takes rows p, p + MLP_SPLIT, ...; 16-byte loads, 4 in flight per thread,
+// fp32 sums); the cluster's partial sums meet in the first CTA's shared memory and are
+// added in rank order, so the result does not depend on scheduling.  Blocks at or past
+// the device count n_kept score -inf.
+constexpr int MLP_SPLIT = 4;
+__global__ void __cluster_dims__(1, MLP_SPLIT, 1) __launch_bounds__(256)
+    mlp_block_scores_kernel(const bf16* __restrict__ a, int64_t lda, int F, int blk,
+                            const int32_t* __restrict__ n_kept, int n_cap, float* __restrict__ scores) {
+  namespace cg = cooperative_groups;
+  const int i = blockIdx.x, part = blockIdx.y;
   int nk = n_kept ? *n_kept : n_cap;
   nk = nk < 0 ? 0 : (nk > n_cap ? n_cap : nk);
-  if (i >= nk) {
-    if (threadIdx.x == 0) scores[i] = -INFINITY;
+  if (i >= nk) {  // uniform over the cluster (same block)
+    if (part == 0 && threadIdx.x == 0) scores[i] = -INFINITY;
     return;
   }
   __shared__ float s_w[8];
+  __shared__ float s_part;
   float acc = 0.f;
-  const int vpr = F / 8;  // 16-byte vectors per row
-  const int total = blk * vpr;
-  const bf16* ab = a + (int64_t)i * blk * lda;
-  for (int e0 = threadIdx.x; e0 < total; e0 += 4 * 256) {  // 4 vectors in flight per thread
+  const int vpr = F / 8;                                    // 16-byte vectors per row
+  const int nrow = (blk - part + MLP_SPLIT - 1) / MLP_SPLIT;  // this CTA's rows of the block
+  const int total = nrow * vpr;
+  const bf16* ab = a + ((int64_t)i * blk + part) * lda;
+  for (int e0 = threadIdx.x; e0 < total; e0 += 4 * 256) {
     uint4 u[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int e = e0 + q * 256;
       const int r = e / vpr, c = e - r * vpr;
-      u[q] = (e < total) ? __ldcs(reinterpret_cast<const uint4*>(ab + (int64_t)r * lda) + c) : make_uint4(0, 0, 0, 0);
+      u[q] = (e < total) ? __ldcs(reinterpret_cast<const uint4*>(ab + (int64_t)r * MLP_SPLIT * lda) + c)
+                         : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -221,8 +230,16 @@ __global__ void __launch_bounds__(256) mlp_block_scores_kernel(const bf16* __res
   if (threadIdx.x == 0) {
     float t = 0.f;
     for (int w = 0; w < 8; ++w) t += s_w[w];
+    s_part = t;
+  }
+  cg::cluster_group cluster = cg::this_cluster();
+  cluster.sync();  // every CTA's partial is in its shared memory
+  if (part == 0 && threadIdx.x == 0) {
+    float t = 0.f;
+    for (int r = 0; r < MLP_SPLIT; ++r) t += *cluster.map_shared_rank(&s_part, r);
     scores[i] = t;
   }
+  cluster.sync();  // the partials are read before any CTA of the cluster exits
 }
 
 // out[i] = outer[pos[i]] for i < *n_pos, -1 after (pos indexes the outer list)
@@ -368,7 +385,8 @@ extern "C" jenga_status jenga_mlp_block_scores(const void* a, int64_t lda, int F
   cudaStream_t st = (cudaStream_t)stream;
   {
     const int _ps = ::jenga::prof_begin("mlp_block_scores", st);
-    mlp_block_scores_kernel<<<n_cap, 256, 0, st>>>((const bf16*)a, lda, F, blk, n_kept, n_cap, scores);
+    mlp_block_scores_kernel<<<dim3(n_cap, MLP_SPLIT), 256, 0, st>>>((const bf16*)a, lda, F, blk, n_kept, n_cap,
+                                                                    scores);
     ::jenga::prof_end(_ps, st);
   }
   JENGA_LAUNCH_CHECK();
