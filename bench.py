@@ -446,7 +446,9 @@ def main():
                 J.jenga_score_blocks(b["qk"][:, :HD], b["qk"][:, HD:], sh.heads, sh.head_dim, blk, out=b["scores"][l],
                                      ws=b["sc_ws"])
                 J.jenga_select(b["scores"][l], "topk_frac", keep[l], out=(idx, nk, mask))
-            J.jenga_sparse_layer_fwd(L, X, idx, nk, blk, kmaxes[l], saved=b["saved"][l], ws=b["fws"])
+            # with exact scoring the retained rows' q and k come from the scoring's q | k
+            J.jenga_sparse_layer_fwd(L, X, idx, nk, blk, kmaxes[l], saved=b["saved"][l], ws=b["fws"],
+                                     qk=b["qk"] if (sparse and pred is None) else None)
         for l in reversed(range(len(layers))):
             idx, nk, _ = b["sel"][l]
             J.jenga_sparse_layer_bwd(layers[l], dX, idx, nk, blk, kmaxes[l], b["saved"][l], b["grads"][l],

@@ -237,6 +237,16 @@ JENGA_API jenga_status jenga_sparse_layer_fwd(const jenga_layer_weights* w, cons
                                     int n_kept_max, void* saved, size_t saved_bytes, void* ws, size_t ws_bytes,
                                     jenga_stream_t stream);
 
+/* jenga_sparse_layer_fwd_qk -- jenga_sparse_layer_fwd that takes the retained rows' q and k
+ * from qk_all, the [S, 2 H D] bf16 post-RoPE q | k of all rows that jenga_layer_score_qk
+ * produced for scoring from the same x (row pitch ld_qk elements, 16-byte aligned rows;
+ * read only), and projects only v (+ LoRA-v): the same kernels made those q and k, so the
+ * result is bit-identical to jenga_sparse_layer_fwd.  Other arguments and errors as there. */
+JENGA_API jenga_status jenga_sparse_layer_fwd_qk(const jenga_layer_weights* w, const jenga_lora* lora, const void* packed,
+                                       void* x, int B, int S, int blk, const int32_t* idx, const int32_t* n_kept,
+                                       int n_kept_max, const void* qk_all, int64_t ld_qk, void* saved,
+                                       size_t saved_bytes, void* ws, size_t ws_bytes, jenga_stream_t stream);
+
 /* jenga_sparse_layer_bwd -- a8 + a9: backward of jenga_sparse_layer_fwd for an upstream
  * gradient G held in dx ([B, S, hidden] bf16).  On return dx holds dL/dx: eliminated
  * rows keep G (identity through the residual), retained rows get the layer backward.

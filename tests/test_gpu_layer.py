@@ -105,3 +105,33 @@ def test_llama7b_shape_s4k_layer(J):
     oi, on, _ = osel.select_topk(gpu["scores"], 32)
     assert on == 32 and np.array_equal(oi, gpu["idx"])
     _check(case, gpu)
+
+
+@pytest.mark.parametrize("shape_name", ["small", "llama7b_s4k"])
+def test_forward_reusing_scoring_qk_is_bit_identical(J, shape_name):
+    """The forward may take the retained rows' q and k from the scoring's q | k of all rows
+    (same x, same kernels): outputs, saved context and gradients are bit-identical."""
+    from tests.layer_harness import bits_to_torch, layer_handle
+    case = small_case(seed=9, S=1024, blk=64) if shape_name == "small" else synth.gen_workload("llama7b_s4k", seed=1,
+                                                                                               lora_b_std=0.02)
+    sh = case.shape
+    L = layer_handle(case.layers[0], sh)
+    HD = sh.heads * sh.head_dim
+    x0 = bits_to_torch(case.x)
+    qk = J.jenga_layer_score_qk(L, x0)
+    sc = J.jenga_score_blocks(qk[:, :HD], qk[:, HD:], sh.heads, sh.head_dim, case.blk)
+    idx, nk, _ = J.jenga_select(sc, "topk_frac", 0.5)
+    kmax = osel.topk_count(0.5, case.S // case.blk)
+    res = []
+    for reuse in (False, True):
+        x = x0.clone()
+        saved = torch.zeros(L.saved_bytes(case.blk, kmax), dtype=torch.uint8, device="cuda")  # padding compares equal
+        J.jenga_sparse_layer_fwd(L, x, idx, nk, case.blk, kmax, saved=saved, qk=qk if reuse else None)
+        dx = bits_to_torch(case.g)
+        grads = J.new_lora_grads(L)
+        J.jenga_sparse_layer_bwd(L, dx, idx, nk, case.blk, kmax, saved, grads, segment_tokens=1024)
+        J.jenga_check_device_status()
+        res.append((x, saved, dx, grads))
+    (xa, sa, da, ga), (xb, sb, db, gb) = res
+    assert torch.equal(xa, xb) and torch.equal(sa, sb) and torch.equal(da, db)
+    assert all(torch.equal(ga[k], gb[k]) for k in ga)

@@ -204,17 +204,27 @@ def jenga_layer_score_qk(layer: LayerHandle, x, out=None, ws=None, stream=None):
     return out
 
 
-def jenga_sparse_layer_fwd(layer: LayerHandle, x, idx, n_kept, blk, n_kept_max, saved=None, ws=None, stream=None):
-    """In place on x [S, h] bf16.  Returns the saved-context buffer for the backward."""
+def jenga_sparse_layer_fwd(layer: LayerHandle, x, idx, n_kept, blk, n_kept_max, saved=None, ws=None, stream=None,
+                           qk=None):
+    """In place on x [S, h] bf16.  Returns the saved-context buffer for the backward.
+
+    qk: optional [S, 2 H D] bf16 q | k of all rows from jenga_layer_score_qk on the same x;
+    the retained rows' q and k are then taken from it (bit-identical) instead of projected."""
     _need_cuda(x, idx, n_kept)
     S = x.shape[-2]
     if saved is None:
         saved = _ws(layer.saved_bytes(blk, n_kept_max), x.device)
     if ws is None:
         ws = _ws(layer.fwd_ws_bytes(blk, n_kept_max), x.device)
-    check(load().jenga_sparse_layer_fwd(ctypes.byref(layer.w), ctypes.byref(layer.lora), _p(layer.packed), _p(x), 1, S,
-                                        blk, _p(idx), _p(n_kept), int(n_kept_max), _p(saved), saved.numel(), _p(ws),
-                                        ws.numel(), _stream(stream)))
+    if qk is None:
+        check(load().jenga_sparse_layer_fwd(ctypes.byref(layer.w), ctypes.byref(layer.lora), _p(layer.packed), _p(x), 1,
+                                            S, blk, _p(idx), _p(n_kept), int(n_kept_max), _p(saved), saved.numel(),
+                                            _p(ws), ws.numel(), _stream(stream)))
+    else:
+        _need_cuda(qk)
+        check(load().jenga_sparse_layer_fwd_qk(ctypes.byref(layer.w), ctypes.byref(layer.lora), _p(layer.packed), _p(x),
+                                               1, S, blk, _p(idx), _p(n_kept), int(n_kept_max), _p(qk), qk.stride(0),
+                                               _p(saved), saved.numel(), _p(ws), ws.numel(), _stream(stream)))
     return saved
 
 

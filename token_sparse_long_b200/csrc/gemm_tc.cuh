@@ -60,6 +60,7 @@ struct EpiParams {
   float alpha = 1.f;
   float beta = 1.f;              // LORA_T: scale of the fp32 copy
   int hd = 0;                    // QKV: H * D (section width)
+  int col0 = 0;                  // QKV: column of this GEMM's first output in the q | k | v layout
   const float2* rope_tab = nullptr;  // QKV: (cos, sin) of position(m) x frequency j, [M rows][64]
   bool tma_out = false;          // set by the launcher: the output tensor map is valid
 };
@@ -469,7 +470,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll 1
         for (int g = 0; g < BN / 128; ++g) {
           const int nh = n0 + g * 128;
-          const bool rope = nh < 2 * ep.hd;
+          const bool rope = ep.col0 + nh < 2 * ep.hd;
 #pragma unroll 1
           for (int hh = 0; hh < 2; ++hh) {
             float u[32];

@@ -348,10 +348,10 @@ extern "C" size_t jenga_layer_fwd_workspace_bytes(const jenga_layer_weights* w, 
   return carve_fwd_ws(c, d, n_kept_max * blk, &f);
 }
 
-extern "C" jenga_status jenga_sparse_layer_fwd(const jenga_layer_weights* w, const jenga_lora* lora,
-                                               const void* packed, void* x, int B, int S, int blk, const int32_t* idx,
-                                               const int32_t* n_kept, int n_kept_max, void* saved, size_t saved_bytes,
-                                               void* ws, size_t ws_bytes, jenga_stream_t stream) {
+static jenga_status layer_fwd(const jenga_layer_weights* w, const jenga_lora* lora, const void* packed, void* x,
+                              int B, int S, int blk, const int32_t* idx, const int32_t* n_kept, int n_kept_max,
+                              void* saved, size_t saved_bytes, void* ws, size_t ws_bytes, const void* qk_all,
+                              int64_t ld_qk, jenga_stream_t stream) {
   Dims d;
   JENGA_TRY(check_weights(w, lora, &d));
   JENGA_CHECK_ARG(packed && x && idx && n_kept, "jenga_sparse_layer_fwd: null pointer");
@@ -392,8 +392,26 @@ extern "C" jenga_status jenga_sparse_layer_fwd(const jenga_layer_weights* w, con
     JENGA_TRY((launch_gemm<32, EPI_LORA_T>({f.xn, nc, h}, {p.aqv, 2 * LORA_R, h}, h, nullptr, nullptr, 0, nc,
                                            2 * LORA_R, e, st, "gemm_lora_t")));
   }
-  // 3. QKV (+ LoRA up-projection as a second K phase) with RoPE at original positions
-  {
+  // 3. QKV (+ LoRA up-projection as a second K phase) with RoPE at original positions.
+  //    With the scoring's q | k of all rows (same x, same kernels, so the same bits), the
+  //    retained rows' q and k are copied from it and only v (+ LoRA-v) is projected.
+  if (qk_all) {
+    {
+      const int _ps = ::jenga::prof_begin("gather_qk_rows", st);
+      gather_rows_bf16_kernel<<<grid_cap((int64_t)nc * (2 * HD / 8), 256), 256, 0, st>>>(
+          (const bf16*)qk_all, ld_qk, s.qkv, 3 * HD, 2 * HD, idx, blk, n_kept, blk, nc);
+      ::jenga::prof_end(_ps, st);
+    }
+    JENGA_LAUNCH_CHECK();
+    EpiParams e = epi_base(idx, blk, n_kept, 0);
+    e.out = s.qkv + 2 * HD;
+    e.ldo = 3 * HD;
+    e.hd = HD;
+    e.col0 = 2 * HD;  // the v section: no RoPE
+    GemmOperand a2{f.tb, nc, LORA_PAD}, b2{p.lorab + (size_t)2 * HD * LORA_PAD, HD, LORA_PAD};
+    JENGA_TRY((launch_gemm<256, EPI_QKV_ROPE>({f.xn, nc, h}, {p.wqkv + (size_t)2 * HD * h, HD, h}, h, &a2, &b2,
+                                              LORA_PAD, nc, HD, e, st, "gemm_v")));
+  } else {
     EpiParams e = epi_base(idx, blk, n_kept, 0);
     e.out = s.qkv;
     e.ldo = 3 * HD;
@@ -447,6 +465,27 @@ extern "C" jenga_status jenga_sparse_layer_fwd(const jenga_layer_weights* w, con
     JENGA_TRY((launch_gemm<256, EPI_SCATTER_ADD>({f.a, nc, F}, {w->wd, h, F}, F, nullptr, nullptr, 0, nc, h, e, st, "gemm_down_scatter")));
   }
   return JENGA_OK;
+}
+
+extern "C" jenga_status jenga_sparse_layer_fwd(const jenga_layer_weights* w, const jenga_lora* lora,
+                                               const void* packed, void* x, int B, int S, int blk, const int32_t* idx,
+                                               const int32_t* n_kept, int n_kept_max, void* saved, size_t saved_bytes,
+                                               void* ws, size_t ws_bytes, jenga_stream_t stream) {
+  return layer_fwd(w, lora, packed, x, B, S, blk, idx, n_kept, n_kept_max, saved, saved_bytes, ws, ws_bytes, nullptr,
+                   0, stream);
+}
+
+extern "C" jenga_status jenga_sparse_layer_fwd_qk(const jenga_layer_weights* w, const jenga_lora* lora,
+                                                  const void* packed, void* x, int B, int S, int blk,
+                                                  const int32_t* idx, const int32_t* n_kept, int n_kept_max,
+                                                  const void* qk_all, int64_t ld_qk, void* saved, size_t saved_bytes,
+                                                  void* ws, size_t ws_bytes, jenga_stream_t stream) {
+  Dims d;
+  JENGA_TRY(check_weights(w, lora, &d));
+  JENGA_CHECK_ARG(qk_all && ld_qk >= 2 * (int64_t)d.HD && ld_qk % 8 == 0 && ((uintptr_t)qk_all & 15) == 0,
+                  "jenga_sparse_layer_fwd_qk: qk_all must be [S, >= 2 H D] bf16, 16-byte aligned rows");
+  return layer_fwd(w, lora, packed, x, B, S, blk, idx, n_kept, n_kept_max, saved, saved_bytes, ws, ws_bytes, qk_all,
+                   ld_qk, stream);
 }
 
 // ==================================================================== backward

@@ -343,6 +343,21 @@ __global__ void rope_table_kernel(float2* __restrict__ tab, int rows, const int3
   }
 }
 
+// dst[m, 0:cols] = src[row(m), 0:cols] for the compact rows m below the device-side valid
+// count (row(m) through the kept-block list), 16-byte vectors; cols % 8 == 0.
+__global__ void gather_rows_bf16_kernel(const bf16* __restrict__ src, int64_t lds, bf16* __restrict__ dst,
+                                        int64_t ldd, int cols, const int32_t* __restrict__ idx, int blk,
+                                        const int32_t* __restrict__ n_valid, int valid_mult, int rows) {
+  const int nv = valid_rows(n_valid, valid_mult, 0, rows);
+  const int vpr = cols / 8;
+  const int64_t total = (int64_t)nv * vpr;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int m = (int)(e / vpr), c = (int)(e - (int64_t)m * vpr);
+    const int64_t r = seq_row(idx, blk, m);
+    reinterpret_cast<uint4*>(dst + (int64_t)m * ldd)[c] = __ldg(reinterpret_cast<const uint4*>(src + r * lds) + c);
+  }
+}
+
 // ---- weight re-layout (pack)
 // dst[(dr0 + c) * ldd + dc0 + r] = src[(sr0 + r) * lds + sc0 + c] for r < R, c < C   (transpose)
 __global__ void transpose_bf16_kernel(const bf16* __restrict__ src, int64_t lds, bf16* __restrict__ dst,
