@@ -78,3 +78,29 @@ def test_package_imports_without_gpu():
     with pytest.raises(Exception):
         import torch
         J.jenga_select(torch.zeros(4), "mean_ge")   # CPU tensor: refused, no CPU path
+
+
+def test_lm_loss_and_predictor_pair_host_checks(lib):
+    null = ctypes.c_void_p(0)
+    p = ctypes.c_void_p(256)
+    # segmented LM loss: the workspace holds one segment's logits (fp32) and gradient rows
+    # (bf16) plus the transposed embedding, so it grows with the segment, not with S
+    seg = lib.jenga_lm_loss_workspace_bytes(32768, 4096, 32000, 4096)
+    full = lib.jenga_lm_loss_workspace_bytes(32768, 4096, 32000, 32768)
+    assert seg >= 4096 * 32000 * 6 + 4096 * 32000 * 2 and full >= 32768 * 32000 * 6
+    assert full > 5 * seg
+    assert lib.jenga_lm_loss_workspace_bytes(100, 64, 64, 4096) == lib.jenga_lm_loss_workspace_bytes(100, 64, 64, 100)
+    # V not a multiple of 64; null pointers; workspace too small
+    assert lib.jenga_lm_loss_segmented(p, p, p, 128, 64, 1000, 64, p, p, p, 1 << 30, null) == _lib.EINVAL
+    assert lib.jenga_lm_loss_segmented(null, p, p, 128, 64, 1024, 64, p, p, p, 1 << 30, null) == _lib.EINVAL
+    assert lib.jenga_lm_loss_segmented(p, p, p, 128, 64, 1024, 64, p, p, p, 16, null) == _lib.EWORKSPACE
+    # Q/K predictor pair: output width above 64 and misaligned inputs are refused
+    assert lib.jenga_predict_qk_workspace_bytes(1, 32768, 5120, 128, 16) >= 256 * 5120 * 4 + 2 * 256 * 16 * 4
+    assert lib.jenga_predict_blocks_qk(p, 1, 1024, 512, 128, p, p, p, p, p, p, 128, 64, 65, 1, p, p, 1 << 30,
+                                       null) == _lib.EINVAL
+    q = ctypes.c_void_p(264)
+    assert lib.jenga_predict_blocks_qk(q, 1, 1024, 512, 128, p, p, p, p, p, p, 128, 64, 16, 1, p, p, 1 << 30,
+                                       null) == _lib.EINVAL
+    # MLP-block criterion: F must be a multiple of 8
+    assert lib.jenga_mlp_block_scores(p, 1004, 1004, 64, null, 4, p, null) == _lib.EINVAL
+    assert lib.jenga_mlp_block_scores(p, 1008, 1008, 64, null, 0, p, null) == 0  # nothing to do
