@@ -120,12 +120,21 @@ __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_bwd_rows_kernel(
   if (m >= valid_rows(n_valid, valid_mult, row_offset, gridDim.x)) return;
   const int nch = h >> 3;
   const float r = rstd[m];
-  float dyg[ROW_MAX_CHUNKS][8], xv[ROW_MAX_CHUNKS][8];
+  float dyg[ROW_MAX_CHUNKS][8], xv[ROW_MAX_CHUNKS][8], bv[ROW_MAX_CHUNKS][8];
   float dot = 0.f;
 #pragma unroll
   for (int i = 0; i < ROW_MAX_CHUNKS; ++i) {
     const int c = threadIdx.x + i * ROW_THREADS;
     if (c < nch) {
+      // the residual base is loaded here too, so its latency overlaps the row reduction
+      if (base_f) {
+        const float4* bp = reinterpret_cast<const float4*>(base_f + (int64_t)m * ldb) + 2 * c;
+        const float4 a = bp[0], b = bp[1];
+        bv[i][0] = a.x; bv[i][1] = a.y; bv[i][2] = a.z; bv[i][3] = a.w;
+        bv[i][4] = b.x; bv[i][5] = b.y; bv[i][6] = b.z; bv[i][7] = b.w;
+      } else {
+        unpack8(reinterpret_cast<const uint4*>(base_b + (int64_t)m * ldb)[c], bv[i]);
+      }
       const float4* dp = reinterpret_cast<const float4*>(dy + (int64_t)m * lddy) + 2 * c;
       float4 a = dp[0], b = dp[1];
       float gv[8];
@@ -150,18 +159,9 @@ __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_bwd_rows_kernel(
   for (int i = 0; i < ROW_MAX_CHUNKS; ++i) {
     const int c = threadIdx.x + i * ROW_THREADS;
     if (c < nch) {
-      float bv[8];
-      if (base_f) {
-        const float4* bp = reinterpret_cast<const float4*>(base_f + (int64_t)m * ldb) + 2 * c;
-        float4 a = bp[0], b = bp[1];
-        bv[0] = a.x; bv[1] = a.y; bv[2] = a.z; bv[3] = a.w;
-        bv[4] = b.x; bv[5] = b.y; bv[6] = b.z; bv[7] = b.w;
-      } else {
-        unpack8(reinterpret_cast<const uint4*>(base_b + (int64_t)m * ldb)[c], bv);
-      }
       float o[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = bv[e] + r * dyg[i][e] - xv[i][e] * k;
+      for (int e = 0; e < 8; ++e) o[e] = bv[i][e] + r * dyg[i][e] - xv[i][e] * k;
       if (out_f) {
         float4* op = reinterpret_cast<float4*>(out_f + (int64_t)m * ldo) + 2 * c;
         op[0] = make_float4(o[0], o[1], o[2], o[3]);
