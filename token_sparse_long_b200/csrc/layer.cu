@@ -107,6 +107,7 @@ struct BwdWs {
   float *dk_acc, *dv_acc;
   bf16 *xn, *g, *dgu, *dhb, *dhlo, *dO, *dqkv, *dqkvlo, *dtb;
   float *gu, *dhn, *dh, *delta, *dq, *dt, *part;
+  float2* rope;  // [T][64] (cos, sin) of the segment rows' positions
 };
 static size_t carve_bwd_ws(Carve& c, const Dims& d, int nc, int T, BwdWs* w) {
   w->dk_acc = c.take<float>((size_t)nc * d.HD);
@@ -126,6 +127,7 @@ static size_t carve_bwd_ws(Carve& c, const Dims& d, int nc, int T, BwdWs* w) {
   w->delta = c.take<float>((size_t)d.H * T);
   w->dq = c.take<float>((size_t)T * d.HD);
   w->dt = c.take<float>((size_t)T * 2 * LORA_R);
+  w->rope = c.take<float2>((size_t)T * 64);
   const int chunks = (T + LG_CHUNK - 1) / LG_CHUNK;
   const int cmax = d.HD > d.h ? d.HD : d.h;
   w->part = c.take<float>((size_t)4 * chunks * cmax * 16);
@@ -305,7 +307,7 @@ extern "C" jenga_status jenga_layer_score_qk(const jenga_layer_weights* w, const
   float2* rope = c.take<float2>((size_t)S * 64);
   {
     const int _ps = ::jenga::prof_begin("rope_table", st);
-    rope_table_kernel<<<grid_cap((int64_t)S * 64, 256), 256, 0, st>>>(rope, S, nullptr, 1, nullptr, 1, p.inv_freq);
+    rope_table_kernel<<<grid_cap((int64_t)S * 64, 256), 256, 0, st>>>(rope, S, nullptr, 1, nullptr, 1, 0, p.inv_freq);
     ::jenga::prof_end(_ps, st);
   }
   JENGA_LAUNCH_CHECK();
@@ -419,7 +421,8 @@ static jenga_status layer_fwd(const jenga_layer_weights* w, const jenga_lora* lo
     e.rope_tab = f.rope;
     {
       const int _ps = ::jenga::prof_begin("rope_table", st);
-      rope_table_kernel<<<grid_cap((int64_t)nc * 64, 256), 256, 0, st>>>(f.rope, nc, idx, blk, n_kept, blk, p.inv_freq);
+      rope_table_kernel<<<grid_cap((int64_t)nc * 64, 256), 256, 0, st>>>(f.rope, nc, idx, blk, n_kept, blk, 0,
+                                                                        p.inv_freq);
       ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();
@@ -599,9 +602,16 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
                                     b.dq, HD, b.dk_acc, b.dv_acc, HD, H, s0, s1, n_kept, blk, nc, st));
     // keys of this segment are complete: RoPE^T and pack dQKV (bf16)
     {
+    const int _ps = ::jenga::prof_begin("rope_table", st);
+    rope_table_kernel<<<grid_cap((int64_t)T * 64, 256), 256, 0, st>>>(b.rope, T, idx, blk, n_kept, blk, s0,
+                                                                       p.inv_freq);
+    ::jenga::prof_end(_ps, st);
+    }
+    JENGA_LAUNCH_CHECK();
+    {
     const int _ps = ::jenga::prof_begin("rope_bwd_pack", st);
-    rope_bwd_pack_kernel<<<grid_cap((int64_t)T * H * 64, 256), 256, 0, st>>>(
-        b.dq, HD, b.dk_acc, b.dv_acc, HD, s0, b.dqkv, b.dqkvlo, 3 * HD, idx, blk, n_kept, blk, T, H, p.inv_freq);
+    rope_bwd_pack_kernel<<<grid_cap((int64_t)T * H * 32, 256), 256, 0, st>>>(
+        b.dq, HD, b.dk_acc, b.dv_acc, HD, s0, b.dqkv, b.dqkvlo, 3 * HD, b.rope, n_kept, blk, T, H);
     ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();

@@ -202,42 +202,47 @@ __global__ void gather_seg_kernel(const bf16* __restrict__ src, int64_t lds, bf1
   }
 }
 
-// dqkv[m] = [rope^T(dq[m]) | rope^T(dk[s0+m]) | dv[s0+m]] as a bf16 hi part (dqkv) and the
-// bf16 residual (dqkv_lo); positions row(s0 + m).
-// One thread per (row, head, pair i < 64).
+// Backward of RoPE on dq / dk (the transpose rotation) and the pack of dQ | dK | dV for the
+// segment's rows [s0, s0 + nv) into bf16 hi and lo halves (hi = bf16(x), lo = bf16(x - hi)).
+// One warp per (row, head): lane l takes frequency pair (2l, 2l + 1), reading its (cos,
+// sin) pairs from the segment's RoPE table (tab[m][j], rope_table_kernel at offset s0),
+// 8-byte loads and bf16x2 stores.
 __global__ void rope_bwd_pack_kernel(const float* __restrict__ dq, int64_t ld_dq, const float* __restrict__ dk,
                                      const float* __restrict__ dv, int64_t ld_acc, int s0, bf16* __restrict__ dqkv,
-                                     bf16* __restrict__ dqkv_lo, int64_t ld_out, const int32_t* __restrict__ idx, int blk,
-                                     const int32_t* __restrict__ n_valid, int valid_mult, int rows, int H,
-                                     const double* __restrict__ inv_freq) {
+                                     bf16* __restrict__ dqkv_lo, int64_t ld_out, const float2* __restrict__ tab,
+                                     const int32_t* __restrict__ n_valid, int valid_mult, int rows, int H) {
   const int nv = valid_rows(n_valid, valid_mult, s0, rows);
-  const int64_t total = (int64_t)nv * H * 64;
+  const int64_t total = (int64_t)nv * H * 32;
   const int HD = H * 128;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-    const int i = (int)(e & 63);
-    const int64_t mh = e >> 6;
-    const int hh = (int)(mh % H);
-    const int m = (int)(mh / H);
-    const int64_t pos = seq_row(idx, blk, s0 + m);
-    const double ang = (double)pos * inv_freq[i];
-    const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
-    float sn, cs;
-    sincosf((float)red, &sn, &cs);
-    const int c1 = hh * 128 + i, c2 = c1 + 64;
-    const float* q = dq + (int64_t)m * ld_dq;
-    const float* kk = dk + (int64_t)(s0 + m) * ld_acc;
-    const float* vv = dv + (int64_t)(s0 + m) * ld_acc;
+    const int ip = (int)(e & 31);
+    const int mh = (int)(e >> 5);
+    const int m = mh / H, hh = mh - m * H;
+    const float4 t = __ldg(reinterpret_cast<const float4*>(tab + (int64_t)m * 64) + ip);  // (cos, sin) x 2
+    const int c1 = hh * 128 + 2 * ip, c2 = c1 + 64;
+    const float2 a1 = *reinterpret_cast<const float2*>(dq + (int64_t)m * ld_dq + c1);
+    const float2 a2 = *reinterpret_cast<const float2*>(dq + (int64_t)m * ld_dq + c2);
+    const float2 b1 = *reinterpret_cast<const float2*>(dk + (int64_t)(s0 + m) * ld_acc + c1);
+    const float2 b2 = *reinterpret_cast<const float2*>(dk + (int64_t)(s0 + m) * ld_acc + c2);
+    const float2 v1 = *reinterpret_cast<const float2*>(dv + (int64_t)(s0 + m) * ld_acc + c1);
+    const float2 v2 = *reinterpret_cast<const float2*>(dv + (int64_t)(s0 + m) * ld_acc + c2);
+    // per frequency: (x1, x2) -> (x1 cos + x2 sin, x2 cos - x1 sin)
+    const float val[6][2] = {{a1.x * t.x + a2.x * t.y, a1.y * t.z + a2.y * t.w},
+                             {a2.x * t.x - a1.x * t.y, a2.y * t.z - a1.y * t.w},
+                             {b1.x * t.x + b2.x * t.y, b1.y * t.z + b2.y * t.w},
+                             {b2.x * t.x - b1.x * t.y, b2.y * t.z - b1.y * t.w},
+                             {v1.x, v1.y},
+                             {v2.x, v2.y}};
+    const int col[6] = {c1, c2, HD + c1, HD + c2, 2 * HD + c1, 2 * HD + c2};
     bf16* o = dqkv + (int64_t)m * ld_out;
     bf16* ol = dqkv_lo + (int64_t)m * ld_out;
-    const float a1 = q[c1], a2 = q[c2];
-    const float b1 = kk[c1], b2 = kk[c2];
-    const float val[6] = {a1 * cs + a2 * sn, a2 * cs - a1 * sn, b1 * cs + b2 * sn, b2 * cs - b1 * sn, vv[c1], vv[c2]};
-    const int col[6] = {c1, c2, HD + c1, HD + c2, 2 * HD + c1, 2 * HD + c2};
 #pragma unroll
-    for (int e = 0; e < 6; ++e) {
-      const bf16 hi = __float2bfloat16_rn(val[e]);
-      o[col[e]] = hi;
-      ol[col[e]] = __float2bfloat16_rn(val[e] - __bfloat162float(hi));
+    for (int k2 = 0; k2 < 6; ++k2) {
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(val[k2][0], val[k2][1]);
+      const float2 hf = __bfloat1622float2(hi);
+      *reinterpret_cast<__nv_bfloat162*>(o + col[k2]) = hi;
+      *reinterpret_cast<__nv_bfloat162*>(ol + col[k2]) =
+          __floats2bfloat162_rn(val[k2][0] - hf.x, val[k2][1] - hf.y);
     }
   }
 }
@@ -328,13 +333,13 @@ __global__ void lora_grad_reduce_kernel(LoraGradJobs jobs, const float* __restri
 // (position through the kept-block list when idx is given), the angle reduced to [-pi, pi] in
 // float64 before a float sincos.  Rows past the device-side valid count get position 0.
 __global__ void rope_table_kernel(float2* __restrict__ tab, int rows, const int32_t* __restrict__ idx, int blk,
-                                  const int32_t* __restrict__ n_valid, int valid_mult,
+                                  const int32_t* __restrict__ n_valid, int valid_mult, int row_offset,
                                   const double* __restrict__ inv_freq) {
-  const int nv = valid_rows(n_valid, valid_mult, 0, rows);
+  const int nv = valid_rows(n_valid, valid_mult, row_offset, rows);
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < (int64_t)rows * 64;
        e += (int64_t)gridDim.x * blockDim.x) {
     const int m = (int)(e >> 6), j = (int)(e & 63);
-    const int64_t pos = (m < nv) ? (idx ? seq_row(idx, blk, m) : m) : 0;
+    const int64_t pos = (m < nv) ? (idx ? seq_row(idx, blk, row_offset + m) : row_offset + m) : 0;
     const double ang = (double)pos * inv_freq[j];
     const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
     float sn, cs;
