@@ -104,3 +104,18 @@ def test_lm_loss_and_predictor_pair_host_checks(lib):
     # MLP-block criterion: F must be a multiple of 8
     assert lib.jenga_mlp_block_scores(p, 1004, 1004, 64, null, 4, p, null) == _lib.EINVAL
     assert lib.jenga_mlp_block_scores(p, 1008, 1008, 64, null, 0, p, null) == 0  # nothing to do
+
+
+def test_product_path_never_touches_the_oracle():
+    # the oracle is test infrastructure: the package (binding, build script, kernels) must
+    # neither import it nor reference its files
+    pkg = os.path.join(ROOT, "token_sparse_long_b200")
+    hits = []
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                with open(os.path.join(dirpath, f)) as fh:
+                    for n, line in enumerate(fh, 1):
+                        if re.search(r"\b(import\s+oracle|from\s+oracle|oracle/)", line):
+                            hits.append(f"{f}:{n}")
+    assert not hits, hits
