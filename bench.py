@@ -363,6 +363,24 @@ def measure_movement(J, torch, dev, X0, case, ks, hbm):
     return out
 
 
+def max_over_ranks(x, device):
+    """The per-rank value's maximum over the process group (the timing rule for N ranks:
+    the slowest replica sets the step time); x itself with no group or one rank."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_tokens_per_s(S, world, ms):
+    """Whole-job throughput of `world` independent replicas of an S-token step that took
+    ms milliseconds on the slowest rank."""
+    return S * world / (ms / 1e3)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -483,12 +501,7 @@ def main():
         e.record()
         torch.cuda.synchronize()
         barrier()
-        ms = s.elapsed_time(e) / K
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return max_over_ranks(s.elapsed_time(e) / K, dev)
 
     # ---------------- sparse step (headline)
     torch.cuda.reset_peak_memory_stats(dev)
@@ -666,7 +679,7 @@ def main():
                          f"algorithmic flops ({full / 1e12:.1f} TFLOP)"}
 
     if rank == 0:
-        line = {"metric": METRIC, "value": S * world / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        line = {"metric": METRIC, "value": replica_tokens_per_s(S, world, ms), "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": {"workload": args.workload, "seq_len": S, "global_batch": world, "layers": len(layers),
