@@ -62,12 +62,15 @@ def causal_pairs(n):
     return n * (n + 1) / 2.0
 
 
-def work_model(case, ks, seg):
+def work_model(case, ks, seg, scoring="exact"):
     """Algorithmic work per step for each kernel name: (kind, amount) with kind
     'flop' or 'byte'.  GEMM: 2 M N K.  Attention fwd: 2 matmuls per causal pair
     (4 D H pairs); backward: 5 matmul-equivalents per pair (10 D H pairs), shared
     3 : 4 between the dQ and dK/dV kernels in proportion to the matmuls each runs.
-    Scoring: one QK^T product per causal pair per pass (2 D H pairs)."""
+    Scoring ('exact'): q, k of all rows, then one QK^T product per causal pair per pass
+    (2 D H pairs); the forward then takes the retained rows' q, k from the scoring and
+    projects only v.  Scoring 'predictor': one read of X for the block means (the MLP is
+    negligible), and the forward projects q, k and v."""
     sh = case.shape
     S, h, H, D, F = case.S, sh.hidden, sh.heads, sh.head_dim, sh.ffn
     HD = H * D
@@ -79,12 +82,17 @@ def work_model(case, ks, seg):
 
     for k in ks:
         n = k * case.blk
-        add("gemm_lora_t_all", "flop", 2.0 * S * 32 * h)
-        add("gemm_qk_rope_all", "flop", 2.0 * S * 2 * HD * h)
-        add("score_lse_tc", "flop", 2.0 * D * H * causal_pairs(S))
-        add("score_mass_tc", "flop", 2.0 * D * H * causal_pairs(S))
+        if scoring == "exact":
+            add("gemm_lora_t_all", "flop", 2.0 * S * 32 * h)
+            add("gemm_qk_rope_all", "flop", 2.0 * S * 2 * HD * h)
+            add("score_lse_tc", "flop", 2.0 * D * H * causal_pairs(S))
+            add("score_mass_tc", "flop", 2.0 * D * H * causal_pairs(S))
+            add("gemm_v", "flop", 2.0 * n * HD * h)
+            add("gather_qk_rows", "byte", 2.0 * n * 2 * HD * 2)
+        else:
+            add("pred_block_mean", "byte", 2.0 * S * h)
+            add("gemm_qkv_rope", "flop", 2.0 * n * 3 * HD * h)
         add("gemm_lora_t", "flop", 2.0 * n * 32 * h)
-        add("gemm_qkv_rope", "flop", 2.0 * n * 3 * HD * h)
         add("attn_fwd_tc", "flop", 4.0 * D * H * causal_pairs(n))
         add("gemm_o_scatter", "flop", 2.0 * n * h * HD)
         add("gemm_gateup_swiglu", "flop", 2.0 * n * 2 * F * h)
@@ -122,8 +130,8 @@ def traffic_units(name, case, ks, seg):
     return None
 
 
-def step_flops(case, ks):
-    return sum(v for k, v in work_model(case, ks, 4096).values() if k == "flop")
+def step_flops(case, ks, scoring="exact"):
+    return sum(v for k, v in work_model(case, ks, 4096, scoring).values() if k == "flop")
 
 
 # ---------------------------------------------------------------------------- clocks
@@ -253,7 +261,7 @@ def full_step_flops(w, ks):
         pass
     c = C()
     c.shape, c.S, c.blk = w.shape, w.S, w.blk
-    return step_flops(c, ks)
+    return step_flops(c, ks, "predictor" if w.predictor_hidden else "exact")
 
 
 # ---------------------------------------------------------------------------- GPU arm
@@ -524,7 +532,8 @@ def main():
 
     # ---------------- roofline of the dominant kernel (live per-launch events, timed region)
     hbm, tf_burst, tf_sus, peak_src = load_peaks()
-    wm = work_model(case, ks, seg)
+    scoring = "predictor" if pred is not None else "exact"
+    wm = work_model(case, ks, seg, scoring)
     top = max(prof.items(), key=lambda kv: kv[1]["ms"])
     tname, tstat = top
     launches = sum(v["launches"] for v in prof.values())
@@ -672,7 +681,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         dt, fl = oracle_sample(case, BASELINE_TOKENS)
         rate = fl / dt
-        full = step_flops(case, ks)
+        full = step_flops(case, ks, scoring)
         cpu = {"value": S / (full / rate), "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
                "sample": f"oracle scoring + top-50% selection + retained-token fwd+bwd of layer 0 on the first "
                          f"{BASELINE_TOKENS} tokens ({dt:.1f} s, {fl / 1e9:.0f} GFLOP); scaled by the full step's "
@@ -690,7 +699,7 @@ def main():
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "movement": movement,
                 "clocks": clk, "peak_mem_gib": peak_sparse, "dense": dense,
                 **({"predictor": predictor} if predictor is not None else {}), "lm_loss": lm_loss,
-                "step_tflop": step_flops(case, ks) / 1e12, "kernels": kernels}
+                "step_tflop": step_flops(case, ks, scoring) / 1e12, "kernels": kernels}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
