@@ -241,7 +241,11 @@ JENGA_API jenga_status jenga_sparse_layer_fwd(const jenga_layer_weights* w, cons
  * from qk_all, the [S, 2 H D] bf16 post-RoPE q | k of all rows that jenga_layer_score_qk
  * produced for scoring from the same x (row pitch ld_qk elements, 16-byte aligned rows;
  * read only), and projects only v (+ LoRA-v): the same kernels made those q and k, so the
- * result is bit-identical to jenga_sparse_layer_fwd.  Other arguments and errors as there. */
+ * result is bit-identical to jenga_sparse_layer_fwd.  qk_all must be recomputed after ANY
+ * change to x (including jenga_scale_rows), to the weights or to the LoRA tensors: the
+ * library cannot detect a stale buffer, and one silently gives wrong q and k.  qk_all must
+ * hold at least S rows (the library cannot check its row count).  Other arguments and
+ * errors as there. */
 JENGA_API jenga_status jenga_sparse_layer_fwd_qk(const jenga_layer_weights* w, const jenga_lora* lora, const void* packed,
                                        void* x, int B, int S, int blk, const int32_t* idx, const int32_t* n_kept,
                                        int n_kept_max, const void* qk_all, int64_t ld_qk, void* saved,
@@ -346,6 +350,15 @@ JENGA_API jenga_status jenga_test_gemm(const void* A, int64_t lda, const void* B
  * to [-125, 64]), and y_mufu[i] = 2^x[i] by the hardware approximation (ex2.approx.ftz).
  * x, y_fma, y_mufu: device fp32 arrays of n elements.  For accuracy tests only. */
 JENGA_API jenga_status jenga_test_exp2(const float* x, float* y_fma, float* y_mufu, int n, jenga_stream_t stream);
+
+/**
+ * jenga_test_wait_timeout -- exercises the device-side wait bound (no counterpart in the
+ * paper).  Launches one warp that waits on a shared-memory barrier nothing ever completes;
+ * after the current wait budget (jenga_set_wait_budget_ns) it records JENGA_ETIMEOUT (site 8,
+ * detail 0xC0FFEE) in the device error word and returns, with nothing else in flight.  The
+ * next jenga_check_device_status(stream) then returns JENGA_ETIMEOUT.  Set a short budget
+ * first (the default is 2 s) and restore it afterwards.  For tests only. */
+JENGA_API jenga_status jenga_test_wait_timeout(jenga_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -131,62 +131,98 @@ def silu_grad(z):
     return s * (1.0 + z * (1.0 - s))
 
 
-def attention_fwd(q, k, v, chunk=1024):
-    """Causal softmax attention per head (softmax(q k^T / sqrt(D)) v, keys j <= i).
+def head_attention_fwd(args):
+    """Causal softmax attention of ONE head: args = (qh, kh, vh [n, D], chunk).
 
-    Returns o [n, H, D] and the row log-sum-exp [H, n] of the scaled logits."""
-    n, H, D = q.shape
+    o_i = softmax_j(q_i . k_j / sqrt(D)) v over keys j <= i.  Returns o [n, D] and the
+    row log-sum-exp [n] of the scaled logits; rows go in chunks only to bound memory."""
+    qh, kh, vh, chunk = args
+    n, D = qh.shape
     scale = 1.0 / np.sqrt(D)
-    o = np.zeros_like(q)
-    lse = np.zeros((H, n))
+    o = np.zeros_like(qh)
+    lse = np.zeros(n)
     jj = np.arange(n)
-    for h in range(H):
-        for i0 in range(0, n, chunk):
-            i1 = min(n, i0 + chunk)
-            s = (q[i0:i1, h] @ k[:i1, h].T) * scale
-            s = np.where(jj[None, :i1] <= np.arange(i0, i1)[:, None], s, -np.inf)
-            m = s.max(axis=1, keepdims=True)
-            p = np.exp(s - m)
-            l = p.sum(axis=1, keepdims=True)
-            o[i0:i1, h] = (p / l) @ v[:i1, h]
-            lse[h, i0:i1] = (m + np.log(l))[:, 0]
+    for i0 in range(0, n, chunk):
+        i1 = min(n, i0 + chunk)
+        s = (qh[i0:i1] @ kh[:i1].T) * scale
+        s = np.where(jj[None, :i1] <= np.arange(i0, i1)[:, None], s, -np.inf)
+        m = s.max(axis=1, keepdims=True)
+        p = np.exp(s - m)
+        l = p.sum(axis=1, keepdims=True)
+        o[i0:i1] = (p / l) @ vh[:i1]
+        lse[i0:i1] = (m + np.log(l))[:, 0]
     return o, lse
 
 
-def attention_bwd_rows(q, k, v, do, r0, r1, dk_acc, dv_acc, chunk=1024):
-    """Backward of ``attention_fwd`` for the query rows [r0, r1).
+def _heads(t):
+    return [np.ascontiguousarray(t[:, h]) for h in range(t.shape[1])]
 
-    Returns dq for those rows and ADDS their contribution to dk_acc / dv_acc (keys
-    [0, r1)).  dS = P * (dP - rowsum(P * dP)), dP = dO V^T, dQ = dS K / sqrt(D),
-    dK = dS^T Q / sqrt(D), dV = P^T dO (textbook softmax-attention backward)."""
+
+def attention_fwd(q, k, v, chunk=1024, pmap=map):
+    """Causal softmax attention per head (softmax(q k^T / sqrt(D)) v, keys j <= i).
+
+    Returns o [n, H, D] and the row log-sum-exp [H, n] of the scaled logits.  ``pmap``
+    maps ``head_attention_fwd`` over the heads (independent of one another)."""
     n, H, D = q.shape
+    o = np.zeros_like(q)
+    lse = np.zeros((H, n))
+    tasks = [(qh, kh, vh, chunk) for qh, kh, vh in zip(_heads(q), _heads(k), _heads(v))]
+    for h, (oh, lh) in enumerate(pmap(head_attention_fwd, tasks)):
+        o[:, h] = oh
+        lse[h] = lh
+    return o, lse
+
+
+def head_attention_bwd(args):
+    """Backward of ``head_attention_fwd`` for ONE head: args = (qh, kh, vh, doh [n, D],
+    segments, chunk).  The query rows go segment by segment in the order given (each
+    segment (r0, r1) in row chunks); every segment's contribution is added to the key /
+    value gradients of keys [0, r1).  Per chunk, the textbook softmax-attention backward:
+    P = softmax(q k^T / sqrt(D)) (causal), dP = dO V^T, dS = P * (dP - rowsum(P * dP)),
+    dQ = dS K / sqrt(D), dK += dS^T Q / sqrt(D), dV += P^T dO.  Returns dq, dk, dv [n, D]."""
+    qh, kh, vh, doh, segments, chunk = args
+    n, D = qh.shape
     scale = 1.0 / np.sqrt(D)
-    dq = np.zeros((r1 - r0, H, D))
+    dq = np.zeros((n, D))
+    dk = np.zeros((n, D))
+    dv = np.zeros((n, D))
     jj = np.arange(n)
-    for h in range(H):
+    for (r0, r1) in segments:
         for i0 in range(r0, r1, chunk):
             i1 = min(r1, i0 + chunk)
-            s = (q[i0:i1, h] @ k[:i1, h].T) * scale
+            s = (qh[i0:i1] @ kh[:i1].T) * scale
             s = np.where(jj[None, :i1] <= np.arange(i0, i1)[:, None], s, -np.inf)
             m = s.max(axis=1, keepdims=True)
             p = np.exp(s - m)
             p /= p.sum(axis=1, keepdims=True)
-            dp = do[i0:i1, h] @ v[:i1, h].T
+            dp = doh[i0:i1] @ vh[:i1].T
             delta = (p * dp).sum(axis=1, keepdims=True)
             ds = p * (dp - delta)
-            dq[i0 - r0:i1 - r0, h] = (ds @ k[:i1, h]) * scale
-            dk_acc[:i1, h] += (ds.T @ q[i0:i1, h]) * scale
-            dv_acc[:i1, h] += p.T @ do[i0:i1, h]
-    return dq
+            dq[i0:i1] = (ds @ kh[:i1]) * scale
+            dk[:i1] += (ds.T @ qh[i0:i1]) * scale
+            dv[:i1] += p.T @ doh[i0:i1]
+    return dq, dk, dv
+
+
+def attention_bwd(q, k, v, do, segments, chunk=1024, pmap=map):
+    """``head_attention_bwd`` for every head (mapped with ``pmap``): dq, dk, dv [n, H, D]."""
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(q)
+    dv = np.zeros_like(q)
+    tasks = [(qh, kh, vh, dh, segments, chunk) for qh, kh, vh, dh in zip(_heads(q), _heads(k), _heads(v), _heads(do))]
+    for h, (a, b, c) in enumerate(pmap(head_attention_bwd, tasks)):
+        dq[:, h], dk[:, h], dv[:, h] = a, b, c
+    return dq, dk, dv
 
 
 # ------------------------------------------------------------------ layer
 
 
-def layer_fwd(x, pos, W: Weights, rnd=True):
-    """Llama decoder layer on the retained rows x [n, h] at original positions ``pos``.
-
-    Returns (out [n, h], ctx) where ctx holds what the backward needs."""
+def project_qk(x, pos, W: Weights, rnd=True, with_v=False):
+    """The attention input projections of rows x [n, h] at original positions ``pos``:
+    xn = RMSNorm(x) (rounded), q = RoPE(xn Wq^T + s (xn Aq^T) Bq^T), k = RoPE(xn Wk^T)
+    (rounded after RoPE), and with ``with_v`` also v = xn Wv^T + s (xn Av^T) Bv^T (rounded).
+    Returns dict(xn, rstd1, tq, tv, q, k[, v], cos, sin); q, k, v are [n, H, D]."""
     x = np.asarray(x, np.float64)
     n, hdim = x.shape
     H, D, s = W.heads, W.head_dim, W.lora_scale
@@ -196,11 +232,26 @@ def layer_fwd(x, pos, W: Weights, rnd=True):
     tv = xn @ W.av.T
     q_lin = (xn @ W.wq.T + s * (tq @ W.bq.T)).reshape(n, H, D)
     k_lin = (xn @ W.wk.T).reshape(n, H, D)
-    v = _r((xn @ W.wv.T + s * (tv @ W.bv.T)).reshape(n, H, D), rnd)
     cos, sin = rope_cos_sin(pos, D, W.theta)
-    q = _r(rope(q_lin, cos, sin), rnd)
-    k = _r(rope(k_lin, cos, sin), rnd)
-    o, lse = attention_fwd(q, k, v)
+    out = dict(xn=xn, rstd1=rstd1, tq=tq, tv=tv, q=_r(rope(q_lin, cos, sin), rnd), k=_r(rope(k_lin, cos, sin), rnd),
+               cos=cos, sin=sin)
+    if with_v:
+        out["v"] = _r((xn @ W.wv.T + s * (tv @ W.bv.T)).reshape(n, H, D), rnd)
+    return out
+
+
+def layer_fwd(x, pos, W: Weights, rnd=True, pmap=map):
+    """Llama decoder layer on the retained rows x [n, h] at original positions ``pos``.
+
+    Returns (out [n, h], ctx) where ctx holds what the backward needs.  ``pmap`` maps the
+    per-head attention (see ``attention_fwd``)."""
+    x = np.asarray(x, np.float64)
+    n, hdim = x.shape
+    H, D = W.heads, W.head_dim
+    pr = project_qk(x, pos, W, rnd, with_v=True)
+    xn, rstd1, tq, tv, q, k, v, cos, sin = (pr[key] for key in ("xn", "rstd1", "tq", "tv", "q", "k", "v", "cos",
+                                                                 "sin"))
+    o, lse = attention_fwd(q, k, v, pmap=pmap)
     o = _r(o, rnd)
     h = _r(x + o.reshape(n, H * D) @ W.wo.T, rnd)
     hn, rstd2 = rms_norm(h, W.g2, W.eps)
@@ -220,25 +271,30 @@ def _segments(n, seg):
     return [(s0, min(n, s0 + seg)) for s0 in range(0, n, seg)]
 
 
-def layer_bwd(ctx, G, W: Weights, segment_tokens=None):
+def layer_bwd(ctx, G, W: Weights, segment_tokens=None, pmap=map):
     """Backward of ``layer_fwd`` for loss = sum(out * G) (so dOut = G).
 
     Frozen base weights get no gradient.  Returns (dx [n, h], grads) with grads the
     LoRA gradients daq [r, h], dbq [H*D, r], dav, dbv.  ``segment_tokens`` splits the
-    retained rows into consecutive segments processed last-first (module docstring)."""
+    retained rows into consecutive segments processed last-first (module docstring):
+    the MLP block and the o projection are row-local, so every segment's attention-output
+    gradient is formed first; the attention backward then runs per head over the query
+    segments, last first, accumulating the key / value gradients; the projection backward
+    (row-local once a segment's key / value gradients are complete) follows per segment,
+    last first, adding each segment's LoRA gradient contribution in that order."""
     G = np.asarray(G, np.float64)
     x, xn, h, hn = ctx["x"], ctx["xn"], ctx["h"], ctx["hn"]
-    q, k, v, o = ctx["q"], ctx["k"], ctx["v"], ctx["o"]
+    q, k, v = ctx["q"], ctx["k"], ctx["v"]
     cos, sin = ctx["cos"], ctx["sin"]
     n, hdim = x.shape
     H, D, s = W.heads, W.head_dim, W.lora_scale
-    r = W.aq.shape[0]
     dx = np.zeros((n, hdim))
     grads = dict(daq=np.zeros_like(W.aq), dbq=np.zeros_like(W.bq),
                  dav=np.zeros_like(W.av), dbv=np.zeros_like(W.bv))
-    dk_acc = np.zeros((n, H, D))
-    dv_acc = np.zeros((n, H, D))
-    for (s0, s1) in reversed(_segments(n, segment_tokens)):
+    segs = list(reversed(_segments(n, segment_tokens)))
+    dh_all = np.zeros((n, hdim))
+    do_all = np.zeros((n, H, D))
+    for (s0, s1) in segs:
         sl = slice(s0, s1)
         # --- MLP block: out = h + (silu(hn Wg^T) * (hn Wu^T)) Wd^T
         Gs = G[sl]
@@ -247,15 +303,15 @@ def layer_bwd(ctx, G, W: Weights, segment_tokens=None):
         dut = da * silu(gt)
         dgt = da * ut * silu_grad(gt)
         dhn = dgt @ W.wg + dut @ W.wu
-        dh = Gs + rms_norm_bwd(dhn, h[sl], W.g2, ctx["rstd2"][sl])
+        dh_all[sl] = Gs + rms_norm_bwd(dhn, h[sl], W.g2, ctx["rstd2"][sl])
         # --- attention block: h = x + o Wo^T
-        do_full = np.zeros((n, H, D))
-        do_full[sl] = (dh @ W.wo).reshape(s1 - s0, H, D)
-        dq = attention_bwd_rows(q, k, v, do_full, s0, s1, dk_acc, dv_acc)
-        # keys/values of this segment are complete now
-        dq_lin = rope_bwd(dq, cos[sl], sin[sl]).reshape(s1 - s0, H * D)
-        dk_lin = rope_bwd(dk_acc[sl], cos[sl], sin[sl]).reshape(s1 - s0, H * D)
-        dv = dv_acc[sl].reshape(s1 - s0, H * D)
+        do_all[sl] = (dh_all[sl] @ W.wo).reshape(s1 - s0, H, D)
+    dq, dk, dv_h = attention_bwd(q, k, v, do_all, segs, pmap=pmap)
+    for (s0, s1) in segs:
+        sl = slice(s0, s1)
+        dq_lin = rope_bwd(dq[sl], cos[sl], sin[sl]).reshape(s1 - s0, H * D)
+        dk_lin = rope_bwd(dk[sl], cos[sl], sin[sl]).reshape(s1 - s0, H * D)
+        dv = dv_h[sl].reshape(s1 - s0, H * D)
         dtq = s * (dq_lin @ W.bq)                      # [ns, r]
         dtv = s * (dv @ W.bv)
         grads["dbq"] += s * (dq_lin.T @ ctx["tq"][sl])
@@ -263,28 +319,27 @@ def layer_bwd(ctx, G, W: Weights, segment_tokens=None):
         grads["daq"] += dtq.T @ xn[sl]
         grads["dav"] += dtv.T @ xn[sl]
         dxn = dq_lin @ W.wq + dk_lin @ W.wk + dv @ W.wv + dtq @ W.aq + dtv @ W.av
-        dx[sl] = dh + rms_norm_bwd(dxn, x[sl], W.g1, ctx["rstd1"][sl])
-    del r
+        dx[sl] = dh_all[sl] + rms_norm_bwd(dxn, x[sl], W.g1, ctx["rstd1"][sl])
     return _r(dx, ctx["rnd"]), grads
 
 
 # ------------------------------------------------------------------ whole sequence
 
 
-def sparse_layer_fwd(X, idx, n_kept, blk, W: Weights, rnd=True):
+def sparse_layer_fwd(X, idx, n_kept, blk, W: Weights, rnd=True, pmap=map):
     """Layer on the kept blocks of X [S, h]; eliminated rows pass through unchanged."""
     X = np.asarray(X, np.float64)
     rows = retained_rows(idx, n_kept, blk)
     Xo = X.copy()
     if rows.size == 0:
         return Xo, None
-    out, ctx = layer_fwd(X[rows], rows, W, rnd)
+    out, ctx = layer_fwd(X[rows], rows, W, rnd, pmap=pmap)
     Xo[rows] = out
     ctx["rows"] = rows
     return Xo, ctx
 
 
-def sparse_layer_bwd(ctx, G, W: Weights, segment_tokens=None):
+def sparse_layer_bwd(ctx, G, W: Weights, segment_tokens=None, pmap=map):
     """dX = G on eliminated rows; the layer backward on retained rows."""
     G = np.asarray(G, np.float64)
     dX = G.copy()
@@ -293,6 +348,6 @@ def sparse_layer_bwd(ctx, G, W: Weights, segment_tokens=None):
                  dav=np.zeros_like(W.av), dbv=np.zeros_like(W.bv))
         return dX, z
     rows = ctx["rows"]
-    dx, grads = layer_bwd(ctx, G[rows], W, segment_tokens)
+    dx, grads = layer_bwd(ctx, G[rows], W, segment_tokens, pmap=pmap)
     dX[rows] = dx
     return dX, grads

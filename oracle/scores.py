@@ -25,36 +25,51 @@ def _as_f64(a):
     return np.asarray(a, dtype=np.float64)
 
 
-def column_mass(q, k, causal=True, chunk=512):
-    """Per-key softmax column mass, summed over heads.
+def head_column_mass(args):
+    """Softmax column mass of ONE head: args = (qh [S, D], kh [S, D], causal, chunk).
 
-    q, k: [S, H, D].  Returns [S] with mass[j] = sum_h sum_i P^h_ij where
-    P^h_i. = softmax_j(q^h_i . k^h_j / sqrt(D)) over j <= i (all j if not causal).
-    The softmax is the textbook one (subtract the row max, exponentiate, divide by
-    the row sum); rows are processed in chunks only to bound memory.
-    """
-    q = _as_f64(q)
-    k = _as_f64(k)
-    S, H, D = q.shape
+    Returns [S] with mass[j] = sum_i P_ij, P_i. = softmax_j(q_i . k_j / sqrt(D)) over
+    j <= i (all j if not causal).  The softmax is the textbook one (subtract the row max,
+    exponentiate, divide by the row sum); rows are processed in chunks only to bound
+    memory, and a causal chunk of rows [i0, i1) only forms the keys j < i1 (the others
+    have probability exactly 0)."""
+    qh, kh, causal, chunk = args
+    qh = _as_f64(qh)
+    kh = _as_f64(kh)
+    S, D = qh.shape
     scale = 1.0 / np.sqrt(D)
     mass = np.zeros(S, dtype=np.float64)
-    jj = np.arange(S)
-    for h in range(H):
-        kh = k[:, h, :]
-        for i0 in range(0, S, chunk):
-            i1 = min(S, i0 + chunk)
-            s = (q[i0:i1, h, :] @ kh.T) * scale            # [c, S]
-            if causal:
-                ii = np.arange(i0, i1)[:, None]
-                s = np.where(jj[None, :] <= ii, s, -np.inf)
-            m = s.max(axis=1, keepdims=True)
-            p = np.exp(s - m)
-            p /= p.sum(axis=1, keepdims=True)
-            mass += p.sum(axis=0)
+    for i0 in range(0, S, chunk):
+        i1 = min(S, i0 + chunk)
+        kend = i1 if causal else S
+        s = (qh[i0:i1] @ kh[:kend].T) * scale            # [c, kend]
+        if causal:
+            ii = np.arange(i0, i1)[:, None]
+            s = np.where(np.arange(kend)[None, :] <= ii, s, -np.inf)
+        m = s.max(axis=1, keepdims=True)
+        p = np.exp(s - m)
+        p /= p.sum(axis=1, keepdims=True)
+        mass[:kend] += p.sum(axis=0)
     return mass
 
 
-def block_scores_softmax_mass(q, k, blk, causal=True):
+def column_mass(q, k, causal=True, chunk=512, pmap=map):
+    """Per-key softmax column mass, summed over heads (in head order).
+
+    q, k: [S, H, D].  Returns [S] with mass[j] = sum_h sum_i P^h_ij (``head_column_mass``
+    per head).  ``pmap`` maps the per-head function over the heads (the builtin ``map`` by
+    default; a process pool's ``map`` gives the same result, since heads are independent)."""
+    q = _as_f64(q)
+    k = _as_f64(k)
+    S, H, D = q.shape
+    mass = np.zeros(S, dtype=np.float64)
+    tasks = [(np.ascontiguousarray(q[:, h, :]), np.ascontiguousarray(k[:, h, :]), causal, chunk) for h in range(H)]
+    for mh in pmap(head_column_mass, tasks):
+        mass += mh
+    return mass
+
+
+def block_scores_softmax_mass(q, k, blk, causal=True, pmap=map):
     """Score of each token block: sum of ``column_mass`` over the block's keys.
 
     q, k: [S, H, D] (one sequence) or [B, S, H, D].  S must be a multiple of blk.
@@ -63,10 +78,10 @@ def block_scores_softmax_mass(q, k, blk, causal=True):
     q = _as_f64(q)
     k = _as_f64(k)
     if q.ndim == 4:
-        return np.stack([block_scores_softmax_mass(q[b], k[b], blk, causal) for b in range(q.shape[0])])
+        return np.stack([block_scores_softmax_mass(q[b], k[b], blk, causal, pmap) for b in range(q.shape[0])])
     S = q.shape[0]
     assert S % blk == 0
-    mass = column_mass(q, k, causal)
+    mass = column_mass(q, k, causal, pmap=pmap)
     return mass.reshape(S // blk, blk).sum(axis=1)
 
 

@@ -96,6 +96,7 @@ _SIGS = {
     "jenga_test_gemm": (c_int, [c_void_p, c_int64, c_void_p, c_int64, c_int, c_int, c_int, c_void_p, c_int64, c_int,
                                 c_int, c_void_p]),
     "jenga_test_exp2": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_void_p]),
+    "jenga_test_wait_timeout": (c_int, [c_void_p]),
 }
 
 _lib = None

@@ -209,7 +209,9 @@ def jenga_sparse_layer_fwd(layer: LayerHandle, x, idx, n_kept, blk, n_kept_max, 
     """In place on x [S, h] bf16.  Returns the saved-context buffer for the backward.
 
     qk: optional [S, 2 H D] bf16 q | k of all rows from jenga_layer_score_qk on the same x;
-    the retained rows' q and k are then taken from it (bit-identical) instead of projected."""
+    the retained rows' q and k are then taken from it (bit-identical) instead of projected.
+    qk must have been computed from this x, after any change to x (e.g. jenga_scale_rows),
+    and with this layer's weights and LoRA: a stale qk silently gives wrong q and k."""
     _need_cuda(x, idx, n_kept)
     S = x.shape[-2]
     if saved is None:
@@ -222,6 +224,12 @@ def jenga_sparse_layer_fwd(layer: LayerHandle, x, idx, n_kept, blk, n_kept_max, 
                                             _p(ws), ws.numel(), _stream(stream)))
     else:
         _need_cuda(qk)
+        HD = layer.heads * layer.head_dim
+        if qk.dtype != torch.bfloat16 or qk.device != x.device:
+            raise ValueError("qk must be a bf16 tensor on x's device")
+        if qk.dim() != 2 or qk.shape[0] < S or qk.shape[1] < 2 * HD or qk.stride(1) != 1:
+            raise ValueError(f"qk must be [>= {S}, >= {2 * HD}] with a contiguous last dimension, got "
+                             f"{tuple(qk.shape)} strides {qk.stride()}")
         check(load().jenga_sparse_layer_fwd_qk(ctypes.byref(layer.w), ctypes.byref(layer.lora), _p(layer.packed), _p(x),
                                                1, S, blk, _p(idx), _p(n_kept), int(n_kept_max), _p(qk), qk.stride(0),
                                                _p(saved), saved.numel(), _p(ws), ws.numel(), _stream(stream)))
@@ -330,6 +338,12 @@ def jenga_test_gemm(a, b, out_f32=True, bn=256, stream=None):
     check(load().jenga_test_gemm(_p(a), a.stride(0), _p(b), b.stride(0), M, N, K, _p(c), c.stride(0),
                                  1 if out_f32 else 0, bn, _stream(stream)))
     return c
+
+
+def jenga_test_wait_timeout(stream=None):
+    """Launch the wait-bound test hook (see include/jenga.h); read the result with
+    jenga_check_device_status."""
+    check(load().jenga_test_wait_timeout(_stream(stream)))
 
 
 def jenga_test_exp2(x, stream=None):

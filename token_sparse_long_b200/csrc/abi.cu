@@ -137,9 +137,29 @@ jenga_status make_tmap_f32(CUtensorMap* map, const void* base, uint64_t rows, ui
   return JENGA_OK;
 }
 
+// Test hook of the bounded-wait path: one warp initialises an mbarrier that nothing ever
+// arrives on and waits for its first phase.  No copy or tensor-core operation is in flight,
+// so when the wait budget runs out the kernel only records JENGA_ETIMEOUT and returns.
+__global__ void test_wait_timeout_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  const bool ok = mbar_wait_at(&bar, 0, SITE_TEST_WAIT, 0xC0FFEEu);
+  (void)__all_sync(0xffffffffu, ok);
+}
+
 }  // namespace jenga
 
 using namespace jenga;
+
+extern "C" jenga_status jenga_test_wait_timeout(jenga_stream_t stream) {
+  test_wait_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>();
+  JENGA_LAUNCH_CHECK();
+  return JENGA_OK;
+}
 
 extern "C" const char* jenga_status_string(jenga_status st) {
   switch (st) {

@@ -57,6 +57,7 @@ enum ErrSite : unsigned int {
   SITE_INDEX_RANGE = 5,
   SITE_NKEPT_RANGE = 6,
   SITE_ATTN = 7,
+  SITE_TEST_WAIT = 8,
 };
 
 __device__ __forceinline__ void record_device_error(unsigned code, unsigned site, unsigned detail) {
@@ -388,7 +389,8 @@ __device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
 // the multi-function unit (16 results per clock per SM).  Binary split x = j + f with j the
 // integer nearest x (the 1.5 * 2^23 shifter rounds x into the low mantissa bits) and
 // |f| <= 1/2; 2^f is a cubic whose relative error is equal-ripple on [-1/2, 1/2]
-// (coefficients from token_sparse_long_b200/exp2_fit.py, max relative error 7.5e-5);
+// (coefficients: a Lawson IRLS minimax fit, refitted and checked by tests/test_exp2_fit.py;
+// max relative error 7.5e-5);
 // 2^j is added into the exponent field.  Inputs are clamped to [-125, HI], so the result
 // is >= 2^-125.5 for very negative x and finite for large x.
 template <int HI = 64>

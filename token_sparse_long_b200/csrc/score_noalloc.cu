@@ -10,7 +10,7 @@
 // The array is a file-scope __device__ object: every GPU that loads the library holds
 // it (16 MiB) until the process exits.  Its device address is looked up once per device
 // with cudaGetSymbolAddress while that device is current (the first call on the device
-// does this).  All calls share the array; each call overwrites every element it later
+// does this, and the first call in a new context after a device reset does it again).  All calls share the array; each call overwrites every element it later
 // reads, so no clearing is needed, but two calls whose kernels overlap on the GPU (e.g.
 // on different streams) race on it.
 #include <mutex>
@@ -25,18 +25,42 @@ static __device__ __align__(256) unsigned char g_score_scratch[NOALLOC_SCRATCH_B
 
 static std::mutex s_noalloc_mu;
 static void* s_noalloc_ptr[128];
+static void* s_noalloc_ctx[128];  // the CUDA context the cached address belongs to
 
+typedef int (*CtxGetCurrentFn)(void**);
+
+static void* current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  void* ctx = nullptr;
+  if (fn) fn(&ctx);
+  return ctx;
+}
+
+// Device address of the scratch array in the current context.  Looked up with
+// cudaGetSymbolAddress the first time a device is used and again whenever the current
+// context differs from the one the cached address was taken in (a new primary context
+// after cudaDeviceReset loads the module again, possibly at another address).
 static jenga_status noalloc_scratch(void** out) {
   int dev = -1;
   JENGA_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 128) return fail(JENGA_EUNSUPPORTED, "jenga_score_blocks_noalloc: device ordinal %d", dev);
   std::lock_guard<std::mutex> lock(s_noalloc_mu);
-  if (!s_noalloc_ptr[dev]) {
+  void* ctx = current_context();
+  if (!s_noalloc_ptr[dev] || !ctx || ctx != s_noalloc_ctx[dev]) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_score_scratch);
     if (e != cudaSuccess || !p)
       return fail(JENGA_ECUDA, "jenga_score_blocks_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
     s_noalloc_ptr[dev] = p;
+    s_noalloc_ctx[dev] = current_context();  // bound by the lookup if it was not yet
   }
   *out = s_noalloc_ptr[dev];
   return JENGA_OK;
