@@ -19,7 +19,13 @@ Readings (the pages are silent on these):
 * RMSNorm eps 1e-5, learned gains applied after normalisation; RoPE theta 10000 with
   the rotate-half convention (pairs d and d + D/2); LoRA on q_proj and v_proj,
   delta W = scale * B @ A, no dropout, no biases.
-* One index set per layer serves both sub-blocks.
+* One index set per layer serves both sub-blocks, unless an MLP keep mask is given
+  (Jenga summary §4.2.4, extend to the MLP block): then the MLP sub-block runs only on the
+  retained rows whose mask entry is set, and on the others the layer output is h (the
+  attention sub-block's output), so their MLP branch contributes nothing to the forward
+  and its gradient is zero in the backward.  The mask is per retained row (per retained
+  block in ``sparse_layer_fwd``); which blocks to keep is decided elsewhere (the GPU's
+  criterion and selection are passed in, like the attention block list).
 * bf16 storage rounding (``rnd=True``) at: xn (normed attention input), q and k after
   RoPE, v, the attention output o, h (after the attention residual add), hn (normed
   MLP input), a = SiLU(g) * u, the layer output, and the input gradient dX.  All other
@@ -240,11 +246,12 @@ def project_qk(x, pos, W: Weights, rnd=True, with_v=False):
     return out
 
 
-def layer_fwd(x, pos, W: Weights, rnd=True, pmap=map):
+def layer_fwd(x, pos, W: Weights, rnd=True, pmap=map, mlp_keep=None):
     """Llama decoder layer on the retained rows x [n, h] at original positions ``pos``.
 
     Returns (out [n, h], ctx) where ctx holds what the backward needs.  ``pmap`` maps the
-    per-head attention (see ``attention_fwd``)."""
+    per-head attention (see ``attention_fwd``).  ``mlp_keep`` (bool [n], optional): rows
+    whose MLP sub-block runs; the others output h (module docstring)."""
     x = np.asarray(x, np.float64)
     n, hdim = x.shape
     H, D = W.heads, W.head_dim
@@ -260,8 +267,11 @@ def layer_fwd(x, pos, W: Weights, rnd=True, pmap=map):
     ut = hn @ W.wu.T
     a = _r(silu(gt) * ut, rnd)
     out = _r(h + a @ W.wd.T, rnd)
+    if mlp_keep is not None:
+        mlp_keep = np.asarray(mlp_keep, bool)
+        out = np.where(mlp_keep[:, None], out, h)
     ctx = dict(x=x, pos=np.asarray(pos), xn=xn, rstd1=rstd1, tq=tq, tv=tv, q=q, k=k, v=v, o=o,
-               lse=lse, h=h, hn=hn, rstd2=rstd2, gt=gt, ut=ut, a=a, cos=cos, sin=sin, rnd=rnd)
+               lse=lse, h=h, hn=hn, rstd2=rstd2, gt=gt, ut=ut, a=a, cos=cos, sin=sin, rnd=rnd, mlp_keep=mlp_keep)
     return out, ctx
 
 
@@ -296,9 +306,11 @@ def layer_bwd(ctx, G, W: Weights, segment_tokens=None, pmap=map):
     do_all = np.zeros((n, H, D))
     for (s0, s1) in segs:
         sl = slice(s0, s1)
-        # --- MLP block: out = h + (silu(hn Wg^T) * (hn Wu^T)) Wd^T
+        # --- MLP block: out = h + (silu(hn Wg^T) * (hn Wu^T)) Wd^T (rows the MLP keeps)
         Gs = G[sl]
-        da = Gs @ W.wd
+        keep = ctx.get("mlp_keep")
+        Gm = Gs if keep is None else Gs * keep[sl][:, None]
+        da = Gm @ W.wd
         gt, ut = ctx["gt"][sl], ctx["ut"][sl]
         dut = da * silu(gt)
         dgt = da * ut * silu_grad(gt)
@@ -326,14 +338,19 @@ def layer_bwd(ctx, G, W: Weights, segment_tokens=None, pmap=map):
 # ------------------------------------------------------------------ whole sequence
 
 
-def sparse_layer_fwd(X, idx, n_kept, blk, W: Weights, rnd=True, pmap=map):
-    """Layer on the kept blocks of X [S, h]; eliminated rows pass through unchanged."""
+def sparse_layer_fwd(X, idx, n_kept, blk, W: Weights, rnd=True, pmap=map, mlp_keep_blocks=None):
+    """Layer on the kept blocks of X [S, h]; eliminated rows pass through unchanged.
+    ``mlp_keep_blocks`` (bool per retained block, in kept-list order, optional): the blocks
+    whose MLP sub-block runs (``layer_fwd``'s mlp_keep, expanded to rows)."""
     X = np.asarray(X, np.float64)
     rows = retained_rows(idx, n_kept, blk)
     Xo = X.copy()
     if rows.size == 0:
         return Xo, None
-    out, ctx = layer_fwd(X[rows], rows, W, rnd, pmap=pmap)
+    keep = None
+    if mlp_keep_blocks is not None:
+        keep = np.repeat(np.asarray(mlp_keep_blocks, bool)[: int(n_kept)], blk)
+    out, ctx = layer_fwd(X[rows], rows, W, rnd, pmap=pmap, mlp_keep=keep)
     Xo[rows] = out
     ctx["rows"] = rows
     return Xo, ctx

@@ -212,3 +212,66 @@ def test_rounded_mode_stays_close_to_exact():
     d0, _ = oly.layer_bwd(c0, G, W)
     d1, _ = oly.layer_bwd(c1, G, W)
     assert np.abs(d1 - d0).max() / np.sqrt((d0 ** 2).mean()) < 3e-2
+
+
+# ------------------------------------------------------------------ MLP-block keep mask
+def test_mlp_mask_all_kept_is_bit_identical_to_no_mask():
+    W = _weights(9)
+    X, G = _case(9, S=32)
+    idx = np.array([0, 2, 3, 5, 7, -1, -1, -1], np.int32)
+    Xa, ca = oly.sparse_layer_fwd(X, idx, 5, 4, W, rnd=True)
+    dXa, ga = oly.sparse_layer_bwd(ca, G, W, 8)
+    Xb, cb = oly.sparse_layer_fwd(X, idx, 5, 4, W, rnd=True, mlp_keep_blocks=np.ones(5, bool))
+    dXb, gb = oly.sparse_layer_bwd(cb, G, W, 8)
+    assert np.array_equal(Xa, Xb) and np.array_equal(dXa, dXb)
+    assert all(np.array_equal(ga[k], gb[k]) for k in ga)
+
+
+def _hf_run_mlp_mask(W, x_r, pos, G_r, keep_rows):
+    """HF layer whose MLP output is multiplied by the 0/1 row mask: out = h + m * MLP(norm(h))."""
+    from transformers.models.llama import modeling_llama as ml
+    orig = ml.LlamaMLP.forward
+    mask = torch.tensor(keep_rows.astype(np.float64))[None, :, None]
+    ml.LlamaMLP.forward = lambda self, x: orig(self, x) * mask
+    try:
+        return _hf_run(W, x_r, pos, G_r)
+    finally:
+        ml.LlamaMLP.forward = orig
+
+
+def test_mlp_mask_matches_hf_layer_with_masked_mlp_branch():
+    W = _weights(10)
+    X, G = _case(10, S=32)
+    idx = np.array([1, 2, 4, 6, 7, -1, -1, -1], np.int32)
+    keep_blocks = np.array([True, False, True, False, False])
+    Xo, ctx = oly.sparse_layer_fwd(X, idx, 5, 4, W, rnd=False, mlp_keep_blocks=keep_blocks)
+    dX, grads = oly.sparse_layer_bwd(ctx, G, W)
+    rows = retained_rows(idx, 5, 4)
+    out_hf, dx_hf, g_hf = _hf_run_mlp_mask(W, X[rows], rows, G[rows], np.repeat(keep_blocks, 4))
+    np.testing.assert_allclose(Xo[rows], out_hf, rtol=RT, atol=AT)
+    np.testing.assert_allclose(dX[rows], dx_hf, rtol=RT, atol=AT)
+    for key in g_hf:
+        np.testing.assert_allclose(grads[key], g_hf[key], rtol=RT, atol=AT * 10)
+    # MLP-eliminated rows output exactly h = x + attention output
+    h = ctx["h"]
+    dropped = ~np.repeat(keep_blocks, 4)
+    np.testing.assert_array_equal(Xo[rows][dropped], h[dropped])
+
+
+def test_mlp_mask_finite_differences():
+    W = _weights(11, h=16, H=2, D=8, F=24, r=3)
+    X, G = _case(11, S=16, h=16)
+    pos = np.arange(2, 18)
+    keep = np.arange(16) % 3 != 0
+    out, ctx = oly.layer_fwd(X, pos, W, rnd=False, mlp_keep=keep)
+    dx, grads = oly.layer_bwd(ctx, G, W, 5)
+    rng = np.random.default_rng(66)
+    loss = lambda Xv: float((oly.layer_fwd(Xv, pos, W, rnd=False, mlp_keep=keep)[0] * G).sum())  # noqa: E731
+    eps = 1e-6
+    d = rng.standard_normal(X.shape)
+    num = (loss(X + eps * d) - loss(X - eps * d)) / (2 * eps)
+    assert abs(num - (dx * d).sum()) < 1e-6 * max(1.0, abs(num))
+    # and the mask matters: all kept gives a different gradient
+    _, c2 = oly.layer_fwd(X, pos, W, rnd=False)
+    dx2, _ = oly.layer_bwd(c2, G, W, 5)
+    assert np.abs(dx2 - dx).max() > 1e-3
