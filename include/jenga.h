@@ -108,11 +108,14 @@ JENGA_API size_t jenga_profile_report(char* buf, size_t len);
  *   blk      : tokens per block, S % blk == 0; nb = S / blk.
  *   causal   : 1 = query i attends keys j <= i (the scoring the path uses); 0 = all j.
  *   scores   : [B, nb] fp32 out.  Deterministic (fixed reduction order).
- *   ws       : workspace of jenga_score_workspace_bytes(...) bytes (row LSE [B,H,S]
- *              and per-head partial scores [B,H,nb]).
- * fp32 inputs use exact fp32 SIMT dot products (D <= 128); bf16 inputs use the
- * tensor-core kernels and need D == 128.  Errors: EINVAL (shapes), EWORKSPACE,
- * EUNSUPPORTED (D / dtype / mode combination not built). */
+ *   ws       : workspace of jenga_score_workspace_bytes(...) bytes.  After a softmax-mass
+ *              call its first B*H*S floats (from the first 256-byte aligned address of ws)
+ *              hold the negated row log-sum-exp -log2 sum_{j<=i} 2^(log2(e) q_i.k_j/sqrt(D))
+ *              of every (sequence, head, query), a diagnostic; the rest is scratch.
+ * fp32 inputs use exact fp32 SIMT dot products (D <= 128).  bf16 inputs use the single-pass
+ * tensor-core kernel and need D == 128 and blk a multiple of 32 (S itself need not be a
+ * multiple of the 128-token tile).  Errors: EINVAL (shapes), EWORKSPACE, EUNSUPPORTED
+ * (D / dtype / blk / mode combination not built). */
 JENGA_API size_t jenga_score_workspace_bytes(int B, int S, int H, int D, int blk);
 JENGA_API jenga_status jenga_score_blocks(const void* q, int64_t ldq, const void* k, int64_t ldk, int B, int S, int H,
                                 int D, int blk, int causal, jenga_dtype dt, jenga_score_mode mode,
@@ -124,13 +127,19 @@ JENGA_API jenga_status jenga_score_blocks(const void* q, int64_t ldq, const void
  * allow no allocation outside their own pool, or latency-critical code that cannot
  * afford cudaMalloc / cudaFree and the device synchronisation they may cause.  The
  * scratch is one fixed 16 MiB array inside the library image (every GPU that loads the
- * library holds it until the process exits), so B * H * S must stay below about 2M
- * (two fp32 values per (batch, head, token)); larger sizes return JENGA_EWORKSPACE.
+ * library holds it until the process exits).  Limit: jenga_score_workspace_bytes(B, S, H,
+ * D, blk) must not exceed jenga_score_blocks_noalloc_max_bytes(); larger sizes return
+ * JENGA_EWORKSPACE before anything is launched.  That covers every mode: the fp32 path
+ * needs 2*B*H*S*4 bytes, the bf16 single pass about 4*B*H*S*(1 + S/(64*128)) bytes plus
+ * 512*(S/64 + 8) bytes per work slot (at most 160 slots), the block-max mode
+ * 4*B*(S/g)^2 bytes (g = blk for blk 32 or 64, else 128); e.g. 32 heads of 128 with blocks
+ * of 64 fit up to S = 8192.
  * Arguments and results are those of jenga_score_blocks.  The first call on a device
- * looks up the array's device address (cudaGetSymbolAddress, that device current):
- * make that first call before any stream capture.  All calls share the array and each
- * call overwrites what it reads, so nothing needs clearing, but calls whose kernels
- * overlap on the GPU (for example on two streams) race on it.  Allocates nothing.
+ * looks up the array's device address (cudaGetSymbolAddress, that device current), and so
+ * does the first call in a new CUDA context of that device (after a device reset): make
+ * such a first call before any stream capture.  All calls share the array and each call
+ * overwrites what it reads, so nothing needs clearing, but calls whose kernels overlap on
+ * the GPU (for example on two streams) race on it.  Allocates nothing.
  * jenga_score_blocks_noalloc_max_bytes() returns the array size in bytes. */
 JENGA_API size_t jenga_score_blocks_noalloc_max_bytes(void);
 JENGA_API jenga_status jenga_score_blocks_noalloc(const void* q, int64_t ldq, const void* k, int64_t ldk, int B,
@@ -250,6 +259,31 @@ JENGA_API jenga_status jenga_sparse_layer_fwd_qk(const jenga_layer_weights* w, c
                                        void* x, int B, int S, int blk, const int32_t* idx, const int32_t* n_kept,
                                        int n_kept_max, const void* qk_all, int64_t ld_qk, void* saved,
                                        size_t saved_bytes, void* ws, size_t ws_bytes, jenga_stream_t stream);
+
+/* jenga_sparse_layer_fwd_mlp -- jenga_sparse_layer_fwd (or _fwd_qk when qk_all is not null)
+ * with MLP-block token elimination (Jenga summary §4.2.4, extend to the MLP block): after the
+ * gate / up projection of all retained rows, each retained block's MLP informativeness is the
+ * L1 mass of its activation SiLU(gate) * up (jenga_mlp_block_scores), jenga_select(mlp_mode,
+ * mlp_param) picks the blocks the MLP sub-block keeps among the n_kept_max retained positions
+ * (TOPK_FRAC: a fraction of n_kept_max; TOPK: a count; ABS_GE: a threshold), and the down
+ * projection and its in-place residual add run only on those blocks; on the other retained
+ * blocks the layer output is h, the attention sub-block's output.  The keep mask is stored in
+ * `saved`, and jenga_sparse_layer_bwd then runs the MLP backward (gate / up recompute, SwiGLU
+ * backward, the dhn GEMM) only on the kept blocks and passes the upstream gradient straight
+ * through the MLP branch of the others.
+ *   mlp_scores : [n_kept_max] fp32 out (nullable): the criterion per retained position
+ *             (-inf at and past the device count n_kept);
+ *   mlp_pos : [n_kept_max] int32 out (nullable): kept positions in the retained list,
+ *             ascending, then -1 (compose with idx by jenga_compose_block_indices for
+ *             sequence block numbers);  n_mlp : [1] int32 out (nullable): their count.
+ * n_kept_max <= 8192.  Other arguments, workspace and errors as jenga_sparse_layer_fwd. */
+JENGA_API jenga_status jenga_sparse_layer_fwd_mlp(const jenga_layer_weights* w, const jenga_lora* lora,
+                                                  const void* packed, void* x, int B, int S, int blk,
+                                                  const int32_t* idx, const int32_t* n_kept, int n_kept_max,
+                                                  const void* qk_all, int64_t ld_qk, jenga_select_mode mlp_mode,
+                                                  float mlp_param, float* mlp_scores, int32_t* mlp_pos,
+                                                  int32_t* n_mlp, void* saved, size_t saved_bytes, void* ws,
+                                                  size_t ws_bytes, jenga_stream_t stream);
 
 /* jenga_sparse_layer_bwd -- a8 + a9: backward of jenga_sparse_layer_fwd for an upstream
  * gradient G held in dx ([B, S, hidden] bf16).  On return dx holds dL/dx: eliminated

@@ -110,3 +110,19 @@ def block_scores_paper_blockmax(q, k, blk, causal=True):
             if v.any():
                 out[n] += agg[:, cols][v].max()
     return out
+
+
+def row_lse(qh, kh, rows, causal=True):
+    """Natural log-sum-exp of the scaled logits of the given query rows of ONE head:
+    lse_i = log sum_{j <= i} exp(q_i . k_j / sqrt(D)) (all j if not causal), with the
+    textbook max shift.  qh, kh: [S, D]; rows: query indices.  Returns [len(rows)]."""
+    qh = _as_f64(qh)
+    kh = _as_f64(kh)
+    S, D = qh.shape
+    out = np.zeros(len(rows))
+    for n, i in enumerate(rows):
+        kend = int(i) + 1 if causal else S
+        s = (kh[:kend] @ qh[int(i)]) / np.sqrt(D)
+        m = s.max()
+        out[n] = m + np.log(np.exp(s - m).sum())
+    return out

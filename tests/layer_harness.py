@@ -76,14 +76,103 @@ def run_layer_gpu(case, layer_i=0, keep=0.5, seg=4096, mode="topk_frac", handle=
                 grads={k: v.cpu().numpy().astype(np.float64) for k, v in grads.items()}, kmax=kmax)
 
 
-def oracle_layer(case, gpu, layer_i=0, seg=None):
-    """Oracle forward/backward on the GPU's kept-block list and the same inputs."""
+def oracle_layer(case, gpu, layer_i=0, seg=None, pmap=map, X=None, G=None):
+    """Oracle forward/backward on the GPU's kept-block list and the same inputs (the case's
+    X and G unless given as float64 arrays, e.g. a chained layer's GPU input)."""
     W = oly.Weights.from_bits(case.layers[layer_i], case.shape)
-    X = from_bits(case.x)
-    G = from_bits(case.g)
-    Xo, ctx = oly.sparse_layer_fwd(X, gpu["idx"], gpu["n_kept"], case.blk, W, rnd=True)
-    dX, grads = oly.sparse_layer_bwd(ctx, G, W, seg)
+    X = from_bits(case.x) if X is None else X
+    G = from_bits(case.g) if G is None else G
+    Xo, ctx = oly.sparse_layer_fwd(X, gpu["idx"], gpu["n_kept"], case.blk, W, rnd=True, pmap=pmap)
+    dX, grads = oly.sparse_layer_bwd(ctx, G, W, seg, pmap=pmap)
+    del ctx
     return Xo, dX, grads, X, G
+
+
+TOL = 3e-2
+
+
+def retained_mask(S, blk, idx, n_kept):
+    rows = np.zeros(S, bool)
+    for b in np.asarray(idx)[: int(n_kept)]:
+        rows[b * blk:(b + 1) * blk] = True
+    return rows
+
+
+def check_layer_against_oracle(S, blk, idx, n_kept, out, dx, grads_gpu, Xo, dX, grads, X, G):
+    """The layer bars (bf16 outputs and gradients against the oracle on the same inputs
+    and the GPU's kept blocks): max |gpu - oracle| / rms(oracle) <= 3e-2 on the output and
+    the input gradient, one bf16 ulp of the stored value forgiven; the same on the
+    sub-block contributions (out - x <= 3e-2, dX - G <= 6e-2, which a real fault moves by
+    O(1)); LoRA gradients <= 3e-2; eliminated rows exactly x and exactly G.  Returns the
+    errors."""
+    rows = retained_mask(S, blk, idx, n_kept)
+    assert np.array_equal(out[~rows], X[~rows]), "eliminated rows must pass through unchanged"
+    assert np.array_equal(dx[~rows], G[~rows]), "eliminated rows: identity gradient"
+    e = {}
+    if rows.any():
+        e["out"] = rel_max_ulp(out[rows], Xo[rows])
+        e["dx"] = rel_max_ulp(dx[rows], dX[rows])
+        e["out-x"] = rel_delta_ulp(out[rows], Xo[rows], X[rows])
+        e["dx-G"] = rel_delta_ulp(dx[rows], dX[rows], G[rows])
+    for k in grads:
+        if np.abs(grads[k]).max() == 0:
+            assert np.abs(grads_gpu[k]).max() == 0, k
+            e[k] = 0.0
+        else:
+            e[k] = rel_max(grads_gpu[k], grads[k])
+    print("layer errors:", {k: float("%.3g" % v) for k, v in e.items()})
+    for k, v in e.items():
+        assert v < (2 * TOL if k == "dx-G" else TOL), (k, v)
+    return e
+
+
+def oracle_qk_all(case, layer_i=0, X=None):
+    """The oracle's post-RoPE q and k of ALL S rows (positions 0..S-1): [S, H, D] each."""
+    W = oly.Weights.from_bits(case.layers[layer_i], case.shape)
+    X = from_bits(case.x) if X is None else X
+    pr = oly.project_qk(X, np.arange(X.shape[0]), W, rnd=True)
+    return pr["q"], pr["k"]
+
+
+def check_qk_all(qk_gpu, q_o, k_o):
+    """a1: the GPU's [S, 2 H D] q | k of all rows against the oracle's, at the bf16 bar."""
+    g = torch_to_f64(qk_gpu)
+    S = q_o.shape[0]
+    HD = q_o.shape[1] * q_o.shape[2]
+    eq = rel_max_ulp(g[:S, :HD], q_o.reshape(S, HD))
+    ek = rel_max_ulp(g[:S, HD:2 * HD], k_o.reshape(S, HD))
+    same = float(np.mean(g[:S, :2 * HD] == np.concatenate([q_o.reshape(S, HD), k_o.reshape(S, HD)], axis=1)))
+    print(f"a1 q|k of all rows: q err {eq:.3g}, k err {ek:.3g}, bit-equal fraction {same:.4f}")
+    assert eq < TOL and ek < TOL, (eq, ek)
+    return eq, ek
+
+
+def check_scores(gpu_scores, oracle_scores, rtol=2e-2):
+    """Block scores elementwise within rtol relative (bf16 bar 2e-2)."""
+    g = np.asarray(gpu_scores, np.float64).reshape(-1)
+    o = np.asarray(oracle_scores, np.float64).reshape(-1)
+    rel = np.abs(g - o) / np.abs(o)
+    print(f"scores: max rel err {rel.max():.3g} over {o.size} blocks (sum gpu {g.sum():.6g}, oracle {o.sum():.6g})")
+    assert np.all(rel <= rtol), float(rel.max())
+    return float(rel.max())
+
+
+def check_topk_selection(gpu_scores, gpu_idx, gpu_nk, k, oracle_scores=None):
+    """Bit-exact: the oracle's top-k on the GPU's scores gives the GPU's list.  Reported:
+    the top-k on the oracle's own scores differs only in blocks within 1e-3 relative of
+    the k-th largest oracle score (blocks that close to the threshold are not counted)."""
+    oi, on, _ = osel.select_topk(np.asarray(gpu_scores).reshape(-1), k)
+    assert on == int(gpu_nk) and np.array_equal(oi, np.asarray(gpu_idx).reshape(-1)), "selection not bit-exact"
+    if oracle_scores is None or k == 0:
+        return 0
+    o = np.asarray(oracle_scores, np.float64).reshape(-1)
+    oi2, on2, _ = osel.select_topk(o, k)
+    a = set(oi[:on].tolist())
+    b = set(oi2[:on2].tolist())
+    thr = np.sort(o)[::-1][k - 1]
+    far = [n for n in a ^ b if abs(o[n] - thr) > 1e-3 * abs(thr)]
+    print(f"selection on oracle scores: {len(a ^ b)} blocks differ, {len(far)} of them beyond 1e-3 of the threshold")
+    return len(far)
 
 
 def oracle_scores_from_qk(qk_np, heads, head_dim, blk):

@@ -1,0 +1,224 @@
+"""GPU parity at the stated workload configurations, at full size, against the CPU oracle.
+
+Each test runs the CUDA path through the Python binding of the C ABI on the seeded inputs
+of one workload and checks, against the oracle on the same inputs:
+* a1: the q | k of ALL S rows (post-RoPE, bf16) at the 3e-2 bar (scaled by RMS, one bf16
+  ulp forgiven);
+* block scores (bf16 path) elementwise within 2e-2 relative of the oracle's scores
+  computed from the ORACLE's q and k;
+* selection bit-exact: the oracle's top-k on the GPU's scores is the GPU's kept list
+  (and the top-k on the oracle's own scores is reported, blocks within 1e-3 of the
+  threshold not counted);
+* the retained-token layer forward and backward on the GPU's kept blocks and the GPU's
+  layer input: output, input gradient and LoRA gradients at the 3e-2 bar, eliminated rows
+  exactly unchanged / exactly the upstream gradient.
+
+Workloads (seeded synthetic inputs; Jenga summary §4.2-§4.4, Jenga notes §4.2-§4.4):
+* llama7b_s16k: one Llama-2-7B-shaped layer at S = 16384, block 64, 5 % salient rows x3 in
+  8 spans, keep 25 / 50 / 75 % of the blocks and a keep-all dense run;
+* llama7b_x4_s32k: four stacked 7B-shaped layers at S = 32768, block 128, keep
+  80 / 60 / 50 / 40 %, 4 % salient rows x3 redrawn per layer, 4096-token backward
+  segments (up to 26 240 retained rows, 7 segments); every layer is checked on its GPU
+  input, and the oracle's own chained forward is compared with the GPU's final output;
+* llama13b_pred_s32k: one 13B-shaped layer (hidden 5120, 40 heads, FFN 13824) at
+  S = 32768 scored by the block-score predictor MLP (5120 -> 128 -> 1), keep 50 %.
+
+The oracle's per-head attention and scoring run in a process pool (the same results as a
+sequential run); these tests take minutes of CPU time."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import predictor as opred
+from oracle import select as osel
+from oracle.bf16 import from_bits, round_bf16
+from tests.layer_harness import (check_layer_against_oracle, check_qk_all, check_scores, check_topk_selection,
+                                 layer_handle, oracle_layer, oracle_qk_all, bits_to_torch, rel_max, rel_max_ulp,
+                                 torch_to_f64)
+from tests.oracle_pool import oracle_pool
+from oracle import scores as osc
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def J():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import token_sparse_long_b200 as J
+    J._lib.load()
+    return J
+
+
+@pytest.fixture(scope="module")
+def pmap():
+    with oracle_pool() as pm:
+        yield pm
+
+
+def _scores_and_a1(J, case, L, X_t, X_f64, layer_i, pmap):
+    """GPU q | k of all rows and block scores; oracle q, k from the same layer input; checks
+    a1 and the scores; returns the GPU qk, the GPU scores and the oracle scores."""
+    sh = case.shape
+    HD = sh.heads * sh.head_dim
+    qk = J.jenga_layer_score_qk(L, X_t)
+    sc = J.jenga_score_blocks(qk[:, :HD], qk[:, HD:], sh.heads, sh.head_dim, case.blk)
+    torch.cuda.synchronize()
+    q_o, k_o = oracle_qk_all(case, layer_i, X_f64)
+    check_qk_all(qk, q_o, k_o)
+    o_sc = osc.block_scores_softmax_mass(q_o, k_o, case.blk, pmap=pmap)
+    del q_o, k_o
+    g_sc = sc.cpu().numpy().astype(np.float64)
+    check_scores(g_sc, o_sc)
+    assert abs(g_sc.sum() - sh.heads * case.S) < 2e-3 * sh.heads * case.S
+    return qk, g_sc, o_sc
+
+
+def _layer_gpu(J, L, X_t, G_t, idx, nk, blk, kmax, seg, qk=None):
+    """Sparse forward in place on X_t, then the backward in place on G_t; returns numpy."""
+    grads = J.new_lora_grads(L)
+    saved = J.jenga_sparse_layer_fwd(L, X_t, idx, nk, blk, kmax, qk=qk)
+    out = torch_to_f64(X_t)
+    J.jenga_sparse_layer_bwd(L, G_t, idx, nk, blk, kmax, saved, grads, segment_tokens=seg)
+    J.jenga_check_device_status()
+    torch.cuda.synchronize()
+    del saved
+    return out, torch_to_f64(G_t), {k: v.cpu().numpy().astype(np.float64) for k, v in grads.items()}
+
+
+# ------------------------------------------------------------------ llama7b_s16k
+@pytest.fixture(scope="module")
+def s16k(J, pmap):
+    case = synth.gen_workload("llama7b_s16k", seed=0, lora_b_std=0.02)
+    L = layer_handle(case.layers[0], case.shape)
+    X_t = bits_to_torch(case.x)
+    qk, g_sc, o_sc = _scores_and_a1(J, case, L, X_t, from_bits(case.x), 0, pmap)
+    return dict(case=case, L=L, qk=qk, g_sc=g_sc, o_sc=o_sc)
+
+
+@pytest.mark.parametrize("keep", [0.25, 0.5, 0.75, 1.0])
+def test_llama7b_s16k_keep_sweep(J, pmap, s16k, keep):
+    case, L = s16k["case"], s16k["L"]
+    nb = case.S // case.blk
+    X_t = bits_to_torch(case.x)
+    G_t = bits_to_torch(case.g)
+    k = osel.topk_count(keep, nb)
+    if keep < 1.0:
+        idx, nk, _ = J.jenga_select(torch.from_numpy(s16k["g_sc"].astype(np.float32)).cuda(), "topk_frac", keep)
+        check_topk_selection(s16k["g_sc"], idx.cpu().numpy(), int(nk.cpu()[0]), k, s16k["o_sc"])
+        qk = s16k["qk"]
+    else:  # the dense comparator: keep-all, no scoring
+        idx = torch.arange(nb, dtype=torch.int32, device="cuda")
+        nk = torch.tensor([nb], dtype=torch.int32, device="cuda")
+        qk = None
+    out, dx, grads = _layer_gpu(J, L, X_t, G_t, idx, nk, case.blk, k, case.segment_tokens, qk=qk)
+    gpu = dict(idx=idx.cpu().numpy(), n_kept=int(nk.cpu()[0]))
+    Xo, dX, og, X, G = oracle_layer(case, gpu, 0, case.segment_tokens, pmap=pmap)
+    check_layer_against_oracle(case.S, case.blk, gpu["idx"], gpu["n_kept"], out, dx, grads, Xo, dX, og, X, G)
+
+
+# ------------------------------------------------------------------ llama7b_x4_s32k
+def test_llama7b_x4_s32k_chain(J, pmap):
+    """Four stacked layers as the benchmark step runs them (salient rows of layer l >= 1
+    scaled x3 in place before its scoring, the same diagonal applied to dX after its
+    backward); each layer is checked against the oracle on the GPU's input of that layer,
+    its kept blocks and (backward) its upstream gradient."""
+    case = synth.gen_workload("llama7b_x4_s32k", seed=0, lora_b_std=0.02)
+    sh, S, blk, seg = case.shape, case.S, case.blk, case.segment_tokens
+    nb = S // blk
+    HD = sh.heads * sh.head_dim
+    Ls = [layer_handle(p, sh) for p in case.layers]
+    sal = [torch.from_numpy(s.astype(np.int32)).cuda() for s in case.salient]
+    X = bits_to_torch(case.x)
+    ins, outs, sels, saved, qks = [], [], [], [], []
+    for l, L in enumerate(Ls):
+        if l > 0 and len(case.salient[l]):
+            J.jenga_scale_rows(X, sal[l], case.salient_scale)
+        ins.append(X.clone())
+        qk = J.jenga_layer_score_qk(L, X)
+        sc = J.jenga_score_blocks(qk[:, :HD], qk[:, HD:], sh.heads, sh.head_dim, blk)
+        k = osel.topk_count(case.keep[l], nb)
+        idx, nk, _ = J.jenga_select(sc, "topk_frac", case.keep[l])
+        saved.append(J.jenga_sparse_layer_fwd(L, X, idx, nk, blk, k, qk=qk))
+        outs.append(X.clone())
+        sels.append((sc.cpu().numpy().astype(np.float64), idx, nk, k))
+        qks.append(qk if l == 0 else None)
+        del qk
+    dX = bits_to_torch(case.g)
+    gin, gout, grads = [None] * 4, [None] * 4, [None] * 4
+    for l in reversed(range(4)):
+        _, idx, nk, k = sels[l]
+        gin[l] = dX.clone()
+        g = J.new_lora_grads(Ls[l])
+        J.jenga_sparse_layer_bwd(Ls[l], dX, idx, nk, blk, k, saved[l], g, segment_tokens=seg)
+        gout[l] = dX.clone()
+        grads[l] = {kk: v.cpu().numpy().astype(np.float64) for kk, v in g.items()}
+        if l > 0 and len(case.salient[l]):
+            J.jenga_scale_rows(dX, sal[l], case.salient_scale)
+    J.jenga_check_device_status()
+    torch.cuda.synchronize()
+    del saved
+    for l in range(4):
+        g_sc, idx, nk, k = sels[l]
+        x_in = torch_to_f64(ins[l])
+        if l == 0:  # a1 and the scores on the first layer's input
+            q_o, k_o = oracle_qk_all(case, 0, x_in)
+            check_qk_all(qks[0], q_o, k_o)
+            o_sc = osc.block_scores_softmax_mass(q_o, k_o, blk, pmap=pmap)
+            del q_o, k_o
+            check_scores(g_sc, o_sc)
+        else:
+            o_sc = None
+        assert abs(g_sc.sum() - sh.heads * S) < 2e-3 * sh.heads * S
+        check_topk_selection(g_sc, idx.cpu().numpy(), int(nk.cpu()[0]), k, o_sc)
+        gpu = dict(idx=idx.cpu().numpy(), n_kept=int(nk.cpu()[0]))
+        assert gpu["n_kept"] == k == (205, 154, 128, 103)[l]
+        Xo, dXo, og, Xi, Gi = oracle_layer(case, gpu, l, seg, pmap=pmap, X=x_in, G=torch_to_f64(gin[l]))
+        print(f"layer {l}: {k} of {nb} blocks kept")
+        check_layer_against_oracle(S, blk, gpu["idx"], gpu["n_kept"], torch_to_f64(outs[l]), torch_to_f64(gout[l]),
+                                   grads[l], Xo, dXo, og, Xi, Gi)
+        del Xo, dXo, Xi, Gi
+    # the oracle's own chain (its outputs feed its next layer) against the GPU's output
+    from oracle import layer as oly
+    Xc = from_bits(case.x)
+    for l in range(4):
+        if l > 0 and len(case.salient[l]):
+            Xc[case.salient[l]] = round_bf16(Xc[case.salient[l]] * case.salient_scale)
+        W = oly.Weights.from_bits(case.layers[l], sh)
+        Xc, _ = oly.sparse_layer_fwd(Xc, sels[l][1].cpu().numpy(), sels[l][3], blk, W, rnd=True, pmap=pmap)
+    e_chain = rel_max_ulp(torch_to_f64(outs[3]), Xc)
+    print(f"four-layer chained forward (oracle on its own outputs, GPU kept blocks): {e_chain:.3g}")
+    assert e_chain < 3e-2
+
+
+# ------------------------------------------------------------------ llama13b_pred_s32k
+def test_llama13b_predictor_layer(J, pmap):
+    """13B-shaped layer scored by the block-score predictor MLP: the predicted scores
+    against the oracle's predictor (max error 1e-3 of the scores' rms), bit-exact top-50%
+    selection on them, then the layer forward / backward against the oracle."""
+    case = synth.gen_workload("llama13b_pred_s32k", seed=0, lora_b_std=0.02)
+    sh, S, blk = case.shape, case.S, case.blk
+    nb = S // blk
+    pr = case.predictor
+    w1 = bits_to_torch(pr["w1"])
+    b1 = torch.from_numpy(pr["b1"]).cuda()
+    w2 = bits_to_torch(pr["w2"]).reshape(-1)
+    b2 = torch.from_numpy(pr["b2"]).cuda()
+    X_t = bits_to_torch(case.x)
+    G_t = bits_to_torch(case.g)
+    p_sc = J.jenga_predict_blocks(X_t, blk, w1, b1, w2, b2)
+    g_sc = p_sc.cpu().numpy().astype(np.float64)
+    X = from_bits(case.x)
+    o_sc = opred.predict_blocks(X, blk, from_bits(pr["w1"]), pr["b1"], from_bits(pr["w2"]), pr["b2"])
+    err = rel_max(g_sc, o_sc)
+    print(f"predictor scores: max err {err:.3g} of the scores' rms")
+    assert err < 1e-3
+    k = osel.topk_count(0.5, nb)
+    idx, nk, _ = J.jenga_select(p_sc, "topk_frac", 0.5)
+    check_topk_selection(g_sc, idx.cpu().numpy(), int(nk.cpu()[0]), k)
+    L = layer_handle(case.layers[0], sh)
+    out, dx, grads = _layer_gpu(J, L, X_t, G_t, idx, nk, blk, k, case.segment_tokens)
+    gpu = dict(idx=idx.cpu().numpy(), n_kept=int(nk.cpu()[0]))
+    Xo, dX, og, X, G = oracle_layer(case, gpu, 0, case.segment_tokens, pmap=pmap)
+    check_layer_against_oracle(S, blk, gpu["idx"], gpu["n_kept"], out, dx, grads, Xo, dX, og, X, G)

@@ -89,6 +89,56 @@ def test_score_bf16_against_oracle(J, S, H, causal):
     assert abs(got.sum() - H * S) < 2e-3 * H * S
 
 
+@pytest.mark.parametrize("B,S,H,blk,causal", [(1, 4160, 2, 64, True), (1, 4160, 2, 64, False), (1, 1024, 3, 32, True),
+                                             (1, 1056, 2, 32, False), (1, 2048, 4, 128, True), (1, 96, 2, 32, True),
+                                             (3, 320, 2, 64, True), (2, 640, 1, 128, False)])
+def test_score_bf16_shapes_against_oracle(J, B, S, H, blk, causal):
+    """Single-pass scoring at ragged lengths (S % 128 = 64 or 32: a partial last query and
+    key tile), 32-key chunks (blk 32), blk 128, S below one tile, and several sequences (the
+    tile rows past a sequence's end belong to the next one and must be masked)."""
+    g = torch.Generator(device="cuda").manual_seed(S * 7 + H + blk)
+    q = (torch.randn(B, S, H * 128, device="cuda", generator=g) * 0.3).to(torch.bfloat16)
+    k = (torch.randn(B, S, H * 128, device="cuda", generator=g) * 0.3).to(torch.bfloat16)
+    sc = J.jenga_score_blocks(q, k, H, 128, blk, causal=causal)
+    J.jenga_check_device_status()
+    got = sc.cpu().numpy().astype(np.float64)
+    for b in range(B):
+        ref = osc.block_scores_softmax_mass(torch_to_f64(q[b]).reshape(S, H, 128), torch_to_f64(k[b]).reshape(S, H, 128),
+                                            blk, causal=causal)
+        assert np.all(np.abs(got[b] - ref) / np.abs(ref) < 2e-2), (b, np.abs(got[b] - ref).max())
+        assert abs(got[b].sum() - H * S) < 2e-3 * H * S
+
+
+def test_score_bf16_32_heads_s4096_and_row_lse(J):
+    """The layer workload's scoring shape (32 heads x 128, S 4096, blocks of 64) against the
+    oracle, and the row log-sum-exps the kernel leaves at the start of its workspace against
+    the oracle's for a sample of rows."""
+    S, H, blk = 4096, 32, 64
+    g = torch.Generator(device="cuda").manual_seed(4096)
+    q = (torch.randn(S, H * 128, device="cuda", generator=g) * 0.2).to(torch.bfloat16)
+    k = (torch.randn(S, H * 128, device="cuda", generator=g) * 0.2).to(torch.bfloat16)
+    lib = J._lib.load()
+    ws = torch.zeros(lib.jenga_score_workspace_bytes(1, S, H, 128, blk), dtype=torch.uint8, device="cuda")
+    sc = J.jenga_score_blocks(q, k, H, 128, blk, ws=ws)
+    J.jenga_check_device_status()
+    qf = torch_to_f64(q).reshape(S, H, 128)
+    kf = torch_to_f64(k).reshape(S, H, 128)
+    from tests.oracle_pool import oracle_pool
+    with oracle_pool() as pm:
+        ref = osc.block_scores_softmax_mass(qf, kf, blk, pmap=pm)
+    got = sc.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - ref) / np.abs(ref) < 2e-2), np.abs(got - ref).max()
+    off = (-ws.data_ptr()) % 256
+    neg_l2 = ws[off:off + H * S * 4].view(torch.float32).reshape(H, S).double().cpu().numpy()
+    rows = np.r_[0, 1, 127, 128, 129, 2047, 4095, np.random.default_rng(0).integers(0, S, 24)]
+    for h in (0, 17, 31):
+        want = osc.row_lse(qf[:, h], kf[:, h], rows) / np.log(2.0)  # log2 units
+        got_l = -neg_l2[h, rows]
+        err = np.abs(got_l - want)
+        assert np.all(err <= 2e-4 * (1 + np.abs(want))), (h, [(int(r), float(a), float(b)) for r, a, b in
+                                                             zip(rows[:8], got_l[:8], want[:8])], float(err.max()))
+
+
 def test_score_bf16_large_logit_jump(J):
     # one key far along the sequence whose logit exceeds every earlier one by > 60 (log2
     # units): rows that reach it must leave the pass-1 fast path and rescale exactly
@@ -154,6 +204,24 @@ def test_score_paper_blockmax(J):
     sc = J.jenga_score_blocks(q, k, H, D, blk, mode="paper_blockmax")
     ref = osc.block_scores_paper_blockmax(torch_to_f64(q).reshape(S, H, D), torch_to_f64(k).reshape(S, H, D), blk)
     assert np.allclose(sc.cpu().numpy(), ref, rtol=1e-4, atol=1e-5)
+
+
+@pytest.mark.parametrize("S,H,blk,causal", [(4096, 32, 64, True), (1024, 3, 32, True), (1024, 2, 128, False),
+                                             (2048, 2, 256, True), (4160, 2, 64, True), (640, 4, 128, True)])
+def test_score_paper_blockmax_bf16_tcgen05(J, S, H, blk, causal):
+    """Eq. (2) block-max scores on the tensor-core path (bf16, head_dim 128) against the
+    oracle's block_scores_paper_blockmax on the same bf16 values: blocks of 32, 64, 128
+    and 256 tokens (several 128-token sub-tiles per block), a ragged S, causal and not."""
+    g = torch.Generator(device="cuda").manual_seed(S + H + blk)
+    q = (torch.randn(S, H * 128, device="cuda", generator=g) * 0.5).to(torch.bfloat16)
+    k = (torch.randn(S, H * 128, device="cuda", generator=g) * 0.5).to(torch.bfloat16)
+    sc = J.jenga_score_blocks(q, k, H, 128, blk, causal=causal, mode="paper_blockmax")
+    J.jenga_check_device_status()
+    ref = osc.block_scores_paper_blockmax(torch_to_f64(q).reshape(S, H, 128), torch_to_f64(k).reshape(S, H, 128), blk,
+                                          causal=causal)
+    got = sc.cpu().numpy().astype(np.float64)
+    rel = np.abs(got - ref) / np.abs(ref)
+    assert np.all(rel < 2e-3), rel.max()
 
 
 # ------------------------------------------------------------------ selection

@@ -137,3 +137,18 @@ def test_golden_score_fp32_regression():
     np.testing.assert_allclose(sc, gold["scores"], rtol=1e-12)
     assert abs(sum(gold["scores"]) - 4 * 512) < 1e-9
     assert list(c.salient) == gold["salient_rows"]
+
+
+def test_row_lse_against_library_logsumexp_and_softmax_normalisation():
+    from scipy.special import logsumexp
+    S, D = 50, 16
+    q, k = _rand_qk(9, S, 1, D, 3.0)
+    rows = [0, 1, 7, 49]
+    got = osc.row_lse(q[:, 0], k[:, 0], rows)
+    for n, i in enumerate(rows):
+        s = (q[i, 0] @ k[: i + 1, 0].T) / np.sqrt(D)
+        assert abs(got[n] - logsumexp(s)) < 1e-12
+        assert abs(np.exp(s - got[n]).sum() - 1.0) < 1e-12
+    assert abs(osc.row_lse(q[:, 0], k[:, 0], [0])[0] - (q[0, 0] @ k[0, 0]) / np.sqrt(D)) < 1e-12
+    full = osc.row_lse(q[:, 0], k[:, 0], [3], causal=False)[0]
+    assert abs(full - logsumexp((k[:, 0] @ q[3, 0]) / np.sqrt(D))) < 1e-12

@@ -53,6 +53,11 @@ def test_noalloc_matches_workspace_entry_point_twice(lib):
     got, ref = _scores_both(lib, q, k, 3, 128, 64, _lib.BF16)
     assert np.all(np.abs(got - ref) <= 2e-2 * np.abs(ref))
     assert abs(got.sum() - 3 * 1024) < 2e-3 * 3 * 1024
+    # and against the CPU oracle on the same bf16 values (the scoring tests' 2e-2 bar)
+    from oracle import scores as osc
+    f64 = lambda t: t.float().cpu().numpy().astype(np.float64).reshape(1024, 3, 128)
+    want = osc.block_scores_softmax_mass(f64(q), f64(k), 64)
+    assert np.all(np.abs(got - want) <= 2e-2 * np.abs(want))
     # call 2: different data and shape (fp32, 4 heads x 64, S 512, blocks of 32); the
     # scratch still holds call 1's values and must not leak into this result
     q2 = torch.randn(512, 4 * 64, device="cuda", generator=g, dtype=torch.float32)
@@ -69,7 +74,8 @@ def test_noalloc_rejects_sizes_beyond_its_array(lib):
     assert cap == 16 << 20
     null = ctypes.c_void_p(0)
     p = ctypes.c_void_p(256)
-    # B*H*S = 32 * 131072 needs 32 MiB of scratch: refused on the host, nothing launched
+    # S = 131072 at 32 heads needs far more than 16 MiB of scratch: refused on the host,
+    # nothing launched
     st = lib.jenga_score_blocks_noalloc(p, 4096, p, 4096, 1, 131072, 32, 128, 128, 1, _lib.BF16, 0, p, null)
     assert st == _lib.EWORKSPACE
     assert "fixed" in _lib.last_error()

@@ -77,6 +77,10 @@ _SIGS = {
     "jenga_sparse_layer_fwd_qk": (c_int, [POINTER(LayerWeights), POINTER(Lora), c_void_p, c_void_p, c_int, c_int, c_int,
                                           c_void_p, c_void_p, c_int, c_void_p, c_int64, c_void_p, c_size_t, c_void_p,
                                           c_size_t, c_void_p]),
+    "jenga_sparse_layer_fwd_mlp": (c_int, [POINTER(LayerWeights), POINTER(Lora), c_void_p, c_void_p, c_int, c_int,
+                                           c_int, c_void_p, c_void_p, c_int, c_void_p, c_int64, c_int, c_float,
+                                           c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p, c_size_t,
+                                           c_void_p]),
     "jenga_layer_bwd_workspace_bytes": (c_size_t, [POINTER(LayerWeights), c_int, c_int, c_int, c_int]),
     "jenga_sparse_layer_bwd": (c_int, [POINTER(LayerWeights), POINTER(Lora), c_void_p, c_void_p, c_int, c_int, c_int,
                                        c_void_p, c_void_p, c_int, c_void_p, c_size_t, POINTER(LoraGrads), c_int,

@@ -236,6 +236,38 @@ def jenga_sparse_layer_fwd(layer: LayerHandle, x, idx, n_kept, blk, n_kept_max, 
     return saved
 
 
+def jenga_sparse_layer_fwd_mlp(layer: LayerHandle, x, idx, n_kept, blk, n_kept_max, mlp_mode, mlp_param, saved=None,
+                               ws=None, stream=None, qk=None, mlp_pos=None, n_mlp=None, mlp_scores=None):
+    """jenga_sparse_layer_fwd with MLP-block elimination: the MLP sub-block keeps the retained
+    blocks that jenga_select(mlp_mode, mlp_param) picks on their SiLU(gate) * up mass.
+    Returns (saved, mlp_scores fp32 [n_kept_max], mlp_pos int32 [n_kept_max], n_mlp int32 [1])."""
+    _need_cuda(x, idx, n_kept)
+    S = x.shape[-2]
+    if saved is None:
+        saved = _ws(layer.saved_bytes(blk, n_kept_max), x.device)
+    if ws is None:
+        ws = _ws(layer.fwd_ws_bytes(blk, n_kept_max), x.device)
+    if mlp_pos is None:
+        mlp_pos = torch.empty(max(int(n_kept_max), 1), dtype=torch.int32, device=x.device)
+    if n_mlp is None:
+        n_mlp = torch.empty(1, dtype=torch.int32, device=x.device)
+    if mlp_scores is None:
+        mlp_scores = torch.empty(max(int(n_kept_max), 1), dtype=torch.float32, device=x.device)
+    ld_qk = 0
+    if qk is not None:
+        _need_cuda(qk)
+        HD = layer.heads * layer.head_dim
+        if qk.dtype != torch.bfloat16 or qk.device != x.device or qk.dim() != 2 or qk.shape[0] < S \
+                or qk.shape[1] < 2 * HD or qk.stride(1) != 1:
+            raise ValueError("qk must be a bf16 [>= S, >= 2 H D] tensor on x's device, last dimension contiguous")
+        ld_qk = qk.stride(0)
+    check(load().jenga_sparse_layer_fwd_mlp(ctypes.byref(layer.w), ctypes.byref(layer.lora), _p(layer.packed), _p(x), 1,
+                                            S, blk, _p(idx), _p(n_kept), int(n_kept_max), _p(qk), ld_qk,
+                                            SELECT_MODES[mlp_mode], float(mlp_param), _p(mlp_scores), _p(mlp_pos),
+                                            _p(n_mlp), _p(saved), saved.numel(), _p(ws), ws.numel(), _stream(stream)))
+    return saved, mlp_scores, mlp_pos, n_mlp
+
+
 def new_lora_grads(layer: LayerHandle):
     dev = layer.t["aq"].device
     return {k: torch.zeros(layer.t[k[1:]].shape, dtype=torch.float32, device=dev) for k in ("daq", "dbq", "dav", "dbv")}

@@ -29,6 +29,12 @@
 // tile i overlaps the gradient products of tile i-1 and the score products of tile i+1.
 // Causal masking, keys / queries past the valid count, and the segment bounds are applied
 // in the epilogue.  Every wait is bounded; waits that guard collective TMEM loads are voted.
+// Operands are fp16 (3 more mantissa bits than bf16): fp16 copies of q, k, v, the segment's dO
+// scaled by a power of two s_dO (max per-head row norm <= 1), P scaled by 2^8 (P <= 1) and
+// dS scaled by s_dS = 2^floor(log2(2^14 / Vmax)) with Vmax the largest per-head row norm of v,
+// so |dS s_dS| <= |P (dP - Delta)| s_dS <= 2 |dO_i| |v| s_dS <= 2^15 can never overflow
+// (gscal[2] = s_dO, gscal[3] = s_dS, set on the device before the launch).  The fp32 results
+// are divided by the scales again before they leave the kernels.
 #pragma once
 
 #include "common.cuh"
@@ -85,6 +91,15 @@ __device__ __forceinline__ void st_row16_sw128(uint8_t* tile, int r, int quad, c
   }
 }
 
+// fp16 forms of the instruction descriptors (operand format fields 0 = fp16)
+__host__ __device__ constexpr uint32_t idesc_f16(uint32_t bf16_desc) { return bf16_desc & ~((7u << 7) | (7u << 10)); }
+
+// two floats -> packed fp16 pair (round to nearest even), a in the low half
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 __device__ __forceinline__ void st_row32_sw128(uint8_t* tile, int r, int half, const uint32_t* pk) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
@@ -102,7 +117,7 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
                             int64_t delta_ld, const __grid_constant__ CUtensorMap tmDK,
                             const __grid_constant__ CUtensorMap tmDV, int s0, int s1,
                             const int32_t* __restrict__ n_valid, int valid_mult, int n_cap, float scale_log2,
-                            float scale) {
+                            float scale, const float* __restrict__ gscal) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DKV_BAR_OFF);
@@ -185,7 +200,7 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
     // (Q, dO) from the ring, independent of the gradient products.  One accumulator each:
     // tile i + 1's product starts as soon as the epilogue has read tile i's.
     const bool s_chain = (warp == 1);
-    constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64);
+    constexpr uint32_t idesc_s = idesc_f16(umma_idesc_bf16(128, 64));
     const uint32_t ta = s_chain ? tK : tV;
     const uint32_t acc_s = s_chain ? tS : tP;
     const int b_s_off = s_chain ? 0 : 2 * ABT_BOX64;  // Q or dO
@@ -209,7 +224,7 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
     // gradient products: warp 3 dV += P^T dO, warp 4 dK += dS^T Q, each as soon as the
     // epilogue has written tile i's P^T / dS^T
     const bool p_chain = (warp == 3);
-    constexpr uint32_t idesc_g = umma_idesc_bf16_bmn(128, 128);
+    constexpr uint32_t idesc_g = idesc_f16(umma_idesc_bf16_bmn(128, 128));
     const uint32_t acc_g = p_chain ? tdV : tdK;
     const int gbuf_off = p_chain ? DKV_PT_OFF : DKV_DST_OFF;  // P^T or dS^T tiles
     const int b_g_off = p_chain ? 2 * ABT_BOX64 : 0;          // dO or Q
@@ -255,6 +270,8 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
     // the staging tiles become the P^T / dS^T buffers only after every copy is done
     asm volatile("bar.sync 1, %0;" ::"n"(32 * DKV_EPI_WARPS) : "memory");
     const uint64_t sl2x2 = f2pack(scale_log2, scale_log2);
+    const float s_dO = __ldg(gscal + 2), s_dS = __ldg(gscal + 3);
+    const uint64_t pscale2 = f2pack(256.f, 256.f), dscale2 = f2pack(s_dS, s_dS);
     for (int i = 0; ok && i < nq; ++i) {
       const int s = i & 1, rs = i % DKV_STAGES;
       const int qbase = (qa0 + i) * 64 + quad * 16;
@@ -290,14 +307,14 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
           const uint64_t d23 = fmul2(
               p23, fadd2(f2pack(__uint_as_float(dp[4 * c4 + 2]), __uint_as_float(dp[4 * c4 + 3])), f2pack(Dq.z, Dq.w)));
           float a, bb;
-          f2unpack(p01, a, bb);
-          pk[2 * c4] = pack_bf2(a, bb);
-          f2unpack(p23, a, bb);
-          pk[2 * c4 + 1] = pack_bf2(a, bb);
-          f2unpack(d01, a, bb);
-          dk[2 * c4] = pack_bf2(a, bb);
-          f2unpack(d23, a, bb);
-          dk[2 * c4 + 1] = pack_bf2(a, bb);
+          f2unpack(fmul2(p01, pscale2), a, bb);
+          pk[2 * c4] = pack_h2(a, bb);
+          f2unpack(fmul2(p23, pscale2), a, bb);
+          pk[2 * c4 + 1] = pack_h2(a, bb);
+          f2unpack(fmul2(d01, dscale2), a, bb);
+          dk[2 * c4] = pack_h2(a, bb);
+          f2unpack(fmul2(d23, dscale2), a, bb);
+          dk[2 * c4 + 1] = pack_h2(a, bb);
         }
       } else {  // causal diagonal or the segment's ragged end
 #pragma unroll
@@ -314,10 +331,10 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
             p[e] = pe;
             d[e] = valid ? pe * (__uint_as_float(dp[c]) + Ds[e]) : 0.f;  // L, Delta past n are unset
           }
-          pk[2 * c4] = pack_bf2(p[0], p[1]);
-          pk[2 * c4 + 1] = pack_bf2(p[2], p[3]);
-          dk[2 * c4] = pack_bf2(d[0], d[1]);
-          dk[2 * c4 + 1] = pack_bf2(d[2], d[3]);
+          pk[2 * c4] = pack_h2(p[0] * 256.f, p[1] * 256.f);
+          pk[2 * c4 + 1] = pack_h2(p[2] * 256.f, p[3] * 256.f);
+          dk[2 * c4] = pack_h2(d[0] * s_dS, d[1] * s_dS);
+          dk[2 * c4 + 1] = pack_h2(d[2] * s_dS, d[3] * s_dS);
         }
       }
       // buffer s was last read by the gradient products of tile i-2
@@ -348,7 +365,7 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
         uint32_t a[32];
         tmem_ld32_nowait((t ? tdK : tdV) + lo + c0, a);
         tmem_wait_ld();
-        const float f = t ? scale : 1.f;
+        const float f = t ? scale / (s_dS * s_dO) : 1.f / (256.f * s_dO);
         uint8_t* dst = t ? bk : bv;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
@@ -382,7 +399,7 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
                           const float* __restrict__ lse, int64_t lse_ld, const float* __restrict__ delta,
                           int64_t delta_ld, const __grid_constant__ CUtensorMap tmDQ, int s0,
                           const int32_t* __restrict__ n_valid, int valid_mult, int n_cap, float scale_log2,
-                          float scale) {
+                          float scale, const float* __restrict__ gscal) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DQ_BAR_OFF);
@@ -458,7 +475,7 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     // A (Q, dO) from tensor memory, B (K, V) from the ring
     const bool s_chain = (warp <= 2);
     const int par = (warp - 1) & 1;
-    constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64);
+    constexpr uint32_t idesc_s = idesc_f16(umma_idesc_bf16(128, 64));
     const uint32_t ta = s_chain ? tQ : tDO;
     const uint32_t acc0 = tmem + (s_chain ? 0 : 128);
     const int b_off = s_chain ? 0 : 2 * ABT_BOX64;  // K or V
@@ -481,7 +498,7 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
   } else if (warp == 5 && lane == 0) {
     // dQ += dS K as soon as the epilogue has written tile j's dS (A: smem K-major, B: the
     // ring's K tile MN-major)
-    constexpr uint32_t idesc_g = umma_idesc_bf16_bmn(128, 128);
+    constexpr uint32_t idesc_g = idesc_f16(umma_idesc_bf16_bmn(128, 128));
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
       const int b = j & 1, rs = j % DQ_STAGES;
@@ -513,6 +530,8 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
     const float L = qvalid ? lse[(int64_t)h * lse_ld + q] : 0.f;  // -L, log2 units
     const float Dq = qvalid ? delta[(int64_t)h * delta_ld + q - s0] : 0.f;  // -Delta
     const uint64_t sl2x2 = f2pack(scale_log2, scale_log2), nL2 = f2pack(L, L), nD2 = f2pack(Dq, Dq);
+    const float s_dO = __ldg(gscal + 2), s_dS = __ldg(gscal + 3);
+    const uint64_t dscale2 = f2pack(s_dS, s_dS);
     bool ok = true;
     if (quad < 2) {
       // quad 0 copies Q, quad 1 dO from their staging tiles into tensor memory
@@ -551,8 +570,8 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
               exp2_mufu_x2(ffma2(f2pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, nL2));
           const uint64_t d2 = fmul2(p2, fadd2(f2pack(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), nD2));
           float a, bb;
-          f2unpack(d2, a, bb);
-          dk[c >> 1] = pack_bf2(a, bb);
+          f2unpack(fmul2(d2, dscale2), a, bb);
+          dk[c >> 1] = pack_h2(a, bb);
         }
       } else {
 #pragma unroll
@@ -564,7 +583,7 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
             const float pe = valid ? fast_exp2(fmaf(__uint_as_float(sv[c + e]), scale_log2, L)) : 0.f;
             d2[e] = valid ? pe * (__uint_as_float(dp[c + e]) + Dq) : 0.f;
           }
-          dk[c >> 1] = pack_bf2(d2[0], d2[1]);
+          dk[c >> 1] = pack_h2(d2[0] * s_dS, d2[1] * s_dS);
         }
       }
       if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait_at(&ds_free[s], ((j >> 1) - 1) & 1, 137, j))) {
@@ -587,11 +606,12 @@ __global__ void __launch_bounds__(ABT_THREADS, 1)
       uint32_t a[32];
       tmem_ld32_nowait(tdQ + lo + quad * 32, a);
       tmem_wait_ld();
+      const float f = scale / (s_dS * s_dO);
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         *reinterpret_cast<float4*>(box + r * 128 + ((c ^ (r & 7)) << 4)) =
-            make_float4(__uint_as_float(a[4 * c]) * scale, __uint_as_float(a[4 * c + 1]) * scale,
-                        __uint_as_float(a[4 * c + 2]) * scale, __uint_as_float(a[4 * c + 3]) * scale);
+            make_float4(__uint_as_float(a[4 * c]) * f, __uint_as_float(a[4 * c + 1]) * f,
+                        __uint_as_float(a[4 * c + 2]) * f, __uint_as_float(a[4 * c + 3]) * f);
       fence_proxy_async_smem();
     }
     const bool all_fin = bar_and(fin, 1, 32 * DQ_EPI_WARPS);

@@ -40,7 +40,8 @@ enum GemmEpi : int {
   EPI_SWIGLU = 3,       // 64-col groups (gate, up) -> out[m, n/2 + j] = bf16(silu(g) * u)
   EPI_QKV_ROPE = 4,     // q/k/v sections of width hd; RoPE(pos(m)) on q and k -> bf16
   EPI_SWIGLU_BWD = 5,   // acc = dA; aux = (g, u) interleaved fp32 -> out = (dg, du) interleaved fp16
-  EPI_LORA_T = 6,       // out fp32 [m, 0:N] = beta * acc ; aux bf16 [m, 0:64] = bf16(alpha * acc), zero padded
+  EPI_LORA_T = 6,       // out fp32 [m, 0:N] = beta * acc ; aux bf16 [m, 0:64] = (hi, lo) of alpha * acc:
+                        // cols 0..N-1 bf16(alpha acc), cols 32..32+N-1 bf16(alpha acc - hi), else 0
 };
 
 struct EpiParams {
@@ -63,7 +64,22 @@ struct EpiParams {
   int col0 = 0;                  // QKV: column of this GEMM's first output in the q | k | v layout
   const float2* rope_tab = nullptr;  // QKV: (cos, sin) of position(m) x frequency j, [M rows][64]
   bool tma_out = false;          // set by the launcher: the output tensor map is valid
+  // optional keep mask per block of mask_blk compact rows (indexed by (row_offset + m) /
+  // mask_blk): 128-row tiles with no kept row are skipped by every role (no loads, no MMAs,
+  // no stores), and the scatter-add epilogue leaves the rows of masked blocks untouched
+  const uint8_t* blk_mask = nullptr;
+  int mask_blk = 1;
 };
+
+// Does the 128-row tile at local row m0 hold a row of a kept block (always, without a mask)?
+__device__ __forceinline__ bool gemm_tile_live(const EpiParams& p, int m0, int valid) {
+  if (!p.blk_mask) return true;
+  const int r0 = p.row_offset + m0;
+  const int r1 = p.row_offset + min(m0 + 128, valid);
+  for (int b = r0 / p.mask_blk; b * p.mask_blk < r1; ++b)
+    if (__ldg(p.blk_mask + b)) return true;
+  return false;
+}
 
 __device__ __forceinline__ int epi_valid_rows(const EpiParams& p) {
   int v = p.m_host;
@@ -222,6 +238,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
     const int n0 = (tile % ntn) * BN, m0 = (tile / ntn) * GEMM_BM;
+    if (!gemm_tile_live(ep, m0, valid)) continue;
     for (int kb = 0; kb < nkb; ++kb, ++g) {
       const int s = g % STAGES;
       if (g >= STAGES && !mbar_wait(&empty[s], ((g / STAGES) - 1) & 1, SITE_GEMM_PRODUCER)) {
@@ -248,7 +265,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // idesc: kind::f16 instruction descriptor (bf16 or fp16 operands, fp32 accumulate)
     bool ok = true;
     int g = 0, it = 0;
-    for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
+    for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+      if (!gemm_tile_live(ep, (tile / ntn) * GEMM_BM, valid)) continue;
       const int buf = it & 1;
       // the epilogue must have read this accumulator's previous tile (two tiles ago)
       if (it >= 2 && !mbar_wait(&acc_empty[buf], ((it >> 1) - 1) & 1, SITE_GEMM_MMA)) break;
@@ -271,6 +289,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         umma_commit(&empty[s]);
       }
       if (ok) umma_commit(&acc_full[buf]);
+      ++it;  // live tiles only: the accumulator parity follows the tiles actually computed
     }
   } else if (warp >= 2) {
     // ---------------- epilogue
@@ -300,9 +319,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       ++nst;
     };
     int it = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-    const int buf = it & 1;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     const int n0 = (tile % ntn) * BN, m0 = (tile / ntn) * GEMM_BM;
+    if (!gemm_tile_live(ep, m0, valid)) continue;
+    const int buf = it & 1;
     const int m = m0 + r;
     // warp vote: the tcgen05.ld calls below are collective, so all lanes take one path
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (it >> 1) & 1, SITE_GEMM_EPILOGUE));
@@ -362,6 +382,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               d[q] = make_float4(v[4 * q] * ep.alpha, v[4 * q + 1] * ep.alpha, v[4 * q + 2] * ep.alpha,
                                  v[4 * q + 3] * ep.alpha);
           } else {  // scatter-add into the residual rows
+            if (ep.blk_mask && !__ldg(ep.blk_mask + (m + ep.row_offset) / ep.mask_blk)) continue;
             const int64_t row = map_row(ep, m + ep.row_offset);
             if (row < 0 || row >= ep.x_rows) {
               record_device_error(JENGA_EINTERNAL, SITE_INDEX_RANGE, (unsigned)row);
@@ -447,21 +468,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           store_f16x32(o + 64, v);
         }
       } else if (EPI == EPI_LORA_T) {
-        // N <= 32 (t_q, t_v): fp32 copy + scaled bf16 copy padded to 64 columns
+        // N <= 32 (t_q, t_v): fp32 copy + the scaled value as a bf16 hi + lo pair (columns
+        // 0..31 and 32..63 of the K-padded operand of the next product)
         tmem_ld32(tbase, v);
         if (row_ok) {
           float* o = reinterpret_cast<float*>(ep.out) + (int64_t)m * ep.ldo;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (i < N) o[i] = v[i] * ep.beta;
-          float w[32];
+          float w[32], lo[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) w[i] = i < N ? v[i] * ep.alpha : 0.f;
+          for (int i = 0; i < 32; ++i) {
+            w[i] = i < N ? v[i] * ep.alpha : 0.f;
+            lo[i] = w[i] - __bfloat162float(__float2bfloat16_rn(w[i]));
+          }
           bf16* a = reinterpret_cast<bf16*>(ep.aux) + (int64_t)m * ep.ld_aux;
           store_bf16x32(a, w);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) w[i] = 0.f;
-          store_bf16x32(a + 32, w);
+          store_bf16x32(a + 32, lo);
         }
       } else if (EPI == EPI_QKV_ROPE) {
         // tile = BN/128 heads; section = (n / hd): 0 q, 1 k, 2 v; RoPE on q and k with this
@@ -517,6 +540,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    ++it;
     }
     if (lane == 0 && nst > 0) bulk_wait_group_read<0>();  // staging outlives the stores' reads
   }

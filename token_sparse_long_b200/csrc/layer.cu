@@ -7,11 +7,11 @@ namespace jenga {
 
 jenga_status attn_forward(const bf16* q, const bf16* k, const bf16* v, int64_t ld, bf16* o, int64_t ldo, float* lse,
                           int64_t lse_ld, int H, const int32_t* n_valid, int valid_mult, int n_cap, cudaStream_t st);
-jenga_status attn_backward_segment(const bf16* q, const bf16* k, const bf16* v, int64_t ld, const bf16* o,
-                                   int64_t ldo, const float* lse, int64_t lse_ld, const bf16* dO, int64_t ld_do,
-                                   float* delta, int64_t delta_ld, float* dq, int64_t ld_dq, float* dk_acc,
-                                   float* dv_acc, int64_t ld_acc, int H, int s0, int s1, const int32_t* n_valid,
-                                   int valid_mult, int n_cap, cudaStream_t st);
+jenga_status attn_backward_segment(const void* q16, const void* k16, const void* v16, int64_t ld, const float* lse,
+                                   int64_t lse_ld, const void* dO16, int64_t ld_do, const float* delta,
+                                   int64_t delta_ld, float* dq, int64_t ld_dq, float* dk_acc, float* dv_acc,
+                                   int64_t ld_acc, int H, int s0, int s1, const int32_t* n_valid, int valid_mult,
+                                   int n_cap, const float* gscal, cudaStream_t st);
 
 constexpr int LORA_R = 16;
 constexpr int LORA_PAD = 64;  // padded K of the LoRA operand pairs
@@ -77,6 +77,7 @@ static size_t carve_packed(Carve& c, const Dims& d, Packed* p) {
 struct Saved {
   bf16 *xr, *qkv, *o, *hres;
   float *t, *lse, *rstd1, *rstd2;
+  uint8_t* mlp_mask;  // [n_kept_max]: 1 = the MLP sub-block runs on this retained block
 };
 
 static size_t carve_saved(Carve& c, const Dims& d, int nc, Saved* s) {
@@ -88,18 +89,25 @@ static size_t carve_saved(Carve& c, const Dims& d, int nc, Saved* s) {
   s->lse = c.take<float>((size_t)d.H * nc);
   s->rstd1 = c.take<float>(nc);
   s->rstd2 = c.take<float>(nc);
+  s->mlp_mask = c.take<uint8_t>(nc > 0 ? (size_t)nc : 1);  // >= n_kept_max entries (one per retained block)
   return c.used();
 }
 
 struct FwdWs {
   bf16 *xn, *tb, *a;
   float2* rope;  // [nc][64] (cos, sin) of the retained rows' positions
+  float* mlp_scores;  // MLP-block criterion per retained block
+  int32_t *mlp_pos, *n_mlp;
 };
 static size_t carve_fwd_ws(Carve& c, const Dims& d, int nc, FwdWs* w) {
   w->xn = c.take<bf16>((size_t)nc * d.h);
   w->tb = c.take<bf16>((size_t)nc * LORA_PAD);
   w->a = c.take<bf16>((size_t)nc * d.F);
   w->rope = c.take<float2>((size_t)nc * 64);
+  const size_t nbk = nc > 0 ? (size_t)nc : 1;  // >= n_kept_max
+  w->mlp_scores = c.take<float>(nbk);
+  w->mlp_pos = c.take<int32_t>(nbk);
+  w->n_mlp = c.take<int32_t>(1);
   return c.used();
 }
 
@@ -108,10 +116,16 @@ struct BwdWs {
   bf16 *xn, *g, *dgu, *dhb, *dhlo, *dO, *dqkv, *dqkvlo, *dtb;
   float *gu, *dhn, *dh, *delta, *dq, *dt, *part;
   float2* rope;  // [T][64] (cos, sin) of the segment rows' positions
+  __half* qkv16;   // [nc, 3 HD] fp16 copy of the saved q | k | v (attention backward operands)
+  float* dOf;      // [T, HD] fp32 dO of the segment (scaled to fp16 into dO)
+  float* gscal;    // [4] norms and scales of the fp16 attention backward
 };
 static size_t carve_bwd_ws(Carve& c, const Dims& d, int nc, int T, BwdWs* w) {
   w->dk_acc = c.take<float>((size_t)nc * d.HD);
   w->dv_acc = c.take<float>((size_t)nc * d.HD);
+  w->qkv16 = c.take<__half>((size_t)nc * 3 * d.HD);
+  w->dOf = c.take<float>((size_t)T * d.HD);
+  w->gscal = c.take<float>(4);
   w->xn = c.take<bf16>((size_t)T * d.h);
   w->gu = c.take<float>((size_t)T * 2 * d.F);
   w->g = c.take<bf16>((size_t)T * d.h);
@@ -234,9 +248,15 @@ extern "C" jenga_status jenga_layer_pack(const jenga_layer_weights* w, const jen
   JENGA_TRY(copy2d(wk, h, p.wqkv + (size_t)HD * h, h, HD, h, st));
   JENGA_TRY(copy2d(wv, h, p.wqkv + (size_t)2 * HD * h, h, HD, h, st));
   // LoRA up-projection as a K=64 operand: rows of q -> cols 0..15 = Bq, rows of v -> cols 16..31 = Bv
+  // The A operand of that phase is [s t (bf16), s t - bf16(s t) (bf16)] (EPI_LORA_T), so the
+  // B columns repeat: q rows cols 0..15 and 32..47 = Bq, v rows cols 16..31 and 48..63 = Bv;
+  // the LoRA term then carries the rounding residual of s t (about 16 mantissa bits).
   JENGA_TRY(zero(p.lorab, (int64_t)3 * HD * LORA_PAD, st));
-  JENGA_TRY(copy2d((const bf16*)lora->bq, LORA_R, p.lorab, LORA_PAD, HD, LORA_R, st));
-  JENGA_TRY(copy2d((const bf16*)lora->bv, LORA_R, p.lorab + (size_t)2 * HD * LORA_PAD + LORA_R, LORA_PAD, HD, LORA_R, st));
+  for (int half = 0; half < 2; ++half) {
+    JENGA_TRY(copy2d((const bf16*)lora->bq, LORA_R, p.lorab + half * 2 * LORA_R, LORA_PAD, HD, LORA_R, st));
+    JENGA_TRY(copy2d((const bf16*)lora->bv, LORA_R, p.lorab + (size_t)2 * HD * LORA_PAD + LORA_R + half * 2 * LORA_R,
+                     LORA_PAD, HD, LORA_R, st));
+  }
   // LoRA down-projection [Aq; Av] (32 x h)
   JENGA_TRY(copy2d((const bf16*)lora->aq, h, p.aqv, h, LORA_R, h, st));
   JENGA_TRY(copy2d((const bf16*)lora->av, h, p.aqv + (size_t)LORA_R * h, h, LORA_R, h, st));
@@ -264,8 +284,9 @@ extern "C" jenga_status jenga_layer_pack(const jenga_layer_weights* w, const jen
   JENGA_TRY(transpose((const bf16*)lora->bq, LORA_R, p.bcat, 3 * HD, HD, LORA_R, st));
   JENGA_TRY(transpose((const bf16*)lora->bv, LORA_R, p.bcat + (size_t)LORA_R * 3 * HD + 2 * HD, 3 * HD, HD, LORA_R, st));
   // [Aq; Av]^T padded to 64 columns: [h, 64]
-  JENGA_TRY(zero(p.aqvT, (int64_t)h * LORA_PAD, st));
+  // (columns 32..63 repeat 0..31: the A operand carries dt's hi and lo halves, EPI_LORA_T)
   JENGA_TRY(transpose(p.aqv, h, p.aqvT, LORA_PAD, 2 * LORA_R, h, st));
+  JENGA_TRY(transpose(p.aqv, h, p.aqvT + 2 * LORA_R, LORA_PAD, 2 * LORA_R, h, st));
   {
   const int _ps = ::jenga::prof_begin("inv_freq", st);
   inv_freq_kernel<<<1, 64, 0, st>>>(p.inv_freq, d.D, log2((double)w->rope_theta));
@@ -350,10 +371,17 @@ extern "C" size_t jenga_layer_fwd_workspace_bytes(const jenga_layer_weights* w, 
   return carve_fwd_ws(c, d, n_kept_max * blk, &f);
 }
 
+// mlp_mode < 0: the MLP sub-block runs on every retained block.  Otherwise the MLP-block
+// criterion (jenga_mlp_block_scores over a = SiLU(g) * u of the retained blocks) is selected
+// with jenga_select(mlp_mode, mlp_param) over the n_kept_max retained positions, and the MLP
+// sub-block (down projection and its residual add here; its backward later) runs only on
+// the kept positions (Jenga summary §4.2.4).
 static jenga_status layer_fwd(const jenga_layer_weights* w, const jenga_lora* lora, const void* packed, void* x,
                               int B, int S, int blk, const int32_t* idx, const int32_t* n_kept, int n_kept_max,
                               void* saved, size_t saved_bytes, void* ws, size_t ws_bytes, const void* qk_all,
-                              int64_t ld_qk, jenga_stream_t stream) {
+                              int64_t ld_qk, jenga_stream_t stream, int mlp_mode = -1, float mlp_param = 0.f,
+                              int32_t* mlp_pos_out = nullptr, int32_t* n_mlp_out = nullptr,
+                              float* mlp_scores_out = nullptr) {
   Dims d;
   JENGA_TRY(check_weights(w, lora, &d));
   JENGA_CHECK_ARG(packed && x && idx && n_kept, "jenga_sparse_layer_fwd: null pointer");
@@ -459,12 +487,25 @@ static jenga_status layer_fwd(const jenga_layer_weights* w, const jenga_lora* lo
     e.ldo = F;
     JENGA_TRY((launch_gemm<256, EPI_SWIGLU>({f.xn, nc, h}, {p.wgu, 2 * F, h}, h, nullptr, nullptr, 0, nc, 2 * F, e, st, "gemm_gateup_swiglu")));
   }
-  // 8. down_proj with the in-place residual add into X
+  // 8. the blocks the MLP sub-block runs on: all retained blocks, or the ones the MLP-block
+  //    criterion keeps (a mask over retained positions, saved for the backward)
+  if (mlp_mode < 0) {
+    JENGA_CUDA_TRY(cudaMemsetAsync(s.mlp_mask, 1, (size_t)n_kept_max, st));
+  } else {
+    float* msc = mlp_scores_out ? mlp_scores_out : f.mlp_scores;
+    JENGA_TRY(jenga_mlp_block_scores(f.a, F, F, blk, n_kept, n_kept_max, msc, stream));
+    JENGA_TRY(jenga_select(msc, 1, n_kept_max, (jenga_select_mode)mlp_mode, mlp_param,
+                           mlp_pos_out ? mlp_pos_out : f.mlp_pos, n_mlp_out ? n_mlp_out : f.n_mlp, s.mlp_mask,
+                           nullptr, 0, stream));
+  }
+  // 9. down_proj with the in-place residual add into X (kept MLP blocks only)
   {
     EpiParams e = epi_base(idx, blk, n_kept, 0);
     e.x = X;
     e.ldx = h;
     e.x_rows = S;
+    e.blk_mask = s.mlp_mask;
+    e.mask_blk = blk;
     JENGA_TRY((launch_gemm<256, EPI_SCATTER_ADD>({f.a, nc, F}, {w->wd, h, F}, F, nullptr, nullptr, 0, nc, h, e, st, "gemm_down_scatter")));
   }
   return JENGA_OK;
@@ -489,6 +530,25 @@ extern "C" jenga_status jenga_sparse_layer_fwd_qk(const jenga_layer_weights* w, 
                   "jenga_sparse_layer_fwd_qk: qk_all must be [S, >= 2 H D] bf16, 16-byte aligned rows");
   return layer_fwd(w, lora, packed, x, B, S, blk, idx, n_kept, n_kept_max, saved, saved_bytes, ws, ws_bytes, qk_all,
                    ld_qk, stream);
+}
+
+extern "C" jenga_status jenga_sparse_layer_fwd_mlp(const jenga_layer_weights* w, const jenga_lora* lora,
+                                                   const void* packed, void* x, int B, int S, int blk,
+                                                   const int32_t* idx, const int32_t* n_kept, int n_kept_max,
+                                                   const void* qk_all, int64_t ld_qk, jenga_select_mode mlp_mode,
+                                                   float mlp_param, float* mlp_scores, int32_t* mlp_pos,
+                                                   int32_t* n_mlp, void* saved, size_t saved_bytes, void* ws,
+                                                   size_t ws_bytes, jenga_stream_t stream) {
+  Dims d;
+  JENGA_TRY(check_weights(w, lora, &d));
+  JENGA_CHECK_ARG(mlp_mode == JENGA_SELECT_TOPK_FRAC || mlp_mode == JENGA_SELECT_TOPK || mlp_mode == JENGA_SELECT_ABS_GE,
+                  "jenga_sparse_layer_fwd_mlp: MLP selection mode must be TOPK_FRAC, TOPK or ABS_GE");
+  JENGA_CHECK_ARG(n_kept_max <= 8192, "jenga_sparse_layer_fwd_mlp: n_kept_max <= 8192");
+  if (qk_all)
+    JENGA_CHECK_ARG(ld_qk >= 2 * (int64_t)d.HD && ld_qk % 8 == 0 && ((uintptr_t)qk_all & 15) == 0,
+                    "jenga_sparse_layer_fwd_mlp: qk_all must be [S, >= 2 H D] bf16, 16-byte aligned rows");
+  return layer_fwd(w, lora, packed, x, B, S, blk, idx, n_kept, n_kept_max, saved, saved_bytes, ws, ws_bytes, qk_all,
+                   ld_qk, stream, (int)mlp_mode, mlp_param, mlp_pos, n_mlp, mlp_scores);
 }
 
 // ==================================================================== backward
@@ -540,6 +600,15 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
 
   JENGA_CUDA_TRY(cudaMemsetAsync(b.dk_acc, 0, (size_t)nc * HD * sizeof(float), st));
   JENGA_CUDA_TRY(cudaMemsetAsync(b.dv_acc, 0, (size_t)nc * HD * sizeof(float), st));
+  // fp16 operands of the attention backward: q | k | v copies and the largest per-head v norm
+  JENGA_CUDA_TRY(cudaMemsetAsync(b.gscal, 0, 4 * sizeof(float), st));
+  {
+    const int _ps = ::jenga::prof_begin("qkv_to_f16", st);
+    qkv_to_f16_kernel<<<grid_cap((int64_t)nc * (3 * HD / 8), 256), 256, 0, st>>>(
+        s.qkv, 3 * HD, b.qkv16, 3 * HD, nc, 3 * HD, 2 * HD, reinterpret_cast<unsigned int*>(b.gscal));
+    ::jenga::prof_end(_ps, st);
+  }
+  JENGA_LAUNCH_CHECK();
   const int nseg = (nc + segment_tokens - 1) / segment_tokens;
   for (int sg = nseg - 1; sg >= 0; --sg) {
     const int s0 = sg * segment_tokens;
@@ -548,10 +617,13 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
     // --- MLP block (recomputed): hn, (g, u)
     JENGA_TRY(rmsnorm(s.hres + (size_t)s0 * h, h, nullptr, 1, s0, n_kept, blk, T, h, w->rms_eps,
                       (const bf16*)w->mlp_norm, nullptr, b.xn, nullptr, st));
+    // the MLP GEMMs skip the 128-row tiles whose blocks the MLP sub-block did not run on
     {
       EpiParams e = epi_base(idx, blk, n_kept, s0);
       e.out = b.gu;
       e.ldo = 2 * F;
+      e.blk_mask = s.mlp_mask;
+      e.mask_blk = blk;
       JENGA_TRY((launch_gemm<256, EPI_STORE_F32>({b.xn, T, h}, {p.wgu, 2 * F, h}, h, nullptr, nullptr, 0, T, 2 * F, e, st, "gemm_gateup_recompute")));
     }
     // upstream gradient rows of this segment
@@ -569,6 +641,8 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
       e.ldo = 2 * F;
       e.aux = b.gu;
       e.ld_aux = 2 * F;
+      e.blk_mask = s.mlp_mask;
+      e.mask_blk = blk;
       JENGA_TRY((launch_gemm<256, EPI_SWIGLU_BWD>({b.g, T, h}, {p.wdT, F, h}, h, nullptr, nullptr, 0, T, F, e, st, "gemm_da_swiglu_bwd")));
     }
     // dhn = [dg, du] [Wg; Wu]
@@ -576,6 +650,8 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
       EpiParams e = epi_base(idx, blk, n_kept, s0);
       e.out = b.dhn;
       e.ldo = h;
+      e.blk_mask = s.mlp_mask;
+      e.mask_blk = blk;
       JENGA_TRY((launch_gemm<256, EPI_STORE_F32>({b.dgu, T, 2 * F}, {p.wguT, h, 2 * F}, 2 * F, nullptr, nullptr, 0, T,
                                                  h, e, st, "gemm_dhn", nullptr, nullptr, 0, /*f16_inputs=*/true)));
     }
@@ -584,22 +660,39 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
     const int _ps = ::jenga::prof_begin("rmsnorm_bwd_rows", st);
     rmsnorm_bwd_rows_kernel<<<T, ROW_THREADS, 0, st>>>(b.dhn, h, s.hres + (size_t)s0 * h, h, s.rstd2 + s0,
                                                         (const bf16*)w->mlp_norm, nullptr, b.g, h, b.dh, b.dhb,
-                                                        b.dhlo, h, nullptr, 0, idx, blk, s0, n_kept, blk, h, S);
+                                                        b.dhlo, h, nullptr, 0, idx, blk, s0, n_kept, blk, h, S,
+                                                        s.mlp_mask, blk);
     ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();
-    // --- attention block: dO = dh Wo
+    // --- attention block: dO = dh Wo (fp32), then its fp16 form with a power-of-two scale and
+    //     the scaled Delta
     {
       EpiParams e = epi_base(idx, blk, n_kept, s0);
-      e.out = b.dO;
+      e.out = b.dOf;
       e.ldo = HD;
       // dh enters as a bf16 hi + lo pair (two K phases over the same weights)
       GemmOperand a2{b.dhlo, T, h}, b2{p.woT, HD, h};
-      JENGA_TRY((launch_gemm<256, EPI_STORE_BF16>({b.dhb, T, h}, {p.woT, HD, h}, h, &a2, &b2, h, T, HD, e, st,
-                                                  "gemm_do")));
+      JENGA_TRY((launch_gemm<256, EPI_STORE_F32>({b.dhb, T, h}, {p.woT, HD, h}, h, &a2, &b2, h, T, HD, e, st,
+                                                 "gemm_do")));
     }
-    JENGA_TRY(attn_backward_segment(s.qkv, s.qkv + HD, s.qkv + 2 * HD, 3 * HD, s.o, HD, s.lse, nc, b.dO, HD, b.delta, T,
-                                    b.dq, HD, b.dk_acc, b.dv_acc, HD, H, s0, s1, n_kept, blk, nc, st));
+    JENGA_CUDA_TRY(cudaMemsetAsync(b.gscal + 1, 0, sizeof(float), st));
+    {
+      const int _ps = ::jenga::prof_begin("do_norm_max", st);
+      do_norm_max_kernel<<<grid_cap((int64_t)T * H * 32, 256), 256, 0, st>>>(
+          b.dOf, HD, T, H, s0, n_kept, blk, reinterpret_cast<unsigned int*>(b.gscal));
+      ::jenga::prof_end(_ps, st);
+    }
+    JENGA_LAUNCH_CHECK();
+    {
+      const int _ps = ::jenga::prof_begin("do_to_f16_delta", st);
+      do_to_f16_delta_kernel<<<grid_cap((int64_t)T * H * 32, 256), 256, 0, st>>>(
+          b.dOf, HD, s.o, HD, reinterpret_cast<__half*>(b.dO), HD, b.delta, T, T, H, s0, n_kept, blk, b.gscal);
+      ::jenga::prof_end(_ps, st);
+    }
+    JENGA_LAUNCH_CHECK();
+    JENGA_TRY(attn_backward_segment(b.qkv16, b.qkv16 + HD, b.qkv16 + 2 * HD, 3 * HD, s.lse, nc, b.dO, HD, b.delta, T,
+                                    b.dq, HD, b.dk_acc, b.dv_acc, HD, H, s0, s1, n_kept, blk, nc, b.gscal, st));
     // keys of this segment are complete: RoPE^T and pack dQKV (bf16)
     {
     const int _ps = ::jenga::prof_begin("rope_table", st);

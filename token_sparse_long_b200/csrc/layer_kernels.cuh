@@ -114,12 +114,15 @@ __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_bwd_rows_kernel(
     const float* __restrict__ rstd, const bf16* __restrict__ gain, const float* __restrict__ base_f,
     const bf16* __restrict__ base_b, int64_t ldb, float* __restrict__ out_f, bf16* __restrict__ out_b,
     bf16* __restrict__ out_lo, int64_t ldo, bf16* __restrict__ dst, int64_t ldd, const int32_t* __restrict__ idx, int blk, int row_offset,
-    const int32_t* __restrict__ n_valid, int valid_mult, int h, int64_t dst_rows) {
+    const int32_t* __restrict__ n_valid, int valid_mult, int h, int64_t dst_rows,
+    const uint8_t* __restrict__ keep_mask = nullptr, int mask_blk = 1) {
   __shared__ float red[ROW_THREADS / 32];
   const int m = blockIdx.x;
   if (m >= valid_rows(n_valid, valid_mult, row_offset, gridDim.x)) return;
   const int nch = h >> 3;
-  const float r = rstd[m];
+  // a row of a masked block (keep_mask entry 0) has no sub-block gradient: out = base
+  const bool live = !keep_mask || __ldg(keep_mask + (row_offset + m) / mask_blk);
+  const float r = live ? rstd[m] : 0.f;
   float dyg[ROW_MAX_CHUNKS][8], xv[ROW_MAX_CHUNKS][8], bv[ROW_MAX_CHUNKS][8];
   float dot = 0.f;
 #pragma unroll
@@ -135,16 +138,24 @@ __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_bwd_rows_kernel(
       } else {
         unpack8(reinterpret_cast<const uint4*>(base_b + (int64_t)m * ldb)[c], bv[i]);
       }
-      const float4* dp = reinterpret_cast<const float4*>(dy + (int64_t)m * lddy) + 2 * c;
-      float4 a = dp[0], b = dp[1];
-      float gv[8];
-      unpack8(reinterpret_cast<const uint4*>(gain)[c], gv);
-      unpack8(reinterpret_cast<const uint4*>(x + (int64_t)m * ldx)[c], xv[i]);
-      const float d[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      if (live) {
+        const float4* dp = reinterpret_cast<const float4*>(dy + (int64_t)m * lddy) + 2 * c;
+        float4 a = dp[0], b = dp[1];
+        float gv[8];
+        unpack8(reinterpret_cast<const uint4*>(gain)[c], gv);
+        unpack8(reinterpret_cast<const uint4*>(x + (int64_t)m * ldx)[c], xv[i]);
+        const float d[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        dyg[i][e] = d[e] * gv[e];
-        dot = fmaf(dyg[i][e], xv[i][e], dot);
+        for (int e = 0; e < 8; ++e) {
+          dyg[i][e] = d[e] * gv[e];
+          dot = fmaf(dyg[i][e], xv[i][e], dot);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          dyg[i][e] = 0.f;
+          xv[i][e] = 0.f;
+        }
       }
     }
   }
@@ -429,6 +440,114 @@ __global__ void bf16_to_f16_inplace_kernel(uint16_t* __restrict__ x, int64_t n) 
 __global__ void zero_bf16_kernel(bf16* __restrict__ dst, int64_t n) {
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
     dst[e] = __float2bfloat16_rn(0.f);
+}
+
+// ---------------------------------------------------------------- fp16 operands of the
+// attention backward (attn_bwd_tc.cuh): fp16 copies of q | k | v, a power-of-two scale for
+// the segment's dO, and a dS scale that cannot overflow.
+// gscal (fp32 words): [0] max over rows and heads of |v_row,head|_2 (float bits, atomicMax),
+// [1] the same for the segment's dO, [2] s_dO, [3] s_dS.
+
+// out = fp16(in) for rows x cols (bf16 -> fp16, 8 values per thread and step); with
+// vnorm_col0 >= 0 the per-head row norms of columns [vnorm_col0, cols) (the v section) are
+// max-reduced into gscal[0].
+__global__ void qkv_to_f16_kernel(const bf16* __restrict__ in, int64_t ldi, __half* __restrict__ out, int64_t ldo,
+                                  int rows, int cols, int vnorm_col0, unsigned int* __restrict__ gmax) {
+  const int vpr = cols / 8;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < (int64_t)rows * vpr;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int r = (int)(e / vpr), c = (int)(e - (int64_t)r * vpr) * 8;
+    float f[8];
+    unpack8(*reinterpret_cast<const uint4*>(in + (int64_t)r * ldi + c), f);
+    uint4 o;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half2 h = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
+      ow[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(out + (int64_t)r * ldo + c) = o;
+  }
+  if (vnorm_col0 < 0) return;
+  // per (row, v head): one warp sums the squares of the head's 128 values
+  const int H = (cols - vnorm_col0) / 128;
+  const int lane = threadIdx.x & 31;
+  for (int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < (int64_t)rows * H;
+       w += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    const int r = (int)(w / H), hh = (int)(w - (int64_t)r * H);
+    float f[4];
+    const uint2 u = *reinterpret_cast<const uint2*>(in + (int64_t)r * ldi + vnorm_col0 + hh * 128 + lane * 4);
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+    const float2 a = __bfloat1622float2(p2[0]), b = __bfloat1622float2(p2[1]);
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+    float ss = f[0] * f[0] + f[1] * f[1] + f[2] * f[2] + f[3] * f[3];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) atomicMax(gmax, __float_as_uint(sqrtf(ss)));  // non-negative: bit order = value order
+  }
+}
+
+// gscal[1] = max over the segment's valid rows and heads of |dO_row,head|_2 (dO fp32 [T, ld]).
+__global__ void do_norm_max_kernel(const float* __restrict__ dO, int64_t ld, int T, int H, int s0,
+                                   const int32_t* __restrict__ n_valid, int valid_mult,
+                                   unsigned int* __restrict__ gscal_bits) {
+  const int nv = valid_rows(n_valid, valid_mult, s0, T);
+  const int lane = threadIdx.x & 31;
+  for (int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < (int64_t)nv * H;
+       w += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    const int r = (int)(w / H), hh = (int)(w - (int64_t)r * H);
+    const float4 v = *reinterpret_cast<const float4*>(dO + (int64_t)r * ld + hh * 128 + lane * 4);
+    float ss = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) atomicMax(gscal_bits + 1, __float_as_uint(sqrtf(ss)));
+  }
+}
+
+__device__ __forceinline__ float pow2_floor(float x) {  // largest power of two <= x (x > 0, finite)
+  return exp2f(floorf(log2f(x)));
+}
+
+// dO16 = fp16(dO s_dO) with s_dO the power of two that brings the largest per-head row norm
+// into (1/2, 1]; delta[h, r] = -sum_d dO16[r, h, d] o[r, h, d] (the scaled Delta, negated);
+// s_dS = the largest power of two with 2 s_dS Vmax <= 2^15 (so |dS s_dS| <= 2 |dO16_i| |v| s_dS
+// <= 2^15 < 65504).  Rows past the valid count get zeros.  gscal[2] = s_dO, gscal[3] = s_dS.
+__global__ void do_to_f16_delta_kernel(const float* __restrict__ dO, int64_t ld, const bf16* __restrict__ o,
+                                       int64_t ldo, __half* __restrict__ dO16, int64_t ld16,
+                                       float* __restrict__ delta, int64_t delta_ld, int T, int H, int s0,
+                                       const int32_t* __restrict__ n_valid, int valid_mult,
+                                       float* __restrict__ gscal) {
+  const int nv = valid_rows(n_valid, valid_mult, s0, T);
+  const float dmax = __uint_as_float(reinterpret_cast<const unsigned int*>(gscal)[1]);
+  const float vmax = __uint_as_float(reinterpret_cast<const unsigned int*>(gscal)[0]);
+  const float s_dO = (dmax > 0.f && dmax < INFINITY) ? 1.f / exp2f(ceilf(log2f(dmax))) : 1.f;
+  const float s_dS = (vmax > 0.f && vmax < INFINITY) ? fminf(pow2_floor(16384.f / vmax), 0x1p60f) : 1.f;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    gscal[2] = s_dO;
+    gscal[3] = s_dS;
+  }
+  const int lane = threadIdx.x & 31;
+  for (int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < (int64_t)T * H;
+       w += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    const int r = (int)(w / H), hh = (int)(w - (int64_t)r * H);
+    const int c = hh * 128 + lane * 4;
+    float d = 0.f;
+    uint2 packed = make_uint2(0u, 0u);
+    if (r < nv) {
+      const float4 v = *reinterpret_cast<const float4*>(dO + (int64_t)r * ld + c);
+      const __half2 h01 = __floats2half2_rn(v.x * s_dO, v.y * s_dO), h23 = __floats2half2_rn(v.z * s_dO, v.w * s_dO);
+      packed = make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
+      const uint2 ob = *reinterpret_cast<const uint2*>(o + (int64_t)(s0 + r) * ldo + c);
+      const __nv_bfloat162* op = reinterpret_cast<const __nv_bfloat162*>(&ob);
+      const float2 o01 = __bfloat1622float2(op[0]), o23 = __bfloat1622float2(op[1]);
+      const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+      d = f01.x * o01.x + f01.y * o01.y + f23.x * o23.x + f23.y * o23.y;
+    }
+    *reinterpret_cast<uint2*>(dO16 + (int64_t)r * ld16 + c) = packed;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+    if (lane == 0) delta[(int64_t)hh * delta_ld + r] = -d;
+  }
 }
 
 __global__ void inv_freq_kernel(double* __restrict__ out, int D, double log2_theta) {

@@ -2,15 +2,16 @@
 //
 // score[b, n] = sum_h sum_{j in block n} sum_{i >= j} P^h_ij,  P^h_i. = softmax_j(q_i.k_j / sqrt(D))
 //
-// Two passes, memory linear in S (the notes' FlashAttention-integrated scoring, §4.3):
-//   pass 1: per (head, query) the row log-sum-exp of the causal logits;
-//   pass 2: per (head, key) the column mass sum_i exp(s_ij - LSE_i);
-//   reduce: per block, sum over its keys and over heads in a fixed order (deterministic).
-// fp32 inputs: exact fp32 SIMT dot products.  bf16 inputs (head_dim 128): tensor-core
-// tiles of 64 queries x 64 keys.
-#include "attn_frag.cuh"
-#include "score_tc.cuh"
-#include "score_mass_tc.cuh"
+// Memory linear in S (the notes' FlashAttention-integrated scoring, §4.3).
+// bf16 inputs (head_dim 128): one tcgen05 pass (score_fused_tc.cuh) that keeps, per query
+// row, the log-sum-exp of every key chunk next to the row's running sum, and turns them into
+// chunk masses once the row's log-sum-exp is final; a deterministic reduction over heads and
+// query tiles gives the block scores.
+// fp32 inputs: exact fp32 SIMT dot products in two passes (per (head, query) the row
+// log-sum-exp; per (head, key) the column mass sum_i exp(s_ij - LSE_i)), then the same kind
+// of fixed-order reduction.
+#include "score_fused_tc.cuh"
+#include "score_blockmax_tc.cuh"
 
 namespace jenga {
 
@@ -93,153 +94,7 @@ __global__ void __launch_bounds__(256) score_mass_f32_kernel(const float* __rest
   if (lane == 0) mass[((int64_t)b * H + h) * S + j] = acc;
 }
 
-// ------------------------------------------------------------------ bf16 tensor-core path
-// pass 1: 64 query rows per CTA (4 warps x 16), key tiles streamed, online max / sum.
-__global__ void __launch_bounds__(128) score_lse_bf16_kernel(const bf16* __restrict__ q, int64_t ldq,
-                                                             const bf16* __restrict__ k, int64_t ldk, int S, int H,
-                                                             int causal, float scale_log2,
-                                                             float* __restrict__ lse) {
-  extern __shared__ __align__(128) uint8_t sm[];
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int qt = gridDim.x - 1 - blockIdx.x;
-  const int q0 = qt * AT_ROWS;
-  const bf16* qh = q + (int64_t)b * S * ldq + h * AT_D;
-  const bf16* kh = k + (int64_t)b * S * ldk + h * AT_D;
-  uint8_t* sQ = sm;
-  uint8_t* sK[2] = {sm + AT_TILE_BYTES, sm + 2 * AT_TILE_BYTES};
-  load_tile_async(sQ, qh, ldq, q0, S);
-  load_tile_async(sK[0], kh, ldk, 0, S);
-  cp_async_commit();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int row0 = q0 + warp * 16 + g, row1 = row0 + 8;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  uint32_t qa[8][4];
-  const int nkt = causal ? qt + 1 : S / AT_ROWS;
-  for (int kt = 0; kt < nkt; ++kt) {
-    if (kt + 1 < nkt) {
-      load_tile_async(sK[(kt + 1) & 1], kh, ldk, (kt + 1) * AT_ROWS, S);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    if (kt == 0) {
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) ld_a(sQ, warp * 16, ks * 16, qa[ks]);
-    }
-    float s[8][4];
-    mm_regs_x_rowsT(qa, sK[kt & 1], s);
-    const bool diag = causal && (kt == qt);
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int col = kt * AT_ROWS + j * 8 + 2 * t + e;
-        s[j][e] = (!diag || col <= row0) ? s[j][e] * scale_log2 : -INFINITY;
-        s[j][2 + e] = (!diag || col <= row1) ? s[j][2 + e] * scale_log2 : -INFINITY;
-        mx0 = fmaxf(mx0, s[j][e]);
-        mx1 = fmaxf(mx1, s[j][2 + e]);
-      }
-    }
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    l0 *= exp2f(m0 - mn0);
-    l1 *= exp2f(m1 - mn1);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      l0 += exp2f(s[j][0] - mn0) + exp2f(s[j][1] - mn0);
-      l1 += exp2f(s[j][2] - mn1) + exp2f(s[j][3] - mn1);
-    }
-    m0 = mn0;
-    m1 = mn1;
-    __syncthreads();
-  }
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  if (t == 0) {
-    float* lb = lse + ((int64_t)b * H + h) * S;
-    lb[row0] = (m0 + log2f(l0)) * SC_LN2;
-    lb[row1] = (m1 + log2f(l1)) * SC_LN2;
-  }
-}
-
-// pass 2: 64 keys per CTA (K fragments in registers), query tiles streamed;
-// each key accumulates exp(s_ij - LSE_i) over the queries i it is visible to.
-__global__ void __launch_bounds__(128) score_mass_bf16_kernel(const bf16* __restrict__ q, int64_t ldq,
-                                                              const bf16* __restrict__ k, int64_t ldk, int S, int H,
-                                                              int causal, float scale_log2,
-                                                              const float* __restrict__ lse,
-                                                              float* __restrict__ mass) {
-  extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ float sL[2][AT_ROWS];
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int kt = blockIdx.x;  // early key tiles see the most queries: launched first
-  const int k0 = kt * AT_ROWS;
-  const bf16* qh = q + (int64_t)b * S * ldq + h * AT_D;
-  const bf16* kh = k + (int64_t)b * S * ldk + h * AT_D;
-  const float* lb = lse + ((int64_t)b * H + h) * S;
-  uint8_t* sK = sm;
-  uint8_t* sQ[2] = {sm + AT_TILE_BYTES, sm + 2 * AT_TILE_BYTES};
-  const int qt_begin = causal ? kt : 0;
-  const int qt_end = S / AT_ROWS;
-  load_tile_async(sK, kh, ldk, k0, S);
-  load_tile_async(sQ[0], qh, ldq, qt_begin * AT_ROWS, S);
-  if (threadIdx.x < AT_ROWS) sL[0][threadIdx.x] = lb[qt_begin * AT_ROWS + threadIdx.x] * SC_LOG2E;
-  cp_async_commit();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int krow0 = k0 + warp * 16 + g, krow1 = krow0 + 8;
-  float acc0 = 0.f, acc1 = 0.f;
-  uint32_t ka[8][4];
-  for (int qt = qt_begin; qt < qt_end; ++qt) {
-    const int buf = (qt - qt_begin) & 1;
-    if (qt + 1 < qt_end) {
-      load_tile_async(sQ[buf ^ 1], qh, ldq, (qt + 1) * AT_ROWS, S);
-      if (threadIdx.x < AT_ROWS) sL[buf ^ 1][threadIdx.x] = lb[(qt + 1) * AT_ROWS + threadIdx.x] * SC_LOG2E;
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    if (qt == qt_begin) {
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) ld_a(sK, warp * 16, ks * 16, ka[ks]);
-    }
-    float s[8][4];
-    mm_regs_x_rowsT(ka, sQ[buf], s);
-    const bool diag = causal && (qt == kt);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int cl = j * 8 + 2 * t + e;
-        const int col = qt * AT_ROWS + cl;
-        const float L = sL[buf][cl];
-        acc0 += (!diag || col >= krow0) ? exp2f(s[j][e] * scale_log2 - L) : 0.f;
-        acc1 += (!diag || col >= krow1) ? exp2f(s[j][2 + e] * scale_log2 - L) : 0.f;
-      }
-    }
-    __syncthreads();
-  }
-  acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
-  acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
-  acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
-  acc1 += __shfl_xor_sync(0xffffffffu, acc1, 2);
-  if (t == 0) {
-    float* mb = mass + ((int64_t)b * H + h) * S;
-    mb[krow0] = acc0;
-    mb[krow1] = acc1;
-  }
-}
-
-// ------------------------------------------------------------------ block reduce (both paths)
+// ------------------------------------------------------------------ block reduce (fp32 path)
 // scores[b, n] = sum over the block's keys of (sum_h mass[b, h, key]) ; fixed order.
 __global__ void __launch_bounds__(1024) score_reduce_kernel(const float* __restrict__ mass, int S, int H, int blk,
                                                             float* __restrict__ scores) {
@@ -320,13 +175,44 @@ __global__ void score_blockmax_sum_kernel(const float* __restrict__ part, int nb
 
 using namespace jenga;
 
+// bf16 path: chunk width (keys) of the single-pass kernel for a block size (0: unsupported)
+static int score_chunk(int blk) { return blk % 64 == 0 ? 64 : (blk % 32 == 0 ? 32 : 0); }
+
+struct ScoreWs {  // byte offsets of the bf16 path's workspace regions
+  size_t lse, part, scratch, total;
+  int grid;
+};
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// bf16 block-max path: sub-tile group size for a block size (0: unsupported)
+static int blockmax_group(int blk) { return (blk == 32 || blk == 64) ? blk : (blk % 128 == 0 ? 128 : 0); }
+
+static ScoreWs score_ws_layout(int B, int S, int H, int blk) {
+  ScoreWs w{};
+  const int ch = score_chunk(blk);
+  if (!ch) return w;
+  const int nt = (S + SF_ROWS - 1) / SF_ROWS;
+  const long n_items = (long)nt * H * B;
+  w.grid = (int)(n_items < SF_GRID_CAP ? n_items : SF_GRID_CAP);
+  w.lse = 0;
+  w.part = align256((size_t)B * H * S * sizeof(float));
+  w.scratch = w.part + align256((size_t)B * H * nt * nt * (SF_ROWS / ch) * sizeof(float));
+  w.total = w.scratch + (size_t)w.grid * sf_scratch_floats_per_cta(nt, ch) * sizeof(float);
+  return w;
+}
+
 extern "C" size_t jenga_score_workspace_bytes(int B, int S, int H, int D, int blk) {
   (void)D;
   if (B < 1 || S < 1 || H < 1 || blk < 1) return 0;
   const size_t nb = (size_t)S / blk;
-  size_t a = 2 * (size_t)B * H * S * sizeof(float);  // LSE + column mass
-  size_t c = (size_t)B * nb * nb * sizeof(float);    // block-max partials
-  return (a > c ? a : c) + 256;
+  size_t a = 2 * (size_t)B * H * S * sizeof(float);  // fp32 path: row LSE + column mass
+  const int bg = blockmax_group(blk);
+  const size_t ng = bg ? (size_t)S / bg : 0;
+  size_t c = (size_t)B * (ng > nb ? ng * ng : nb * nb) * sizeof(float);  // block-max partials
+  size_t d = score_ws_layout(B, S, H, blk).total;    // bf16 single pass
+  size_t m = a > c ? a : c;
+  return (m > d ? m : d) + 256;
 }
 
 extern "C" jenga_status jenga_score_blocks(const void* q, int64_t ldq, const void* k, int64_t ldk, int B, int S,
@@ -346,10 +232,41 @@ extern "C" jenga_status jenga_score_blocks(const void* q, int64_t ldq, const voi
   const float scale = 1.f / sqrtf((float)D);
   const int nb = S / blk;
   if (mode == JENGA_SCORE_PAPER_BLOCKMAX) {
+    if (dt == JENGA_BF16) {
+      const int g = blockmax_group(blk);
+      if (D != 128 || !g || ldq % 8 || ldk % 8 || ((uintptr_t)q & 15) || ((uintptr_t)k & 15))
+        return fail(JENGA_EUNSUPPORTED,
+                    "jenga_score_blocks: bf16 block-max path needs D == 128, blk 32, 64 or a multiple of 128 and "
+                    "16-byte aligned rows");
+      CUtensorMap tq, tk;
+      jenga_status s1 = make_tmap_bf16(&tq, q, (uint64_t)B * S, (uint64_t)H * D, ldq, 128);
+      if (s1 != JENGA_OK) return s1;
+      s1 = make_tmap_bf16(&tk, k, (uint64_t)B * S, (uint64_t)H * D, ldk, 128);
+      if (s1 != JENGA_OK) return s1;
+      const int nt = (S + 127) / 128;
+      const int pairs = causal ? nt * (nt + 1) / 2 : nt * nt;
+      JENGA_CUDA_TRY(
+          cudaFuncSetAttribute(score_blockmax_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BM_SMEM));
+      {
+        const int _ps = ::jenga::prof_begin("score_blockmax_tc", st);
+        score_blockmax_tc_kernel<<<dim3(pairs, B), BM_THREADS, BM_SMEM, st>>>(
+            tq, tk, S, H, g, causal ? 1 : 0, scale / (float)H, wsf);
+        ::jenga::prof_end(_ps, st);
+      }
+      JENGA_LAUNCH_CHECK();
+      {
+        const int _ps = ::jenga::prof_begin("score_blockmax_colsum", st);
+        score_blockmax_colsum_kernel<<<dim3((nb + 127) / 128, B), 128, 0, st>>>(wsf, nb, blk / g, causal ? 1 : 0,
+                                                                                 scores);
+        ::jenga::prof_end(_ps, st);
+      }
+      JENGA_LAUNCH_CHECK();
+      return JENGA_OK;
+    }
     {
     const int _ps = ::jenga::prof_begin("score_blockmax_f32", st);
     score_blockmax_f32_kernel<<<dim3(nb, nb, B), 256, 0, st>>>(q, ldq, k, ldk, S, H, D, blk, causal ? 1 : 0,
-                                                              dt == JENGA_BF16 ? 1 : 0, scale, wsf);
+                                                              0, scale, wsf);
     ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();
@@ -382,58 +299,46 @@ extern "C" jenga_status jenga_score_blocks(const void* q, int64_t ldq, const voi
     }
     JENGA_LAUNCH_CHECK();
   } else {
-    if (D != AT_D || S % AT_ROWS || ldq % 8 || ldk % 8 || ((uintptr_t)q & 15) || ((uintptr_t)k & 15))
-      return fail(JENGA_EUNSUPPORTED, "jenga_score_blocks: bf16 path needs D == 128, S % 64 == 0, aligned rows");
+    const int ch = score_chunk(blk);
+    if (D != 128 || !ch || ldq % 8 || ldk % 8 || ((uintptr_t)q & 15) || ((uintptr_t)k & 15))
+      return fail(JENGA_EUNSUPPORTED,
+                  "jenga_score_blocks: bf16 path needs D == 128, blk a multiple of 32 and 16-byte aligned rows");
+    const ScoreWs w = score_ws_layout(B, S, H, blk);
+    char* base = (char*)wsf;
+    float* neg_lse = (float*)(base + w.lse);
+    float* part = (float*)(base + w.part);
+    float* scratch = (float*)(base + w.scratch);
+    CUtensorMap tq, tk;
+    jenga_status s1 = make_tmap_bf16(&tq, q, (uint64_t)B * S, (uint64_t)H * D, ldq, SF_ROWS);
+    if (s1 != JENGA_OK) return s1;
+    s1 = make_tmap_bf16(&tk, k, (uint64_t)B * S, (uint64_t)H * D, ldk, SF_ROWS);
+    if (s1 != JENGA_OK) return s1;
+    int grid = sm_count();
+    if (grid > w.grid) grid = w.grid;
     const float sl2 = SC_LOG2E * scale;
-    if (S % SCT_ROWS == 0) {
-      // tcgen05 path: 128-token tiles, TMA-fed, accumulators in tensor memory
-      CUtensorMap tq, tk;
-      jenga_status s1 = make_tmap_bf16(&tq, q, (uint64_t)B * S, (uint64_t)H * D, ldq, SCT_ROWS);
-      if (s1 != JENGA_OK) return s1;
-      s1 = make_tmap_bf16(&tk, k, (uint64_t)B * S, (uint64_t)H * D, ldk, SCT_ROWS);
-      if (s1 != JENGA_OK) return s1;
-      JENGA_CUDA_TRY(cudaFuncSetAttribute(score_lse_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SCT_SMEM));
-      JENGA_CUDA_TRY(cudaFuncSetAttribute(score_mass_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMT_SMEM));
-      dim3 gt(S / SCT_ROWS, H, B);
-      {
-        const int _ps = ::jenga::prof_begin("score_lse_tc", st);
-        score_lse_tc_kernel<<<gt, SCT_THREADS, SCT_SMEM, st>>>(tq, tk, S, H, causal ? 1 : 0, sl2, lse);
-        ::jenga::prof_end(_ps, st);
-      }
-      JENGA_LAUNCH_CHECK();
-      {
-        const int _ps = ::jenga::prof_begin("score_mass_tc", st);
-        score_mass_tc_kernel<<<gt, SMT_THREADS, SMT_SMEM, st>>>(tq, tk, S, H, causal ? 1 : 0, sl2, lse, mass);
-        ::jenga::prof_end(_ps, st);
-      }
-      JENGA_LAUNCH_CHECK();
-      {
-        const int _ps = ::jenga::prof_begin("score_reduce", st);
-        score_reduce_kernel<<<dim3(nb, B), 1024, 0, st>>>(mass, S, H, blk, scores);
-        ::jenga::prof_end(_ps, st);
-      }
-      JENGA_LAUNCH_CHECK();
-      return JENGA_OK;
-    }
-    dim3 g(S / AT_ROWS, H, B);
-    JENGA_CUDA_TRY(
-        cudaFuncSetAttribute(score_lse_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 3 * AT_TILE_BYTES));
-    JENGA_CUDA_TRY(
-        cudaFuncSetAttribute(score_mass_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 3 * AT_TILE_BYTES));
     {
-    const int _ps = ::jenga::prof_begin("score_lse_bf16", st);
-    score_lse_bf16_kernel<<<g, 128, 3 * AT_TILE_BYTES, st>>>((const bf16*)q, ldq, (const bf16*)k, ldk, S, H,
-                                                              causal ? 1 : 0, sl2, lse);
-    ::jenga::prof_end(_ps, st);
+      const int _ps = ::jenga::prof_begin("score_fused_tc", st);
+      if (ch == 64) {
+        JENGA_CUDA_TRY(
+            cudaFuncSetAttribute(score_fused_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, SF_SMEM));
+        score_fused_tc_kernel<64><<<grid, SF_THREADS, SF_SMEM, st>>>(tq, tk, S, H, B, causal ? 1 : 0, sl2, neg_lse,
+                                                                     part, scratch);
+      } else {
+        JENGA_CUDA_TRY(
+            cudaFuncSetAttribute(score_fused_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, SF_SMEM));
+        score_fused_tc_kernel<32><<<grid, SF_THREADS, SF_SMEM, st>>>(tq, tk, S, H, B, causal ? 1 : 0, sl2, neg_lse,
+                                                                     part, scratch);
+      }
+      ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();
     {
-    const int _ps = ::jenga::prof_begin("score_mass_bf16", st);
-    score_mass_bf16_kernel<<<g, 128, 3 * AT_TILE_BYTES, st>>>((const bf16*)q, ldq, (const bf16*)k, ldk, S, H,
-                                                               causal ? 1 : 0, sl2, lse, mass);
-    ::jenga::prof_end(_ps, st);
+      const int _ps = ::jenga::prof_begin("score_chunk_reduce", st);
+      score_chunk_reduce_kernel<<<dim3(nb, B), 256, 0, st>>>(part, S, H, blk, ch, causal ? 1 : 0, scores);
+      ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();
+    return JENGA_OK;
   }
   {
   const int _ps = ::jenga::prof_begin("score_reduce", st);

@@ -79,8 +79,9 @@ extern "C" jenga_status jenga_score_blocks_noalloc(const void* q, int64_t ldq, c
   const size_t need = jenga_score_workspace_bytes(B, S, H, D, blk);
   if (need > NOALLOC_SCRATCH_BYTES)
     return fail(JENGA_EWORKSPACE,
-                "jenga_score_blocks_noalloc: these sizes need %zu bytes of scratch, above the library's fixed "
-                "%zu-byte array (B*H*S must stay below about 2M); use jenga_score_blocks with a workspace",
+                "jenga_score_blocks_noalloc: these sizes need %zu bytes of scratch "
+                "(jenga_score_workspace_bytes), above the library's fixed %zu-byte array; use "
+                "jenga_score_blocks with a workspace",
                 need, NOALLOC_SCRATCH_BYTES);
   void* scratch = nullptr;
   jenga_status s = noalloc_scratch(&scratch);
