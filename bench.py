@@ -697,6 +697,30 @@ def main():
     if not args.no_movement:
         movement = measure_movement(J, torch, dev, X0, case, ks, hbm)
 
+    # ---------------- paper-form block-max score (Eq. 2) on layer 0's q | k of all S rows
+    paper = None
+    if not args.no_movement and pred is None:
+        bq = buffers(ks)
+        J.jenga_layer_score_qk(layers[0], X0, out=bq["qk"], ws=bq["qk_ws"])
+        qk = bq["qk"]
+        fn = lambda: J.jenga_score_blocks(qk[:, :HD], qk[:, HD:], sh.heads, sh.head_dim, blk, mode="paper_blockmax",
+                                          out=bq["scores"][0], ws=bq["sc_ws"])
+        for _ in range(2):
+            fn()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
+        for _ in range(3):
+            fn()
+        ev1.record()
+        torch.cuda.synchronize()
+        J.jenga_check_device_status()
+        t = ev0.elapsed_time(ev1) / 3 / 1e3
+        fl = 2.0 * sh.head_dim * sh.heads * causal_pairs(S)
+        paper = {"ms": t * 1e3, "tflops": fl / t / 1e12, "frac_bf16_sustained": fl / t / 1e12 / tf_sus,
+                 "work": "one QK^T product per causal (query, key) pair and head (2 D H flop per pair)"}
+        del bq
+        torch.cuda.empty_cache()
+
     # ---------------- segmented LM-head loss (segment-based peak cutting)
     lm_loss = None
     if not args.no_lm_loss:
@@ -724,7 +748,7 @@ def main():
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "movement": movement,
                 "clocks": clk, "peak_mem_gib": peak_sparse, "dense": dense,
                 **({"predictor": predictor} if predictor is not None else {}), "lm_loss": lm_loss,
-                "step_tflop": step_flops(case, ks, scoring) / 1e12, "kernels": kernels}
+                "paper_blockmax_score": paper, "step_tflop": step_flops(case, ks, scoring) / 1e12, "kernels": kernels}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -151,7 +151,8 @@ def head_attention_fwd(args):
     for i0 in range(0, n, chunk):
         i1 = min(n, i0 + chunk)
         s = (qh[i0:i1] @ kh[:i1].T) * scale
-        s = np.where(jj[None, :i1] <= np.arange(i0, i1)[:, None], s, -np.inf)
+        # keys j < i0 are visible to every row of the chunk; only the diagonal block is masked
+        s[:, i0:] = np.where(jj[None, i0:i1] <= np.arange(i0, i1)[:, None], s[:, i0:], -np.inf)
         m = s.max(axis=1, keepdims=True)
         p = np.exp(s - m)
         l = p.sum(axis=1, keepdims=True)
@@ -197,7 +198,7 @@ def head_attention_bwd(args):
         for i0 in range(r0, r1, chunk):
             i1 = min(r1, i0 + chunk)
             s = (qh[i0:i1] @ kh[:i1].T) * scale
-            s = np.where(jj[None, :i1] <= np.arange(i0, i1)[:, None], s, -np.inf)
+            s[:, i0:] = np.where(jj[None, i0:i1] <= np.arange(i0, i1)[:, None], s[:, i0:], -np.inf)
             m = s.max(axis=1, keepdims=True)
             p = np.exp(s - m)
             p /= p.sum(axis=1, keepdims=True)

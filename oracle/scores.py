@@ -43,9 +43,9 @@ def head_column_mass(args):
         i1 = min(S, i0 + chunk)
         kend = i1 if causal else S
         s = (qh[i0:i1] @ kh[:kend].T) * scale            # [c, kend]
-        if causal:
+        if causal:  # keys j < i0 are visible to every row of the chunk: mask the diagonal block
             ii = np.arange(i0, i1)[:, None]
-            s = np.where(np.arange(kend)[None, :] <= ii, s, -np.inf)
+            s[:, i0:] = np.where(np.arange(i0, kend)[None, :] <= ii, s[:, i0:], -np.inf)
         m = s.max(axis=1, keepdims=True)
         p = np.exp(s - m)
         p /= p.sum(axis=1, keepdims=True)

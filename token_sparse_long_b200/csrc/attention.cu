@@ -26,8 +26,10 @@ __device__ __forceinline__ int attn_rows(const int32_t* n_valid, int mult, int c
 }
 
 // ------------------------------------------------------------------ host launchers
-jenga_status attn_forward(const bf16* q, const bf16* k, const bf16* v, int64_t ld, bf16* o, int64_t ldo, float* lse,
-                          int64_t lse_ld, int H, const int32_t* n_valid, int valid_mult, int n_cap, cudaStream_t st) {
+// v16: an fp16 copy of v (row pitch ld_v16), the B operand of the PV product (fp16 P).
+jenga_status attn_forward(const bf16* q, const bf16* k, const void* v16, int64_t ld, int64_t ld_v16, bf16* o,
+                          int64_t ldo, float* lse, int64_t lse_ld, int H, const int32_t* n_valid, int valid_mult,
+                          int n_cap, cudaStream_t st) {
   if (n_cap <= 0) return JENGA_OK;
   if (n_cap % AT_ROWS) return fail(JENGA_EINVAL, "attention: rows must be a multiple of 64");
   const float scale_log2 = LOG2E / sqrtf((float)AT_D);
@@ -38,7 +40,7 @@ jenga_status attn_forward(const bf16* q, const bf16* k, const bf16* v, int64_t l
     jenga_status s1;
     if ((s1 = make_tmap_bf16(&tq, q, n_cap, (uint64_t)H * AT_D, ld, ATC_ROWS)) != JENGA_OK) return s1;
     if ((s1 = make_tmap_bf16(&tk, k, n_cap, (uint64_t)H * AT_D, ld, ATC_ROWS)) != JENGA_OK) return s1;
-    if ((s1 = make_tmap_bf16(&tv, v, n_cap, (uint64_t)H * AT_D, ld, ATC_ROWS)) != JENGA_OK) return s1;
+    if ((s1 = make_tmap_f16(&tv, v16, n_cap, (uint64_t)H * AT_D, ld_v16, ATC_ROWS)) != JENGA_OK) return s1;
     JENGA_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATC_SMEM));
     const int _ps = ::jenga::prof_begin("attn_fwd_tc", st);
     attn_fwd_tc_kernel<<<dim3((n_cap + ATC_ROWS - 1) / ATC_ROWS, H), ATC_THREADS, ATC_SMEM, st>>>(

@@ -12,8 +12,11 @@
 //               half-row maxima): load S_j, mask (causal diagonal, keys past n; only on
 //               those tiles), online max with lazy rescaling (O and l are rescaled in TMEM
 //               only when the running max grows by more than 2^8), P = 2^(s log2e /
-//               sqrt(D) - m) as bf16 pairs into tensor memory P[j % 2] (one exponential in
-//               four on the FMA pipe, exp2_fma), row sums in fp32
+//               sqrt(D) - m) x 2^6 as fp16 pairs into tensor memory P[j % 2] (P <= 2^8 under
+//               the lazy rescale, so the scaled value stays below 2^14; one exponential in
+//               four on the FMA pipe, exp2_fma), row sums in fp32; V is an fp16 copy of v
+//               (fp16 has 3 more mantissa bits than bf16 for P and v, which the PV product
+//               needs at long sequence lengths)
 // The softmax of tile j overlaps the PV product of tile j-1 and the QK^T product of
 // tile j+1; with P double-buffered it waits only for the PV product of tile j-2.  Output o = O / l (bf16) and the negated row log-sum-exp in log2 units (the
 // backward adds it to the scaled logits directly).
@@ -141,7 +144,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     }
   } else if (warp == 2 && lane == 0) {
     // O += P_j V_j once the softmax has written P_j
-    constexpr uint32_t idesc_o = umma_idesc_bf16_bmn(128, 128);
+    constexpr uint32_t idesc_o = umma_idesc_bf16_bmn(128, 128) & ~((7u << 7) | (7u << 10));  // fp16 P, V
     for (int j = 0; j < nj; ++j) {
       const int sv = j % ATC_V_STAGES, b = j & 1;
       if (!mbar_wait_at(&p_full[b], (j >> 1) & 1, 103, (qt << 16) | j)) break;
@@ -241,7 +244,8 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
           const float x1 = fmaf(__uint_as_float(v[c + 1]), scale_log2, -m_used);
           const float a = fast_exp2(x0);
           const float b2 = ((c & 3) == 2) ? exp2_fma<64>(x1) : fast_exp2(x1);  // 1 in 4 on the FMA pipe
-          pk[c >> 1] = pack_bf2(a, b2);
+          const __half2 hp = __floats2half2_rn(a * 64.f, b2 * 64.f);
+          pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&hp);
           ps[(c >> 1) & 3] += a + b2;
         }
       } else {  // masked entries are -inf: ex2 gives exactly 0 (exp2_fma would floor at 2^-125)
@@ -249,7 +253,8 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         for (int c = 0; c < 64; c += 2) {
           const float a = fast_exp2(fmaf(__uint_as_float(v[c]), scale_log2, -m_used));
           const float b2 = fast_exp2(fmaf(__uint_as_float(v[c + 1]), scale_log2, -m_used));
-          pk[c >> 1] = pack_bf2(a, b2);
+          const __half2 hp = __floats2half2_rn(a * 64.f, b2 * 64.f);
+          pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&hp);
           ps[(c >> 1) & 3] += a + b2;
         }
       }
@@ -262,7 +267,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
           !__all_sync(0xffffffffu, mbar_wait_at(&p_free[pb], ((j >> 1) - 1) & 1, 108, (qt << 16) | j)))
         ok = false;
       if (ok) {
-        tmem_st32(tP + lane_off + pb * 64 + hf * 32, pk);  // keys 64 hf .. 64 hf + 63 as bf16 pairs
+        tmem_st32(tP + lane_off + pb * 64 + hf * 32, pk);  // keys 64 hf .. 64 hf + 63 as fp16 pairs
         tmem_wait_st();
       }
       tc_fence_before();
@@ -278,7 +283,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     const float l_row = l + xm[(1 - hf) * 128 + r];
     if (__all_sync(0xffffffffu, fin)) {  // warp-uniform: the loads below are collective
       tc_fence_after();
-      const float inv = 1.f / l_row;
+      const float inv = 1.f / (64.f * l_row);  // P entered the PV product scaled by 2^6
       const bool row_ok = qrow < n;
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {

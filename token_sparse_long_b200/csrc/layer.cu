@@ -5,8 +5,9 @@
 
 namespace jenga {
 
-jenga_status attn_forward(const bf16* q, const bf16* k, const bf16* v, int64_t ld, bf16* o, int64_t ldo, float* lse,
-                          int64_t lse_ld, int H, const int32_t* n_valid, int valid_mult, int n_cap, cudaStream_t st);
+jenga_status attn_forward(const bf16* q, const bf16* k, const void* v16, int64_t ld, int64_t ld_v16, bf16* o,
+                          int64_t ldo, float* lse, int64_t lse_ld, int H, const int32_t* n_valid, int valid_mult,
+                          int n_cap, cudaStream_t st);
 jenga_status attn_backward_segment(const void* q16, const void* k16, const void* v16, int64_t ld, const float* lse,
                                    int64_t lse_ld, const void* dO16, int64_t ld_do, const float* delta,
                                    int64_t delta_ld, float* dq, int64_t ld_dq, float* dk_acc, float* dv_acc,
@@ -98,6 +99,7 @@ struct FwdWs {
   float2* rope;  // [nc][64] (cos, sin) of the retained rows' positions
   float* mlp_scores;  // MLP-block criterion per retained block
   int32_t *mlp_pos, *n_mlp;
+  __half* v16;        // [nc, HD] fp16 copy of v (the PV product's operand)
 };
 static size_t carve_fwd_ws(Carve& c, const Dims& d, int nc, FwdWs* w) {
   w->xn = c.take<bf16>((size_t)nc * d.h);
@@ -108,6 +110,7 @@ static size_t carve_fwd_ws(Carve& c, const Dims& d, int nc, FwdWs* w) {
   w->mlp_scores = c.take<float>(nbk);
   w->mlp_pos = c.take<int32_t>(nbk);
   w->n_mlp = c.take<int32_t>(1);
+  w->v16 = c.take<__half>((size_t)nc * d.HD);
   return c.used();
 }
 
@@ -466,7 +469,14 @@ static jenga_status layer_fwd(const jenga_layer_weights* w, const jenga_lora* lo
     ::jenga::prof_end(_ps, st);
   }
   JENGA_LAUNCH_CHECK();
-  JENGA_TRY(attn_forward(s.qkv, s.qkv + HD, s.qkv + 2 * HD, 3 * HD, s.o, HD, s.lse, nc, d.H, n_kept, blk, nc, st));
+  {
+    const int _ps = ::jenga::prof_begin("v_to_f16", st);
+    qkv_to_f16_kernel<<<grid_cap((int64_t)nc * (HD / 8), 256), 256, 0, st>>>(s.qkv + 2 * HD, 3 * HD, f.v16, HD, nc, HD,
+                                                                              -1, nullptr);
+    ::jenga::prof_end(_ps, st);
+  }
+  JENGA_LAUNCH_CHECK();
+  JENGA_TRY(attn_forward(s.qkv, s.qkv + HD, f.v16, 3 * HD, HD, s.o, HD, s.lse, nc, d.H, n_kept, blk, nc, st));
   // 5. o_proj with the in-place residual add into X (and a compact copy of h)
   {
     EpiParams e = epi_base(idx, blk, n_kept, 0);

@@ -351,16 +351,27 @@ __global__ void __launch_bounds__(SF_THREADS, 1)
       const int rows_valid = S - t * SF_ROWS;  // >= 1
       const float4 L4 = reinterpret_cast<const float4*>(Lsm)[lane];
       float* out = part + (((int64_t)b * H + h) * nt + t) * nch_row;
-      for (int c = ew; c < nchunk; c += SF_EPI_WARPS) {
-        const float4 a = *reinterpret_cast<const float4*>(my_lp + (size_t)c * 128 + 4 * lane);
-        float s = 0.f;
-        s += (4 * lane + 0 < rows_valid) ? fast_exp2(a.x - L4.x) : 0.f;
-        s += (4 * lane + 1 < rows_valid) ? fast_exp2(a.y - L4.y) : 0.f;
-        s += (4 * lane + 2 < rows_valid) ? fast_exp2(a.z - L4.z) : 0.f;
-        s += (4 * lane + 3 < rows_valid) ? fast_exp2(a.w - L4.w) : 0.f;
+      // four chunks per warp and step: their loads are in flight together
+      for (int c0 = ew; c0 < nchunk; c0 += 4 * SF_EPI_WARPS) {
+        float4 a[4];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0) out[c] = s;
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + u * SF_EPI_WARPS;
+          a[u] = c < nchunk ? *reinterpret_cast<const float4*>(my_lp + (size_t)c * 128 + 4 * lane)
+                            : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + u * SF_EPI_WARPS;
+          float s = 0.f;
+          s += (4 * lane + 0 < rows_valid) ? fast_exp2(a[u].x - L4.x) : 0.f;
+          s += (4 * lane + 1 < rows_valid) ? fast_exp2(a[u].y - L4.y) : 0.f;
+          s += (4 * lane + 2 < rows_valid) ? fast_exp2(a[u].z - L4.z) : 0.f;
+          s += (4 * lane + 3 < rows_valid) ? fast_exp2(a[u].w - L4.w) : 0.f;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+          if (lane == 0 && c < nchunk) out[c] = s;
+        }
       }
       // the next item overwrites the scratch and Lsm only after every warp read them
       asm volatile("bar.sync 1, %0;" ::"n"(32 * SF_EPI_WARPS) : "memory");
