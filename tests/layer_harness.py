@@ -101,10 +101,12 @@ def retained_mask(S, blk, idx, n_kept):
 def check_layer_against_oracle(S, blk, idx, n_kept, out, dx, grads_gpu, Xo, dX, grads, X, G):
     """The layer bars (bf16 outputs and gradients against the oracle on the same inputs
     and the GPU's kept blocks): max |gpu - oracle| / rms(oracle) <= 3e-2 on the output and
-    the input gradient, one bf16 ulp of the stored value forgiven; the same on the
-    sub-block contributions (out - x <= 3e-2, dX - G <= 6e-2, which a real fault moves by
-    O(1)); LoRA gradients <= 3e-2; eliminated rows exactly x and exactly G.  Returns the
-    errors."""
+    the input gradient, one bf16 ulp of the stored value forgiven; LoRA gradients <= 3e-2;
+    eliminated rows exactly x and exactly G.  Diagnostics beyond the stated bar: the same
+    measure on the sub-block contributions, which a real fault moves by O(1): out - x <= 3e-2
+    with two ulps forgiven (h and out are both stored in bf16 at the magnitude of the
+    residual stream, which the salient-row scaling of chained layers makes large), and
+    dX - G <= 6e-2 (one rounding).  Returns the errors."""
     rows = retained_mask(S, blk, idx, n_kept)
     assert np.array_equal(out[~rows], X[~rows]), "eliminated rows must pass through unchanged"
     assert np.array_equal(dx[~rows], G[~rows]), "eliminated rows: identity gradient"
@@ -112,7 +114,7 @@ def check_layer_against_oracle(S, blk, idx, n_kept, out, dx, grads_gpu, Xo, dX, 
     if rows.any():
         e["out"] = rel_max_ulp(out[rows], Xo[rows])
         e["dx"] = rel_max_ulp(dx[rows], dX[rows])
-        e["out-x"] = rel_delta_ulp(out[rows], Xo[rows], X[rows])
+        e["out-x"] = rel_delta_ulp(out[rows], Xo[rows], X[rows], roundings=2)
         e["dx-G"] = rel_delta_ulp(dx[rows], dX[rows], G[rows])
     for k in grads:
         if np.abs(grads[k]).max() == 0:
@@ -248,14 +250,14 @@ def rel_max_ulp(gpu, ref):
     return float(ex.max() / (rms if rms > 0 else 1.0))
 
 
-def rel_delta_ulp(gpu, ref, base):
+def rel_delta_ulp(gpu, ref, base, roundings=1):
     """Error of a sub-block's contribution (result - base) stored in bf16:
-    max over elements of (|gpu - ref| - ulp_bf16(ref))_+ / rms(ref - base).
-    One bf16 ulp of the stored result is forgiven (its final rounding may land on
-    either neighbour); everything else counts against the 3e-2 bar."""
+    max over elements of (|gpu - ref| - roundings * ulp_bf16(ref))_+ / rms(ref - base).
+    One bf16 ulp of the stored result is forgiven per bf16 rounding taken at the result's
+    magnitude (each may land on either neighbour); everything else counts against the bar."""
     gpu = np.asarray(gpu, np.float64)
     ref = np.asarray(ref, np.float64)
     d = ref - np.asarray(base, np.float64)
     rms = np.sqrt((d * d).mean())
-    ex = np.maximum(np.abs(gpu - ref) - bf16_ulp(ref), 0.0)
+    ex = np.maximum(np.abs(gpu - ref) - roundings * bf16_ulp(ref), 0.0)
     return float(ex.max() / (rms if rms > 0 else 1.0))

@@ -27,9 +27,10 @@ __device__ __forceinline__ int attn_rows(const int32_t* n_valid, int mult, int c
 
 // ------------------------------------------------------------------ host launchers
 // v16: an fp16 copy of v (row pitch ld_v16), the B operand of the PV product (fp16 P).
+// o_lo (nullable): bf16 rounding residual of o (same layout), so that hi + lo carries ~16 bits.
 jenga_status attn_forward(const bf16* q, const bf16* k, const void* v16, int64_t ld, int64_t ld_v16, bf16* o,
                           int64_t ldo, float* lse, int64_t lse_ld, int H, const int32_t* n_valid, int valid_mult,
-                          int n_cap, cudaStream_t st) {
+                          int n_cap, cudaStream_t st, bf16* o_lo) {
   if (n_cap <= 0) return JENGA_OK;
   if (n_cap % AT_ROWS) return fail(JENGA_EINVAL, "attention: rows must be a multiple of 64");
   const float scale_log2 = LOG2E / sqrtf((float)AT_D);
@@ -44,7 +45,7 @@ jenga_status attn_forward(const bf16* q, const bf16* k, const void* v16, int64_t
     JENGA_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATC_SMEM));
     const int _ps = ::jenga::prof_begin("attn_fwd_tc", st);
     attn_fwd_tc_kernel<<<dim3((n_cap + ATC_ROWS - 1) / ATC_ROWS, H), ATC_THREADS, ATC_SMEM, st>>>(
-        tq, tk, tv, o, ldo, lse, lse_ld, n_valid, valid_mult, n_cap, scale_log2);
+        tq, tk, tv, o, ldo, lse, lse_ld, n_valid, valid_mult, n_cap, scale_log2, o_lo);
     ::jenga::prof_end(_ps, st);
     JENGA_LAUNCH_CHECK();
     return JENGA_OK;

@@ -30,9 +30,9 @@
 // Causal masking, keys / queries past the valid count, and the segment bounds are applied
 // in the epilogue.  Every wait is bounded; waits that guard collective TMEM loads are voted.
 // Operands are fp16 (3 more mantissa bits than bf16): fp16 copies of q, k, v, the segment's dO
-// scaled by a power of two s_dO (max per-head row norm <= 1), P scaled by 2^8 (P <= 1) and
-// dS scaled by s_dS = 2^floor(log2(2^14 / Vmax)) with Vmax the largest per-head row norm of v,
-// so |dS s_dS| <= |P (dP - Delta)| s_dS <= 2 |dO_i| |v| s_dS <= 2^15 can never overflow
+// scaled by a power of two s_dO (max per-head row norm in (2^13, 2^14]), P scaled by 2^8 (P <= 1)
+// and dS scaled by s_dS = 2^floor(log2(1 / Vmax)) with Vmax the largest per-head row norm of v,
+// so |dS s_dS| <= |P (dP - Delta)| s_dS <= |dO_i| |v_j - o_i| s_dS <= 2^15 can never overflow
 // (gscal[2] = s_dO, gscal[3] = s_dS, set on the device before the launch).  The fp32 results
 // are divided by the scales again before they leave the kernels.
 #pragma once

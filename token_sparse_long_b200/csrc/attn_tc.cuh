@@ -44,7 +44,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ o, int64_t ldo,
                        float* __restrict__ lse, int64_t lse_ld, const int32_t* __restrict__ n_valid, int valid_mult,
-                       int n_cap, float scale_log2) {
+                       int n_cap, float scale_log2, bf16* __restrict__ o_lo) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ATC_BAR_OFF);
@@ -293,13 +293,23 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         tmem_wait_ld();
         if (row_ok) {
           uint4* dst = reinterpret_cast<uint4*>(o + (int64_t)qrow * ldo + col + c0);
+          uint4* dlo = o_lo ? reinterpret_cast<uint4*>(o_lo + (int64_t)qrow * ldo + col + c0) : nullptr;
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
-            uint32_t w[4];
+            uint32_t w[4], wl[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              w[i] = pack_bf2(__uint_as_float(ob[q4 * 8 + 2 * i]) * inv, __uint_as_float(ob[q4 * 8 + 2 * i + 1]) * inv);
+            for (int i = 0; i < 4; ++i) {
+              const float x0 = __uint_as_float(ob[q4 * 8 + 2 * i]) * inv;
+              const float x1 = __uint_as_float(ob[q4 * 8 + 2 * i + 1]) * inv;
+              w[i] = pack_bf2(x0, x1);
+              // the rounding residual (o = hi + lo to ~16 bits) for the backward's Delta = dO . o,
+              // which cancels strongly on rows that attend to few keys
+              const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
+              const float2 hf2 = __bfloat1622float2(hb);
+              wl[i] = pack_bf2(x0 - hf2.x, x1 - hf2.y);
+            }
             dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
+            if (dlo) dlo[q4] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
           }
         }
       }

@@ -7,7 +7,7 @@ namespace jenga {
 
 jenga_status attn_forward(const bf16* q, const bf16* k, const void* v16, int64_t ld, int64_t ld_v16, bf16* o,
                           int64_t ldo, float* lse, int64_t lse_ld, int H, const int32_t* n_valid, int valid_mult,
-                          int n_cap, cudaStream_t st);
+                          int n_cap, cudaStream_t st, bf16* o_lo);
 jenga_status attn_backward_segment(const void* q16, const void* k16, const void* v16, int64_t ld, const float* lse,
                                    int64_t lse_ld, const void* dO16, int64_t ld_do, const float* delta,
                                    int64_t delta_ld, float* dq, int64_t ld_dq, float* dk_acc, float* dv_acc,
@@ -79,6 +79,7 @@ struct Saved {
   bf16 *xr, *qkv, *o, *hres;
   float *t, *lse, *rstd1, *rstd2;
   uint8_t* mlp_mask;  // [n_kept_max]: 1 = the MLP sub-block runs on this retained block
+  bf16* olo;          // [nc, HD] bf16 rounding residual of o (the backward's Delta uses hi + lo)
 };
 
 static size_t carve_saved(Carve& c, const Dims& d, int nc, Saved* s) {
@@ -91,6 +92,7 @@ static size_t carve_saved(Carve& c, const Dims& d, int nc, Saved* s) {
   s->rstd1 = c.take<float>(nc);
   s->rstd2 = c.take<float>(nc);
   s->mlp_mask = c.take<uint8_t>(nc > 0 ? (size_t)nc : 1);  // >= n_kept_max entries (one per retained block)
+  s->olo = c.take<bf16>((size_t)nc * d.HD);
   return c.used();
 }
 
@@ -476,7 +478,7 @@ static jenga_status layer_fwd(const jenga_layer_weights* w, const jenga_lora* lo
     ::jenga::prof_end(_ps, st);
   }
   JENGA_LAUNCH_CHECK();
-  JENGA_TRY(attn_forward(s.qkv, s.qkv + HD, f.v16, 3 * HD, HD, s.o, HD, s.lse, nc, d.H, n_kept, blk, nc, st));
+  JENGA_TRY(attn_forward(s.qkv, s.qkv + HD, f.v16, 3 * HD, HD, s.o, HD, s.lse, nc, d.H, n_kept, blk, nc, st, s.olo));
   // 5. o_proj with the in-place residual add into X (and a compact copy of h)
   {
     EpiParams e = epi_base(idx, blk, n_kept, 0);
@@ -697,7 +699,7 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
     {
       const int _ps = ::jenga::prof_begin("do_to_f16_delta", st);
       do_to_f16_delta_kernel<<<grid_cap((int64_t)T * H * 32, 256), 256, 0, st>>>(
-          b.dOf, HD, s.o, HD, reinterpret_cast<__half*>(b.dO), HD, b.delta, T, T, H, s0, n_kept, blk, b.gscal);
+          b.dOf, HD, s.o, s.olo, HD, reinterpret_cast<__half*>(b.dO), HD, b.delta, T, T, H, s0, n_kept, blk, b.gscal);
       ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();

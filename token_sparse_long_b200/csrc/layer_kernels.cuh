@@ -509,19 +509,26 @@ __device__ __forceinline__ float pow2_floor(float x) {  // largest power of two 
 }
 
 // dO16 = fp16(dO s_dO) with s_dO the power of two that brings the largest per-head row norm
-// into (1/2, 1]; delta[h, r] = -sum_d dO16[r, h, d] o[r, h, d] (the scaled Delta, negated);
-// s_dS = the largest power of two with 2 s_dS Vmax <= 2^15 (so |dS s_dS| <= 2 |dO16_i| |v| s_dS
-// <= 2^15 < 65504).  Rows past the valid count get zeros.  gscal[2] = s_dO, gscal[3] = s_dS.
+// into (2^13, 2^14]; delta[h, r] = -sum_d dO16[r, h, d] o[r, h, d] (the scaled Delta, negated;
+// o = the bf16 o plus its stored rounding residual o_lo when given); s_dS = the largest power of
+// two <= 1 / Vmax (so |dS s_dS| <= |dO16_i| |v_j - o_i| s_dS <= 2^14 2 Vmax s_dS <= 2^15 < 65504).
+// Rows past the valid count get zeros.  gscal[2] = s_dO, gscal[3] = s_dS.
 __global__ void do_to_f16_delta_kernel(const float* __restrict__ dO, int64_t ld, const bf16* __restrict__ o,
-                                       int64_t ldo, __half* __restrict__ dO16, int64_t ld16,
+                                       const bf16* __restrict__ o_lo, int64_t ldo, __half* __restrict__ dO16,
+                                       int64_t ld16,
                                        float* __restrict__ delta, int64_t delta_ld, int T, int H, int s0,
                                        const int32_t* __restrict__ n_valid, int valid_mult,
                                        float* __restrict__ gscal) {
   const int nv = valid_rows(n_valid, valid_mult, s0, T);
   const float dmax = __uint_as_float(reinterpret_cast<const unsigned int*>(gscal)[1]);
   const float vmax = __uint_as_float(reinterpret_cast<const unsigned int*>(gscal)[0]);
-  const float s_dO = (dmax > 0.f && dmax < INFINITY) ? 1.f / exp2f(ceilf(log2f(dmax))) : 1.f;
-  const float s_dS = (vmax > 0.f && vmax < INFINITY) ? fminf(pow2_floor(16384.f / vmax), 0x1p60f) : 1.f;
+  // dO's largest per-head row norm (and so every element) scaled to at most 2^14: fp16's range
+  // above 1 holds the rows with large gradients, and ordinary rows stay far from the subnormal
+  // range (a scale to norm <= 1 put their elements near 2^-14 when a few rows dominated)
+  const float s_dO = (dmax > 0.f && dmax < INFINITY) ? exp2f(14.f - ceilf(log2f(dmax))) : 1.f;
+  // |dS| <= |dP - Delta| = |dO16_i . (v_j - o_i)| <= 2^14 * 2 Vmax, so 2^15 / (2^15 Vmax) keeps
+  // |dS s_dS| <= 2^15 < 65504
+  const float s_dS = (vmax > 0.f && vmax < INFINITY) ? fminf(pow2_floor(1.f / vmax), 0x1p60f) : 1.f;
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     gscal[2] = s_dO;
     gscal[3] = s_dS;
@@ -539,7 +546,13 @@ __global__ void do_to_f16_delta_kernel(const float* __restrict__ dO, int64_t ld,
       packed = make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
       const uint2 ob = *reinterpret_cast<const uint2*>(o + (int64_t)(s0 + r) * ldo + c);
       const __nv_bfloat162* op = reinterpret_cast<const __nv_bfloat162*>(&ob);
-      const float2 o01 = __bfloat1622float2(op[0]), o23 = __bfloat1622float2(op[1]);
+      float2 o01 = __bfloat1622float2(op[0]), o23 = __bfloat1622float2(op[1]);
+      if (o_lo) {  // o = hi + lo (the forward's rounding residual)
+        const uint2 lb = *reinterpret_cast<const uint2*>(o_lo + (int64_t)(s0 + r) * ldo + c);
+        const __nv_bfloat162* lp = reinterpret_cast<const __nv_bfloat162*>(&lb);
+        const float2 l01 = __bfloat1622float2(lp[0]), l23 = __bfloat1622float2(lp[1]);
+        o01.x += l01.x; o01.y += l01.y; o23.x += l23.x; o23.y += l23.y;
+      }
       const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
       d = f01.x * o01.x + f01.y * o01.y + f23.x * o23.x + f23.y * o23.y;
     }

@@ -14,7 +14,8 @@
 // integrated with the attention computation, memory linear in S: Jenga notes §4.3).
 //
 // Persistent grid (at most one CTA per SM, a fixed scratch slot per CTA); work items are
-// (128-query tile, head, sequence), longest first, dealt to the CTAs in snake order.  Per CTA,
+// (128-query tile, head, sequence), head-major with the longest query tiles of each head first,
+// dealt to the CTAs in snake order.  Per CTA,
 // 608 threads:
 //   warp 0       TMA: the item's first key-tile pairs, then (once the previous item's MMAs are
 //                done) its query tile, then the remaining key pairs through a 3-stage ring
@@ -190,9 +191,13 @@ __global__ void __launch_bounds__(SF_THREADS, 1)
     const int G = (int)gridDim.x;
     return r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
   };
+  // items in (sequence, head)-major order, query tiles longest first within each head: the
+  // ~148 items in flight at a time belong to one or two heads, so their key tiles stay in L2
+  // (an order that interleaved heads had every head's keys in flight and read them from DRAM
+  // again for each query tile)
   auto decode = [&](int u, int& t, int& h, int& b) {
-    t = nt - 1 - u / HB;
-    const int hb = u % HB;
+    const int hb = u / nt;
+    t = nt - 1 - u % nt;
     h = hb % H;
     b = hb / H;
   };
