@@ -113,9 +113,9 @@ def work_model(case, ks, seg, scoring="exact"):
 # dram__bytes_write.sum; the capture and its command are in profiles/).  attn_bwd_dkdv_tc:
 # its traffic is dominated by the fp32 dK / dV accumulators (read and written back by the
 # L2's reduce-adds) and the K / V reads, both proportional to the keys [0, segment end) a
-# launch covers, so the unit is a key row; captured on llama7b_s16k (one launch over 4096
-# keys: 269.6 MB read + 85.9 MB written).
-TRAFFIC_PER_UNIT = {"attn_bwd_dkdv_tc": ("key row", (269.571584e6 + 85.910528e6) / 4096)}
+# launch covers, so the unit is a key row; captured on one 7B-shaped layer at S = 16384, keep
+# 50 % (the launch of the backward segment over keys 0 .. 8191: 470.9 MB read + 213.5 MB written).
+TRAFFIC_PER_UNIT = {"attn_bwd_dkdv_tc": ("key row", (470.904832e6 + 213.455360e6) / 8192)}
 
 
 def traffic_units(name, case, ks, seg):

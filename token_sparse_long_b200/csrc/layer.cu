@@ -613,6 +613,8 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
   JENGA_CUDA_TRY(cudaMemsetAsync(b.dk_acc, 0, (size_t)nc * HD * sizeof(float), st));
   JENGA_CUDA_TRY(cudaMemsetAsync(b.dv_acc, 0, (size_t)nc * HD * sizeof(float), st));
   // fp16 operands of the attention backward: q | k | v copies and the largest per-head v norm
+  if ((int64_t)nc * (3 * HD / 8) >= (int64_t)1 << 31)
+    return fail(JENGA_EUNSUPPORTED, "jenga_sparse_layer_bwd: retained rows x 3 H D too large");
   JENGA_CUDA_TRY(cudaMemsetAsync(b.gscal, 0, 4 * sizeof(float), st));
   {
     const int _ps = ::jenga::prof_begin("qkv_to_f16", st);

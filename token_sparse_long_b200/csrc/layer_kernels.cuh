@@ -453,10 +453,11 @@ __global__ void zero_bf16_kernel(bf16* __restrict__ dst, int64_t n) {
 // max-reduced into gscal[0].
 __global__ void qkv_to_f16_kernel(const bf16* __restrict__ in, int64_t ldi, __half* __restrict__ out, int64_t ldo,
                                   int rows, int cols, int vnorm_col0, unsigned int* __restrict__ gmax) {
-  const int vpr = cols / 8;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < (int64_t)rows * vpr;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int r = (int)(e / vpr), c = (int)(e - (int64_t)r * vpr) * 8;
+  // rows x (cols / 8) < 2^31 (checked by the caller): 32-bit index arithmetic
+  const unsigned vpr = (unsigned)cols / 8u;
+  const unsigned total = (unsigned)rows * vpr;
+  for (unsigned e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
+    const unsigned r = e / vpr, c = (e - r * vpr) * 8u;
     float f[8];
     unpack8(*reinterpret_cast<const uint4*>(in + (int64_t)r * ldi + c), f);
     uint4 o;
@@ -469,21 +470,29 @@ __global__ void qkv_to_f16_kernel(const bf16* __restrict__ in, int64_t ldi, __ha
     *reinterpret_cast<uint4*>(out + (int64_t)r * ldo + c) = o;
   }
   if (vnorm_col0 < 0) return;
-  // per (row, v head): one warp sums the squares of the head's 128 values
+  // per (row, v head): one warp sums the squares of the head's 128 values; the maxima are
+  // reduced over the warp's rows, then over the block, then one atomicMax per block
   const int H = (cols - vnorm_col0) / 128;
   const int lane = threadIdx.x & 31;
-  for (int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < (int64_t)rows * H;
-       w += ((int64_t)gridDim.x * blockDim.x) >> 5) {
-    const int r = (int)(w / H), hh = (int)(w - (int64_t)r * H);
-    float f[4];
+  const unsigned nw = (unsigned)rows * (unsigned)H;
+  float best = 0.f;
+  for (unsigned w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < nw; w += (gridDim.x * blockDim.x) >> 5) {
+    const unsigned r = w / (unsigned)H, hh = w - r * (unsigned)H;
     const uint2 u = *reinterpret_cast<const uint2*>(in + (int64_t)r * ldi + vnorm_col0 + hh * 128 + lane * 4);
     const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u);
     const float2 a = __bfloat1622float2(p2[0]), b = __bfloat1622float2(p2[1]);
-    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
-    float ss = f[0] * f[0] + f[1] * f[1] + f[2] * f[2] + f[3] * f[3];
+    float ss = a.x * a.x + a.y * a.y + b.x * b.x + b.y * b.y;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) atomicMax(gmax, __float_as_uint(sqrtf(ss)));  // non-negative: bit order = value order
+    best = fmaxf(best, ss);
+  }
+  __shared__ float wmax[32];
+  if (lane == 0) wmax[threadIdx.x >> 5] = best;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.f;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) m = fmaxf(m, wmax[i]);
+    if (m > 0.f) atomicMax(gmax, __float_as_uint(sqrtf(m)));  // non-negative: bit order = value order
   }
 }
 
@@ -493,14 +502,24 @@ __global__ void do_norm_max_kernel(const float* __restrict__ dO, int64_t ld, int
                                    unsigned int* __restrict__ gscal_bits) {
   const int nv = valid_rows(n_valid, valid_mult, s0, T);
   const int lane = threadIdx.x & 31;
-  for (int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < (int64_t)nv * H;
-       w += ((int64_t)gridDim.x * blockDim.x) >> 5) {
-    const int r = (int)(w / H), hh = (int)(w - (int64_t)r * H);
+  const unsigned nw = (unsigned)nv * (unsigned)H;
+  float best = 0.f;
+  for (unsigned w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < nw; w += (gridDim.x * blockDim.x) >> 5) {
+    const unsigned r = w / (unsigned)H, hh = w - r * (unsigned)H;
     const float4 v = *reinterpret_cast<const float4*>(dO + (int64_t)r * ld + hh * 128 + lane * 4);
     float ss = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) atomicMax(gscal_bits + 1, __float_as_uint(sqrtf(ss)));
+    best = fmaxf(best, ss);
+  }
+  // one atomicMax per block (the warps' maxima reduced in shared memory first)
+  __shared__ float wmax[32];
+  if (lane == 0) wmax[threadIdx.x >> 5] = best;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.f;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) m = fmaxf(m, wmax[i]);
+    if (m > 0.f) atomicMax(gscal_bits + 1, __float_as_uint(sqrtf(m)));
   }
 }
 

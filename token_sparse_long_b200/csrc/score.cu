@@ -179,7 +179,7 @@ using namespace jenga;
 static int score_chunk(int blk) { return blk % 64 == 0 ? 64 : (blk % 32 == 0 ? 32 : 0); }
 
 struct ScoreWs {  // byte offsets of the bf16 path's workspace regions
-  size_t lse, part, scratch, total;
+  size_t lse, part, counter, scratch, total;
   int grid;
 };
 
@@ -197,7 +197,8 @@ static ScoreWs score_ws_layout(int B, int S, int H, int blk) {
   w.grid = (int)(n_items < SF_GRID_CAP ? n_items : SF_GRID_CAP);
   w.lse = 0;
   w.part = align256((size_t)B * H * S * sizeof(float));
-  w.scratch = w.part + align256((size_t)B * H * nt * nt * (SF_ROWS / ch) * sizeof(float));
+  w.counter = w.part + align256((size_t)B * H * nt * nt * (SF_ROWS / ch) * sizeof(float));
+  w.scratch = w.counter + 256;
   w.total = w.scratch + (size_t)w.grid * sf_scratch_floats_per_cta(nt, ch) * sizeof(float);
   return w;
 }
@@ -308,6 +309,8 @@ extern "C" jenga_status jenga_score_blocks(const void* q, int64_t ldq, const voi
     float* neg_lse = (float*)(base + w.lse);
     float* part = (float*)(base + w.part);
     float* scratch = (float*)(base + w.scratch);
+    unsigned int* counter = (unsigned int*)(base + w.counter);
+    JENGA_CUDA_TRY(cudaMemsetAsync(counter, 0, sizeof(unsigned int), st));
     CUtensorMap tq, tk;
     jenga_status s1 = make_tmap_bf16(&tq, q, (uint64_t)B * S, (uint64_t)H * D, ldq, SF_ROWS);
     if (s1 != JENGA_OK) return s1;
@@ -322,12 +325,12 @@ extern "C" jenga_status jenga_score_blocks(const void* q, int64_t ldq, const voi
         JENGA_CUDA_TRY(
             cudaFuncSetAttribute(score_fused_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, SF_SMEM));
         score_fused_tc_kernel<64><<<grid, SF_THREADS, SF_SMEM, st>>>(tq, tk, S, H, B, causal ? 1 : 0, sl2, neg_lse,
-                                                                     part, scratch);
+                                                                     part, scratch, counter);
       } else {
         JENGA_CUDA_TRY(
             cudaFuncSetAttribute(score_fused_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, SF_SMEM));
         score_fused_tc_kernel<32><<<grid, SF_THREADS, SF_SMEM, st>>>(tq, tk, S, H, B, causal ? 1 : 0, sl2, neg_lse,
-                                                                     part, scratch);
+                                                                     part, scratch, counter);
       }
       ::jenga::prof_end(_ps, st);
     }

@@ -15,7 +15,7 @@
 //
 // Persistent grid (at most one CTA per SM, a fixed scratch slot per CTA); work items are
 // (128-query tile, head, sequence), head-major with the longest query tiles of each head first,
-// dealt to the CTAs in snake order.  Per CTA,
+// taken from a global counter as CTAs become free.  Per CTA,
 // 608 threads:
 //   warp 0       TMA: the item's first key-tile pairs, then (once the previous item's MMAs are
 //                done) its query tile, then the remaining key pairs through a 3-stage ring
@@ -140,7 +140,8 @@ template <int CH>
 __global__ void __launch_bounds__(SF_THREADS, 1)
     score_fused_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, int S,
                           int H, int B, int causal, float sl2, float* __restrict__ neg_lse,
-                          float* __restrict__ part, float* __restrict__ scratch) {
+                          float* __restrict__ part, float* __restrict__ scratch,
+                          unsigned int* __restrict__ work_counter) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* fix = smem;
@@ -152,7 +153,10 @@ __global__ void __launch_bounds__(SF_THREADS, 1)
   uint64_t* s_empty = s_full + 2;        // [2]
   uint64_t* fix_full = s_empty + 2;
   uint64_t* fix_empty = fix_full + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(fix_empty + 1);
+  uint64_t* item_full = fix_empty + 1;   // [4] work-item queue: slot written
+  uint64_t* item_empty = item_full + 4;  // [4] ... and read by every consumer
+  int* item_q = reinterpret_cast<int*>(item_empty + 4);  // [4]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(item_q + 4);
   float* Lsm = reinterpret_cast<float*>(smem + SF_L_OFF);
 
   constexpr int CPT = SF_ROWS / CH;  // chunks per key tile
@@ -175,6 +179,10 @@ __global__ void __launch_bounds__(SF_THREADS, 1)
     }
     mbar_init(fix_full, 1);
     mbar_init(fix_empty, 2);
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(&item_full[s], 1);
+      mbar_init(&item_empty[s], 2 + SF_EPI_WARPS);  // the two issuing threads and the epilogue warps
+    }
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -186,10 +194,13 @@ __global__ void __launch_bounds__(SF_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  // item r of this CTA: snake order over the longest-first list
-  auto item_of = [&](int r) -> int {
-    const int G = (int)gridDim.x;
-    return r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+  // Work items are taken from a global counter (dynamic balance: a CTA that finishes early
+  // takes the next item); the producer thread fetches item r and publishes it in queue slot
+  // r % 4 for the issuing and epilogue warps.  Item numbers >= n_items end every role's loop.
+  auto take_item = [&](int r, int& u) -> bool {  // the consumers' read of slot r % 4
+    if (!mbar_wait(&item_full[r & 3], (uint32_t)((r >> 2) & 1), SITE_SCORE_TC)) return false;
+    u = item_q[r & 3];
+    return true;
   };
   // items in (sequence, head)-major order, query tiles longest first within each head: the
   // ~148 items in flight at a time belong to one or two heads, so their key tiles stay in L2
@@ -208,7 +219,10 @@ __global__ void __launch_bounds__(SF_THREADS, 1)
     bool ok = true;
     long P = 0;  // key pairs streamed so far
     for (int r = 0; ok; ++r) {
-      const int u = item_of(r);
+      if (r >= 4 && !mbar_wait(&item_empty[r & 3], (uint32_t)(((r >> 2) - 1) & 1), SITE_SCORE_TC)) break;
+      const int u = (int)atomicAdd(work_counter, 1u);
+      item_q[r & 3] = u;
+      mbar_arrive(&item_full[r & 3]);
       if (u >= n_items) break;
       int t, h, b;
       decode(u, t, h, b);
@@ -249,7 +263,9 @@ __global__ void __launch_bounds__(SF_THREADS, 1)
     bool ok = true;
     long P = 0;
     for (int r = 0; ok; ++r) {
-      const int u = item_of(r);
+      int u;
+      if (!take_item(r, u)) break;
+      mbar_arrive(&item_empty[r & 3]);
       if (u >= n_items) break;
       int t, h, b;
       decode(u, t, h, b);
@@ -293,7 +309,12 @@ __global__ void __launch_bounds__(SF_THREADS, 1)
     bool ok = true;
     long P = 0;
     for (int it = 0;; ++it) {
-      const int u = item_of(it);
+      int u = 0;
+      const bool got = __all_sync(0xffffffffu, take_item(it, u));
+      __syncwarp();
+      if (got && lane == 0) mbar_arrive(&item_empty[it & 3]);
+      // all epilogue warps leave together (they meet at named barriers inside the item)
+      if (!bar_and(got && ok, 1, 32 * SF_EPI_WARPS)) break;
       if (u >= n_items) break;
       int t, h, b;
       decode(u, t, h, b);
