@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-movement", action="store_true", help="skip the standalone gather/scatter/select timing")
     ap.add_argument("--no-lm-loss", action="store_true", help="skip the segmented LM-head loss timing")
+    ap.add_argument("--oracle-one-thread", action="store_true",
+                    help="time the CPU oracle on one thread over the two small workloads, in full, and exit")
     return ap.parse_args()
 
 
@@ -96,7 +98,6 @@ def work_model(case, ks, seg, scoring="exact"):
         add("gemm_o_scatter", "flop", 2.0 * n * h * HD)
         add("gemm_gateup_swiglu", "flop", 2.0 * n * 2 * F * h)
         add("gemm_down_scatter", "flop", 2.0 * n * h * F)
-        add("gemm_gateup_recompute", "flop", 2.0 * n * 2 * F * h)
         add("gemm_da_swiglu_bwd", "flop", 2.0 * n * F * h)
         add("gemm_dhn", "flop", 2.0 * n * h * 2 * F)
         add("gemm_do", "flop", 2.0 * n * HD * h)
@@ -415,8 +416,42 @@ def replica_tokens_per_s(S, world, ms):
     return S * world / (ms / 1e3)
 
 
+def oracle_one_thread():
+    """The CPU oracle on one host thread, each small workload in full: ``score_fp32`` (S 512,
+    4 heads x 64, blocks of 32: fp32 block scores, mean-threshold selection, gather, scatter-add
+    of 2 x the gathered rows) and ``llama7b_s4k`` (one 7B-shaped layer at S 4096, blocks of 64,
+    keep 50 %: q/k of all rows, block scores, top-k selection, retained-token forward and
+    backward).  Inputs and oracle weights are built before the clock starts."""
+    from threadpoolctl import threadpool_limits
+    from oracle import movement as omv
+    from oracle import scores as osc
+    from oracle import select as osel
+    out = {}
+    with threadpool_limits(1):
+        c = synth.gen_score_case(0)
+        q = c.q.reshape(c.S, c.H, c.D).astype(np.float64)
+        k = c.k.reshape(c.S, c.H, c.D).astype(np.float64)
+        x = c.x.astype(np.float64)
+        t0 = time.perf_counter()
+        sc = osc.block_scores_softmax_mass(q, k, c.blk)
+        (idx, n, _), _ = osel.select_mean_ge(sc)
+        xg = omv.gather(x, idx, n, c.blk)
+        omv.scatter_add(x, xg, idx, n, c.blk, 2.0, "f32")
+        dt = time.perf_counter() - t0
+        out["score_fp32"] = {"seconds": dt, "tokens_per_s": c.S / dt, "kept_blocks": int(n)}
+        w = synth.WORKLOADS["llama7b_s4k"]
+        case = synth.gen_workload("llama7b_s4k", seed=0)
+        Ws = oracle_weights(case)
+        dt, flops = oracle_sample(case, case.S, list(w.keep), Ws)
+        out["llama7b_s4k"] = {"seconds": dt, "tokens_per_s": case.S / dt, "gflop": flops / 1e9}
+    print(json.dumps({"oracle_one_thread": out, "threads": 1}), flush=True)
+
+
 def main():
     args = parse()
+    if args.oracle_one_thread:
+        oracle_one_thread()
+        return
     if args.impl == "reference":
         run_reference(args)
         return

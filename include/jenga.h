@@ -188,7 +188,8 @@ JENGA_API jenga_status jenga_scale_rows(void* x, int64_t ldx, int B, int S, int 
  * run only on the retained rows (Jenga summary §4.1, §4.4.1).  bf16 storage, fp32
  * accumulation.  RoPE uses each token's ORIGINAL position (rotate-half, pairs d and
  * d + D/2, angle pos * theta^(-2i/D)); attention is causal among retained tokens.
- * head_dim must be 128, hidden and ffn multiples of 128, lora rank 16. */
+ * head_dim must be 128, heads at most 64 with heads * 128 a multiple of 256, hidden a
+ * multiple of 256 up to 8192, ffn a multiple of 256, lora rank 16. */
 typedef struct jenga_layer_weights {
   int hidden, heads, head_dim, ffn;
   float rms_eps, rope_theta;
@@ -220,7 +221,14 @@ typedef struct jenga_lora_grads { /* fp32, ACCUMULATED into (+=) */
 } jenga_lora_grads;
 
 /* Packed (re-laid-out) copies of the frozen weights the kernels read: fused QKV,
- * gate/up interleaved in 64-row groups, and the transposes the backward needs.
+ * gate/up interleaved in 64-row groups, and the transposes the backward needs.  The
+ * backward's copies (the transposes of Wo, Wq | Wk | Wv and [Wg; Wu], and of the LoRA
+ * matrices) are fp16, because the backward products run on fp16 operands: a weight whose
+ * magnitude exceeds 65504 (fp16's largest finite value) makes jenga_check_device_status
+ * report JENGA_EINVAL (site 9, detail = element index).  The LoRA matrices are read at pack
+ * time: pack again after changing them.  The LoRA operand of the dX product is divided by
+ * a power of two chosen here from Bq, Bv and lora->scale, which keeps it in fp16's range
+ * for a backward LoRA scale up to max(lora->scale, 1).
  * Built once per layer with jenga_layer_pack; read-only afterwards. */
 JENGA_API size_t jenga_layer_pack_bytes(const jenga_layer_weights* w, const jenga_lora* lora);
 JENGA_API jenga_status jenga_layer_pack(const jenga_layer_weights* w, const jenga_lora* lora, void* packed,
@@ -237,7 +245,11 @@ JENGA_API jenga_status jenga_layer_score_qk(const jenga_layer_weights* w, const 
 /* jenga_sparse_layer_fwd -- a5 + a6 + a7: the layer on the kept blocks of x, in place.
  *   x      : [B, S, hidden] bf16, updated in place on retained rows only.
  *   idx, n_kept : from jenga_select; n_kept_max: host bound on every n_kept[b].
- *   saved  : jenga_layer_saved_bytes(...) bytes; written here, read by the backward.
+ *   saved  : jenga_layer_saved_bytes(...) bytes; written here, read by the backward.  It
+ *            holds, per retained row, the gathered input, q | k | v, the attention output,
+ *            the residual h, the MLP pre-activations (gate, up) in fp16 (so the backward
+ *            does not recompute them; a pre-activation above 65504 in magnitude becomes
+ *            infinite there), the LoRA down-projections and the row statistics.
  *   ws     : jenga_layer_fwd_workspace_bytes(...) bytes of scratch. */
 JENGA_API size_t jenga_layer_saved_bytes(const jenga_layer_weights* w, int B, int blk, int n_kept_max);
 JENGA_API size_t jenga_layer_fwd_workspace_bytes(const jenga_layer_weights* w, int B, int blk, int n_kept_max);
@@ -268,8 +280,8 @@ JENGA_API jenga_status jenga_sparse_layer_fwd_qk(const jenga_layer_weights* w, c
  * (TOPK_FRAC: a fraction of n_kept_max; TOPK: a count; ABS_GE: a threshold), and the down
  * projection and its in-place residual add run only on those blocks; on the other retained
  * blocks the layer output is h, the attention sub-block's output.  The keep mask is stored in
- * `saved`, and jenga_sparse_layer_bwd then runs the MLP backward (gate / up recompute, SwiGLU
- * backward, the dhn GEMM) only on the kept blocks and passes the upstream gradient straight
+ * `saved`, and jenga_sparse_layer_bwd then runs the MLP backward (the dA GEMM with the SwiGLU
+ * derivative, the dhn GEMM) only on the kept blocks and passes the upstream gradient straight
  * through the MLP branch of the others.
  *   mlp_scores : [n_kept_max] fp32 out (nullable): the criterion per retained position
  *             (-inf at and past the device count n_kept);

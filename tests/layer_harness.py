@@ -208,8 +208,10 @@ def smoke_check():
     print("smoke ok: n_kept", gpu["n_kept"], "of", case.S // case.blk, "blocks")
 
 
-def split_saved(saved, nc, h, H, D=128, r=16):
-    """View the saved-context buffer as its parts (layout of the library's forward)."""
+def split_saved(saved, nc, h, H, D=128, r=16, F=None):
+    """View the saved-context buffer as its parts (layout of the library's forward); with
+    the FFN width F also the MLP keep mask, o's rounding residual and the fp16 (gate, up)
+    pre-activations (interleaved in groups of 64: g 0..63, u 0..63, g 64..127, ...)."""
     buf = saved
     off = 0
     out = {}
@@ -217,7 +219,7 @@ def split_saved(saved, nc, h, H, D=128, r=16):
     def take(name, n, dtype, shape):
         nonlocal off
         off = (off + 255) // 256 * 256
-        nbytes = n * (2 if dtype == torch.bfloat16 else 4)
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
         out[name] = buf[off:off + nbytes].view(dtype).reshape(shape)
         off += nbytes
 
@@ -230,7 +232,18 @@ def split_saved(saved, nc, h, H, D=128, r=16):
     take("lse", H * nc, torch.float32, (H, nc))  # negated row log-sum-exp, log2 units
     take("rstd1", nc, torch.float32, (nc,))
     take("rstd2", nc, torch.float32, (nc,))
+    if F is not None:
+        take("mlp_mask", max(nc, 1), torch.uint8, (max(nc, 1),))
+        take("olo", nc * HD, torch.bfloat16, (nc, HD))
+        take("gu", nc * 2 * F, torch.float16, (nc, 2 * F))
     return out
+
+
+def deinterleave_gu(gu, F):
+    """(g, u) [n, F] each from the interleaved [n, 2F] gate/up layout (groups of 64)."""
+    n = gu.shape[0]
+    v = gu.reshape(n, F // 64, 2, 64)
+    return v[:, :, 0, :].reshape(n, F), v[:, :, 1, :].reshape(n, F)
 
 
 def bf16_ulp(v):

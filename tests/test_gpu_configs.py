@@ -34,8 +34,8 @@ from oracle import predictor as opred
 from oracle import select as osel
 from oracle.bf16 import from_bits, round_bf16
 from tests.layer_harness import (check_layer_against_oracle, check_qk_all, check_scores, check_topk_selection,
-                                 layer_handle, oracle_layer, oracle_qk_all, bits_to_torch, rel_max, rel_max_ulp,
-                                 torch_to_f64)
+                                 layer_handle, oracle_layer, oracle_qk_all, bits_to_torch, bf16_ulp, rel_max,
+                                 rel_max_ulp, torch_to_f64)
 from tests.oracle_pool import oracle_pool
 from oracle import scores as osc
 
@@ -159,6 +159,13 @@ def test_llama7b_x4_s32k_chain(J, pmap):
     J.jenga_check_device_status()
     torch.cuda.synchronize()
     del saved
+    # the in-place salient scaling between layers: bit-exact against its definition (the
+    # per-layer checks below start from the GPU's scaled input, so this pins the step between)
+    for l in range(1, 4):
+        want = torch_to_f64(outs[l - 1])
+        sl = case.salient[l]
+        want[sl] = round_bf16(want[sl] * case.salient_scale)
+        assert np.array_equal(torch_to_f64(ins[l]), want), f"salient scaling before layer {l}"
     for l in range(4):
         g_sc, idx, nk, k = sels[l]
         x_in = torch_to_f64(ins[l])
@@ -187,9 +194,18 @@ def test_llama7b_x4_s32k_chain(J, pmap):
             Xc[case.salient[l]] = round_bf16(Xc[case.salient[l]] * case.salient_scale)
         W = oly.Weights.from_bits(case.layers[l], sh)
         Xc, _ = oly.sparse_layer_fwd(Xc, sels[l][1].cpu().numpy(), sels[l][3], blk, W, rnd=True, pmap=pmap)
-    e_chain = rel_max_ulp(torch_to_f64(outs[3]), Xc)
-    print(f"four-layer chained forward (oracle on its own outputs, GPU kept blocks): {e_chain:.3g}")
-    assert e_chain < 3e-2
+    g3 = torch_to_f64(outs[3])
+    e_chain = rel_max_ulp(g3, Xc)
+    # per row against the row's own rms: the x3 scaling of the salient rows before layers 1-3
+    # multiplies the error an earlier layer left in such a row along with the row (a row
+    # salient in three layers carries 27x its layer-0 error), which the whole-tensor measure
+    # above then compares with the rms of all rows; per row the scaling cancels
+    ex = np.maximum(np.abs(g3 - Xc) - bf16_ulp(Xc), 0.0)
+    e_rows = float((ex.max(axis=1) / np.sqrt((Xc * Xc).mean(axis=1))).max())
+    print(f"four-layer chained forward (oracle on its own outputs, GPU kept blocks): {e_chain:.3g} of the "
+          f"output rms, {e_rows:.3g} per row of the row's rms")
+    # four layers, each within 3e-2, errors adding along the residual stream
+    assert e_rows < 4 * 3e-2
 
 
 # ------------------------------------------------------------------ llama13b_pred_s32k

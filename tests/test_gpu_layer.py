@@ -219,3 +219,28 @@ def test_mlp_elimination_against_oracle(J, S, blk, keep, mlp_keep, seg):
     h_gpu = torch_to_f64(parts["h"])[: nk * blk]
     assert np.array_equal(out[rows][drop], h_gpu[drop])
     assert drop.any() and (~drop).any()
+
+
+def test_pack_reports_weight_outside_fp16_range(J):
+    """The backward's weight copies are fp16: a frozen weight beyond fp16's largest finite
+    value (65504) is reported through the device status (JENGA_EINVAL) at pack time, and the
+    status word is cleared by the read."""
+    from token_sparse_long_b200 import LayerHandle
+    from tests.layer_harness import bits_to_torch
+    case = small_case(seed=3)
+    sh, p = case.shape, case.layers[0]
+    t = {k: bits_to_torch(getattr(p, k)) for k in ("wq", "wk", "wv", "wo", "wg", "wu", "wd", "attn_norm",
+                                                    "mlp_norm", "aq", "bq", "av", "bv")}
+    J.jenga_check_device_status()
+    LayerHandle(**t, heads=sh.heads, head_dim=sh.head_dim, rms_eps=sh.rms_eps, rope_theta=sh.rope_theta,
+                lora_scale=sh.lora_scale)
+    torch.cuda.synchronize()
+    J.jenga_check_device_status()  # in range: no error
+    t["wo"][1, 2] = 1.0e5
+    LayerHandle(**t, heads=sh.heads, head_dim=sh.head_dim, rms_eps=sh.rms_eps, rope_theta=sh.rope_theta,
+                lora_scale=sh.lora_scale)
+    torch.cuda.synchronize()
+    with pytest.raises(J._lib.JengaError) as ei:
+        J.jenga_check_device_status()
+    assert ei.value.status == 1  # JENGA_EINVAL
+    J.jenga_check_device_status()  # cleared by the read

@@ -1,14 +1,15 @@
 """Per-step GPU parity of the layer forward: each saved intermediate (gathered x,
-q/k/v after RoPE, LoRA t, attention output and its log-sum-exp, h) against the
-oracle's value of the same step, so that a fault is pinned to the step that makes it."""
+q/k/v after RoPE, LoRA t, attention output and its log-sum-exp, h, the MLP pre-activations)
+against the oracle's value of the same step, so that a fault is pinned to the step that
+makes it."""
 import numpy as np
 import pytest
 import torch
 
 from oracle import layer as oly
 from oracle.bf16 import from_bits
-from tests.layer_harness import (bits_to_torch, layer_handle, rel_delta_ulp, rel_max, rel_max_ulp, small_case,
-                                 split_saved, torch_to_f64)
+from tests.layer_harness import (bits_to_torch, deinterleave_gu, layer_handle, rel_delta_ulp, rel_max, rel_max_ulp,
+                                 small_case, split_saved, torch_to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,7 +38,7 @@ def test_forward_intermediates(J, keep_blocks):
     saved = J.jenga_sparse_layer_fwd(L, x, idx, nk, case.blk, kmax)
     J.jenga_check_device_status()
     nc = kmax * case.blk
-    parts = split_saved(saved, nc, sh.hidden, sh.heads)
+    parts = split_saved(saved, nc, sh.hidden, sh.heads, F=sh.ffn)
     W = oly.Weights.from_bits(case.layers[0], sh)
     rows = (np.asarray(keep_blocks)[:, None] * case.blk + np.arange(case.blk)[None]).reshape(-1)
     X = from_bits(case.x)
@@ -56,6 +57,13 @@ def test_forward_intermediates(J, keep_blocks):
     errs["o"] = rel_max_ulp(torch_to_f64(parts["o"]), ctx["o"].reshape(nc, HD))
     errs["h"] = rel_delta_ulp(torch_to_f64(parts["h"]), ctx["h"], X[rows])
     errs["out"] = rel_delta_ulp(torch_to_f64(x)[rows], out, X[rows])
+    # the saved (gate, up) pre-activations: fp16 storage of the fp32-accumulated products
+    g16, u16 = deinterleave_gu(parts["gu"].cpu().double().numpy(), sh.ffn)
+    errs["g"] = rel_max(g16, ctx["gt"])
+    errs["u"] = rel_max(u16, ctx["ut"])
+    assert (parts["mlp_mask"][:kmax].cpu().numpy() == 1).all()
     print(errs)
     for k, v in errs.items():
         assert v < 3e-2, (k, errs)
+    # g and u are one fp16 rounding (2^-11 relative) plus fp32 accumulation away from the oracle
+    assert errs["g"] < 2e-3 and errs["u"] < 2e-3, errs

@@ -58,6 +58,7 @@ enum ErrSite : unsigned int {
   SITE_NKEPT_RANGE = 6,
   SITE_ATTN = 7,
   SITE_TEST_WAIT = 8,
+  SITE_PACK_RANGE = 9,  // a weight outside fp16's range at pack time (detail: element index)
 };
 
 __device__ __forceinline__ void record_device_error(unsigned code, unsigned site, unsigned detail) {

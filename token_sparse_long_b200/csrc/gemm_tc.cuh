@@ -4,8 +4,9 @@
 //
 // All operands are K-major (row-major [rows, K]).  The optional second and third
 // operand pairs extend the reduction: they fold the LoRA up-projection into the QKV
-// projection, carry the low half of a bf16 hi + lo split operand, and fold the LoRA
-// down-projection's input gradient into the dX GEMM.
+// projection and the LoRA down-projection's input gradient into the dX GEMM.  A
+// gradient operand enters as fp16 rows scaled by powers of two into fp16's range; the
+// epilogue multiplies each output row by the inverse scale (EpiParams::row_scale).
 //
 // Structure: persistent, one CTA per SM walking the 128 x BN output tiles in a fixed
 // stride (tile = blockIdx.x, + gridDim.x, ...; N tiles fastest), 192 threads:
@@ -37,11 +38,14 @@ enum GemmEpi : int {
   EPI_STORE_BF16 = 0,   // out[m, n] = bf16(acc * alpha)
   EPI_STORE_F32 = 1,    // out[m, n] = acc * alpha (fp32)
   EPI_SCATTER_ADD = 2,  // x[row(m), n] = bf16(x + acc); aux[m, n] = same value (optional)
-  EPI_SWIGLU = 3,       // 64-col groups (gate, up) -> out[m, n/2 + j] = bf16(silu(g) * u)
+  EPI_SWIGLU = 3,       // 64-col groups (gate, up) -> out[m, n/2 + j] = bf16(silu(g) * u);
+                        // with aux: (g, u) also stored fp16 in the interleaved layout
   EPI_QKV_ROPE = 4,     // q/k/v sections of width hd; RoPE(pos(m)) on q and k -> bf16
-  EPI_SWIGLU_BWD = 5,   // acc = dA; aux = (g, u) interleaved fp32 -> out = (dg, du) interleaved fp16
-  EPI_LORA_T = 6,       // out fp32 [m, 0:N] = beta * acc ; aux bf16 [m, 0:64] = (hi, lo) of alpha * acc:
-                        // cols 0..N-1 bf16(alpha acc), cols 32..32+N-1 bf16(alpha acc - hi), else 0
+  EPI_SWIGLU_BWD = 5,   // acc = dA; aux = (g, u) interleaved fp32 (fp16 with aux_f16) -> out = (dg, du)
+                        // interleaved fp16
+  EPI_LORA_T = 6,       // out fp32 [m, 0:N] = beta * acc (* row factor) ; aux [m, 0:64] = (hi, lo) of
+                        // a = alpha * acc (/ *aux_div): cols 0..N-1 round(a), cols 32..32+N-1
+                        // round(a - hi), else 0 (bf16, or fp16 with aux_f16)
 };
 
 struct EpiParams {
@@ -69,6 +73,12 @@ struct EpiParams {
   // no stores), and the scatter-add epilogue leaves the rows of masked blocks untouched
   const uint8_t* blk_mask = nullptr;
   int mask_blk = 1;
+  // STORE_F32, LORA_T: optional per-row factor of the accumulator (local row m), the inverse
+  // power-of-two scale of an fp16 A operand whose rows were scaled into fp16's range
+  const float* row_scale = nullptr;
+  // LORA_T: the aux copy is fp16 (else bf16) and is divided by *aux_div (device scalar)
+  bool aux_f16 = false;
+  const float* aux_div = nullptr;
 };
 
 // Does the 128-row tile at local row m0 hold a row of a kept block (always, without a mask)?
@@ -331,8 +341,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     {
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * (BN < 32 ? 32 : BN);
       const bool row_ok = m < valid;
+      const float rfac = (EPI == EPI_STORE_F32 || EPI == EPI_LORA_T) && ep.row_scale && row_ok
+                             ? __ldg(ep.row_scale + m)
+                             : 1.f;
       float v[32];
       if (EPI == EPI_STORE_BF16 || EPI == EPI_STORE_F32 || EPI == EPI_SCATTER_ADD) {
+        const float oscale = EPI == EPI_STORE_F32 ? ep.alpha * rfac : ep.alpha;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           tmem_ld32(tbase + c * 32, v);
@@ -347,8 +361,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
             for (int q = 0; q < 8; ++q)
               *reinterpret_cast<float4*>(sb + lane * 128 + ((q ^ (lane & 7)) << 4)) =
-                  make_float4(v[4 * q] * ep.alpha, v[4 * q + 1] * ep.alpha, v[4 * q + 2] * ep.alpha,
-                              v[4 * q + 3] * ep.alpha);
+                  make_float4(v[4 * q] * oscale, v[4 * q + 1] * oscale, v[4 * q + 2] * oscale,
+                              v[4 * q + 3] * oscale);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -379,8 +393,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             float4* d = reinterpret_cast<float4*>(reinterpret_cast<float*>(ep.out) + (int64_t)m * ep.ldo + n);
 #pragma unroll
             for (int q = 0; q < 8; ++q)
-              d[q] = make_float4(v[4 * q] * ep.alpha, v[4 * q + 1] * ep.alpha, v[4 * q + 2] * ep.alpha,
-                                 v[4 * q + 3] * ep.alpha);
+              d[q] = make_float4(v[4 * q] * oscale, v[4 * q + 1] * oscale, v[4 * q + 2] * oscale,
+                                 v[4 * q + 3] * oscale);
           } else {  // scatter-add into the residual rows
             if (ep.blk_mask && !__ldg(ep.blk_mask + (m + ep.row_offset) / ep.mask_blk)) continue;
             const int64_t row = map_row(ep, m + ep.row_offset);
@@ -409,6 +423,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             if (n >= N) continue;
             const bool tma = ep.tma_out && m0 + quarter * 32 + 32 <= valid;
             if (!tma && !row_ok) continue;
+            if (ep.aux) {  // the pre-activations, saved for the backward
+              __half* ga = reinterpret_cast<__half*>(ep.aux) + (int64_t)m * ep.ld_aux + n + hh * 32;
+              store_f16x32(ga, v);
+              store_f16x32(ga + 64, u);
+            }
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = silu_f(v[i]) * u[i];
             if (tma) {  // the group's 64 outputs form one bf16 tile
@@ -433,14 +452,33 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const bool tma = ep.tma_out && m0 + quarter * 32 + 32 <= valid;
           if (!tma && !row_ok) continue;
           const int64_t col = (int64_t)(j >> 6) * 128 + (j & 63);
-          const float* gu = reinterpret_cast<const float*>(ep.aux) + (int64_t)m * ep.ld_aux + col;
           float gv[32], uv[32], dg[32];
+          if (ep.aux_f16) {
+            const __half* gu = reinterpret_cast<const __half*>(ep.aux) + (int64_t)m * ep.ld_aux + col;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 a = reinterpret_cast<const float4*>(gu)[q];
-            const float4 b = reinterpret_cast<const float4*>(gu + 64)[q];
-            gv[4 * q] = a.x; gv[4 * q + 1] = a.y; gv[4 * q + 2] = a.z; gv[4 * q + 3] = a.w;
-            uv[4 * q] = b.x; uv[4 * q + 1] = b.y; uv[4 * q + 2] = b.z; uv[4 * q + 3] = b.w;
+            for (int q = 0; q < 4; ++q) {
+              const uint4 a = reinterpret_cast<const uint4*>(gu)[q];
+              const uint4 b = reinterpret_cast<const uint4*>(gu + 64)[q];
+              const __half2* ah = reinterpret_cast<const __half2*>(&a);
+              const __half2* bh = reinterpret_cast<const __half2*>(&b);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 fa = __half22float2(ah[e]), fb = __half22float2(bh[e]);
+                gv[8 * q + 2 * e] = fa.x;
+                gv[8 * q + 2 * e + 1] = fa.y;
+                uv[8 * q + 2 * e] = fb.x;
+                uv[8 * q + 2 * e + 1] = fb.y;
+              }
+            }
+          } else {
+            const float* gu = reinterpret_cast<const float*>(ep.aux) + (int64_t)m * ep.ld_aux + col;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 a = reinterpret_cast<const float4*>(gu)[q];
+              const float4 b = reinterpret_cast<const float4*>(gu + 64)[q];
+              gv[4 * q] = a.x; gv[4 * q + 1] = a.y; gv[4 * q + 2] = a.z; gv[4 * q + 3] = a.w;
+              uv[4 * q] = b.x; uv[4 * q + 1] = b.y; uv[4 * q + 2] = b.z; uv[4 * q + 3] = b.w;
+            }
           }
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
@@ -468,23 +506,33 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           store_f16x32(o + 64, v);
         }
       } else if (EPI == EPI_LORA_T) {
-        // N <= 32 (t_q, t_v): fp32 copy + the scaled value as a bf16 hi + lo pair (columns
-        // 0..31 and 32..63 of the K-padded operand of the next product)
+        // N <= 32 (t_q, t_v): fp32 copy (times the row factor) + the scaled value as a hi + lo
+        // pair (columns 0..31 and 32..63 of the K-padded operand of the next product), bf16
+        // or, with aux_f16, fp16 divided by *aux_div
         tmem_ld32(tbase, v);
         if (row_ok) {
           float* o = reinterpret_cast<float*>(ep.out) + (int64_t)m * ep.ldo;
+          const float ob = ep.beta * rfac;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (i < N) o[i] = v[i] * ep.beta;
+            if (i < N) o[i] = v[i] * ob;
+          const float as = ep.aux_div ? ep.alpha / __ldg(ep.aux_div) : ep.alpha;
           float w[32], lo[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            w[i] = i < N ? v[i] * ep.alpha : 0.f;
-            lo[i] = w[i] - __bfloat162float(__float2bfloat16_rn(w[i]));
+            w[i] = i < N ? v[i] * as : 0.f;
+            lo[i] = w[i] - (ep.aux_f16 ? __half2float(__float2half_rn(w[i]))
+                                       : __bfloat162float(__float2bfloat16_rn(w[i])));
           }
-          bf16* a = reinterpret_cast<bf16*>(ep.aux) + (int64_t)m * ep.ld_aux;
-          store_bf16x32(a, w);
-          store_bf16x32(a + 32, lo);
+          if (ep.aux_f16) {
+            __half* a = reinterpret_cast<__half*>(ep.aux) + (int64_t)m * ep.ld_aux;
+            store_f16x32(a, w);
+            store_f16x32(a + 32, lo);
+          } else {
+            bf16* a = reinterpret_cast<bf16*>(ep.aux) + (int64_t)m * ep.ld_aux;
+            store_bf16x32(a, w);
+            store_bf16x32(a + 32, lo);
+          }
         }
       } else if (EPI == EPI_QKV_ROPE) {
         // tile = BN/128 heads; section = (n / hd): 0 q, 1 k, 2 v; RoPE on q and k with this

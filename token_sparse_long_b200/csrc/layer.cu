@@ -41,7 +41,8 @@ static jenga_status check_weights(const jenga_layer_weights* w, const jenga_lora
   JENGA_CHECK_ARG(w && lora, "layer: null weights");
   JENGA_CHECK_ARG(w->head_dim == 128, "layer: head_dim must be 128 (got %d)", w->head_dim);
   JENGA_CHECK_ARG(w->hidden > 0 && w->hidden % 256 == 0 && w->hidden <= 8192, "layer: hidden must be a multiple of 256, <= 8192");
-  JENGA_CHECK_ARG(w->heads > 0 && w->ffn > 0 && w->ffn % 256 == 0, "layer: ffn must be a multiple of 256");
+  JENGA_CHECK_ARG(w->heads > 0 && w->heads <= 64, "layer: heads must be in [1, 64] (got %d)", w->heads);
+  JENGA_CHECK_ARG(w->ffn > 0 && w->ffn % 256 == 0, "layer: ffn must be a multiple of 256");
   JENGA_CHECK_ARG(lora->rank == LORA_R, "layer: LoRA rank must be 16");
   JENGA_CHECK_ARG(w->wq && w->wk && w->wv && w->wo && w->wg && w->wu && w->wd && w->attn_norm && w->mlp_norm,
                   "layer: null weight pointer");
@@ -55,9 +56,13 @@ static jenga_status check_weights(const jenga_layer_weights* w, const jenga_lora
   return JENGA_OK;
 }
 
+// The backward operands woT, wqkvT, bcat and aqvT (and wguT) are stored fp16: the products
+// that read them take fp16 A operands (row-scaled gradients), and one tcgen05 product has
+// one operand type.  aqvT carries the factor lora_c (lora_l1_divisor_kernel).
 struct Packed {
   bf16 *wqkv, *lorab, *aqv, *wgu, *woT, *wdT, *wguT, *wqkvT, *bcat, *aqvT;
   double* inv_freq;
+  float* lora_c;
 };
 
 static size_t carve_packed(Carve& c, const Dims& d, Packed* p) {
@@ -72,6 +77,7 @@ static size_t carve_packed(Carve& c, const Dims& d, Packed* p) {
   p->bcat = c.take<bf16>((size_t)2 * LORA_R * 3 * d.HD);
   p->aqvT = c.take<bf16>((size_t)d.h * LORA_PAD);
   p->inv_freq = c.take<double>(64);
+  p->lora_c = c.take<float>(4);
   return c.used();
 }
 
@@ -80,6 +86,7 @@ struct Saved {
   float *t, *lse, *rstd1, *rstd2;
   uint8_t* mlp_mask;  // [n_kept_max]: 1 = the MLP sub-block runs on this retained block
   bf16* olo;          // [nc, HD] bf16 rounding residual of o (the backward's Delta uses hi + lo)
+  __half* gu;         // [nc, 2F] fp16 MLP pre-activations (g, u) in the interleaved gate/up layout
 };
 
 static size_t carve_saved(Carve& c, const Dims& d, int nc, Saved* s) {
@@ -93,6 +100,7 @@ static size_t carve_saved(Carve& c, const Dims& d, int nc, Saved* s) {
   s->rstd2 = c.take<float>(nc);
   s->mlp_mask = c.take<uint8_t>(nc > 0 ? (size_t)nc : 1);  // >= n_kept_max entries (one per retained block)
   s->olo = c.take<bf16>((size_t)nc * d.HD);
+  s->gu = c.take<__half>((size_t)nc * 2 * d.F);
   return c.used();
 }
 
@@ -118,8 +126,10 @@ static size_t carve_fwd_ws(Carve& c, const Dims& d, int nc, FwdWs* w) {
 
 struct BwdWs {
   float *dk_acc, *dv_acc;
-  bf16 *xn, *g, *dgu, *dhb, *dhlo, *dO, *dqkv, *dqkvlo, *dtb;
-  float *gu, *dhn, *dh, *delta, *dq, *dt, *part;
+  bf16 *xn, *g, *dgu, *dO;
+  __half *dh16, *dqkv16, *dtb;  // fp16 A operands: dh and dQKV row-scaled, the LoRA term / lora_c
+  float *rs_dh, *rs_qkv;        // their per-row inverse scales
+  float *dhn, *dh, *delta, *dq, *dt, *part;
   float2* rope;  // [T][64] (cos, sin) of the segment rows' positions
   __half* qkv16;   // [nc, 3 HD] fp16 copy of the saved q | k | v (attention backward operands)
   float* dOf;      // [T, HD] fp32 dO of the segment (scaled to fp16 into dO)
@@ -132,15 +142,14 @@ static size_t carve_bwd_ws(Carve& c, const Dims& d, int nc, int T, BwdWs* w) {
   w->dOf = c.take<float>((size_t)T * d.HD);
   w->gscal = c.take<float>(4);
   w->xn = c.take<bf16>((size_t)T * d.h);
-  w->gu = c.take<float>((size_t)T * 2 * d.F);
   w->g = c.take<bf16>((size_t)T * d.h);
   w->dgu = c.take<bf16>((size_t)T * 2 * d.F);
-  w->dhb = c.take<bf16>((size_t)T * d.h);
+  w->dh16 = c.take<__half>((size_t)T * d.h);
   w->dO = c.take<bf16>((size_t)T * d.HD);
-  w->dqkv = c.take<bf16>((size_t)T * 3 * d.HD);
-  w->dtb = c.take<bf16>((size_t)T * LORA_PAD);
-  w->dhlo = c.take<bf16>((size_t)T * d.h);
-  w->dqkvlo = c.take<bf16>((size_t)T * 3 * d.HD);
+  w->dqkv16 = c.take<__half>((size_t)T * 3 * d.HD);
+  w->dtb = c.take<__half>((size_t)T * LORA_PAD);
+  w->rs_dh = c.take<float>(T);
+  w->rs_qkv = c.take<float>(T);
   w->dhn = c.take<float>((size_t)T * d.h);
   w->dh = c.take<float>((size_t)T * d.h);
   w->delta = c.take<float>((size_t)d.H * T);
@@ -276,13 +285,6 @@ extern "C" jenga_status jenga_layer_pack(const jenga_layer_weights* w, const jen
   JENGA_TRY(transpose((const bf16*)w->wo, HD, p.woT, h, h, HD, st));          // Wo [h, HD] -> [HD, h]
   JENGA_TRY(transpose((const bf16*)w->wd, F, p.wdT, h, h, F, st));            // Wd [h, F]  -> [F, h]
   JENGA_TRY(transpose(p.wgu, h, p.wguT, 2 * F, 2 * F, h, st));                // [2F, h]    -> [h, 2F]
-  {  // the dhn product runs on fp16 operands (dg, du carry 3 more mantissa bits than bf16)
-    const int _ps = ::jenga::prof_begin("bf16_to_f16_inplace", st);
-    bf16_to_f16_inplace_kernel<<<grid_cap((int64_t)h * 2 * F, 256), 256, 0, st>>>((uint16_t*)p.wguT,
-                                                                                (int64_t)h * 2 * F);
-    ::jenga::prof_end(_ps, st);
-  }
-  JENGA_LAUNCH_CHECK();
   JENGA_TRY(transpose(p.wqkv, h, p.wqkvT, 3 * HD, 3 * HD, h, st));            // [3HD, h]   -> [h, 3HD]
   // dt = dqkv * bcat^T : rows 0..15 = [Bq^T | 0 | 0], rows 16..31 = [0 | 0 | Bv^T]
   JENGA_TRY(zero(p.bcat, (int64_t)2 * LORA_R * 3 * HD, st));
@@ -292,6 +294,31 @@ extern "C" jenga_status jenga_layer_pack(const jenga_layer_weights* w, const jen
   // (columns 32..63 repeat 0..31: the A operand carries dt's hi and lo halves, EPI_LORA_T)
   JENGA_TRY(transpose(p.aqv, h, p.aqvT, LORA_PAD, 2 * LORA_R, h, st));
   JENGA_TRY(transpose(p.aqv, h, p.aqvT + 2 * LORA_R, LORA_PAD, 2 * LORA_R, h, st));
+  {  // the divisor of the fp16 LoRA operand of the dX product (from bcat while it is bf16)
+    const int _ps = ::jenga::prof_begin("lora_l1_divisor", st);
+    lora_l1_divisor_kernel<<<1, 1024, 0, st>>>(p.bcat, 2 * LORA_R, 3 * HD, lora->scale, p.lora_c);
+    ::jenga::prof_end(_ps, st);
+  }
+  JENGA_LAUNCH_CHECK();
+  // the backward products run on fp16 operands: re-encode their weight operands in place
+  {
+    struct {
+      bf16* w;
+      int64_t n;
+      const float* mul;
+    } conv[5] = {{p.wguT, (int64_t)h * 2 * F, nullptr},
+                 {p.woT, (int64_t)HD * h, nullptr},
+                 {p.wqkvT, (int64_t)h * 3 * HD, nullptr},
+                 {p.bcat, (int64_t)2 * LORA_R * 3 * HD, nullptr},
+                 {p.aqvT, (int64_t)h * LORA_PAD, p.lora_c}};
+    for (int i = 0; i < 5; ++i) {
+      const int _ps = ::jenga::prof_begin("bf16_to_f16_inplace", st);
+      bf16_to_f16_inplace_kernel<<<grid_cap(conv[i].n, 256), 256, 0, st>>>((uint16_t*)conv[i].w, conv[i].n,
+                                                                          conv[i].mul);
+      ::jenga::prof_end(_ps, st);
+      JENGA_LAUNCH_CHECK();
+    }
+  }
   {
   const int _ps = ::jenga::prof_begin("inv_freq", st);
   inv_freq_kernel<<<1, 64, 0, st>>>(p.inv_freq, d.D, log2((double)w->rope_theta));
@@ -497,6 +524,8 @@ static jenga_status layer_fwd(const jenga_layer_weights* w, const jenga_lora* lo
     EpiParams e = epi_base(idx, blk, n_kept, 0);
     e.out = f.a;
     e.ldo = F;
+    e.aux = s.gu;  // (g, u) saved for the backward's SwiGLU derivative
+    e.ld_aux = 2 * F;
     JENGA_TRY((launch_gemm<256, EPI_SWIGLU>({f.xn, nc, h}, {p.wgu, 2 * F, h}, h, nullptr, nullptr, 0, nc, 2 * F, e, st, "gemm_gateup_swiglu")));
   }
   // 8. the blocks the MLP sub-block runs on: all retained blocks, or the ones the MLP-block
@@ -628,18 +657,7 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
     const int s0 = sg * segment_tokens;
     const int s1 = (s0 + segment_tokens < nc) ? s0 + segment_tokens : nc;
     const int T = s1 - s0;
-    // --- MLP block (recomputed): hn, (g, u)
-    JENGA_TRY(rmsnorm(s.hres + (size_t)s0 * h, h, nullptr, 1, s0, n_kept, blk, T, h, w->rms_eps,
-                      (const bf16*)w->mlp_norm, nullptr, b.xn, nullptr, st));
-    // the MLP GEMMs skip the 128-row tiles whose blocks the MLP sub-block did not run on
-    {
-      EpiParams e = epi_base(idx, blk, n_kept, s0);
-      e.out = b.gu;
-      e.ldo = 2 * F;
-      e.blk_mask = s.mlp_mask;
-      e.mask_blk = blk;
-      JENGA_TRY((launch_gemm<256, EPI_STORE_F32>({b.xn, T, h}, {p.wgu, 2 * F, h}, h, nullptr, nullptr, 0, T, 2 * F, e, st, "gemm_gateup_recompute")));
-    }
+    // --- MLP block (the forward saved the pre-activations (g, u) in fp16)
     // upstream gradient rows of this segment
     {
     const int _ps = ::jenga::prof_begin("gather_seg", st);
@@ -648,13 +666,15 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
     ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();
-    // dA = G Wd ; (dg, du) from SiLU(g) * u
+    // dA = G Wd ; (dg, du) from SiLU(g) * u; the MLP GEMMs skip the 128-row tiles whose
+    // blocks the MLP sub-block did not run on
     {
       EpiParams e = epi_base(idx, blk, n_kept, s0);
       e.out = b.dgu;
       e.ldo = 2 * F;
-      e.aux = b.gu;
+      e.aux = s.gu + (size_t)s0 * 2 * F;
       e.ld_aux = 2 * F;
+      e.aux_f16 = true;
       e.blk_mask = s.mlp_mask;
       e.mask_blk = blk;
       JENGA_TRY((launch_gemm<256, EPI_SWIGLU_BWD>({b.g, T, h}, {p.wdT, F, h}, h, nullptr, nullptr, 0, T, F, e, st, "gemm_da_swiglu_bwd")));
@@ -673,8 +693,8 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
     {
     const int _ps = ::jenga::prof_begin("rmsnorm_bwd_rows", st);
     rmsnorm_bwd_rows_kernel<<<T, ROW_THREADS, 0, st>>>(b.dhn, h, s.hres + (size_t)s0 * h, h, s.rstd2 + s0,
-                                                        (const bf16*)w->mlp_norm, nullptr, b.g, h, b.dh, b.dhb,
-                                                        b.dhlo, h, nullptr, 0, idx, blk, s0, n_kept, blk, h, S,
+                                                        (const bf16*)w->mlp_norm, nullptr, b.g, h, b.dh, b.dh16,
+                                                        b.rs_dh, h, nullptr, 0, idx, blk, s0, n_kept, blk, h, S,
                                                         s.mlp_mask, blk);
     ::jenga::prof_end(_ps, st);
     }
@@ -685,10 +705,10 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
       EpiParams e = epi_base(idx, blk, n_kept, s0);
       e.out = b.dOf;
       e.ldo = HD;
-      // dh enters as a bf16 hi + lo pair (two K phases over the same weights)
-      GemmOperand a2{b.dhlo, T, h}, b2{p.woT, HD, h};
-      JENGA_TRY((launch_gemm<256, EPI_STORE_F32>({b.dhb, T, h}, {p.woT, HD, h}, h, &a2, &b2, h, T, HD, e, st,
-                                                 "gemm_do")));
+      // dh enters as fp16 rows scaled into [2^13, 2^14); the epilogue undoes the row scale
+      e.row_scale = b.rs_dh;
+      JENGA_TRY((launch_gemm<256, EPI_STORE_F32>({b.dh16, T, h}, {p.woT, HD, h}, h, nullptr, nullptr, 0, T, HD, e,
+                                                 st, "gemm_do", nullptr, nullptr, 0, /*f16_inputs=*/true)));
     }
     JENGA_CUDA_TRY(cudaMemsetAsync(b.gscal + 1, 0, sizeof(float), st));
     {
@@ -717,12 +737,13 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
     JENGA_LAUNCH_CHECK();
     {
     const int _ps = ::jenga::prof_begin("rope_bwd_pack", st);
-    rope_bwd_pack_kernel<<<grid_cap((int64_t)T * H * 32, 256), 256, 0, st>>>(
-        b.dq, HD, b.dk_acc, b.dv_acc, HD, s0, b.dqkv, b.dqkvlo, 3 * HD, b.rope, n_kept, blk, T, H);
+    rope_bwd_pack_kernel<<<T, ROW_THREADS, 0, st>>>(b.dq, HD, b.dk_acc, b.dv_acc, HD, s0, b.dqkv16, b.rs_qkv,
+                                                     3 * HD, b.rope, n_kept, blk, T, H);
     ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();
-    // dt = s [dq Bq, dv Bv]  (fp32, and bf16 K-padded for the dX GEMM)
+    // dt = s [dq Bq, dv Bv]: fp32 (the row scale undone) for the LoRA gradients, and the
+    // still row-scaled value / lora_c as the fp16 K-padded LoRA operand of the dX product
     {
       EpiParams e = epi_base(idx, blk, n_kept, s0);
       e.out = b.dt;
@@ -731,8 +752,12 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
       e.ld_aux = LORA_PAD;
       e.alpha = ls;
       e.beta = ls;
-      JENGA_TRY((launch_gemm<32, EPI_LORA_T>({b.dqkv, T, 3 * HD}, {p.bcat, 2 * LORA_R, 3 * HD}, 3 * HD, nullptr, nullptr,
-                                             0, T, 2 * LORA_R, e, st, "gemm_dt")));
+      e.row_scale = b.rs_qkv;
+      e.aux_f16 = true;
+      e.aux_div = p.lora_c;
+      JENGA_TRY((launch_gemm<32, EPI_LORA_T>({b.dqkv16, T, 3 * HD}, {p.bcat, 2 * LORA_R, 3 * HD}, 3 * HD, nullptr,
+                                             nullptr, 0, T, 2 * LORA_R, e, st, "gemm_dt", nullptr, nullptr, 0,
+                                             /*f16_inputs=*/true)));
     }
     // xn of the segment (recomputed from the saved gathered input)
     JENGA_TRY(rmsnorm(s.xr + (size_t)s0 * h, h, nullptr, 1, s0, n_kept, blk, T, h, w->rms_eps,
@@ -742,10 +767,11 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
       const int chunks = (T + LG_CHUNK - 1) / LG_CHUNK;
       const int cmax = HD > h ? HD : h;
       LoraGradJobs jobs;
-      jobs.j[0] = {b.dqkv, 3 * HD, s.t + (size_t)s0 * 2 * LORA_R, HD, ls, grads->dbq, LORA_R, 1};
-      jobs.j[1] = {b.dqkv + 2 * HD, 3 * HD, s.t + (size_t)s0 * 2 * LORA_R + LORA_R, HD, ls, grads->dbv, LORA_R, 1};
-      jobs.j[2] = {b.xn, h, b.dt, h, 1.f, grads->daq, 1, h};
-      jobs.j[3] = {b.xn, h, b.dt + LORA_R, h, 1.f, grads->dav, 1, h};
+      jobs.j[0] = {b.dqkv16, 3 * HD, s.t + (size_t)s0 * 2 * LORA_R, HD, ls, grads->dbq, LORA_R, 1, b.rs_qkv, 1};
+      jobs.j[1] = {b.dqkv16 + 2 * HD, 3 * HD, s.t + (size_t)s0 * 2 * LORA_R + LORA_R, HD, ls, grads->dbv, LORA_R, 1,
+                   b.rs_qkv, 1};
+      jobs.j[2] = {b.xn, h, b.dt, h, 1.f, grads->daq, 1, h, nullptr, 0};
+      jobs.j[3] = {b.xn, h, b.dt + LORA_R, h, 1.f, grads->dav, 1, h, nullptr, 0};
       {
         const int _ps = ::jenga::prof_begin("lora_grad_partial", st);
         lora_grad_partial_kernel<<<dim3((cmax + LG_COLS - 1) / LG_COLS, chunks, 4), 256, 0, st>>>(
@@ -765,11 +791,13 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
       EpiParams e = epi_base(idx, blk, n_kept, s0);
       e.out = b.dhn;
       e.ldo = h;
-      // dQKV enters as a bf16 hi + lo pair; the third K phase adds dt [Aq; Av]
-      GemmOperand a2{b.dqkvlo, T, 3 * HD}, b2{p.wqkvT, h, 3 * HD};
-      GemmOperand a3{b.dtb, T, LORA_PAD}, b3{p.aqvT, h, LORA_PAD};
-      JENGA_TRY((launch_gemm<256, EPI_STORE_F32>({b.dqkv, T, 3 * HD}, {p.wqkvT, h, 3 * HD}, 3 * HD, &a2, &b2, 3 * HD,
-                                                 T, h, e, st, "gemm_dxn", &a3, &b3, LORA_PAD)));
+      // dQKV enters as fp16 rows scaled into [2^13, 2^14); the second K phase adds the LoRA
+      // term (s_m dt / lora_c) (lora_c [Aq; Av]); the epilogue undoes the row scale
+      e.row_scale = b.rs_qkv;
+      GemmOperand a2{b.dtb, T, LORA_PAD}, b2{p.aqvT, h, LORA_PAD};
+      JENGA_TRY((launch_gemm<256, EPI_STORE_F32>({b.dqkv16, T, 3 * HD}, {p.wqkvT, h, 3 * HD}, 3 * HD, &a2, &b2,
+                                                 LORA_PAD, T, h, e, st, "gemm_dxn", nullptr, nullptr, 0,
+                                                 /*f16_inputs=*/true)));
     }
     // dX[rows] = dh + RMSNorm_bwd(dxn)  (written in place into the gradient buffer)
     {

@@ -24,6 +24,30 @@ __device__ __forceinline__ float block_sum_256(float v, float* red) {
   return t;
 }
 
+__device__ __forceinline__ float block_max_256(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int w = 0; w < ROW_THREADS / 32; ++w) t = fmaxf(t, red[w]);
+  return t;
+}
+
+// Row scale of an fp16 GEMM operand: sc = 2^(13 - e) for amax in [2^e, 2^(e+1)), so the
+// row's largest magnitude lands in [2^13, 2^14) (fp16 keeps 11 significant bits up to
+// 65504); r = 1 / sc.  Both are powers of two built from their exponent bits, so the
+// scaling and its undoing in the GEMM epilogue are exact.
+__device__ __forceinline__ void pow2_row_scale(float amax, float& sc, float& r) {
+  int e = (int)((__float_as_uint(amax) >> 23) & 255u) - 127;
+  e = e < -113 ? -113 : (e > 127 ? 127 : e);
+  sc = __uint_as_float((uint32_t)(127 + 13 - e) << 23);
+  r = __uint_as_float((uint32_t)(127 - 13 + e) << 23);
+}
+
 __device__ __forceinline__ void unpack8(const uint4& u, float* f) {
   const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
@@ -107,13 +131,14 @@ __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_rows_kernel(
 
 // RMSNorm backward fused with the residual:
 //   out[m] = base[m] + r g dy - x r^3 / h * sum(dy g x)
-// base: fp32 (base_f) or bf16 (base_b); outputs: fp32 out_f, bf16 out_b, and/or the
-// bf16 scatter into dst[row(m)] (in place, pitch ldd).
+// base: fp32 (base_f) or bf16 (base_b); outputs: fp32 out_f, the fp16 GEMM operand out_h
+// (row m scaled by the power of two of pow2_row_scale, its inverse in out_rs[m]), and/or
+// the bf16 scatter into dst[row(m)] (in place, pitch ldd).
 __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_bwd_rows_kernel(
     const float* __restrict__ dy, int64_t lddy, const bf16* __restrict__ x, int64_t ldx,
     const float* __restrict__ rstd, const bf16* __restrict__ gain, const float* __restrict__ base_f,
-    const bf16* __restrict__ base_b, int64_t ldb, float* __restrict__ out_f, bf16* __restrict__ out_b,
-    bf16* __restrict__ out_lo, int64_t ldo, bf16* __restrict__ dst, int64_t ldd, const int32_t* __restrict__ idx, int blk, int row_offset,
+    const bf16* __restrict__ base_b, int64_t ldb, float* __restrict__ out_f, __half* __restrict__ out_h,
+    float* __restrict__ out_rs, int64_t ldo, bf16* __restrict__ dst, int64_t ldd, const int32_t* __restrict__ idx, int blk, int row_offset,
     const int32_t* __restrict__ n_valid, int valid_mult, int h, int64_t dst_rows,
     const uint8_t* __restrict__ keep_mask = nullptr, int mask_blk = 1) {
   __shared__ float red[ROW_THREADS / 32];
@@ -166,30 +191,43 @@ __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_bwd_rows_kernel(
     if (threadIdx.x == 0) record_device_error(JENGA_EINTERNAL, SITE_INDEX_RANGE, (unsigned)drow);
     return;
   }
+  float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < ROW_MAX_CHUNKS; ++i) {
     const int c = threadIdx.x + i * ROW_THREADS;
     if (c < nch) {
-      float o[8];
+      float* o = bv[i];  // the output overwrites the residual base in registers
 #pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = bv[i][e] + r * dyg[i][e] - xv[i][e] * k;
+      for (int e = 0; e < 8; ++e) {
+        o[e] = bv[i][e] + r * dyg[i][e] - xv[i][e] * k;
+        amax = fmaxf(amax, fabsf(o[e]));
+      }
       if (out_f) {
         float4* op = reinterpret_cast<float4*>(out_f + (int64_t)m * ldo) + 2 * c;
         op[0] = make_float4(o[0], o[1], o[2], o[3]);
         op[1] = make_float4(o[4], o[5], o[6], o[7]);
       }
-      if (out_b) {
-        const uint4 hi = pack8(o);
-        reinterpret_cast<uint4*>(out_b + (int64_t)m * ldo)[c] = hi;
-        if (out_lo) {  // residual o - bf16(o), so that hi + lo carries ~16 mantissa bits
-          float hv[8], lo[8];
-          unpack8(hi, hv);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) lo[e] = o[e] - hv[e];
-          reinterpret_cast<uint4*>(out_lo + (int64_t)m * ldo)[c] = pack8(lo);
-        }
-      }
       if (dst) reinterpret_cast<uint4*>(dst + drow * ldd)[c] = pack8(o);
+    }
+  }
+  if (out_h) {  // block-uniform branch: the reduction's barriers are reached by every thread
+    amax = block_max_256(amax, red);
+    float sc, rs;
+    pow2_row_scale(amax, sc, rs);
+    if (threadIdx.x == 0) out_rs[m] = rs;
+#pragma unroll
+    for (int i = 0; i < ROW_MAX_CHUNKS; ++i) {
+      const int c = threadIdx.x + i * ROW_THREADS;
+      if (c < nch) {
+        uint4 u;
+        uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __half2 hv = __floats2half2_rn(bv[i][2 * e] * sc, bv[i][2 * e + 1] * sc);
+          w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        reinterpret_cast<uint4*>(out_h + (int64_t)m * ldo)[c] = u;
+      }
     }
   }
 }
@@ -213,54 +251,75 @@ __global__ void gather_seg_kernel(const bf16* __restrict__ src, int64_t lds, bf1
   }
 }
 
-// Backward of RoPE on dq / dk (the transpose rotation) and the pack of dQ | dK | dV for the
-// segment's rows [s0, s0 + nv) into bf16 hi and lo halves (hi = bf16(x), lo = bf16(x - hi)).
-// One warp per (row, head): lane l takes frequency pair (2l, 2l + 1), reading its (cos,
-// sin) pairs from the segment's RoPE table (tab[m][j], rope_table_kernel at offset s0),
-// 8-byte loads and bf16x2 stores.
-__global__ void rope_bwd_pack_kernel(const float* __restrict__ dq, int64_t ld_dq, const float* __restrict__ dk,
-                                     const float* __restrict__ dv, int64_t ld_acc, int s0, bf16* __restrict__ dqkv,
-                                     bf16* __restrict__ dqkv_lo, int64_t ld_out, const float2* __restrict__ tab,
-                                     const int32_t* __restrict__ n_valid, int valid_mult, int rows, int H) {
-  const int nv = valid_rows(n_valid, valid_mult, s0, rows);
-  const int64_t total = (int64_t)nv * H * 32;
-  const int HD = H * 128;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-    const int ip = (int)(e & 31);
-    const int mh = (int)(e >> 5);
-    const int m = mh / H, hh = mh - m * H;
-    const float4 t = __ldg(reinterpret_cast<const float4*>(tab + (int64_t)m * 64) + ip);  // (cos, sin) x 2
-    const int c1 = hh * 128 + 2 * ip, c2 = c1 + 64;
-    const float2 a1 = *reinterpret_cast<const float2*>(dq + (int64_t)m * ld_dq + c1);
-    const float2 a2 = *reinterpret_cast<const float2*>(dq + (int64_t)m * ld_dq + c2);
-    const float2 b1 = *reinterpret_cast<const float2*>(dk + (int64_t)(s0 + m) * ld_acc + c1);
-    const float2 b2 = *reinterpret_cast<const float2*>(dk + (int64_t)(s0 + m) * ld_acc + c2);
-    const float2 v1 = *reinterpret_cast<const float2*>(dv + (int64_t)(s0 + m) * ld_acc + c1);
-    const float2 v2 = *reinterpret_cast<const float2*>(dv + (int64_t)(s0 + m) * ld_acc + c2);
-    // per frequency: (x1, x2) -> (x1 cos + x2 sin, x2 cos - x1 sin)
-    const float val[6][2] = {{a1.x * t.x + a2.x * t.y, a1.y * t.z + a2.y * t.w},
-                             {a2.x * t.x - a1.x * t.y, a2.y * t.z - a1.y * t.w},
-                             {b1.x * t.x + b2.x * t.y, b1.y * t.z + b2.y * t.w},
-                             {b2.x * t.x - b1.x * t.y, b2.y * t.z - b1.y * t.w},
-                             {v1.x, v1.y},
-                             {v2.x, v2.y}};
-    const int col[6] = {c1, c2, HD + c1, HD + c2, 2 * HD + c1, 2 * HD + c2};
-    bf16* o = dqkv + (int64_t)m * ld_out;
-    bf16* ol = dqkv_lo + (int64_t)m * ld_out;
+// Backward of RoPE on dq / dk (the transpose rotation) and the pack of dQ | dK | dV of the
+// segment's rows [s0, s0 + nv) into one fp16 GEMM operand, each row scaled by the power of
+// two of pow2_row_scale (its inverse in rs[m]).  One CTA per row: thread e of the row's
+// H x 32 (head, frequency pair) items takes pair (2 ip, 2 ip + 1) of head hh, reading its
+// (cos, sin) pairs from the segment's RoPE table (tab[m][j], rope_table_kernel at offset
+// s0); the rotated values wait in registers for the row's largest magnitude.
+constexpr int RB_ITEMS = 8;  // items per thread: H <= RB_ITEMS * ROW_THREADS / 32 = 64
+__global__ void __launch_bounds__(ROW_THREADS) rope_bwd_pack_kernel(
+    const float* __restrict__ dq, int64_t ld_dq, const float* __restrict__ dk, const float* __restrict__ dv,
+    int64_t ld_acc, int s0, __half* __restrict__ dqkv, float* __restrict__ rs, int64_t ld_out,
+    const float2* __restrict__ tab, const int32_t* __restrict__ n_valid, int valid_mult, int rows, int H) {
+  __shared__ float red[ROW_THREADS / 32];
+  const int m = blockIdx.x;
+  if (m >= valid_rows(n_valid, valid_mult, s0, rows)) return;
+  const int HD = H * 128, items = H * 32;
+  float val[RB_ITEMS][12];
+  float amax = 0.f;
 #pragma unroll
-    for (int k2 = 0; k2 < 6; ++k2) {
-      const __nv_bfloat162 hi = __floats2bfloat162_rn(val[k2][0], val[k2][1]);
-      const float2 hf = __bfloat1622float2(hi);
-      *reinterpret_cast<__nv_bfloat162*>(o + col[k2]) = hi;
-      *reinterpret_cast<__nv_bfloat162*>(ol + col[k2]) =
-          __floats2bfloat162_rn(val[k2][0] - hf.x, val[k2][1] - hf.y);
+  for (int k = 0; k < RB_ITEMS; ++k) {
+    const int e = threadIdx.x + k * ROW_THREADS;
+    if (e < items) {
+      const int ip = e & 31, hh = e >> 5;
+      const float4 t = __ldg(reinterpret_cast<const float4*>(tab + (int64_t)m * 64) + ip);  // (cos, sin) x 2
+      const int c1 = hh * 128 + 2 * ip, c2 = c1 + 64;
+      const float2 a1 = *reinterpret_cast<const float2*>(dq + (int64_t)m * ld_dq + c1);
+      const float2 a2 = *reinterpret_cast<const float2*>(dq + (int64_t)m * ld_dq + c2);
+      const float2 b1 = *reinterpret_cast<const float2*>(dk + (int64_t)(s0 + m) * ld_acc + c1);
+      const float2 b2 = *reinterpret_cast<const float2*>(dk + (int64_t)(s0 + m) * ld_acc + c2);
+      const float2 v1 = *reinterpret_cast<const float2*>(dv + (int64_t)(s0 + m) * ld_acc + c1);
+      const float2 v2 = *reinterpret_cast<const float2*>(dv + (int64_t)(s0 + m) * ld_acc + c2);
+      // per frequency: (x1, x2) -> (x1 cos + x2 sin, x2 cos - x1 sin)
+      val[k][0] = a1.x * t.x + a2.x * t.y;
+      val[k][1] = a1.y * t.z + a2.y * t.w;
+      val[k][2] = a2.x * t.x - a1.x * t.y;
+      val[k][3] = a2.y * t.z - a1.y * t.w;
+      val[k][4] = b1.x * t.x + b2.x * t.y;
+      val[k][5] = b1.y * t.z + b2.y * t.w;
+      val[k][6] = b2.x * t.x - b1.x * t.y;
+      val[k][7] = b2.y * t.z - b1.y * t.w;
+      val[k][8] = v1.x;
+      val[k][9] = v1.y;
+      val[k][10] = v2.x;
+      val[k][11] = v2.y;
+#pragma unroll
+      for (int j = 0; j < 12; ++j) amax = fmaxf(amax, fabsf(val[k][j]));
+    }
+  }
+  amax = block_max_256(amax, red);
+  float sc, r;
+  pow2_row_scale(amax, sc, r);
+  if (threadIdx.x == 0) rs[m] = r;
+  __half* o = dqkv + (int64_t)m * ld_out;
+#pragma unroll
+  for (int k = 0; k < RB_ITEMS; ++k) {
+    const int e = threadIdx.x + k * ROW_THREADS;
+    if (e < items) {
+      const int ip = e & 31, hh = e >> 5;
+      const int c1 = hh * 128 + 2 * ip, c2 = c1 + 64;
+      const int col[6] = {c1, c2, HD + c1, HD + c2, 2 * HD + c1, 2 * HD + c2};
+#pragma unroll
+      for (int j = 0; j < 6; ++j)
+        *reinterpret_cast<__half2*>(o + col[j]) = __floats2half2_rn(val[k][2 * j] * sc, val[k][2 * j + 1] * sc);
     }
   }
 }
 
-// Split-K partials of  P[chunk][c][r] = sum_{m in chunk} X[m, c] * Y[m, r]   (r < 16)
-// X bf16 [rows, ldx] (columns [0, C)), Y fp32 [rows, ldy] (columns [0, 16)).
-// grid (C / 64, chunks), 256 threads = 64 columns x 4 groups of 4 r.
+// Split-K partials of  P[chunk][c][r] = sum_{m in chunk} X[m, c] * xs[m] * Y[m, r]   (r < 16)
+// X bf16 or fp16 [rows, ldx] (columns [0, C)), xs an optional per-row factor, Y fp32
+// [rows, ldy] (columns [0, 16)).
 constexpr int LG_CHUNK = 512;   // rows per partial sum
 constexpr int LG_COLS = 512;    // columns per block (2 per thread)
 
@@ -268,13 +327,15 @@ constexpr int LG_COLS = 512;    // columns per block (2 per thread)
 // (r < 16).  The four of a layer segment (dB_q, dB_v from dQ / dV and t; dA_q, dA_v from
 // xn and dt) run in one launch, blockIdx.z = job.
 struct LoraGradJob {
-  const bf16* X;
+  const void* X;   // bf16, or fp16 when x_f16
   int64_t ldx;
   const float* Y;  // 16 consecutive fp32 per row, row pitch ldy
   int C;
   float scale;
   float* out;
   int64_t so_c, so_r;
+  const float* xs;  // per-row factor of X (the inverse of its fp16 row scale), or null
+  int x_f16;
 };
 struct LoraGradJobs {
   LoraGradJob j[4];
@@ -295,7 +356,16 @@ __global__ void __launch_bounds__(256) lora_grad_partial_kernel(LoraGradJobs job
   for (int e = threadIdx.x; e < LG_CHUNK * 4; e += 256) {
     const int rr = e >> 2, q = e & 3;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (m0 + rr < m1) v = *reinterpret_cast<const float4*>(jb.Y + (int64_t)(m0 + rr) * ldy + 4 * q);
+    if (m0 + rr < m1) {
+      v = *reinterpret_cast<const float4*>(jb.Y + (int64_t)(m0 + rr) * ldy + 4 * q);
+      if (jb.xs) {  // X's row factor rides on Y
+        const float f = __ldg(jb.xs + m0 + rr);
+        v.x *= f;
+        v.y *= f;
+        v.z *= f;
+        v.w *= f;
+      }
+    }
     reinterpret_cast<float4*>(sY)[e] = v;
   }
   __syncthreads();
@@ -303,9 +373,10 @@ __global__ void __launch_bounds__(256) lora_grad_partial_kernel(LoraGradJobs job
 #pragma unroll
   for (int r = 0; r < 16; ++r) acc[r] = 0ull;
   if (c < jb.C) {
-    const bf16* xp = jb.X + (int64_t)m0 * jb.ldx + c;
+    const uint16_t* xp = reinterpret_cast<const uint16_t*>(jb.X) + (int64_t)m0 * jb.ldx + c;
     for (int m = m0; m < m1; ++m, xp += jb.ldx) {
-      const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(xp));
+      const float2 x = jb.x_f16 ? __half22float2(*reinterpret_cast<const __half2*>(xp))
+                                : __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(xp));
       const uint64_t x2 = f2pack(x.x, x.y);
       const float4* yr = reinterpret_cast<const float4*>(sY + (m - m0) * 16);
 #pragma unroll
@@ -427,13 +498,44 @@ __global__ void zero_tail_rows_kernel(bf16* __restrict__ x, int64_t ld, int cols
   }
 }
 
-// In-place bf16 -> fp16 re-encoding (exact for magnitudes in [2^-14, 65504]; the frozen
-// gate/up weights used by the fp16 dhn product are well inside that range).
-__global__ void bf16_to_f16_inplace_kernel(uint16_t* __restrict__ x, int64_t n) {
+// In-place bf16 -> fp16 re-encoding of a backward weight operand, times an optional
+// power-of-two factor *mul (exact for magnitudes in [2^-14, 65504] after the factor, which
+// frozen weights are well inside; smaller ones keep fp16's subnormal spacing 2^-24).  A
+// finite value that would overflow fp16 records JENGA_EINVAL at SITE_PACK_RANGE.
+__global__ void bf16_to_f16_inplace_kernel(uint16_t* __restrict__ x, int64_t n, const float* __restrict__ mul) {
+  const float f0 = mul ? *mul : 1.f;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
-    const float f = __uint_as_float((uint32_t)x[e] << 16);
+    const float f = __uint_as_float((uint32_t)x[e] << 16) * f0;
     const __half hv = __float2half_rn(f);
+    if (fabsf(f) < INFINITY && __hisinf(hv)) record_device_error(JENGA_EINVAL, SITE_PACK_RANGE, (unsigned)e);
     x[e] = *reinterpret_cast<const uint16_t*>(&hv);
+  }
+}
+
+// c[0] = the power of two >= 2 max(lscale, 1) max_j sum_k |b[j, k]| over the rows of the LoRA
+// up-projection operand b [rows, cols] (bf16), at least 1.  It divides the fp16 LoRA operand
+// s_m dt_m of the dX product (and multiplies the matching [Aq; Av] columns): a dQKV row
+// scaled below 2^14 gives |s_m dt_m| <= lscale 2^14 max_j sum_k |b[j, k]|, so the stored
+// s_m dt_m / c stays below 2^13 for a backward LoRA scale up to max(lscale, 1).
+// One CTA of 32 warps, warp j < rows sums row j.
+__global__ void lora_l1_divisor_kernel(const bf16* __restrict__ b, int rows, int cols, float lscale,
+                                       float* __restrict__ c) {
+  __shared__ float rmax[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float s = 0.f;
+  if (warp < rows)
+    for (int k = lane; k < cols; k += 32) s += fabsf(__bfloat162float(b[(int64_t)warp * cols + k]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) rmax[warp] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float mx = 0.f;
+    for (int w = 0; w < 32; ++w) mx = fmaxf(mx, rmax[w]);
+    const float need = 2.f * fmaxf(lscale, 1.f) * mx;
+    float v = 1.f;
+    while (v < need && v < 0x1p100f) v *= 2.f;
+    c[0] = v;
   }
 }
 
