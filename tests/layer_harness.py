@@ -106,7 +106,7 @@ def check_layer_against_oracle(S, blk, idx, n_kept, out, dx, grads_gpu, Xo, dX, 
     measure on the sub-block contributions, which a real fault moves by O(1): out - x <= 3e-2
     with two ulps forgiven (h and out are both stored in bf16 at the magnitude of the
     residual stream, which the salient-row scaling of chained layers makes large), and
-    dX - G <= 6e-2 (one rounding).  Returns the errors."""
+    dX - G <= 3e-2 (one rounding forgiven).  Returns the errors."""
     rows = retained_mask(S, blk, idx, n_kept)
     assert np.array_equal(out[~rows], X[~rows]), "eliminated rows must pass through unchanged"
     assert np.array_equal(dx[~rows], G[~rows]), "eliminated rows: identity gradient"
@@ -124,7 +124,7 @@ def check_layer_against_oracle(S, blk, idx, n_kept, out, dx, grads_gpu, Xo, dX, 
             e[k] = rel_max(grads_gpu[k], grads[k])
     print("layer errors:", {k: float("%.3g" % v) for k, v in e.items()})
     for k, v in e.items():
-        assert v < (2 * TOL if k == "dx-G" else TOL), (k, v)
+        assert v < TOL, (k, v)
     return e
 
 

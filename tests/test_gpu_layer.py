@@ -6,8 +6,7 @@ selection difference cannot cascade.  Bars:
   <= 3e-2, with one bf16 ulp of the stored value forgiven (that final rounding may land
   on either neighbour);
 * the same measured on the sub-block contributions alone (out - x, dX - G), which a
-  real fault moves by O(1): <= 3e-2 forward, <= 6e-2 backward (the backward chains four
-  bf16 GEMM-operand roundings: dA, dh, dO, dQKV);
+  real fault moves by O(1): <= 3e-2 both ways;
 * LoRA gradients (fp32): max |gpu - oracle| / rms(oracle) <= 3e-2;
 * eliminated rows exactly unchanged (x) and exactly the identity gradient (G)."""
 import numpy as np

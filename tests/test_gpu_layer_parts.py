@@ -57,7 +57,8 @@ def test_forward_intermediates(J, keep_blocks):
     errs["o"] = rel_max_ulp(torch_to_f64(parts["o"]), ctx["o"].reshape(nc, HD))
     errs["h"] = rel_delta_ulp(torch_to_f64(parts["h"]), ctx["h"], X[rows])
     errs["out"] = rel_delta_ulp(torch_to_f64(x)[rows], out, X[rows])
-    # the saved (gate, up) pre-activations: fp16 storage of the fp32-accumulated products
+    # the saved (gate, up) pre-activations (fp16); the oracle forms them from its own hn,
+    # which differs from the GPU's by the bf16 roundings of h, so they take the common bar
     g16, u16 = deinterleave_gu(parts["gu"].cpu().double().numpy(), sh.ffn)
     errs["g"] = rel_max(g16, ctx["gt"])
     errs["u"] = rel_max(u16, ctx["ut"])
@@ -65,5 +66,3 @@ def test_forward_intermediates(J, keep_blocks):
     print(errs)
     for k, v in errs.items():
         assert v < 3e-2, (k, errs)
-    # g and u are one fp16 rounding (2^-11 relative) plus fp32 accumulation away from the oracle
-    assert errs["g"] < 2e-3 and errs["u"] < 2e-3, errs

@@ -43,9 +43,8 @@ enum GemmEpi : int {
   EPI_QKV_ROPE = 4,     // q/k/v sections of width hd; RoPE(pos(m)) on q and k -> bf16
   EPI_SWIGLU_BWD = 5,   // acc = dA; aux = (g, u) interleaved fp32 (fp16 with aux_f16) -> out = (dg, du)
                         // interleaved fp16
-  EPI_LORA_T = 6,       // out fp32 [m, 0:N] = beta * acc (* row factor) ; aux [m, 0:64] = (hi, lo) of
-                        // a = alpha * acc (/ *aux_div): cols 0..N-1 round(a), cols 32..32+N-1
-                        // round(a - hi), else 0 (bf16, or fp16 with aux_f16)
+  EPI_LORA_T = 6,       // out fp32 [m, 0:N] = beta * acc ; aux bf16 [m, 0:64] = (hi, lo) of alpha * acc:
+                        // cols 0..N-1 bf16(alpha acc), cols 32..32+N-1 bf16(alpha acc - hi), else 0
 };
 
 struct EpiParams {
@@ -73,12 +72,14 @@ struct EpiParams {
   // no stores), and the scatter-add epilogue leaves the rows of masked blocks untouched
   const uint8_t* blk_mask = nullptr;
   int mask_blk = 1;
-  // STORE_F32, LORA_T: optional per-row factor of the accumulator (local row m), the inverse
+  // STORE_F32: optional per-row factor of the accumulator (local row m), the inverse
   // power-of-two scale of an fp16 A operand whose rows were scaled into fp16's range
   const float* row_scale = nullptr;
-  // LORA_T: the aux copy is fp16 (else bf16) and is divided by *aux_div (device scalar)
+  // SWIGLU_BWD: the saved (g, u) are fp16 (else fp32)
   bool aux_f16 = false;
-  const float* aux_div = nullptr;
+  // STORE_F32 only: split the reduction into ksplit consecutive ranges of k-blocks, one per
+  // CTA tile; range ks writes its partial product to rows [ks * M, ks * M + M) of out
+  int ksplit = 1;
 };
 
 // Does the 128-row tile at local row m0 hold a row of a kept block (always, without a mask)?
@@ -216,9 +217,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const int valid = epi_valid_rows(ep);
   const int ntn = (N + BN - 1) / BN;
   const int ntm = (min(valid, ep.m_host) + GEMM_BM - 1) / GEMM_BM;  // tiles past the valid rows are skipped
-  const int ntiles = ntn * ntm;
+  const int nbase = ntn * ntm;  // output tiles; each runs as ksplit work tiles
+  const int ntiles = nbase * ep.ksplit;
   if ((int)blockIdx.x >= ntiles) return;  // uniform per CTA
   const int nkb = nkb1 + nkb2 + nkb3;
+  // k-block range of work tile `tile` (the whole reduction without a split)
+  auto kb_range = [&](int tile, int& lo, int& hi) {
+    const int ks = tile / nbase;
+    lo = (int)((int64_t)nkb * ks / ep.ksplit);
+    hi = (int)((int64_t)nkb * (ks + 1) / ep.ksplit);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -247,9 +255,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     int g = 0;  // k-blocks issued by this CTA so far (ring position)
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
-    const int n0 = (tile % ntn) * BN, m0 = (tile / ntn) * GEMM_BM;
+    const int bt = tile % nbase;
+    const int n0 = (bt % ntn) * BN, m0 = (bt / ntn) * GEMM_BM;
     if (!gemm_tile_live(ep, m0, valid)) continue;
-    for (int kb = 0; kb < nkb; ++kb, ++g) {
+    int kb_lo, kb_hi;
+    kb_range(tile, kb_lo, kb_hi);
+    for (int kb = kb_lo; kb < kb_hi; ++kb, ++g) {
       const int s = g % STAGES;
       if (g >= STAGES && !mbar_wait(&empty[s], ((g / STAGES) - 1) & 1, SITE_GEMM_PRODUCER)) {
         ok = false;
@@ -276,13 +287,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     bool ok = true;
     int g = 0, it = 0;
     for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
-      if (!gemm_tile_live(ep, (tile / ntn) * GEMM_BM, valid)) continue;
+      if (!gemm_tile_live(ep, ((tile % nbase) / ntn) * GEMM_BM, valid)) continue;
+      int kb_lo, kb_hi;
+      kb_range(tile, kb_lo, kb_hi);
       const int buf = it & 1;
       // the epilogue must have read this accumulator's previous tile (two tiles ago)
       if (it >= 2 && !mbar_wait(&acc_empty[buf], ((it >> 1) - 1) & 1, SITE_GEMM_MMA)) break;
       tc_fence_after();
       const uint32_t acc = tmem + buf * (BN < 32 ? 32 : BN);
-      for (int kb = 0; kb < nkb; ++kb, ++g) {
+      for (int kb = kb_lo; kb < kb_hi; ++kb, ++g) {
         const int s = g % STAGES;
         if (!mbar_wait(&full[s], (g / STAGES) & 1, SITE_GEMM_MMA)) {
           ok = false;
@@ -294,7 +307,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
         for (int k = 0; k < GEMM_BK / 16; ++k) {
           umma_bf16(acc, umma_desc_k_sw128(sa + k * 32), umma_desc_k_sw128(sb + k * 32), idesc,
-                    (kb > 0 || k > 0) ? 1u : 0u);
+                    (kb > kb_lo || k > 0) ? 1u : 0u);
         }
         umma_commit(&empty[s]);
       }
@@ -330,8 +343,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     };
     int it = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const int n0 = (tile % ntn) * BN, m0 = (tile / ntn) * GEMM_BM;
+    const int bt = tile % nbase;
+    const int n0 = (bt % ntn) * BN, m0 = (bt / ntn) * GEMM_BM;
     if (!gemm_tile_live(ep, m0, valid)) continue;
+    // split reduction: range ks stores its partial in the ks-th block of M output rows
+    const int orow0 = EPI == EPI_STORE_F32 ? (tile / nbase) * ep.m_host : 0;
     const int buf = it & 1;
     const int m = m0 + r;
     // warp vote: the tcgen05.ld calls below are collective, so all lanes take one path
@@ -341,9 +357,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     {
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * (BN < 32 ? 32 : BN);
       const bool row_ok = m < valid;
-      const float rfac = (EPI == EPI_STORE_F32 || EPI == EPI_LORA_T) && ep.row_scale && row_ok
-                             ? __ldg(ep.row_scale + m)
-                             : 1.f;
+      const float rfac = EPI == EPI_STORE_F32 && ep.row_scale && row_ok ? __ldg(ep.row_scale + m) : 1.f;
       float v[32];
       if (EPI == EPI_STORE_BF16 || EPI == EPI_STORE_F32 || EPI == EPI_SCATTER_ADD) {
         const float oscale = EPI == EPI_STORE_F32 ? ep.alpha * rfac : ep.alpha;
@@ -366,7 +380,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&tmOut, sb, n, m0 + quarter * 32);
+              tma_store_2d(&tmOut, sb, n, orow0 + m0 + quarter * 32);
               bulk_commit_group();
             }
             ++nst;
@@ -390,7 +404,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             for (int i = 0; i < 32; ++i) v[i] *= ep.alpha;
             store_bf16x32(reinterpret_cast<bf16*>(ep.out) + (int64_t)m * ep.ldo + n, v);
           } else if (EPI == EPI_STORE_F32) {
-            float4* d = reinterpret_cast<float4*>(reinterpret_cast<float*>(ep.out) + (int64_t)m * ep.ldo + n);
+            float4* d = reinterpret_cast<float4*>(reinterpret_cast<float*>(ep.out) + (int64_t)(orow0 + m) * ep.ldo + n);
 #pragma unroll
             for (int q = 0; q < 8; ++q)
               d[q] = make_float4(v[4 * q] * oscale, v[4 * q + 1] * oscale, v[4 * q + 2] * oscale,
@@ -506,33 +520,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           store_f16x32(o + 64, v);
         }
       } else if (EPI == EPI_LORA_T) {
-        // N <= 32 (t_q, t_v): fp32 copy (times the row factor) + the scaled value as a hi + lo
-        // pair (columns 0..31 and 32..63 of the K-padded operand of the next product), bf16
-        // or, with aux_f16, fp16 divided by *aux_div
+        // N <= 32 (t_q, t_v): fp32 copy + the scaled value as a bf16 hi + lo pair (columns
+        // 0..31 and 32..63 of the K-padded operand of the next product)
         tmem_ld32(tbase, v);
         if (row_ok) {
           float* o = reinterpret_cast<float*>(ep.out) + (int64_t)m * ep.ldo;
-          const float ob = ep.beta * rfac;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (i < N) o[i] = v[i] * ob;
-          const float as = ep.aux_div ? ep.alpha / __ldg(ep.aux_div) : ep.alpha;
+            if (i < N) o[i] = v[i] * ep.beta;
           float w[32], lo[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            w[i] = i < N ? v[i] * as : 0.f;
-            lo[i] = w[i] - (ep.aux_f16 ? __half2float(__float2half_rn(w[i]))
-                                       : __bfloat162float(__float2bfloat16_rn(w[i])));
+            w[i] = i < N ? v[i] * ep.alpha : 0.f;
+            lo[i] = w[i] - __bfloat162float(__float2bfloat16_rn(w[i]));
           }
-          if (ep.aux_f16) {
-            __half* a = reinterpret_cast<__half*>(ep.aux) + (int64_t)m * ep.ld_aux;
-            store_f16x32(a, w);
-            store_f16x32(a + 32, lo);
-          } else {
-            bf16* a = reinterpret_cast<bf16*>(ep.aux) + (int64_t)m * ep.ld_aux;
-            store_bf16x32(a, w);
-            store_bf16x32(a + 32, lo);
-          }
+          bf16* a = reinterpret_cast<bf16*>(ep.aux) + (int64_t)m * ep.ld_aux;
+          store_bf16x32(a, w);
+          store_bf16x32(a + 32, lo);
         }
       } else if (EPI == EPI_QKV_ROPE) {
         // tile = BN/128 heads; section = (n / hd): 0 q, 1 k, 2 v; RoPE on q and k with this
@@ -637,11 +641,14 @@ jenga_status launch_gemm(const GemmOperand& A1, const GemmOperand& B1, int K1, c
   CUtensorMap tout = ta1;
   EpiParams p = ep;
   p.m_host = M;
+  if (ep.ksplit < 1 || (ep.ksplit > 1 && EPI != EPI_STORE_F32))
+    return fail(JENGA_EINVAL, "gemm: a split reduction needs the fp32 store epilogue");
+  if (ep.ksplit > (K1 + K2 + K3) / GEMM_BK) p.ksplit = (K1 + K2 + K3) / GEMM_BK;  // >= 1 k-block per range
   {
     jenga_status ts = JENGA_EUNSUPPORTED;
     const bool al = ((reinterpret_cast<uintptr_t>(ep.out) & 15) == 0);
     if (al && EPI == EPI_STORE_F32 && ep.ldo % 4 == 0)
-      ts = make_tmap_f32(&tout, ep.out, (uint64_t)M, (uint64_t)N, (uint64_t)ep.ldo, 32);
+      ts = make_tmap_f32(&tout, ep.out, (uint64_t)M * p.ksplit, (uint64_t)N, (uint64_t)ep.ldo, 32);
     else if (al && (EPI == EPI_STORE_BF16 || EPI == EPI_QKV_ROPE) && ep.ldo % 8 == 0)
       ts = make_tmap_bf16(&tout, ep.out, (uint64_t)M, (uint64_t)N, (uint64_t)ep.ldo, 32);
     else if (al && EPI == EPI_SWIGLU && ep.ldo % 8 == 0)
@@ -654,7 +661,7 @@ jenga_status launch_gemm(const GemmOperand& A1, const GemmOperand& B1, int K1, c
   JENGA_CUDA_TRY(
       cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL));
   // persistent: one CTA per SM (or per tile when there are fewer tiles)
-  const int ntiles = ((N + BN - 1) / BN) * ((M + GEMM_BM - 1) / GEMM_BM);
+  const int ntiles = ((N + BN - 1) / BN) * ((M + GEMM_BM - 1) / GEMM_BM) * p.ksplit;
   dim3 grid(ntiles < sm_count() ? ntiles : sm_count());
   // operand format fields (bits 7-9: A, 10-12: B) are 1 for bf16 and 0 for fp16
   const uint32_t idesc = f16_inputs ? (umma_idesc_bf16(GEMM_BM, BN) & ~((7u << 7) | (7u << 10)))

@@ -124,11 +124,22 @@ static size_t carve_fwd_ws(Carve& c, const Dims& d, int nc, FwdWs* w) {
   return c.used();
 }
 
+// The dt product (M = segment rows, N = 32, K = 3 H D) has one output tile per 128 rows: its
+// reduction is split into up to DT_SPLIT_MAX ranges so that about one work tile per SM runs.
+constexpr int DT_SPLIT_MAX = 8;
+static int dt_split(int T, int K) {
+  const int ntm = (T + 127) / 128;
+  int ks = sm_count() / (ntm > 0 ? ntm : 1);
+  ks = ks < 1 ? 1 : (ks > DT_SPLIT_MAX ? DT_SPLIT_MAX : ks);
+  return ks < K / 64 ? ks : K / 64;
+}
+
 struct BwdWs {
   float *dk_acc, *dv_acc;
   bf16 *xn, *g, *dgu, *dO;
   __half *dh16, *dqkv16, *dtb;  // fp16 A operands: dh and dQKV row-scaled, the LoRA term / lora_c
   float *rs_dh, *rs_qkv;        // their per-row inverse scales
+  float* dtpart;                // [DT_SPLIT_MAX][T][32] partial sums of the split dt product
   float *dhn, *dh, *delta, *dq, *dt, *part;
   float2* rope;  // [T][64] (cos, sin) of the segment rows' positions
   __half* qkv16;   // [nc, 3 HD] fp16 copy of the saved q | k | v (attention backward operands)
@@ -150,6 +161,7 @@ static size_t carve_bwd_ws(Carve& c, const Dims& d, int nc, int T, BwdWs* w) {
   w->dtb = c.take<__half>((size_t)T * LORA_PAD);
   w->rs_dh = c.take<float>(T);
   w->rs_qkv = c.take<float>(T);
+  w->dtpart = c.take<float>((size_t)DT_SPLIT_MAX * T * 2 * LORA_R);
   w->dhn = c.take<float>((size_t)T * d.h);
   w->dh = c.take<float>((size_t)T * d.h);
   w->delta = c.take<float>((size_t)d.H * T);
@@ -220,8 +232,12 @@ static jenga_status rmsnorm(const bf16* x, int64_t ldx, const int32_t* idx, int 
   if (rows <= 0) return JENGA_OK;
   {
   const int _ps = ::jenga::prof_begin("rmsnorm_rows", st);
-  rmsnorm_rows_kernel<<<rows, ROW_THREADS, 0, st>>>(x, ldx, idx, blk, row_offset, n_valid, mult, h, eps, gain, xr, h,
-                                                    xn, h, rstd, x_rows ? x_rows : rows);
+  if (h <= 16 * ROW_THREADS)
+    rmsnorm_rows_kernel<2><<<rows, ROW_THREADS, 0, st>>>(x, ldx, idx, blk, row_offset, n_valid, mult, h, eps, gain,
+                                                         xr, h, xn, h, rstd, x_rows ? x_rows : rows);
+  else
+    rmsnorm_rows_kernel<4><<<rows, ROW_THREADS, 0, st>>>(x, ldx, idx, blk, row_offset, n_valid, mult, h, eps, gain,
+                                                         xr, h, xn, h, rstd, x_rows ? x_rows : rows);
   ::jenga::prof_end(_ps, st);
   }
   JENGA_LAUNCH_CHECK();
@@ -692,7 +708,8 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
     // dh = G + RMSNorm_bwd(dhn)
     {
     const int _ps = ::jenga::prof_begin("rmsnorm_bwd_rows", st);
-    rmsnorm_bwd_rows_kernel<<<T, ROW_THREADS, 0, st>>>(b.dhn, h, s.hres + (size_t)s0 * h, h, s.rstd2 + s0,
+    (h <= 16 * ROW_THREADS ? rmsnorm_bwd_rows_kernel<2> : rmsnorm_bwd_rows_kernel<4>)<<<T, ROW_THREADS, 0, st>>>(
+        b.dhn, h, s.hres + (size_t)s0 * h, h, s.rstd2 + s0,
                                                         (const bf16*)w->mlp_norm, nullptr, b.g, h, b.dh, b.dh16,
                                                         b.rs_dh, h, nullptr, 0, idx, blk, s0, n_kept, blk, h, S,
                                                         s.mlp_mask, blk);
@@ -737,27 +754,28 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
     JENGA_LAUNCH_CHECK();
     {
     const int _ps = ::jenga::prof_begin("rope_bwd_pack", st);
-    rope_bwd_pack_kernel<<<T, ROW_THREADS, 0, st>>>(b.dq, HD, b.dk_acc, b.dv_acc, HD, s0, b.dqkv16, b.rs_qkv,
-                                                     3 * HD, b.rope, n_kept, blk, T, H);
+    (H <= ROW_THREADS / 8 ? rope_bwd_pack_kernel<4> : rope_bwd_pack_kernel<8>)<<<T, ROW_THREADS, 0, st>>>(
+        b.dq, HD, b.dk_acc, b.dv_acc, HD, s0, b.dqkv16, b.rs_qkv, 3 * HD, b.rope, n_kept, blk, T, H);
     ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();
     // dt = s [dq Bq, dv Bv]: fp32 (the row scale undone) for the LoRA gradients, and the
-    // still row-scaled value / lora_c as the fp16 K-padded LoRA operand of the dX product
+    // still row-scaled value / lora_c as the fp16 K-padded LoRA operand of the dX product;
+    // the product's reduction is split over ranges (partial sums, then lora_t_reduce)
     {
+      const int ks = dt_split(T, 3 * HD);
       EpiParams e = epi_base(idx, blk, n_kept, s0);
-      e.out = b.dt;
+      e.out = b.dtpart;
       e.ldo = 2 * LORA_R;
-      e.aux = b.dtb;
-      e.ld_aux = LORA_PAD;
-      e.alpha = ls;
-      e.beta = ls;
-      e.row_scale = b.rs_qkv;
-      e.aux_f16 = true;
-      e.aux_div = p.lora_c;
-      JENGA_TRY((launch_gemm<32, EPI_LORA_T>({b.dqkv16, T, 3 * HD}, {p.bcat, 2 * LORA_R, 3 * HD}, 3 * HD, nullptr,
-                                             nullptr, 0, T, 2 * LORA_R, e, st, "gemm_dt", nullptr, nullptr, 0,
-                                             /*f16_inputs=*/true)));
+      e.ksplit = ks;
+      JENGA_TRY((launch_gemm<32, EPI_STORE_F32>({b.dqkv16, T, 3 * HD}, {p.bcat, 2 * LORA_R, 3 * HD}, 3 * HD, nullptr,
+                                                nullptr, 0, T, 2 * LORA_R, e, st, "gemm_dt", nullptr, nullptr, 0,
+                                                /*f16_inputs=*/true)));
+      const int _ps = ::jenga::prof_begin("lora_t_reduce", st);
+      lora_t_reduce_kernel<<<grid_cap((int64_t)T * 32, 256), 256, 0, st>>>(
+          b.dtpart, ks, T, n_kept, blk, s0, ls, b.rs_qkv, p.lora_c, b.dt, 2 * LORA_R, b.dtb, LORA_PAD);
+      ::jenga::prof_end(_ps, st);
+      JENGA_LAUNCH_CHECK();
     }
     // xn of the segment (recomputed from the saved gathered input)
     JENGA_TRY(rmsnorm(s.xr + (size_t)s0 * h, h, nullptr, 1, s0, n_kept, blk, T, h, w->rms_eps,
@@ -802,9 +820,9 @@ extern "C" jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, con
     // dX[rows] = dh + RMSNorm_bwd(dxn)  (written in place into the gradient buffer)
     {
     const int _ps = ::jenga::prof_begin("rmsnorm_bwd_rows", st);
-    rmsnorm_bwd_rows_kernel<<<T, ROW_THREADS, 0, st>>>(b.dhn, h, s.xr + (size_t)s0 * h, h, s.rstd1 + s0,
-                                                        (const bf16*)w->attn_norm, b.dh, nullptr, h, nullptr, nullptr,
-                                                        nullptr, h, dX, h, idx, blk, s0, n_kept, blk, h, S);
+    (h <= 16 * ROW_THREADS ? rmsnorm_bwd_rows_kernel<2> : rmsnorm_bwd_rows_kernel<4>)<<<T, ROW_THREADS, 0, st>>>(
+        b.dhn, h, s.xr + (size_t)s0 * h, h, s.rstd1 + s0, (const bf16*)w->attn_norm, b.dh, nullptr, h, nullptr,
+        nullptr, nullptr, h, dX, h, idx, blk, s0, n_kept, blk, h, S, nullptr, 1);
     ::jenga::prof_end(_ps, st);
     }
     JENGA_LAUNCH_CHECK();

@@ -9,7 +9,9 @@
 namespace jenga {
 
 constexpr int ROW_THREADS = 256;
-constexpr int ROW_MAX_CHUNKS = 4;  // 8-element chunks per thread: hidden <= 8192
+// 8-element chunks per thread of the one-CTA-per-row kernels (a template argument MAXC: 2 for
+// hidden <= 4096, 4 for hidden <= 8192, so the row's registers do not cap the resident CTAs)
+constexpr int ROW_MAX_CHUNKS = 4;
 
 __device__ __forceinline__ float block_sum_256(float v, float* red) {
 #pragma unroll
@@ -82,6 +84,7 @@ __device__ __forceinline__ int64_t seq_row(const int32_t* idx, int blk, int c) {
 
 // xn[m] = bf16(x[row(m)] * rstd * gain); rstd[m]; optionally xr[m] = x[row(m)] (gathered copy).
 // One CTA per compact row m in [0, rows); row(m) = seq_row(idx, blk, row_offset + m).
+template <int MAXC>
 __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_rows_kernel(
     const bf16* __restrict__ x, int64_t ldx, const int32_t* __restrict__ idx, int blk, int row_offset,
     const int32_t* __restrict__ n_valid, int valid_mult, int h, float eps, const bf16* __restrict__ gain,
@@ -98,11 +101,11 @@ __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_rows_kernel(
   }
   const uint4* src = reinterpret_cast<const uint4*>(x + row * ldx);
   const int nch = h >> 3;
-  float v[ROW_MAX_CHUNKS][8];
-  uint4 raw[ROW_MAX_CHUNKS];
+  float v[MAXC][8];
+  uint4 raw[MAXC];
   float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < ROW_MAX_CHUNKS; ++i) {
+  for (int i = 0; i < MAXC; ++i) {
     const int c = threadIdx.x + i * ROW_THREADS;
     if (c < nch) {
       raw[i] = src[c];
@@ -116,7 +119,7 @@ __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_rows_kernel(
   if (threadIdx.x == 0 && rstd_out) rstd_out[m] = r;
   const uint4* gp = reinterpret_cast<const uint4*>(gain);
 #pragma unroll
-  for (int i = 0; i < ROW_MAX_CHUNKS; ++i) {
+  for (int i = 0; i < MAXC; ++i) {
     const int c = threadIdx.x + i * ROW_THREADS;
     if (c < nch) {
       if (xr) reinterpret_cast<uint4*>(xr + (int64_t)m * ldr)[c] = raw[i];
@@ -134,6 +137,7 @@ __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_rows_kernel(
 // base: fp32 (base_f) or bf16 (base_b); outputs: fp32 out_f, the fp16 GEMM operand out_h
 // (row m scaled by the power of two of pow2_row_scale, its inverse in out_rs[m]), and/or
 // the bf16 scatter into dst[row(m)] (in place, pitch ldd).
+template <int MAXC>
 __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_bwd_rows_kernel(
     const float* __restrict__ dy, int64_t lddy, const bf16* __restrict__ x, int64_t ldx,
     const float* __restrict__ rstd, const bf16* __restrict__ gain, const float* __restrict__ base_f,
@@ -148,10 +152,10 @@ __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_bwd_rows_kernel(
   // a row of a masked block (keep_mask entry 0) has no sub-block gradient: out = base
   const bool live = !keep_mask || __ldg(keep_mask + (row_offset + m) / mask_blk);
   const float r = live ? rstd[m] : 0.f;
-  float dyg[ROW_MAX_CHUNKS][8], xv[ROW_MAX_CHUNKS][8], bv[ROW_MAX_CHUNKS][8];
+  float dyg[MAXC][8], xv[MAXC][8], bv[MAXC][8];
   float dot = 0.f;
 #pragma unroll
-  for (int i = 0; i < ROW_MAX_CHUNKS; ++i) {
+  for (int i = 0; i < MAXC; ++i) {
     const int c = threadIdx.x + i * ROW_THREADS;
     if (c < nch) {
       // the residual base is loaded here too, so its latency overlaps the row reduction
@@ -193,7 +197,7 @@ __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_bwd_rows_kernel(
   }
   float amax = 0.f;
 #pragma unroll
-  for (int i = 0; i < ROW_MAX_CHUNKS; ++i) {
+  for (int i = 0; i < MAXC; ++i) {
     const int c = threadIdx.x + i * ROW_THREADS;
     if (c < nch) {
       float* o = bv[i];  // the output overwrites the residual base in registers
@@ -216,7 +220,7 @@ __global__ void __launch_bounds__(ROW_THREADS) rmsnorm_bwd_rows_kernel(
     pow2_row_scale(amax, sc, rs);
     if (threadIdx.x == 0) out_rs[m] = rs;
 #pragma unroll
-    for (int i = 0; i < ROW_MAX_CHUNKS; ++i) {
+    for (int i = 0; i < MAXC; ++i) {
       const int c = threadIdx.x + i * ROW_THREADS;
       if (c < nch) {
         uint4 u;
@@ -257,7 +261,8 @@ __global__ void gather_seg_kernel(const bf16* __restrict__ src, int64_t lds, bf1
 // H x 32 (head, frequency pair) items takes pair (2 ip, 2 ip + 1) of head hh, reading its
 // (cos, sin) pairs from the segment's RoPE table (tab[m][j], rope_table_kernel at offset
 // s0); the rotated values wait in registers for the row's largest magnitude.
-constexpr int RB_ITEMS = 8;  // items per thread: H <= RB_ITEMS * ROW_THREADS / 32 = 64
+// RB items per thread (a template argument: 4 for H <= 32, 8 for H <= 64)
+template <int RB>
 __global__ void __launch_bounds__(ROW_THREADS) rope_bwd_pack_kernel(
     const float* __restrict__ dq, int64_t ld_dq, const float* __restrict__ dk, const float* __restrict__ dv,
     int64_t ld_acc, int s0, __half* __restrict__ dqkv, float* __restrict__ rs, int64_t ld_out,
@@ -266,10 +271,10 @@ __global__ void __launch_bounds__(ROW_THREADS) rope_bwd_pack_kernel(
   const int m = blockIdx.x;
   if (m >= valid_rows(n_valid, valid_mult, s0, rows)) return;
   const int HD = H * 128, items = H * 32;
-  float val[RB_ITEMS][12];
+  float val[RB][12];
   float amax = 0.f;
 #pragma unroll
-  for (int k = 0; k < RB_ITEMS; ++k) {
+  for (int k = 0; k < RB; ++k) {
     const int e = threadIdx.x + k * ROW_THREADS;
     if (e < items) {
       const int ip = e & 31, hh = e >> 5;
@@ -304,7 +309,7 @@ __global__ void __launch_bounds__(ROW_THREADS) rope_bwd_pack_kernel(
   if (threadIdx.x == 0) rs[m] = r;
   __half* o = dqkv + (int64_t)m * ld_out;
 #pragma unroll
-  for (int k = 0; k < RB_ITEMS; ++k) {
+  for (int k = 0; k < RB; ++k) {
     const int e = threadIdx.x + k * ROW_THREADS;
     if (e < items) {
       const int ip = e & 31, hh = e >> 5;
@@ -374,11 +379,12 @@ __global__ void __launch_bounds__(256) lora_grad_partial_kernel(LoraGradJobs job
   for (int r = 0; r < 16; ++r) acc[r] = 0ull;
   if (c < jb.C) {
     const uint16_t* xp = reinterpret_cast<const uint16_t*>(jb.X) + (int64_t)m0 * jb.ldx + c;
-    for (int m = m0; m < m1; ++m, xp += jb.ldx) {
-      const float2 x = jb.x_f16 ? __half22float2(*reinterpret_cast<const __half2*>(xp))
-                                : __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(xp));
+    const bool xh = jb.x_f16;
+    auto rank_update = [&](uint32_t xw, int mr) {  // row mr (chunk-relative) of X and Y
+      const float2 x = xh ? __half22float2(*reinterpret_cast<const __half2*>(&xw))
+                          : __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw));
       const uint64_t x2 = f2pack(x.x, x.y);
-      const float4* yr = reinterpret_cast<const float4*>(sY + (m - m0) * 16);
+      const float4* yr = reinterpret_cast<const float4*>(sY + mr * 16);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float4 y = yr[q];
@@ -387,7 +393,17 @@ __global__ void __launch_bounds__(256) lora_grad_partial_kernel(LoraGradJobs job
         acc[4 * q + 2] = ffma2(x2, f2pack(y.z, y.z), acc[4 * q + 2]);
         acc[4 * q + 3] = ffma2(x2, f2pack(y.w, y.w), acc[4 * q + 3]);
       }
+    };
+    int m = m0;
+    // eight rows' X pairs in flight per step (the loop is load-latency bound otherwise)
+    for (; m + 8 <= m1; m += 8, xp += 8 * jb.ldx) {
+      uint32_t xw[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) xw[u] = *reinterpret_cast<const uint32_t*>(xp + u * jb.ldx);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) rank_update(xw[u], m - m0 + u);
     }
+    for (; m < m1; ++m, xp += jb.ldx) rank_update(*reinterpret_cast<const uint32_t*>(xp), m - m0);
     float lo[16], hi[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) f2unpack(acc[r], lo[r], hi[r]);
@@ -397,6 +413,30 @@ __global__ void __launch_bounds__(256) lora_grad_partial_kernel(LoraGradJobs job
       reinterpret_cast<float4*>(p)[q] = make_float4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
       reinterpret_cast<float4*>(p + 16)[q] = make_float4(hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
     }
+  }
+}
+
+// The LoRA term of the dX product from the split dt product (ksplit partial sums of
+// acc = dQKV' [Bq; Bv]^T over ranges of the reduction, dQKV' the row-scaled fp16 operand):
+//   dt[m, j] = ls r_m sum_ks part[ks][m][j]          (fp32, for the LoRA gradients)
+//   aux[m, j], aux[m, 32 + j] = fp16 hi, lo of ls sum_ks part[ks][m][j] / c
+// (the K-padded fp16 operand of the dX product; c = *cdiv, r_m = rs[m]).  The partial sums
+// are added in range order.
+__global__ void lora_t_reduce_kernel(const float* __restrict__ part, int ksplit, int rows,
+                                     const int32_t* __restrict__ n_valid, int valid_mult, int row_offset, float ls,
+                                     const float* __restrict__ rs, const float* __restrict__ cdiv,
+                                     float* __restrict__ dt, int64_t ld_dt, __half* __restrict__ aux, int64_t ld_aux) {
+  const int nv = valid_rows(n_valid, valid_mult, row_offset, rows);
+  const float ic = 1.f / __ldg(cdiv);  // a power of two: exact
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < nv * 32; e += gridDim.x * blockDim.x) {
+    const int m = e >> 5, j = e & 31;
+    float a = 0.f;
+    for (int ks = 0; ks < ksplit; ++ks) a += part[((int64_t)ks * rows + m) * 32 + j];
+    dt[(int64_t)m * ld_dt + j] = a * ls * __ldg(rs + m);
+    const float w = a * ls * ic;
+    const __half hi = __float2half_rn(w);
+    aux[(int64_t)m * ld_aux + j] = hi;
+    aux[(int64_t)m * ld_aux + 32 + j] = __float2half_rn(w - __half2float(hi));
   }
 }
 

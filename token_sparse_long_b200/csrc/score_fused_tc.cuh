@@ -63,21 +63,6 @@ __device__ __forceinline__ uint64_t sf_exp2_pair(uint64_t x2, int pair) {
   return ((SF_EMU_PAIRS >> (pair & 15)) & 1u) ? exp2_fma_x2<64>(x2) : exp2_mufu_x2(x2);
 }
 
-#ifndef SF_EXP_F16X2
-#define SF_EXP_F16X2 0
-#endif
-
-// 2^x for a pair of logits in fp16 (one ex2.approx.f16x2: both exponentials in one operation
-// of the exponential unit); x2 holds two fp32 arguments, rounded to fp16 first
-__device__ __forceinline__ uint32_t sf_exp2_h2(uint64_t x2) {
-  float a, b;
-  f2unpack(x2, a, b);
-  uint32_t h, e;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(b), "f"(a));
-  asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
-  return e;
-}
-
 __device__ __forceinline__ float sf_lg2(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -98,27 +83,6 @@ __device__ __forceinline__ void sf_update(const uint32_t* v, int cb, int limit, 
     float part[NH];
 #pragma unroll
     for (int hh = 0; hh < NH; ++hh) {
-#if SF_EXP_F16X2
-      // fp16 exponentials summed in four fp16 pairs of CH / 8 terms each (terms <= 1 while
-      // the reference max holds; an overflow makes the sum infinite and takes the exact path)
-      __half2 acch[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acch[i] = __float2half2_rn(0.f);
-#pragma unroll
-      for (int pr = 0; pr < CH / 2; ++pr) {
-        const int c = hh * CH + 2 * pr;
-        const uint64_t x2 = ffma2(f2pack(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), sl2x2, nm2);
-        const uint32_t e = sf_exp2_h2(x2);
-        acch[pr & 3] = __hadd2(acch[pr & 3], *reinterpret_cast<const __half2*>(&e));
-      }
-      float s[8];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __half22float2(acch[i]);
-        s[2 * i] = f.x;
-        s[2 * i + 1] = f.y;
-      }
-#else
       uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int pr = 0; pr < CH / 2; ++pr) {
@@ -129,7 +93,6 @@ __device__ __forceinline__ void sf_update(const uint32_t* v, int cb, int limit, 
       float s[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) f2unpack(acc2[i], s[2 * i], s[2 * i + 1]);
-#endif
       part[hh] = ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
     }
     float tot = part[0];
