@@ -303,7 +303,12 @@ JENGA_API jenga_status jenga_sparse_layer_fwd_mlp(const jenga_layer_weights* w, 
  * Frozen base weights get no gradient; LoRA gradients are ACCUMULATED into grads.
  * The retained rows are processed in consecutive segments of segment_tokens rows
  * (multiple of 128; last one short), last segment first, so per-segment scratch is
- * bounded by the segment length (Jenga summary §4.4.2). */
+ * bounded by the segment length (Jenga summary §4.4.2).  Precision: fp32 accumulation
+ * throughout; the products with the frozen weights take the gradient rows as fp16, each
+ * row scaled by the power of two that puts its largest magnitude in [2^13, 2^14) (undone
+ * exactly in the product's epilogue); the attention backward runs on fp16 copies of q, k,
+ * v and of the segment's dO scaled by a power of two.  Deterministic: a fixed reduction
+ * order everywhere, so repeated calls give identical bits. */
 JENGA_API size_t jenga_layer_bwd_workspace_bytes(const jenga_layer_weights* w, int B, int blk, int n_kept_max,
                                        int segment_tokens);
 JENGA_API jenga_status jenga_sparse_layer_bwd(const jenga_layer_weights* w, const jenga_lora* lora, const void* packed,

@@ -243,3 +243,25 @@ def test_pack_reports_weight_outside_fp16_range(J):
         J.jenga_check_device_status()
     assert ei.value.status == 1  # JENGA_EINVAL
     J.jenga_check_device_status()  # cleared by the read
+
+
+def test_step_is_deterministic(J):
+    """Scoring (with its dynamically dealt work items), selection, forward and the segmented
+    backward use fixed reduction orders: two runs on the same inputs give identical bits."""
+    case = small_case(seed=5, S=1024, blk=64)
+    a = run_layer_gpu(case, keep=0.5, seg=256)
+    b = run_layer_gpu(case, keep=0.5, seg=256, handle=a["handle"])
+    assert np.array_equal(a["scores"], b["scores"])
+    assert np.array_equal(a["idx"], b["idx"]) and a["n_kept"] == b["n_kept"]
+    assert np.array_equal(a["out"], b["out"])
+    assert np.array_equal(a["dx"], b["dx"])
+    for k in a["grads"]:
+        assert np.array_equal(a["grads"][k], b["grads"][k]), k
+    # the scoring alone with many CTAs taking work items from the shared counter
+    g = torch.Generator(device="cuda").manual_seed(7)
+    q = (torch.randn(8192, 32 * 128, device="cuda", generator=g) * 0.3).to(torch.bfloat16)
+    k = (torch.randn(8192, 32 * 128, device="cuda", generator=g) * 0.3).to(torch.bfloat16)
+    s1 = J.jenga_score_blocks(q, k, 32, 128, 128)
+    s2 = J.jenga_score_blocks(q, k, 32, 128, 128)
+    J.jenga_check_device_status()
+    assert torch.equal(s1, s2)
