@@ -9,9 +9,9 @@
 namespace jenga {
 
 constexpr int ROW_THREADS = 256;
-// 8-element chunks per thread of the one-CTA-per-row kernels (a template argument MAXC: 2 for
-// hidden <= 4096, 4 for hidden <= 8192, so the row's registers do not cap the resident CTAs)
-constexpr int ROW_MAX_CHUNKS = 4;
+// The one-CTA-per-row kernels take the 8-element chunks per thread as a template argument
+// MAXC (2 for hidden <= 4096, 4 for hidden <= 8192), so a row's registers do not cap the
+// resident CTAs.
 
 __device__ __forceinline__ float block_sum_256(float v, float* red) {
 #pragma unroll
