@@ -45,8 +45,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-movement", action="store_true", help="skip the standalone gather/scatter/select timing")
     ap.add_argument("--no-lm-loss", action="store_true", help="skip the segmented LM-head loss timing")
-    ap.add_argument("--oracle-one-thread", action="store_true",
-                    help="time the CPU oracle on one thread over the two small workloads, in full, and exit")
+    ap.add_argument("--cpu-baseline-one-thread", action="store_true",
+                    help="the cpu_baseline leg on one host thread: the CPU oracle over the two small workloads, "
+                         "in full, then exit")
     return ap.parse_args()
 
 
@@ -416,8 +417,9 @@ def replica_tokens_per_s(S, world, ms):
     return S * world / (ms / 1e3)
 
 
-def oracle_one_thread():
-    """The CPU oracle on one host thread, each small workload in full: ``score_fp32`` (S 512,
+def cpu_baseline_one_thread():
+    """The cpu_baseline leg's one-thread figure: the CPU oracle on one host thread, each small
+    workload in full: ``score_fp32`` (S 512,
     4 heads x 64, blocks of 32: fp32 block scores, mean-threshold selection, gather, scatter-add
     of 2 x the gathered rows) and ``llama7b_s4k`` (one 7B-shaped layer at S 4096, blocks of 64,
     keep 50 %: q/k of all rows, block scores, top-k selection, retained-token forward and
@@ -444,13 +446,13 @@ def oracle_one_thread():
         Ws = oracle_weights(case)
         dt, flops = oracle_sample(case, case.S, list(w.keep), Ws)
         out["llama7b_s4k"] = {"seconds": dt, "tokens_per_s": case.S / dt, "gflop": flops / 1e9}
-    print(json.dumps({"oracle_one_thread": out, "threads": 1}), flush=True)
+    print(json.dumps({"cpu_baseline_one_thread": out, "kind": "oracle", "cores": 1}), flush=True)
 
 
 def main():
     args = parse()
-    if args.oracle_one_thread:
-        oracle_one_thread()
+    if args.cpu_baseline_one_thread:
+        cpu_baseline_one_thread()
         return
     if args.impl == "reference":
         run_reference(args)
