@@ -419,11 +419,11 @@ def replica_tokens_per_s(S, world, ms):
 
 def cpu_baseline_one_thread():
     """The cpu_baseline leg's one-thread figure: the CPU oracle on one host thread, each small
-    workload in full: ``score_fp32`` (S 512,
-    4 heads x 64, blocks of 32: fp32 block scores, mean-threshold selection, gather, scatter-add
-    of 2 x the gathered rows) and ``llama7b_s4k`` (one 7B-shaped layer at S 4096, blocks of 64,
-    keep 50 %: q/k of all rows, block scores, top-k selection, retained-token forward and
-    backward).  Inputs and oracle weights are built before the clock starts."""
+    workload in full: ``score_fp32`` (S 512, 4 heads x 64, blocks of 32: fp32 block scores,
+    mean-threshold selection, gather, scatter-add of 2 x the gathered rows) and ``llama7b_s4k``
+    (one 7B-shaped layer at S 4096, blocks of 64, keep 50 %: q/k of all rows, block scores,
+    top-k selection, retained-token forward and backward).  Inputs and oracle weights are
+    built before the clock starts."""
     from threadpoolctl import threadpool_limits
     from oracle import movement as omv
     from oracle import scores as osc
